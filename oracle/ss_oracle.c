@@ -1,0 +1,289 @@
+/*
+ * ss_oracle.c -- plain float64 CPU reference for the Mamba-1 selective scan (S6)
+ * forward pass and its single-token decode state update.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or helper with the CUDA library under
+ * selective_state_space_18_b200/csrc, and it never calls it.
+ *
+ * What it computes (nnterp docs, "selective_scan" component, SelectiveScan class
+ * description; TransformerLens "ssm_mixer" module, compute_ssm_state):
+ *
+ *   dt_t   = softplus(dt_raw[b,c,t] + dt_bias[c])      (or no softplus when disabled)
+ *   h_t[n] = exp(dt_t * A[c,n]) * h_{t-1}[n] + dt_t * B[b,n,t] * x[b,c,t]
+ *   y_t    = sum_n C[b,n,t] * h_t[n] + D[c] * x[b,c,t]
+ *   out_t  = y_t * silu(z[b,c,t])                        (only when z is given)
+ *
+ * with h_{-1} = h0[b,c,:] (zeros when h0 is NULL), and h_last = h_{L-1}.
+ * Enforced boundary reset (the "s6_reset" blog draft, "Enforced Boundary Resetting";
+ * the packed-sequence workload fixes the flag on each document's FIRST token):
+ * at a flagged token the state is zeroed before that token's update, so
+ * h_t = dt_t * B_t * x_t there.
+ *
+ * Layouts are channel-first as the nnterp page states for the kernel's tensors:
+ * x, dt, z, y [batch, channels, seq]; B, C [batch, state_dim, seq];
+ * A [channels, state_dim]; D, dt_bias [channels]; reset [batch, seq];
+ * h0, h_last, decode state [batch, channels, state_dim].  Every array is
+ * contiguous float64 except reset (uint8).
+ *
+ * Two independent orderings of the same recurrence are provided:
+ *   ss_oracle_scan      -- the token loop, in sequence order;
+ *   ss_oracle_tree_scan -- an inclusive associative scan (recursive doubling) of
+ *                          the affine maps h -> a*h + u with an explicit reset
+ *                          flag ("s6_reset", "Associative Boundary Resetting").
+ * The test suite pins each against closed forms and against the other.
+ *
+ * Parallelism: OpenMP over independent (batch, channel) rows only, so that the
+ * benchmark's CPU-baseline timing can use the host's cores.  Nothing else is
+ * blocked, fused or reordered.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORC_OK = 0, ORC_ERR_NULL = 1, ORC_ERR_SHAPE = 2, ORC_ERR_NOMEM = 3 };
+
+/* softplus(r) = log(1 + e^r), evaluated without overflow for large r. */
+static double orc_softplus(double r)
+{
+    if (r > 0.0)
+        return r + log1p(exp(-r));
+    return log1p(exp(r));
+}
+
+/* silu(v) = v * sigmoid(v) = v / (1 + e^{-v}). */
+static double orc_silu(double v)
+{
+    return v / (1.0 + exp(-v));
+}
+
+/* Step size of token t of row (b,c): bias added before the softplus, per channel
+ * (nnterp selective_scan: dt = softplus(dt_proj(x) + dt_bias)). */
+static double orc_step(const double *dt, const double *dt_bias, int dt_softplus,
+                       int64_t idx, int64_t c)
+{
+    double r = dt[idx] + (dt_bias ? dt_bias[c] : 0.0);
+    return dt_softplus ? orc_softplus(r) : r;
+}
+
+int ss_oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * Token loop.  h_all (nullable) receives the state after every token,
+ * [batch, channels, seq, state_dim] -- the "state after each token" the nnterp
+ * page reads from the token loop.
+ */
+int ss_oracle_scan(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
+                   const double *x, const double *dt, const double *A, const double *B,
+                   const double *C, const double *D, const double *z, const double *dt_bias,
+                   const uint8_t *reset, const double *h0, int dt_softplus,
+                   double *y, double *h_last, double *h_all, int nthreads)
+{
+    if (!x || !dt || !A || !B || !C || !y)
+        return ORC_ERR_NULL;
+    if (batch <= 0 || channels <= 0 || state_dim <= 0 || seq <= 0)
+        return ORC_ERR_SHAPE;
+    if (nthreads <= 0)
+        nthreads = 1;
+    const int64_t rows = batch * channels;
+    int status = ORC_OK;
+
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1)
+    for (int64_t row = 0; row < rows; ++row) {
+        const int64_t b = row / channels;
+        const int64_t c = row % channels;
+        double *h = (double *)malloc((size_t)state_dim * sizeof(double));
+        if (!h) {
+#pragma omp atomic write
+            status = ORC_ERR_NOMEM;
+            continue;
+        }
+        for (int64_t n = 0; n < state_dim; ++n)
+            h[n] = h0 ? h0[row * state_dim + n] : 0.0;
+
+        for (int64_t t = 0; t < seq; ++t) {
+            const int64_t idx = row * seq + t;
+            const double d = orc_step(dt, dt_bias, dt_softplus, idx, c);
+            const double xv = x[idx];
+            if (reset && reset[b * seq + t]) {
+                /* state zeroed before this token's update */
+                for (int64_t n = 0; n < state_dim; ++n)
+                    h[n] = 0.0;
+            }
+            double acc = 0.0;
+            for (int64_t n = 0; n < state_dim; ++n) {
+                const double Bn = B[(b * state_dim + n) * seq + t];
+                const double Cn = C[(b * state_dim + n) * seq + t];
+                h[n] = exp(d * A[c * state_dim + n]) * h[n] + d * Bn * xv;
+                acc += Cn * h[n];
+            }
+            double yv = acc + (D ? D[c] : 0.0) * xv;
+            if (z)
+                yv *= orc_silu(z[idx]);
+            y[idx] = yv;
+            if (h_all)
+                for (int64_t n = 0; n < state_dim; ++n)
+                    h_all[(row * seq + t) * state_dim + n] = h[n];
+        }
+        if (h_last)
+            for (int64_t n = 0; n < state_dim; ++n)
+                h_last[row * state_dim + n] = h[n];
+        free(h);
+    }
+    return status;
+}
+
+/*
+ * Element of the associative scan: the affine map h -> (r ? u : a*h + u).
+ * Composition "left then right" ("s6_reset", Associative Boundary Resetting:
+ * the binary operator (A_i, Bx_i) o (A_j, Bx_j) = (A_i A_j, A_j Bx_i + Bx_j),
+ * extended by a flag that records whether the segment contains a reset; when
+ * it does, the incoming state is discarded so the decay no longer matters).
+ */
+typedef struct {
+    double a, u;
+    int r;
+} orc_elem;
+
+static orc_elem orc_combine(orc_elem left, orc_elem right)
+{
+    orc_elem out;
+    if (right.r) {
+        out = right;
+    } else if (left.r) {
+        out.a = 1.0; /* unused: the segment discards its input state */
+        out.u = right.a * left.u + right.u;
+        out.r = 1;
+    } else {
+        out.a = left.a * right.a;
+        out.u = right.a * left.u + right.u;
+        out.r = 0;
+    }
+    return out;
+}
+
+/*
+ * Associative-scan ordering of the same recurrence: for every (b, c, n) the
+ * sequence of maps is reduced to inclusive prefixes by recursive doubling
+ * (Hillis-Steele), then h_t = prefix_t applied to h0.
+ */
+int ss_oracle_tree_scan(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
+                        const double *x, const double *dt, const double *A, const double *B,
+                        const double *C, const double *D, const double *z,
+                        const double *dt_bias, const uint8_t *reset, const double *h0,
+                        int dt_softplus, double *y, double *h_last, int nthreads)
+{
+    if (!x || !dt || !A || !B || !C || !y)
+        return ORC_ERR_NULL;
+    if (batch <= 0 || channels <= 0 || state_dim <= 0 || seq <= 0)
+        return ORC_ERR_SHAPE;
+    if (nthreads <= 0)
+        nthreads = 1;
+    const int64_t rows = batch * channels;
+    int status = ORC_OK;
+
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1)
+    for (int64_t row = 0; row < rows; ++row) {
+        const int64_t b = row / channels;
+        const int64_t c = row % channels;
+        orc_elem *e = (orc_elem *)malloc((size_t)seq * sizeof(orc_elem));
+        double *hs = (double *)malloc((size_t)(seq * state_dim) * sizeof(double));
+        double *steps = (double *)malloc((size_t)seq * sizeof(double));
+        if (!e || !hs || !steps) {
+            free(e);
+            free(hs);
+            free(steps);
+#pragma omp atomic write
+            status = ORC_ERR_NOMEM;
+            continue;
+        }
+        for (int64_t t = 0; t < seq; ++t)
+            steps[t] = orc_step(dt, dt_bias, dt_softplus, row * seq + t, c);
+
+        for (int64_t n = 0; n < state_dim; ++n) {
+            const double An = A[c * state_dim + n];
+            for (int64_t t = 0; t < seq; ++t) {
+                e[t].a = exp(steps[t] * An);
+                e[t].u = steps[t] * B[(b * state_dim + n) * seq + t] * x[row * seq + t];
+                e[t].r = reset ? (reset[b * seq + t] != 0) : 0;
+            }
+            for (int64_t d = 1; d < seq; d *= 2) {
+                /* descending t: element t - d still holds the previous round's value */
+                for (int64_t t = seq - 1; t >= d; --t)
+                    e[t] = orc_combine(e[t - d], e[t]);
+            }
+            const double hin = h0 ? h0[row * state_dim + n] : 0.0;
+            for (int64_t t = 0; t < seq; ++t)
+                hs[t * state_dim + n] = e[t].r ? e[t].u : e[t].a * hin + e[t].u;
+        }
+
+        for (int64_t t = 0; t < seq; ++t) {
+            const int64_t idx = row * seq + t;
+            double acc = 0.0;
+            for (int64_t n = 0; n < state_dim; ++n)
+                acc += C[(b * state_dim + n) * seq + t] * hs[t * state_dim + n];
+            double yv = acc + (D ? D[c] : 0.0) * x[idx];
+            if (z)
+                yv *= orc_silu(z[idx]);
+            y[idx] = yv;
+        }
+        if (h_last)
+            for (int64_t n = 0; n < state_dim; ++n)
+                h_last[row * state_dim + n] = hs[(seq - 1) * state_dim + n];
+        free(e);
+        free(hs);
+        free(steps);
+    }
+    return status;
+}
+
+/*
+ * Single-token decode update (nnterp selective_scan: mamba_selective_state_update
+ * on a decode step; the state [batch, channels, state_dim] is updated in place and
+ * is what the next step starts from).  x, dt, z, y are [batch, channels];
+ * B, C are [batch, state_dim].  No reset on this path.
+ */
+int ss_oracle_update(int64_t batch, int64_t channels, int64_t state_dim, double *state,
+                     const double *x, const double *dt, const double *A, const double *B,
+                     const double *C, const double *D, const double *z,
+                     const double *dt_bias, int dt_softplus, double *y, int nthreads)
+{
+    if (!state || !x || !dt || !A || !B || !C || !y)
+        return ORC_ERR_NULL;
+    if (batch <= 0 || channels <= 0 || state_dim <= 0)
+        return ORC_ERR_SHAPE;
+    if (nthreads <= 0)
+        nthreads = 1;
+    const int64_t rows = batch * channels;
+
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+    for (int64_t row = 0; row < rows; ++row) {
+        const int64_t b = row / channels;
+        const int64_t c = row % channels;
+        const double d = orc_step(dt, dt_bias, dt_softplus, row, c);
+        const double xv = x[row];
+        double *h = state + row * state_dim;
+        double acc = 0.0;
+        for (int64_t n = 0; n < state_dim; ++n) {
+            h[n] = exp(d * A[c * state_dim + n]) * h[n] + d * B[b * state_dim + n] * xv;
+            acc += C[b * state_dim + n] * h[n];
+        }
+        double yv = acc + (D ? D[c] : 0.0) * xv;
+        if (z)
+            yv *= orc_silu(z[row]);
+        y[row] = yv;
+    }
+    return ORC_OK;
+}
