@@ -1,0 +1,148 @@
+/*
+ * ss_scan.h -- C ABI of libssscan.so: the Mamba-1 selective scan (S6) forward pass
+ * and its single-token decode state update on NVIDIA B200 (sm_100a).
+ *
+ * What is computed (nnterp documentation, "selective_scan" component: the
+ * SelectiveScan class description and the two kernel calls it names,
+ * mamba_selective_scan on a prompt and mamba_selective_state_update on a decode
+ * step; TransformerLens "ssm_mixer" module, compute_ssm_state):
+ *
+ *   dt_t   = softplus(dt_raw[b,c,t] + dt_bias[c])     (flag SS_DT_SOFTPLUS; else the sum)
+ *   h_t[n] = exp(dt_t * A[c,n]) * h_{t-1}[n] + dt_t * B[b,n,t] * x[b,c,t]
+ *   y_t    = sum_n C[b,n,t] * h_t[n] + D[c] * x[b,c,t]
+ *   out_t  = y_t * silu(z[b,c,t])                       (only when z is not NULL)
+ *
+ * Enforced boundary reset ("s6_reset" blog draft, Enforced Boundary Resetting):
+ * where reset[b,t] != 0 the state is zeroed before token t's update, so
+ * h_t = dt_t * B[b,:,t] * x[b,c,t] there; the mask is shared by all channels.
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers to contiguous, row-major arrays in the
+ *    channel-first layouts below.  The caller owns all memory; the library never
+ *    allocates, frees or keeps a pointer after the call returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  They return after the launch is enqueued, without synchronising.
+ *  - Host-side validation runs first; on any error nothing is launched and the
+ *    status below is returned.  A launch failure reported by the CUDA runtime
+ *    returns SS_ERR_CUDA.
+ *  - Inputs are never modified.  Outputs must not overlap any input, except that
+ *    h_last may be the very same buffer as h0 (chaining in place).
+ *  - A, D, dt_bias, h0, h_last and the decode state are float32.  x, dt, z, B, C and
+ *    y share the element type `dtype` (float32 or bfloat16); y is rounded to it
+ *    round-to-nearest-even.  State and accumulation are float32.
+ *  - Pointers must be aligned to their element size (SS_ERR_ALIGN otherwise);
+ *    16-byte alignment and seq a multiple of 8 enable the vectorised path, any
+ *    other size or alignment takes a predicated scalar path.
+ */
+#ifndef SS_SCAN_H
+#define SS_SCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SS_API __attribute__((visibility("default")))
+#else
+#define SS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *ss_stream_t;
+
+/* Element type of x, dt, z, B, C and y. */
+typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_dtype_t;
+
+/* Status codes. */
+enum {
+    SS_OK = 0,
+    SS_ERR_NULL = 1,        /* a required pointer is NULL                          */
+    SS_ERR_SHAPE = 2,       /* a size is <= 0 or too large for the launch grid     */
+    SS_ERR_DTYPE = 3,       /* dtype is not SS_F32 or SS_BF16                       */
+    SS_ERR_ALIGN = 4,       /* a pointer is not aligned to its element size        */
+    SS_ERR_UNSUPPORTED = 5, /* state_dim not in {4, 8, 16}, or an unknown flag bit */
+    SS_ERR_CUDA = 6,        /* the CUDA runtime reported an error                  */
+    SS_ERR_TIMEOUT = 7,     /* a bounded device-side wait gave up                  */
+    SS_ERR_ALIAS = 8,       /* an output (or the workspace) overlaps an input      */
+    SS_ERR_WORKSPACE = 9    /* workspace smaller than ss_scan_workspace_bytes()    */
+};
+
+/* flags bit 0: apply softplus to dt_raw + dt_bias (mamba's delta_softplus). */
+enum { SS_DT_SOFTPLUS = 1u };
+
+/*
+ * Prompt scan: the recurrence above over all `seq` tokens of every (b, c) row.
+ *
+ *   x, dt_raw, z : [batch, channels, seq]  dtype      (z nullable: no gate)
+ *   A            : [channels, state_dim]   float32    (negative rates)
+ *   B, C         : [batch, state_dim, seq] dtype      (shared by every channel)
+ *   D, dt_bias   : [channels]              float32    (nullable: 0)
+ *   reset        : [batch, seq]            uint8      (nullable: no resets)
+ *   h0           : [batch, channels, state_dim] float32 (nullable: zeros)
+ *   y            : [batch, channels, seq]  dtype      (output)
+ *   h_last       : [batch, channels, state_dim] float32 (nullable output: the state
+ *                  after the last token, what the next decode step starts from)
+ *   workspace    : nullable device buffer of at least ss_scan_workspace_bytes()
+ *                  bytes, 16-byte aligned, zero-filled by the caller before its FIRST
+ *                  use (cudaMemset); every call that completes leaves it ready for the
+ *                  next one.  With a workspace the sequence is split into segments
+ *                  processed by persistent CTAs that pass the scan carry between
+ *                  them, which balances the GPU for any shape.  Without one, each CTA
+ *                  scans one group of channels over the whole sequence.  Calls that
+ *                  share a workspace must be ordered (same stream, or synchronised);
+ *                  after SS_ERR_TIMEOUT is reported, zero it again before reuse.
+ *
+ * state_dim must be 4, 8 or 16.  Returns SS_OK or an error status.
+ */
+SS_API int ss_scan_fwd(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
+                       ss_dtype_t dtype, const void *x, const void *dt_raw, const float *A,
+                       const void *B, const void *C, const float *D, const void *z,
+                       const float *dt_bias, const uint8_t *reset, const float *h0,
+                       uint32_t flags, void *y, float *h_last, void *workspace,
+                       size_t workspace_bytes, ss_stream_t stream);
+
+/* Workspace bytes ss_scan_fwd needs for this shape (0 for an invalid shape). */
+SS_API int64_t ss_scan_workspace_bytes(int64_t batch, int64_t channels, int64_t state_dim,
+                                       int64_t seq);
+
+/*
+ * Device-side status of earlier scans: synchronises `stream`, then reads and clears
+ * the status word of `workspace` (or, for NULL, the word shared by calls made without
+ * a workspace on the current device).  *status becomes SS_OK, or SS_ERR_TIMEOUT if a
+ * bounded wait inside a kernel gave up (its outputs are then invalid).  Returns
+ * SS_OK, or an error status if the query itself failed.
+ */
+SS_API int ss_scan_status(const void *workspace, ss_stream_t stream, int *status);
+
+/*
+ * Decode step: one token of the same recurrence for every (b, c), updating `state`
+ * in place (nnterp selective_scan: the updated state is what the cache receives).
+ *
+ *   state        : [batch, channels, state_dim] float32 (in/out)
+ *   x, dt_raw, z : [batch, channels]        dtype        (z nullable)
+ *   A            : [channels, state_dim]    float32
+ *   B, C         : [batch, state_dim]       dtype
+ *   D, dt_bias   : [channels]               float32      (nullable)
+ *   y            : [batch, channels]        dtype        (output)
+ *
+ * No reset on this path.  Returns SS_OK or an error status.
+ */
+SS_API int ss_state_update(int64_t batch, int64_t channels, int64_t state_dim, ss_dtype_t dtype,
+                    float *state, const void *x, const void *dt_raw, const float *A,
+                    const void *B, const void *C, const float *D, const void *z,
+                    const float *dt_bias, uint32_t flags, void *y, ss_stream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+SS_API const char *ss_status_string(int status);
+
+/* ABI version of this library: (major << 16) | minor. */
+SS_API int ss_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SS_SCAN_H */

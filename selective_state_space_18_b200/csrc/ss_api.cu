@@ -1,0 +1,441 @@
+// ss_api.cu -- the C ABI of libssscan.so (declarations and contracts: ss_scan.h).
+//
+// Host-side validation, dispatch on (state_dim, dtype, reset present, vector path)
+// and launch on the caller's stream.  No allocation, no synchronisation.
+#include "ss_scan.h"
+
+#include <atomic>
+#include <cstring>
+#include <cstdint>
+#include <cudaTypedefs.h> // PFN_cuTensorMapEncodeTiled
+
+#include "ss_scan_fwd.cuh"
+#include "ss_state_update.cuh"
+
+namespace {
+
+constexpr int kAbiMajor = 2, kAbiMinor = 0;
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// [p, p + n) and [q, q + m) intersect (NULL or empty ranges never do).
+bool overlaps(const void *p, size_t n, const void *q, size_t m)
+{
+    if (!p || !q || n == 0 || m == 0)
+        return false;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
+    return a < b + m && b < a + n;
+}
+
+bool mul_ok(int64_t a, int64_t b, int64_t *out) { return !__builtin_mul_overflow(a, b, out); }
+
+// Raise the dynamic shared-memory limit of a kernel once per device; `done_mask`
+// is owned by the caller's kernel instantiation.
+template <typename K> int ensure_smem(K kernel, size_t bytes, std::atomic<uint64_t> &done_mask)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return SS_ERR_CUDA;
+    const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+    if (bit && (done_mask.load(std::memory_order_acquire) & bit))
+        return SS_OK;
+    if (bytes > 48 * 1024 &&
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)) != cudaSuccess)
+        return SS_ERR_CUDA;
+    done_mask.fetch_or(bit, std::memory_order_acq_rel);
+    return SS_OK;
+}
+
+int launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
+}
+
+// Status word of calls made without a workspace (one per device that loads the
+// library); read and cleared by ss_scan_status(NULL, ...).
+__device__ uint32_t g_ss_status_word;
+
+int status_word_address(uint32_t **out)
+{
+    static std::atomic<uintptr_t> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return SS_ERR_CUDA;
+    if (dev < 64) {
+        const uintptr_t v = cache[dev].load(std::memory_order_acquire);
+        if (v) {
+            *out = reinterpret_cast<uint32_t *>(v);
+            return SS_OK;
+        }
+    }
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_ss_status_word) != cudaSuccess)
+        return SS_ERR_CUDA;
+    if (dev < 64)
+        cache[dev].store(reinterpret_cast<uintptr_t>(ptr), std::memory_order_release);
+    *out = static_cast<uint32_t *>(ptr);
+    return SS_OK;
+}
+
+int device_sm_count(int *sms)
+{
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return SS_ERR_CUDA;
+    int v = dev < 64 ? cache[dev].load(std::memory_order_acquire) : 0;
+    if (!v) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return SS_ERR_CUDA;
+        if (dev < 64)
+            cache[dev].store(v, std::memory_order_release);
+    }
+    *sms = v;
+    return SS_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+PFN_cuTensorMapEncodeTiled tensor_map_encoder()
+{
+    static std::atomic<void *> fn{nullptr};
+    void *f = fn.load(std::memory_order_acquire);
+    if (!f) {
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn.store(f, std::memory_order_release);
+    }
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled>(f);
+}
+
+// 2-D map over `rows` rows of `inner` contiguous elements, box = chunk x box_rows.
+template <typename T>
+bool encode_rows(CUtensorMap *map, const void *base, int64_t inner, int64_t rows, uint32_t box_inner,
+                 uint32_t box_rows)
+{
+    PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
+    if (!enc)
+        return false;
+    const CUtensorMapDataType dt = sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const cuuint64_t dims[2] = {cuuint64_t(inner), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(inner) * sizeof(T)};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int N, typename T>
+bool build_maps(const ss::ScanArgs &a, ss::TmaMaps *m)
+{
+    using S = ss::ScanShape<N>;
+    const int64_t rows = a.batch * a.channels, brows = a.batch * N;
+    return encode_rows<T>(&m->x, a.x, a.seq, rows, S::kChunk, S::kChanPerCta) &&
+           encode_rows<T>(&m->dt, a.dt, a.seq, rows, S::kChunk, S::kChanPerCta) &&
+           encode_rows<T>(&m->z, a.z ? a.z : a.x, a.seq, rows, S::kChunk, S::kChanPerCta) &&
+           encode_rows<T>(&m->B, a.B, a.seq, brows, S::kChunk, N) &&
+           encode_rows<T>(&m->C, a.C, a.seq, brows, S::kChunk, N);
+}
+
+template <int N, typename T, bool R, bool V>
+int launch_scan(ss::ScanArgs a, cudaStream_t stream)
+{
+    using S = ss::ScanShape<N>;
+    constexpr size_t kSmem = S::template smem_bytes<T, V>();
+    auto kernel = ss::ss_scan_fwd_kernel<N, T, R, V>;
+    static std::atomic<uint64_t> smem_done{0};
+    static std::atomic<int> occ_cache[64];
+    int st = ensure_smem(kernel, kSmem, smem_done);
+    if (st != SS_OK)
+        return st;
+    const int64_t nchunks = (a.seq + S::kChunk - 1) / S::kChunk;
+    int64_t grid = a.groups;
+    if (a.workspace) {
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || device_sm_count(&sms) != SS_OK)
+            return SS_ERR_CUDA;
+        int occ = dev < 64 ? occ_cache[dev].load(std::memory_order_acquire) : 0;
+        if (!occ) {
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, S::kThreads, kSmem) != cudaSuccess)
+                return SS_ERR_CUDA;
+            occ = occ > 0 ? occ : 1;
+            if (dev < 64)
+                occ_cache[dev].store(occ, std::memory_order_release);
+        }
+        const int64_t resident = int64_t(sms) * occ;
+        // about eight units per resident CTA, segments of at least eight chunks
+        int64_t segs = (8 * resident + a.groups - 1) / a.groups;
+        const int64_t max_segs = nchunks / 8 > 1 ? nchunks / 8 : 1;
+        segs = segs < 1 ? 1 : (segs > max_segs ? max_segs : segs);
+        const int64_t seg_chunks = (nchunks + segs - 1) / segs;
+        a.seg_len = seg_chunks * S::kChunk;
+        a.segments = (nchunks + seg_chunks - 1) / seg_chunks;
+        const int64_t units = a.groups * a.segments;
+        grid = units < resident ? units : resident;
+    } else {
+        a.seg_len = nchunks * S::kChunk;
+        a.segments = 1;
+        if (status_word_address(&a.status) != SS_OK)
+            return SS_ERR_CUDA;
+    }
+    if (grid > 0x7fffffffLL)
+        return SS_ERR_SHAPE;
+    ss::TmaMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (V && !build_maps<N, T>(a, &maps))
+        return SS_ERR_CUDA;
+    kernel<<<unsigned(grid), S::kThreads, kSmem, stream>>>(a, maps);
+    return launch_status();
+}
+
+template <int N, typename T>
+int dispatch_scan_t(const ss::ScanArgs &a, bool vec, cudaStream_t s)
+{
+    const bool r = a.reset != nullptr;
+    if (r)
+        return vec ? launch_scan<N, T, true, true>(a, s) : launch_scan<N, T, true, false>(a, s);
+    return vec ? launch_scan<N, T, false, true>(a, s) : launch_scan<N, T, false, false>(a, s);
+}
+
+template <int N> int64_t scan_groups(int64_t batch, int64_t channels)
+{
+    const int64_t per = ss::ScanShape<N>::kChanPerCta;
+    return batch * ((channels + per - 1) / per);
+}
+
+template <int N>
+int dispatch_scan_n(ss::ScanArgs a, ss_dtype_t dtype, bool vec, size_t ws_bytes, cudaStream_t s)
+{
+    a.groups_per_batch = (a.channels + ss::ScanShape<N>::kChanPerCta - 1) / ss::ScanShape<N>::kChanPerCta;
+    if (!mul_ok(a.batch, a.groups_per_batch, &a.groups) || a.groups > 0x7fffffffLL)
+        return SS_ERR_SHAPE;
+    if (a.workspace && ws_bytes < size_t(ss::scan_workspace_bytes<N>(a.groups)))
+        return SS_ERR_WORKSPACE;
+    if (dtype == SS_BF16)
+        return dispatch_scan_t<N, __nv_bfloat16>(a, vec, s);
+    return dispatch_scan_t<N, float>(a, vec, s);
+}
+
+template <int N, typename T, bool V>
+int launch_update(ss::UpdateArgs a, cudaStream_t stream)
+{
+    const int64_t per_block = int64_t(ss::kUpdateThreads) * ss::kUpdateItems; // row quarters
+    const int64_t quarters = a.channels * (N / 4);
+    a.blocks_per_row = int((quarters + per_block - 1) / per_block);
+    const int64_t blocks = a.batch * a.blocks_per_row;
+    if (blocks > 0x7fffffffLL)
+        return SS_ERR_SHAPE;
+    ss::ss_state_update_kernel<N, T, V><<<unsigned(blocks), ss::kUpdateThreads, 0, stream>>>(a);
+    return launch_status();
+}
+
+template <int N>
+int dispatch_update_n(const ss::UpdateArgs &a, ss_dtype_t dtype, bool vec, cudaStream_t s)
+{
+    if (dtype == SS_BF16)
+        return vec ? launch_update<N, __nv_bfloat16, true>(a, s) : launch_update<N, __nv_bfloat16, false>(a, s);
+    return vec ? launch_update<N, float, true>(a, s) : launch_update<N, float, false>(a, s);
+}
+
+} // namespace
+
+extern "C" {
+
+int ss_abi_version(void) { return (kAbiMajor << 16) | kAbiMinor; }
+
+const char *ss_status_string(int status)
+{
+    switch (status) {
+    case SS_OK: return "SS_OK";
+    case SS_ERR_NULL: return "SS_ERR_NULL: a required pointer is NULL";
+    case SS_ERR_SHAPE: return "SS_ERR_SHAPE: a size is <= 0 or too large";
+    case SS_ERR_DTYPE: return "SS_ERR_DTYPE: dtype must be SS_F32 or SS_BF16";
+    case SS_ERR_ALIGN: return "SS_ERR_ALIGN: a pointer is not aligned to its element size";
+    case SS_ERR_UNSUPPORTED: return "SS_ERR_UNSUPPORTED: state_dim must be 4, 8 or 16; unknown flag bit";
+    case SS_ERR_CUDA: return "SS_ERR_CUDA: the CUDA runtime reported an error";
+    case SS_ERR_TIMEOUT: return "SS_ERR_TIMEOUT: a bounded device-side wait gave up";
+    case SS_ERR_ALIAS: return "SS_ERR_ALIAS: an output overlaps an input";
+    case SS_ERR_WORKSPACE: return "SS_ERR_WORKSPACE: the workspace is smaller than ss_scan_workspace_bytes()";
+    default: return "unknown status";
+    }
+}
+
+int64_t ss_scan_workspace_bytes(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq)
+{
+    if (batch <= 0 || channels <= 0 || seq <= 0)
+        return 0;
+    switch (state_dim) {
+    case 4: return ss::scan_workspace_bytes<4>(scan_groups<4>(batch, channels));
+    case 8: return ss::scan_workspace_bytes<8>(scan_groups<8>(batch, channels));
+    case 16: return ss::scan_workspace_bytes<16>(scan_groups<16>(batch, channels));
+    default: return 0;
+    }
+}
+
+int ss_scan_status(const void *workspace, ss_stream_t stream, int *status)
+{
+    if (!status)
+        return SS_ERR_NULL;
+    uint32_t *word = nullptr;
+    if (workspace) {
+        if (!aligned(workspace, 16))
+            return SS_ERR_ALIGN;
+        word = &static_cast<ss::WsHeader *>(const_cast<void *>(workspace))->status;
+    } else if (status_word_address(&word) != SS_OK) {
+        return SS_ERR_CUDA;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t v = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess ||
+        cudaMemcpyAsync(&v, word, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return SS_ERR_CUDA;
+    if (v && (cudaMemsetAsync(word, 0, sizeof(v), s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess))
+        return SS_ERR_CUDA;
+    *status = (v & (1u << ss::kStatusTimeout)) ? SS_ERR_TIMEOUT : SS_OK;
+    return SS_OK;
+}
+
+int ss_scan_fwd(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, ss_dtype_t dtype,
+                const void *x, const void *dt_raw, const float *A, const void *B, const void *C,
+                const float *D, const void *z, const float *dt_bias, const uint8_t *reset,
+                const float *h0, uint32_t flags, void *y, float *h_last, void *workspace,
+                size_t workspace_bytes, ss_stream_t stream)
+{
+    if (!x || !dt_raw || !A || !B || !C || !y)
+        return SS_ERR_NULL;
+    if (batch <= 0 || channels <= 0 || state_dim <= 0 || seq <= 0)
+        return SS_ERR_SHAPE;
+    if (dtype != SS_F32 && dtype != SS_BF16)
+        return SS_ERR_DTYPE;
+    if (state_dim != 4 && state_dim != 8 && state_dim != 16)
+        return SS_ERR_UNSUPPORTED;
+    if (flags & ~uint32_t(SS_DT_SOFTPLUS))
+        return SS_ERR_UNSUPPORTED;
+    const size_t es = dtype == SS_BF16 ? 2 : 4;
+    int64_t rows = 0, elems = 0, bcel = 0, stel = 0, rsel = 0;
+    if (!mul_ok(batch, channels, &rows) || !mul_ok(rows, seq, &elems) ||
+        !mul_ok(batch * state_dim, seq, &bcel) || !mul_ok(rows, state_dim, &stel) ||
+        !mul_ok(batch, seq, &rsel) || elems > (INT64_MAX / 8))
+        return SS_ERR_SHAPE;
+    const void *typed[] = {x, dt_raw, B, C, z, y};
+    for (const void *p : typed)
+        if (p && !aligned(p, es))
+            return SS_ERR_ALIGN;
+    const void *f32s[] = {A, D, dt_bias, h0, h_last};
+    for (const void *p : f32s)
+        if (p && !aligned(p, 4))
+            return SS_ERR_ALIGN;
+    // outputs must not overlap inputs (h_last may BE h0: each lane reads its own
+    // h0 entries before it writes the same h_last entries)
+    const size_t ybytes = size_t(elems) * es, hbytes = size_t(stel) * 4;
+    const void *in_p[] = {x, dt_raw, z, B, C, A, D, dt_bias, reset, h0};
+    const size_t in_n[] = {ybytes, ybytes, z ? ybytes : 0, size_t(bcel) * es, size_t(bcel) * es,
+                           size_t(channels * state_dim) * 4, D ? size_t(channels) * 4 : 0,
+                           dt_bias ? size_t(channels) * 4 : 0, reset ? size_t(rsel) : 0,
+                           h0 ? hbytes : 0};
+    for (int i = 0; i < 10; ++i) {
+        if (overlaps(y, ybytes, in_p[i], in_n[i]))
+            return SS_ERR_ALIAS;
+        if (h_last && !(i == 9 && in_p[i] == h_last) && overlaps(h_last, hbytes, in_p[i], in_n[i]))
+            return SS_ERR_ALIAS;
+    }
+    if (h_last && overlaps(h_last, hbytes, y, ybytes))
+        return SS_ERR_ALIAS;
+    if (workspace) {
+        if (!aligned(workspace, 16))
+            return SS_ERR_ALIGN;
+        for (int i = 0; i < 10; ++i)
+            if (overlaps(workspace, workspace_bytes, in_p[i], in_n[i]))
+                return SS_ERR_ALIAS;
+        if (overlaps(workspace, workspace_bytes, y, ybytes) ||
+            (h_last && overlaps(workspace, workspace_bytes, h_last, hbytes)))
+            return SS_ERR_ALIAS;
+    }
+
+    const int vec_elems = 16 / int(es);
+    // the vector path loads tiles through TMA tensor maps: 32-bit coordinates
+    bool vec = (seq % vec_elems) == 0 && seq < (int64_t(1) << 31) && rows < (int64_t(1) << 31) &&
+               batch * state_dim < (int64_t(1) << 31);
+    for (const void *p : typed)
+        if (p && !aligned(p, 16))
+            vec = false;
+
+    ss::ScanArgs a{};
+    a.batch = batch;
+    a.channels = channels;
+    a.seq = seq;
+    a.x = x; a.dt = dt_raw; a.B = B; a.C = C; a.z = z;
+    a.A = A; a.D = D; a.dt_bias = dt_bias; a.h0 = h0;
+    a.reset = reset;
+    a.y = y;
+    a.h_last = h_last;
+    a.softplus = (flags & SS_DT_SOFTPLUS) ? 1 : 0;
+    a.workspace = static_cast<uint8_t *>(workspace);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (state_dim) {
+    case 4: return dispatch_scan_n<4>(a, dtype, vec, workspace_bytes, s);
+    case 8: return dispatch_scan_n<8>(a, dtype, vec, workspace_bytes, s);
+    default: return dispatch_scan_n<16>(a, dtype, vec, workspace_bytes, s);
+    }
+}
+
+int ss_state_update(int64_t batch, int64_t channels, int64_t state_dim, ss_dtype_t dtype,
+                    float *state, const void *x, const void *dt_raw, const float *A,
+                    const void *B, const void *C, const float *D, const void *z,
+                    const float *dt_bias, uint32_t flags, void *y, ss_stream_t stream)
+{
+    if (!state || !x || !dt_raw || !A || !B || !C || !y)
+        return SS_ERR_NULL;
+    if (batch <= 0 || channels <= 0 || state_dim <= 0)
+        return SS_ERR_SHAPE;
+    if (dtype != SS_F32 && dtype != SS_BF16)
+        return SS_ERR_DTYPE;
+    if (state_dim != 4 && state_dim != 8 && state_dim != 16)
+        return SS_ERR_UNSUPPORTED;
+    if (flags & ~uint32_t(SS_DT_SOFTPLUS))
+        return SS_ERR_UNSUPPORTED;
+    const size_t es = dtype == SS_BF16 ? 2 : 4;
+    int64_t rows = 0, stel = 0, bnel = 0;
+    if (!mul_ok(batch, channels, &rows) || !mul_ok(rows, state_dim, &stel) ||
+        !mul_ok(batch, state_dim, &bnel) || stel > (INT64_MAX / 8))
+        return SS_ERR_SHAPE;
+    const void *typed[] = {x, dt_raw, B, C, z, y};
+    for (const void *p : typed)
+        if (p && !aligned(p, es))
+            return SS_ERR_ALIGN;
+    const void *f32s[] = {state, A, D, dt_bias};
+    for (const void *p : f32s)
+        if (p && !aligned(p, 4))
+            return SS_ERR_ALIGN;
+    const size_t sbytes = size_t(stel) * 4, ybytes = size_t(rows) * es;
+    const void *in_p[] = {x, dt_raw, z, B, C, A, D, dt_bias};
+    const size_t in_n[] = {ybytes, ybytes, z ? ybytes : 0, size_t(bnel) * es, size_t(bnel) * es,
+                           size_t(channels * state_dim) * 4, D ? size_t(channels) * 4 : 0,
+                           dt_bias ? size_t(channels) * 4 : 0};
+    for (int i = 0; i < 8; ++i)
+        if (overlaps(y, ybytes, in_p[i], in_n[i]) || overlaps(state, sbytes, in_p[i], in_n[i]))
+            return SS_ERR_ALIAS;
+    if (overlaps(y, ybytes, state, sbytes))
+        return SS_ERR_ALIAS;
+
+    const bool vec = aligned(state, 16) && aligned(A, 16) && aligned(B, 4 * es) && aligned(C, 4 * es);
+    ss::UpdateArgs a{};
+    a.batch = batch;
+    a.channels = channels;
+    a.state = state;
+    a.x = x; a.dt = dt_raw; a.B = B; a.C = C; a.z = z;
+    a.A = A; a.D = D; a.dt_bias = dt_bias;
+    a.y = y;
+    a.softplus = (flags & SS_DT_SOFTPLUS) ? 1 : 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (state_dim) {
+    case 4: return dispatch_update_n<4>(a, dtype, vec, s);
+    case 8: return dispatch_update_n<8>(a, dtype, vec, s);
+    default: return dispatch_update_n<16>(a, dtype, vec, s);
+    }
+}
+
+} // extern "C"

@@ -1,0 +1,817 @@
+// ss_scan_fwd.cuh -- prompt-scan kernel of the Mamba-1 selective scan (S6).
+//
+// Recurrence (nnterp "selective_scan" component, SelectiveScan description;
+// TransformerLens "ssm_mixer", compute_ssm_state):
+//   h_t[n] = exp(dt_t A[c,n]) h_{t-1}[n] + dt_t B[b,n,t] x[b,c,t]
+//   y_t    = sum_n C[b,n,t] h_t[n] + D[c] x[b,c,t],   out_t = y_t silu(z_t)
+// with an enforced reset ("s6_reset" blog draft, Enforced Boundary Resetting)
+// folded into the decay: at a flagged token exp(dt A) is replaced by exactly 0 --
+// the zero of the (decay, increment) operator -- so h_t = dt_t B_t x_t there.
+//
+// Cost model.  The N exponentials per (b, t, c) are the bound (MUFU ex2, 16 per
+// clock per SM); the HBM traffic is about 8 bytes per (b, t, c).  The design keeps
+// the exponential unit fed:
+//
+//  * Work split.  A scan lane owns TWO states of one channel and walks the tokens
+//    in order, so each exponential is computed once and the state never leaves
+//    registers.  A scan warp covers 32 / (N/2) channels (4 at N = 16).
+//  * Warp specialisation.  Each CTA has kScanWarps scan warps, one producer warp and
+//    one epilogue warp.  The producer streams x, dt_raw, z (16-byte loads), B and C
+//    (shared by every channel of a batch row) into a two-stage shared-memory ring,
+//    computing dt = softplus(dt_raw + dt_bias) and dt*x on the way.  The epilogue
+//    warp sums the scan lanes' partial outputs over the N/2 state pairs, applies D*x
+//    and the silu(z) gate and stores y.  The scan warps therefore run an
+//    uninterrupted stream of packed fp32x2 multiplies, MUFU ex2 and fused
+//    multiply-adds.  The roles hand chunks of 32 tokens over through mbarriers
+//    (bounded waits).
+//  * Chained segments.  The sequence is cut into segments; a work unit is (channel
+//    group, segment).  Persistent CTAs take units from a global counter in
+//    segment-major order; the scan carry (the state at a segment's end) is passed
+//    to the next segment's CTA through the workspace under an epoch-tagged flag --
+//    the "carry between chunks" of a two-level scan, applied at segment
+//    granularity.  Without a workspace each CTA runs one channel group over the
+//    whole sequence.
+#pragma once
+
+#include "ss_device.cuh"
+#include "ss_sync.cuh"
+
+namespace ss {
+
+struct ScanArgs {
+    int64_t batch, channels, seq;
+    const void *x, *dt, *B, *C, *z;
+    const float *A, *D, *dt_bias, *h0;
+    const uint8_t *reset;
+    void *y;
+    float *h_last;
+    int softplus;
+    int64_t groups_per_batch; // channel groups per batch row
+    int64_t groups;           // batch * groups_per_batch
+    int64_t seg_len;          // tokens per segment (a multiple of the chunk)
+    int64_t segments;         // ceil(seq / seg_len); 1 without a workspace
+    uint8_t *workspace;       // nullptr: one CTA per channel group, one segment
+    uint32_t *status;         // status word when there is no workspace
+};
+
+// Tensor maps of the TMA path: x, dt, z as [batch * channels rows][seq] and B, C as
+// [batch * state_dim rows][seq], boxes of one chunk of tokens.
+struct TmaMaps {
+    CUtensorMap x, dt, z, B, C;
+};
+
+// Workspace layout (bytes): the caller zeroes it once; every complete call leaves
+// it ready for the next one.
+struct WsHeader {
+    uint32_t counter; // next work unit of this call
+    uint32_t status;  // sticky error bits (1 << SS_ERR_TIMEOUT)
+    uint32_t epoch;   // advanced by the last warp of every call; tags the carry flags
+    uint32_t done;    // warps finished in this call
+    uint32_t pad[12];
+};
+static_assert(sizeof(WsHeader) == 64, "workspace header is 64 bytes");
+
+template <int N> struct ScanShape {
+    static_assert(N == 4 || N == 8 || N == 16, "state_dim must be 4, 8 or 16");
+    static constexpr int kPairs = N / 2;               // state pairs = lanes per channel
+    static constexpr int kChanPerWarp = 32 / kPairs;
+    static constexpr int kScanWarps = 2;
+    static constexpr int kProducerWarp = kScanWarps, kEpilogueWarp = kScanWarps + 1;
+    static constexpr int kWarps = kScanWarps + 2;
+    static constexpr int kThreads = 32 * kWarps;
+    static constexpr int kChanPerCta = kScanWarps * kChanPerWarp;
+    static constexpr int kChunk = 32;                  // tokens per pipeline stage
+    static constexpr int kBlocks = kChunk / 8;         // 8-token blocks per chunk
+    static constexpr int kRow = kChunk + 4;            // padded row (floats)
+    static constexpr int kStages = 2, kYStages = 2;
+    // input stage (floats): meta | B,C rows | dt rows | dt*x rows | reset bias
+    static constexpr int kMeta = 8;
+    static constexpr int kBCOff = kMeta;
+    static constexpr int kDTOff = kBCOff + 2 * N * kRow;
+    static constexpr int kDXOff = kDTOff + kChanPerCta * kRow;
+    static constexpr int kRBOff = kDXOff + kChanPerCta * kRow;
+    static constexpr int kInStage = kRBOff + kChunk;
+    // output stage (floats): meta | partial outputs | raw x | raw z
+    static constexpr int kYChan = kPairs * kRow + 4;   // per-channel block, bank-skewed
+    static constexpr int kYPOff = kMeta;
+    static constexpr int kXZOff = kYPOff + kChanPerCta * kYChan;
+    static constexpr int kXZFloats = (kChanPerCta * kChunk * 4) / 4; // room for fp32 x or z
+    static constexpr int kYStage = kXZOff + 2 * kXZFloats;
+    static constexpr int kFloats = kStages * kInStage + kYStages * kYStage;
+    // IO work per chunk
+    static constexpr int kTokTasks = kChanPerCta * kBlocks;       // (channel, 8 tokens)
+    static constexpr int kTokPerLane = kTokTasks / 32;
+    static constexpr int kBCTasks = 2 * N * kBlocks;              // (B/C row, 8 tokens)
+    static constexpr int kBCPerLane = (kBCTasks + 31) / 32;
+    // raw ring filled by TMA (aligned shapes): x, dt, z tiles [channels][chunk] and
+    // B, C tiles [N][chunk] in storage type, several chunks ahead of the producer
+    static constexpr int kRawStages = 4;
+    template <typename T> static constexpr int raw_x_off() { return 0; }
+    template <typename T> static constexpr int raw_dt_off() { return kChanPerCta * kChunk * int(sizeof(T)); }
+    template <typename T> static constexpr int raw_z_off() { return 2 * kChanPerCta * kChunk * int(sizeof(T)); }
+    template <typename T> static constexpr int raw_b_off() { return 3 * kChanPerCta * kChunk * int(sizeof(T)); }
+    template <typename T> static constexpr int raw_c_off() { return raw_b_off<T>() + N * kChunk * int(sizeof(T)); }
+    template <typename T> static constexpr int raw_stage_bytes()
+    {
+        return ((raw_c_off<T>() + N * kChunk * int(sizeof(T))) + 127) / 128 * 128;
+    }
+    // shared memory: [raw ring] [input stages] [output stages] [barriers] [raw meta]
+    template <typename T, bool TMA> static constexpr size_t smem_bytes()
+    {
+        return size_t(TMA ? kRawStages * raw_stage_bytes<T>() : 0) + size_t(kFloats) * 4 +
+               8 * size_t(8 + kRawStages) + 32 * size_t(kRawStages);
+    }
+    static_assert(kTokTasks % 32 == 0, "token tasks fill whole IO lanes");
+    static_assert(kInStage % 4 == 0 && kYStage % 4 == 0, "16-byte aligned stages");
+};
+
+struct ChunkMeta {
+    int64_t t0;   // first token of the chunk
+    int64_t g;    // channel group (b * groups_per_batch + group)
+    int32_t s;    // segment
+    int32_t flags;
+};
+constexpr int kFirst = 1, kLast = 2, kEnd = 4;
+
+// Chunk descriptors live in the first 32 bytes of each stage, field by field.
+__device__ __forceinline__ void write_meta(float *stage, int64_t t0, int64_t g, int32_t s, int32_t flags)
+{
+    int64_t *w = reinterpret_cast<int64_t *>(stage);
+    w[0] = t0;
+    w[1] = g;
+    int32_t *v = reinterpret_cast<int32_t *>(stage + 4);
+    v[0] = s;
+    v[1] = flags;
+}
+
+__device__ __forceinline__ ChunkMeta read_meta(const float *stage)
+{
+    const int64_t *w = reinterpret_cast<const int64_t *>(stage);
+    const int32_t *v = reinterpret_cast<const int32_t *>(stage + 4);
+    ChunkMeta m;
+    m.t0 = w[0];
+    m.g = w[1];
+    m.s = v[0];
+    m.flags = v[1];
+    return m;
+}
+
+// Shared-memory row of state n of B (C rows follow at +N): even states first, then
+// odd ones, so the state pairs of a channel read distinct bank groups.
+template <int N> __device__ __forceinline__ int bc_row(int n)
+{
+    return (n & 1) * (N / 2) + (n >> 1);
+}
+
+// silu on the output gate: the exact form for fp32 outputs; for bf16 outputs the
+// MUFU tanh form 0.5 v (1 + tanh(v / 2)) (one MUFU op instead of two, error in the
+// gate below 2.5e-4 |v|, inside the bf16 output tolerance).
+template <typename T> __device__ __forceinline__ float gate(float v);
+template <> __device__ __forceinline__ float gate<float>(float v) { return silu(v); }
+template <> __device__ __forceinline__ float gate<__nv_bfloat16>(float v)
+{
+    float t;
+    const float h = 0.5f * v;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+    return fmaf(h, t, h);
+}
+
+// softplus(r) = max(r, 0) + log(1 + e), e = exp(-|r|) in (0, 1].  log(1 + e) = e Q(e)
+// with Q a degree-8 polynomial fitted to log1p(e)/e on [0, 1] for relative error
+// (1.5e-7 in fp32 Horner form): no division, one MUFU op.
+__device__ __forceinline__ float softplus_poly(float r)
+{
+    const float e = ex2(-fabsf(r) * kLog2e);
+    float q = 5.232690697e-03f;
+    q = fmaf(q, e, -2.950522892e-02f);
+    q = fmaf(q, e, 7.822594434e-02f);
+    q = fmaf(q, e, -1.366324604e-01f);
+    q = fmaf(q, e, 1.910600743e-01f);
+    q = fmaf(q, e, -2.484298259e-01f);
+    q = fmaf(q, e, 3.331909690e-01f);
+    q = fmaf(q, e, -4.999949315e-01f);
+    q = fmaf(q, e, 9.999999699e-01f);
+    return fmaxf(r, 0.0f) + e * q;
+}
+
+// The same for two tokens at once with packed fp32x2 arithmetic; the polynomial
+// and the final e Q(e) + max(r, 0) run as fp32x2 fused multiply-adds.
+__device__ __forceinline__ float2 softplus_poly2(float2 r)
+{
+    const float2 t = __fmul2_rn(make_float2(-fabsf(r.x), -fabsf(r.y)), make_float2(kLog2e, kLog2e));
+    const float2 e = make_float2(ex2(t.x), ex2(t.y));
+    float2 q = make_float2(5.232690697e-03f, 5.232690697e-03f);
+    q = __ffma2_rn(q, e, make_float2(-2.950522892e-02f, -2.950522892e-02f));
+    q = __ffma2_rn(q, e, make_float2(7.822594434e-02f, 7.822594434e-02f));
+    q = __ffma2_rn(q, e, make_float2(-1.366324604e-01f, -1.366324604e-01f));
+    q = __ffma2_rn(q, e, make_float2(1.910600743e-01f, 1.910600743e-01f));
+    q = __ffma2_rn(q, e, make_float2(-2.484298259e-01f, -2.484298259e-01f));
+    q = __ffma2_rn(q, e, make_float2(3.331909690e-01f, 3.331909690e-01f));
+    q = __ffma2_rn(q, e, make_float2(-4.999949315e-01f, -4.999949315e-01f));
+    q = __ffma2_rn(q, e, make_float2(9.999999699e-01f, 9.999999699e-01f));
+    return __ffma2_rn(e, q, make_float2(fmaxf(r.x, 0.0f), fmaxf(r.y, 0.0f)));
+}
+
+// ---------------------------------------------------------------------------------------
+// producer warp: global -> registers (one chunk ahead) -> shared-memory stage
+// ---------------------------------------------------------------------------------------
+
+template <int N, typename T, bool HAS_RESET, bool VEC>
+struct IoPrefetch {
+    using S = ScanShape<N>;
+    Raw8<T> bc[S::kBCPerLane];
+    Raw8<T> xr[S::kTokPerLane], dr[S::kTokPerLane], zr[S::kTokPerLane];
+    float bias[S::kTokPerLane];
+    uint32_t rbyte;
+
+    __device__ __forceinline__ void load(const ScanArgs &p, int lane, int64_t g, int64_t t0)
+    {
+        const int64_t L = p.seq;
+        const int64_t b = g / p.groups_per_batch;
+        const int64_t c0 = (g % p.groups_per_batch) * S::kChanPerCta;
+        const T *Bb = static_cast<const T *>(p.B) + b * N * L;
+        const T *Cb = static_cast<const T *>(p.C) + b * N * L;
+#pragma unroll
+        for (int m = 0; m < S::kBCPerLane; ++m) {
+            const int q = lane + 32 * m;
+            if (q < S::kBCTasks) {
+                const int r = q % (2 * N), tb = q / (2 * N);
+                const T *src = r < N ? Bb + r * L : Cb + (r - N) * L;
+                if (VEC)
+                    bc[m].load_vec(src, t0 + tb * 8, L);
+                else
+                    bc[m].load_scalar(src, t0 + tb * 8, L);
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < S::kTokPerLane; ++m) {
+            const int q = lane + 32 * m;
+            const int cl = q / S::kBlocks, tb = q % S::kBlocks;
+            int64_t c = c0 + cl;
+            c = c < p.channels ? c : p.channels - 1;
+            const int64_t row = b * p.channels + c;
+            const int64_t t = t0 + tb * 8;
+            const T *xrow = static_cast<const T *>(p.x) + row * L;
+            const T *drow = static_cast<const T *>(p.dt) + row * L;
+            if (VEC) {
+                xr[m].load_vec_stream(xrow, t, L);
+                dr[m].load_vec_stream(drow, t, L);
+                if (p.z)
+                    zr[m].load_vec_stream(static_cast<const T *>(p.z) + row * L, t, L);
+            } else {
+                xr[m].load_scalar(xrow, t, L);
+                dr[m].load_scalar(drow, t, L);
+                if (p.z)
+                    zr[m].load_scalar(static_cast<const T *>(p.z) + row * L, t, L);
+            }
+            bias[m] = p.dt_bias ? __ldg(p.dt_bias + c) : 0.0f;
+        }
+        if (HAS_RESET)
+            rbyte = (lane < S::kChunk && t0 + lane < L) ? uint32_t(__ldg(p.reset + b * L + t0 + lane)) : 0u;
+    }
+
+    // The same registers filled from a raw TMA stage (the reset byte is loaded by
+    // the caller).
+    __device__ __forceinline__ void load_smem(const ScanArgs &p, int lane, int64_t g, const unsigned char *raw)
+    {
+        const int64_t c0 = (g % p.groups_per_batch) * S::kChanPerCta;
+        const T *rbc = reinterpret_cast<const T *>(raw + S::template raw_b_off<T>());
+#pragma unroll
+        for (int m = 0; m < S::kBCPerLane; ++m) {
+            const int q = lane + 32 * m;
+            if (q < S::kBCTasks) {
+                const int r = q % (2 * N), tb = q / (2 * N);
+                bc[m].load_smem(rbc + r * S::kChunk + tb * 8);
+            }
+        }
+        const T *rx = reinterpret_cast<const T *>(raw + S::template raw_x_off<T>());
+        const T *rd = reinterpret_cast<const T *>(raw + S::template raw_dt_off<T>());
+        const T *rz = reinterpret_cast<const T *>(raw + S::template raw_z_off<T>());
+#pragma unroll
+        for (int m = 0; m < S::kTokPerLane; ++m) {
+            const int q = lane + 32 * m;
+            const int cl = q / S::kBlocks, tb = q % S::kBlocks;
+            xr[m].load_smem(rx + cl * S::kChunk + tb * 8);
+            dr[m].load_smem(rd + cl * S::kChunk + tb * 8);
+            if (p.z)
+                zr[m].load_smem(rz + cl * S::kChunk + tb * 8);
+            int64_t c = c0 + cl;
+            c = c < p.channels ? c : p.channels - 1;
+            bias[m] = p.dt_bias ? __ldg(p.dt_bias + c) : 0.0f;
+        }
+    }
+};
+
+template <int N, typename T, bool HAS_RESET, bool VEC>
+__device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane, const IoPrefetch<N, T, HAS_RESET, VEC> &f,
+                                              float *stage, float *ystage, int64_t t0)
+{
+    using S = ScanShape<N>;
+    const int64_t L = p.seq;
+#pragma unroll
+    for (int m = 0; m < S::kBCPerLane; ++m) {
+        const int q = lane + 32 * m;
+        if (q < S::kBCTasks) {
+            const int r = q % (2 * N), tb = q / (2 * N);
+            const int srow = (r < N ? 0 : N) + bc_row<N>(r < N ? r : r - N);
+            float4 *dst = reinterpret_cast<float4 *>(stage + S::kBCOff + srow * S::kRow + tb * 8);
+            dst[0] = make_float4(f.bc[m].get(0), f.bc[m].get(1), f.bc[m].get(2), f.bc[m].get(3));
+            dst[1] = make_float4(f.bc[m].get(4), f.bc[m].get(5), f.bc[m].get(6), f.bc[m].get(7));
+        }
+    }
+    if (HAS_RESET && lane < S::kChunk)
+        stage[S::kRBOff + lane] = f.rbyte ? -INFINITY : 0.0f;
+    const bool softplus_on = p.softplus != 0;
+#pragma unroll
+    for (int m = 0; m < S::kTokPerLane; ++m) {
+        const int q = lane + 32 * m;
+        const int cl = q / S::kBlocks, tb = q % S::kBlocks;
+        const int64_t tl = t0 + tb * 8;
+        float2 dtv[4], dxv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 r = __fadd2_rn(make_float2(f.dr[m].get(2 * k), f.dr[m].get(2 * k + 1)),
+                                        make_float2(f.bias[m], f.bias[m]));
+            float2 d = softplus_on ? softplus_poly2(r) : r;
+            if (tl + 8 > L) { // past the end: decay 1, increment 0
+                d.x = (tl + 2 * k < L) ? d.x : 0.0f;
+                d.y = (tl + 2 * k + 1 < L) ? d.y : 0.0f;
+            }
+            dtv[k] = d;
+            dxv[k] = __fmul2_rn(d, make_float2(f.xr[m].get(2 * k), f.xr[m].get(2 * k + 1)));
+        }
+        float4 *pd = reinterpret_cast<float4 *>(stage + S::kDTOff + cl * S::kRow + tb * 8);
+        float4 *px = reinterpret_cast<float4 *>(stage + S::kDXOff + cl * S::kRow + tb * 8);
+        pd[0] = make_float4(dtv[0].x, dtv[0].y, dtv[1].x, dtv[1].y);
+        pd[1] = make_float4(dtv[2].x, dtv[2].y, dtv[3].x, dtv[3].y);
+        px[0] = make_float4(dxv[0].x, dxv[0].y, dxv[1].x, dxv[1].y);
+        px[1] = make_float4(dxv[2].x, dxv[2].y, dxv[3].x, dxv[3].y);
+        // raw x and z for the epilogue warp, in the output stage's side buffers
+        Raw8<T> *xs = reinterpret_cast<Raw8<T> *>(ystage + S::kXZOff) + cl * S::kBlocks + tb;
+        Raw8<T> *zs = reinterpret_cast<Raw8<T> *>(ystage + S::kXZOff + S::kXZFloats) + cl * S::kBlocks + tb;
+        *xs = f.xr[m];
+        if (p.z)
+            *zs = f.zr[m];
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// epilogue warp: partial outputs -> sum over state pairs, D*x, gate -> y
+// ---------------------------------------------------------------------------------------
+
+template <typename T> __device__ __forceinline__ float2 gate2(float2 v);
+template <> __device__ __forceinline__ float2 gate2<float>(float2 v)
+{
+    return make_float2(silu(v.x), silu(v.y));
+}
+template <> __device__ __forceinline__ float2 gate2<__nv_bfloat16>(float2 v)
+{
+    const float2 h = __fmul2_rn(v, make_float2(0.5f, 0.5f));
+    float2 t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t.x) : "f"(h.x));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t.y) : "f"(h.y));
+    return __ffma2_rn(h, t, h);
+}
+
+template <int N, typename T, bool VEC>
+__device__ __forceinline__ void epilogue_chunk(const ScanArgs &p, int lane, const float *ystage, int64_t g, int64_t t0)
+{
+    using S = ScanShape<N>;
+    const int64_t L = p.seq;
+    const int64_t b = g / p.groups_per_batch;
+    const int64_t c0 = (g % p.groups_per_batch) * S::kChanPerCta;
+#pragma unroll
+    for (int m = 0; m < S::kTokPerLane; ++m) {
+        const int q = lane + 32 * m;
+        const int cl = q / S::kBlocks, tb = q % S::kBlocks;
+        const int64_t c = c0 + cl;
+        float2 o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            o[k] = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int pr = 0; pr < S::kPairs; ++pr) {
+            const float4 *src = reinterpret_cast<const float4 *>(ystage + S::kYPOff + cl * S::kYChan + pr * S::kRow + tb * 8);
+            const float4 v0 = src[0], v1 = src[1];
+            o[0] = __fadd2_rn(o[0], make_float2(v0.x, v0.y));
+            o[1] = __fadd2_rn(o[1], make_float2(v0.z, v0.w));
+            o[2] = __fadd2_rn(o[2], make_float2(v1.x, v1.y));
+            o[3] = __fadd2_rn(o[3], make_float2(v1.z, v1.w));
+        }
+        if (c >= p.channels)
+            continue;
+        const Raw8<T> xs = reinterpret_cast<const Raw8<T> *>(ystage + S::kXZOff)[cl * S::kBlocks + tb];
+        const float Dc = p.D ? __ldg(p.D + c) : 0.0f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            o[k] = __ffma2_rn(make_float2(Dc, Dc), make_float2(xs.get(2 * k), xs.get(2 * k + 1)), o[k]);
+        if (p.z) {
+            const Raw8<T> zs = reinterpret_cast<const Raw8<T> *>(ystage + S::kXZOff + S::kXZFloats)[cl * S::kBlocks + tb];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                o[k] = __fmul2_rn(o[k], gate2<T>(make_float2(zs.get(2 * k), zs.get(2 * k + 1))));
+        }
+        const float out[8] = {o[0].x, o[0].y, o[1].x, o[1].y, o[2].x, o[2].y, o[3].x, o[3].y};
+        T *yrow = static_cast<T *>(p.y) + (b * p.channels + c) * L;
+        store8<T, VEC>(yrow, t0 + tb * 8, L, out);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// producer loops
+// ---------------------------------------------------------------------------------------
+
+// Shared context of the roles of one CTA.
+struct CtaCtx {
+    float *in_base, *y_base;
+    unsigned char *raw_base;
+    uint64_t *in_full, *in_empty, *y_full, *y_empty, *raw_full;
+    int64_t *raw_meta; // per raw stage: t0, g, (s | flags << 32)
+    WsHeader *ws;
+    uint32_t *status;
+};
+
+constexpr uint32_t kNoUnit = 0xffffffffu;
+
+// Next unit of this CTA: from the work counter (chained) or blockIdx.x (static).
+__device__ __forceinline__ uint32_t take_unit(const ScanArgs &p, WsHeader *ws, bool first)
+{
+    if (!ws)
+        return first ? uint32_t(blockIdx.x) : kNoUnit;
+    const uint32_t u = grab_unit(&ws->counter);
+    return int64_t(u) >= p.groups * p.segments ? kNoUnit : u;
+}
+
+template <int N> __device__ __forceinline__ int64_t unit_chunks(const ScanArgs &p, uint32_t u)
+{
+    const int64_t s = int64_t(u) / p.groups;
+    const int64_t rest = p.seq - s * p.seg_len;
+    const int64_t len = rest < p.seg_len ? rest : p.seg_len;
+    return (len + ScanShape<N>::kChunk - 1) / ScanShape<N>::kChunk;
+}
+
+// Register-prefetch producer (any shape and alignment): every lane walks the same
+// unit sequence; lane 0 takes units and broadcasts them.
+template <int N, typename T, bool HAS_RESET, bool VEC>
+__device__ __forceinline__ void producer_ldg(const ScanArgs &p, const CtaCtx &cx, int lane)
+{
+    using S = ScanShape<N>;
+    auto next = [&](bool first) -> uint32_t {
+        uint32_t u = 0;
+        if (lane == 0)
+            u = take_unit(p, cx.ws, first);
+        return __shfl_sync(0xffffffffu, u, 0);
+    };
+    uint32_t u = next(true);
+    int64_t k = 0, nck = u != kNoUnit ? unit_chunks<N>(p, u) : 0;
+    IoPrefetch<N, T, HAS_RESET, VEC> pf;
+    if (u != kNoUnit)
+        pf.load(p, lane, int64_t(u) % p.groups, (int64_t(u) / p.groups) * p.seg_len);
+    for (uint32_t i = 0;; ++i) {
+        const int st = int(i % S::kStages);
+        const uint32_t ph = ((i / S::kStages) & 1u) ^ 1u;
+        // the input stage is free once the scan warps are done with chunk i-2; the
+        // output stage's side buffers once the epilogue warp is
+        if (!mbar_wait(cx.in_empty + st, ph, cx.status) || !mbar_wait(cx.y_empty + st, ph, cx.status))
+            return;
+        float *stage = cx.in_base + st * S::kInStage;
+        float *ystage = cx.y_base + st * S::kYStage;
+        const bool end = (u == kNoUnit);
+        int64_t g = 0, s = 0, t0 = 0;
+        if (!end) {
+            g = int64_t(u) % p.groups;
+            s = int64_t(u) / p.groups;
+            t0 = s * p.seg_len + k * S::kChunk;
+            produce_chunk<N, T, HAS_RESET, VEC>(p, lane, pf, stage, ystage, t0);
+        }
+        if (lane == 0) {
+            const int32_t fl = end ? kEnd : ((k == 0 ? kFirst : 0) | (k + 1 == nck ? kLast : 0));
+            write_meta(stage, t0, g, int32_t(s), fl);
+            write_meta(ystage, t0, g, int32_t(s), fl);
+        }
+        mbar_arrive(cx.in_full + st);
+        if (end)
+            return;
+        if (++k == nck) {
+            u = next(false);
+            k = 0;
+            nck = u != kNoUnit ? unit_chunks<N>(p, u) : 0;
+        }
+        if (u != kNoUnit)
+            pf.load(p, lane, int64_t(u) % p.groups, (int64_t(u) / p.groups) * p.seg_len + k * S::kChunk);
+    }
+}
+
+// TMA producer (16-byte aligned tensors, seq a multiple of the vector width): lane 0
+// keeps kRawStages - 1 chunks of x, dt, z, B, C in flight as 2-D tile loads into
+// the raw ring; the warp converts each landed chunk into the input stage.
+template <int N, typename T, bool HAS_RESET>
+__device__ __forceinline__ void producer_tma(const ScanArgs &p, const TmaMaps &maps, const CtaCtx &cx, int lane)
+{
+    using S = ScanShape<N>;
+    constexpr int RS = S::kRawStages;
+    constexpr int kRawBytes = S::template raw_stage_bytes<T>();
+    const uint32_t tx_bytes = uint32_t(((p.z ? 3 : 2) * S::kChanPerCta + 2 * N) * S::kChunk * sizeof(T));
+    // issue cursor (lane 0 only)
+    uint32_t iu = kNoUnit;
+    int64_t ik = 0, ink = 0;
+    uint32_t issued = 0; // chunks whose loads were issued
+    auto issue = [&](int r) {
+        int64_t *m = cx.raw_meta + 3 * r;
+        if (iu == kNoUnit) {
+            m[2] = int64_t(kEnd) << 32;
+            return;
+        }
+        const int64_t g = int64_t(iu) % p.groups, s = int64_t(iu) / p.groups;
+        const int64_t t0 = s * p.seg_len + ik * S::kChunk;
+        const int64_t b = g / p.groups_per_batch, c0 = (g % p.groups_per_batch) * S::kChanPerCta;
+        const int32_t fl = (ik == 0 ? kFirst : 0) | (ik + 1 == ink ? kLast : 0);
+        m[0] = t0;
+        m[1] = g;
+        m[2] = (int64_t(fl) << 32) | int64_t(s);
+        unsigned char *dst = cx.raw_base + r * kRawBytes;
+        uint64_t *bar = cx.raw_full + r;
+        mbar_arrive_expect_tx(bar, tx_bytes);
+        const int32_t tt = int32_t(t0), xrow = int32_t(b * p.channels + c0), brow = int32_t(b * N);
+        tma_load_2d(dst + S::template raw_x_off<T>(), &maps.x, tt, xrow, bar);
+        tma_load_2d(dst + S::template raw_dt_off<T>(), &maps.dt, tt, xrow, bar);
+        if (p.z)
+            tma_load_2d(dst + S::template raw_z_off<T>(), &maps.z, tt, xrow, bar);
+        tma_load_2d(dst + S::template raw_b_off<T>(), &maps.B, tt, brow, bar);
+        tma_load_2d(dst + S::template raw_c_off<T>(), &maps.C, tt, brow, bar);
+        ++issued;
+        if (++ik == ink) {
+            iu = take_unit(p, cx.ws, false);
+            ik = 0;
+            ink = iu != kNoUnit ? unit_chunks<N>(p, iu) : 0;
+        }
+    };
+    // on a timeout: let the loads still in flight land before the CTA can exit
+    auto drain = [&](uint32_t consumed) {
+        if (lane == 0)
+            for (uint32_t c = consumed; c < issued; ++c)
+                mbar_wait(cx.raw_full + c % RS, (c / RS) & 1u, nullptr);
+    };
+    if (lane == 0) {
+        iu = take_unit(p, cx.ws, true);
+        ink = iu != kNoUnit ? unit_chunks<N>(p, iu) : 0;
+        for (int r = 0; r < RS - 1; ++r)
+            issue(r);
+    }
+    IoPrefetch<N, T, HAS_RESET, true> pf;
+    for (uint32_t i = 0;; ++i) {
+        __syncwarp(); // every lane is done reading the raw stage refilled next
+        if (lane == 0) {
+            fence_proxy_async_smem();
+            issue(int((i + RS - 1) % RS));
+        }
+        __syncwarp();
+        const int r = int(i % RS);
+        const int64_t *m = cx.raw_meta + 3 * r;
+        const int64_t t0 = m[0], g = m[1];
+        const int32_t s = int32_t(m[2] & 0xffffffff), fl = int32_t(m[2] >> 32);
+        const bool end = (fl & kEnd) != 0;
+        if (HAS_RESET && !end) {
+            const int64_t b = g / p.groups_per_batch;
+            pf.rbyte = (lane < S::kChunk && t0 + lane < p.seq) ? uint32_t(__ldg(p.reset + b * p.seq + t0 + lane)) : 0u;
+        }
+        const int st = int(i % S::kStages);
+        const uint32_t ph = ((i / S::kStages) & 1u) ^ 1u;
+        if (!mbar_wait(cx.in_empty + st, ph, cx.status) || !mbar_wait(cx.y_empty + st, ph, cx.status)) {
+            drain(i);
+            return;
+        }
+        float *stage = cx.in_base + st * S::kInStage;
+        float *ystage = cx.y_base + st * S::kYStage;
+        if (!end) {
+            if (!mbar_wait(cx.raw_full + r, (i / RS) & 1u, cx.status)) {
+                drain(i);
+                return;
+            }
+            pf.load_smem(p, lane, g, cx.raw_base + r * kRawBytes);
+            produce_chunk<N, T, HAS_RESET, true>(p, lane, pf, stage, ystage, t0);
+        }
+        if (lane == 0) {
+            write_meta(stage, t0, g, s, end ? kEnd : fl);
+            write_meta(ystage, t0, g, s, end ? kEnd : fl);
+        }
+        mbar_arrive(cx.in_full + st);
+        if (end)
+            return;
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------------------
+
+template <int N, typename T, bool HAS_RESET, bool VEC>
+__global__ void __launch_bounds__(ScanShape<N>::kThreads, 1)
+ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
+{
+    using S = ScanShape<N>;
+    constexpr bool kTma = VEC;
+    constexpr int kRawRing = kTma ? S::kRawStages * S::template raw_stage_bytes<T>() : 0;
+    extern __shared__ __align__(128) unsigned char smem_bytes[];
+    float *const in_base = reinterpret_cast<float *>(smem_bytes + kRawRing);
+    float *const y_base = in_base + S::kStages * S::kInStage;
+    uint64_t *const bars = reinterpret_cast<uint64_t *>(in_base + S::kFloats);
+    uint64_t *const in_full = bars, *const in_empty = bars + 2;
+    uint64_t *const y_full = bars + 4, *const y_empty = bars + 6;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    WsHeader *const ws = reinterpret_cast<WsHeader *>(p.workspace);
+    const bool chained = ws != nullptr;
+    uint32_t *const status = chained ? &ws->status : p.status;
+    const uint32_t epoch = chained ? *reinterpret_cast<volatile uint32_t *>(&ws->epoch) : 0u;
+    uint64_t *const flags = chained ? reinterpret_cast<uint64_t *>(p.workspace + sizeof(WsHeader)) : nullptr;
+    float2 *const carry = chained
+        ? reinterpret_cast<float2 *>(p.workspace + sizeof(WsHeader) + 8 * p.groups * S::kScanWarps)
+        : nullptr;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(in_full + s, 32);
+            mbar_init(in_empty + s, 32 * S::kScanWarps);
+            mbar_init(y_full + s, 32 * S::kScanWarps);
+            mbar_init(y_empty + s, 32);
+        }
+        for (int r = 0; r < S::kRawStages; ++r)
+            mbar_init(bars + 8 + r, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (warp == S::kProducerWarp) {
+        CtaCtx cx;
+        cx.in_base = in_base;
+        cx.y_base = y_base;
+        cx.raw_base = smem_bytes;
+        cx.in_full = in_full;
+        cx.in_empty = in_empty;
+        cx.y_full = y_full;
+        cx.y_empty = y_empty;
+        cx.raw_full = bars + 8;
+        cx.raw_meta = reinterpret_cast<int64_t *>(bars + 8 + S::kRawStages);
+        cx.ws = ws;
+        cx.status = status;
+        if constexpr (kTma)
+            producer_tma<N, T, HAS_RESET>(p, maps, cx, lane);
+        else
+            producer_ldg<N, T, HAS_RESET, VEC>(p, cx, lane);
+    } else if (warp == S::kEpilogueWarp) {
+        // ============================== epilogue warp ============================
+        for (uint32_t j = 0;; ++j) {
+            const int ys = int(j % S::kYStages);
+            if (!mbar_wait(y_full + ys, (j / S::kYStages) & 1u, status))
+                return;
+            const float *ystage = y_base + ys * S::kYStage;
+            const ChunkMeta meta = read_meta(ystage);
+            if (meta.flags & kEnd)
+                break;
+            epilogue_chunk<N, T, VEC>(p, lane, ystage, meta.g, meta.t0);
+            mbar_arrive(y_empty + ys);
+        }
+    } else {
+        // =============================== scan warps ==============================
+        const int cw = lane / S::kPairs;    // channel within the warp
+        const int sub = lane % S::kPairs;   // state pair
+        const int n0 = 2 * sub, n1 = 2 * sub + 1;
+        const int cl = warp * S::kChanPerWarp + cw;  // channel within the CTA
+        float hs0 = 0.0f, hs1 = 0.0f;
+        float2 A0 = make_float2(0.f, 0.f), A1 = make_float2(0.f, 0.f);
+        int64_t row = 0;
+        bool cvalid = false;
+        for (uint32_t j = 0;; ++j) {
+            const int st = int(j % S::kStages);
+            if (!mbar_wait(in_full + st, (j / S::kStages) & 1u, status))
+                return;
+            const float *stage = in_base + st * S::kInStage;
+            const ChunkMeta meta = read_meta(stage);
+            const uint32_t ysi = j % S::kYStages;
+            if (!mbar_wait(y_empty + ysi, ((j / S::kYStages) & 1u) ^ 1u, status))
+                return;
+            if (meta.flags & kEnd) {
+                mbar_arrive(y_full + ysi); // lets the epilogue warp see the end marker
+                break;
+            }
+            if (meta.flags & kFirst) {
+                const int64_t b = meta.g / p.groups_per_batch;
+                const int64_t c_raw = (meta.g % p.groups_per_batch) * S::kChanPerCta + cl;
+                cvalid = c_raw < p.channels;
+                const int64_t c = cvalid ? c_raw : p.channels - 1;
+                row = b * p.channels + c;
+                const float a0 = __ldg(p.A + c * N + n0) * kLog2e;
+                const float a1 = __ldg(p.A + c * N + n1) * kLog2e;
+                A0 = make_float2(a0, a0);
+                A1 = make_float2(a1, a1);
+                if (meta.s == 0) {
+                    hs0 = p.h0 ? __ldg(p.h0 + row * N + n0) : 0.0f;
+                    hs1 = p.h0 ? __ldg(p.h0 + row * N + n1) : 0.0f;
+                } else {
+                    const int64_t slot = meta.g * S::kScanWarps + warp;
+                    const uint64_t want = (uint64_t(epoch) << 32) | uint64_t(meta.s);
+                    if (!flag_wait(flags + slot, want, status))
+                        return;
+                    const float2 h = __ldcg(carry + slot * 32 + lane);
+                    hs0 = h.x;
+                    hs1 = h.y;
+                }
+            }
+            float *yst = y_base + ysi * S::kYStage;
+            {
+                const float *Bs0 = stage + S::kBCOff + bc_row<N>(n0) * S::kRow;
+                const float *Bs1 = stage + S::kBCOff + bc_row<N>(n1) * S::kRow;
+                const float *Cs0 = Bs0 + N * S::kRow;
+                const float *Cs1 = Bs1 + N * S::kRow;
+                const float *rbs = stage + S::kRBOff;
+                const float *dts = stage + S::kDTOff + cl * S::kRow;
+                const float *dxs = stage + S::kDXOff + cl * S::kRow;
+                float *ys = yst + S::kYPOff + cl * S::kYChan + sub * S::kRow;
+#pragma unroll
+                for (int t = 0; t < S::kChunk; t += 4) {
+                    const float4 d4 = *reinterpret_cast<const float4 *>(dts + t);
+                    const float4 u4 = *reinterpret_cast<const float4 *>(dxs + t);
+                    const float4 b0 = *reinterpret_cast<const float4 *>(Bs0 + t);
+                    const float4 b1 = *reinterpret_cast<const float4 *>(Bs1 + t);
+                    const float4 q0 = *reinterpret_cast<const float4 *>(Cs0 + t);
+                    const float4 q1 = *reinterpret_cast<const float4 *>(Cs1 + t);
+                    float4 r4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (HAS_RESET)
+                        r4 = *reinterpret_cast<const float4 *>(rbs + t);
+                    float2 yo[2];
+#pragma unroll
+                    for (int pr = 0; pr < 2; ++pr) {
+                        const float2 dd = pr ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
+                        const float2 uu = pr ? make_float2(u4.z, u4.w) : make_float2(u4.x, u4.y);
+                        const float2 B0 = pr ? make_float2(b0.z, b0.w) : make_float2(b0.x, b0.y);
+                        const float2 B1 = pr ? make_float2(b1.z, b1.w) : make_float2(b1.x, b1.y);
+                        const float2 C0 = pr ? make_float2(q0.z, q0.w) : make_float2(q0.x, q0.y);
+                        const float2 C1 = pr ? make_float2(q1.z, q1.w) : make_float2(q1.x, q1.y);
+                        float2 g0, g1;
+                        if (HAS_RESET) {
+                            const float2 rr = pr ? make_float2(r4.z, r4.w) : make_float2(r4.x, r4.y);
+                            g0 = __ffma2_rn(dd, A0, rr);
+                            g1 = __ffma2_rn(dd, A1, rr);
+                        } else {
+                            g0 = __fmul2_rn(dd, A0);
+                            g1 = __fmul2_rn(dd, A1);
+                        }
+                        const float a0t = ex2(g0.x), a0u = ex2(g0.y);
+                        const float a1t = ex2(g1.x), a1u = ex2(g1.y);
+                        const float2 v0 = __fmul2_rn(uu, B0);
+                        const float2 v1 = __fmul2_rn(uu, B1);
+                        const float h0t = fmaf(a0t, hs0, v0.x);
+                        hs0 = fmaf(a0u, h0t, v0.y);
+                        const float h1t = fmaf(a1t, hs1, v1.x);
+                        hs1 = fmaf(a1u, h1t, v1.y);
+                        const float2 yy = __fmul2_rn(C0, make_float2(h0t, hs0));
+                        yo[pr] = __ffma2_rn(C1, make_float2(h1t, hs1), yy);
+                    }
+                    *reinterpret_cast<float4 *>(ys + t) = make_float4(yo[0].x, yo[0].y, yo[1].x, yo[1].y);
+                }
+            }
+            mbar_arrive(in_empty + st);
+            mbar_arrive(y_full + ysi);
+            if (meta.flags & kLast) {
+                if (int64_t(meta.s) + 1 < p.segments) {
+                    const int64_t slot = meta.g * S::kScanWarps + warp;
+                    __stcg(carry + slot * 32 + lane, make_float2(hs0, hs1));
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0)
+                        st_release_gpu(flags + slot, (uint64_t(epoch) << 32) | uint64_t(meta.s + 1));
+                } else if (p.h_last && cvalid) {
+                    p.h_last[row * N + n0] = hs0;
+                    p.h_last[row * N + n1] = hs1;
+                }
+            }
+        }
+    }
+
+    // The last warp of a chained call to finish resets the work counter and advances
+    // the epoch for the next call.  (Each warp counts itself, so no CTA-wide barrier is
+    // needed after the roles have diverged; a warp that gave up on a wait never gets
+    // here, and then the workspace stays as it is and the status word says why.)
+    if (chained) {
+        __syncwarp();
+        if (lane == 0) {
+            __threadfence();
+            const uint32_t done = atomicAdd(&ws->done, 1u);
+            if (done + 1 == gridDim.x * uint32_t(S::kWarps)) {
+                ws->done = 0;
+                ws->counter = 0;
+                __threadfence();
+                atomicAdd(&ws->epoch, 1u);
+            }
+        }
+    }
+}
+
+// Bytes of workspace a chained call needs for `groups` channel groups.
+template <int N> constexpr int64_t scan_workspace_bytes(int64_t groups)
+{
+    return int64_t(sizeof(WsHeader)) + groups * ScanShape<N>::kScanWarps * (8 + 32 * 8);
+}
+
+} // namespace ss

@@ -1,0 +1,235 @@
+"""ctypes binding of ``libssscan.so`` (C declarations: include/ss_scan.h).
+
+Argument marshalling only: tensors are checked, made contiguous, outputs are
+allocated with torch, and the device pointers plus the current CUDA stream are
+handed to the C entry points of the same names.  Every step of the scan runs in
+the library's kernels; there is no other code path, and a missing library is an
+error, never a fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libssscan.so")
+
+SS_F32, SS_BF16 = 0, 1
+SS_DT_SOFTPLUS = 1
+STATUS = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE", 4: "SS_ERR_ALIGN",
+          5: "SS_ERR_UNSUPPORTED", 6: "SS_ERR_CUDA", 7: "SS_ERR_TIMEOUT", 8: "SS_ERR_ALIAS",
+          9: "SS_ERR_WORKSPACE"}
+EXPORTS = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_scan_status", "ss_state_update",
+           "ss_status_string", "ss_abi_version")
+ABI_MAJOR = 2
+
+_lock = threading.Lock()
+_lib = None
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+
+
+class SSError(RuntimeError):
+    """A non-zero status returned by the library."""
+
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = load_library().ss_status_string(status).decode()
+        super().__init__(f"{fn} failed: {msg} (status {status})")
+
+
+def load_library(path: str = LIB_PATH):
+    """Load (once) and return the ctypes handle of ``libssscan.so``."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise RuntimeError(
+                    f"{path} is not built; run `python -m selective_state_space_18_b200.build`")
+            lib = ctypes.CDLL(path)
+            lib.ss_scan_fwd.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 10 + [
+                ctypes.c_uint32, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+            lib.ss_scan_fwd.restype = ctypes.c_int
+            lib.ss_scan_workspace_bytes.argtypes = [_i64, _i64, _i64, _i64]
+            lib.ss_scan_workspace_bytes.restype = _i64
+            lib.ss_scan_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_int)]
+            lib.ss_scan_status.restype = ctypes.c_int
+            lib.ss_state_update.argtypes = [_i64, _i64, _i64, ctypes.c_int] + [_vp] * 9 + [
+                ctypes.c_uint32, _vp, _vp]
+            lib.ss_state_update.restype = ctypes.c_int
+            lib.ss_status_string.argtypes = [ctypes.c_int]
+            lib.ss_status_string.restype = ctypes.c_char_p
+            lib.ss_abi_version.argtypes = []
+            lib.ss_abi_version.restype = ctypes.c_int
+            if lib.ss_abi_version() >> 16 != ABI_MAJOR:
+                raise RuntimeError(f"{path}: ABI {lib.ss_abi_version() >> 16}, expected {ABI_MAJOR}")
+            _lib = lib
+    return _lib
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SS_F32
+    if t.dtype == torch.bfloat16:
+        return SS_BF16
+    raise TypeError(f"x must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _prep(t, name, device, dtype=None, shape=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t.contiguous()
+
+
+def _out(t, name, device, dtype, shape):
+    """A caller-supplied output: written in place, so it must already be contiguous."""
+    if t.device != device or t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be a {dtype} tensor of shape {tuple(shape)} on {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+_workspaces = {}
+
+
+def scan_workspace(batch, channels, state_dim, seq, device, stream=None):
+    """A zero-initialised workspace for ss_scan_fwd, cached per (device, stream) and
+    grown on demand.  Calls on one stream are ordered, so they may share it."""
+    need = int(load_library().ss_scan_workspace_bytes(batch, channels, state_dim, seq))
+    if need <= 0:
+        raise ValueError("invalid scan shape")
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    key = (device.index, stream.cuda_stream)
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < need:
+        with torch.cuda.stream(stream):
+            ws = torch.zeros(max(need, 1 << 16), dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def ss_scan_status(workspace=None, stream=None, device=None):
+    """Read and clear the device status word of earlier scans (synchronises the
+    stream): 'SS_OK' or 'SS_ERR_TIMEOUT'."""
+    if device is None:
+        device = workspace.device if workspace is not None else torch.device("cuda", torch.cuda.current_device())
+    out = ctypes.c_int(-1)
+    st = load_library().ss_scan_status(_ptr(workspace), _stream(stream, device), ctypes.byref(out))
+    if st != 0:
+        raise SSError("ss_scan_status", st)
+    return STATUS[out.value]
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def ss_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h0=None, *,
+                dt_softplus=True, y=None, h_last=None, return_last_state=True, stream=None,
+                workspace=True):
+    """Prompt scan.  x, dt, z: [batch, channels, seq]; B, C: [batch, state_dim, seq];
+    A: [channels, state_dim] fp32; D, dt_bias: [channels] fp32; reset: [batch, seq]
+    bool/uint8; h0: [batch, channels, state_dim] fp32.  Returns (y, h_last).
+
+    workspace: True (a cached per-stream workspace: segmented, balanced schedule),
+    False (none: one CTA per channel group) or a zero-initialised uint8 tensor."""
+    if x.dim() != 3:
+        raise ValueError("x must be [batch, channels, seq]")
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("ss_scan_fwd runs on CUDA tensors only")
+    bt, ch, L = x.shape
+    n = A.shape[-1]
+    code = _dtype_code(x)
+    x = _prep(x, "x", dev)
+    dt = _prep(dt, "dt", dev, x.dtype, (bt, ch, L))
+    z = _prep(z, "z", dev, x.dtype, (bt, ch, L))
+    B = _prep(B, "B", dev, x.dtype, (bt, n, L))
+    C = _prep(C, "C", dev, x.dtype, (bt, n, L))
+    A = _prep(A, "A", dev, torch.float32, (ch, n))
+    D = _prep(D, "D", dev, torch.float32, (ch,))
+    dt_bias = _prep(dt_bias, "dt_bias", dev, torch.float32, (ch,))
+    h0 = _prep(h0, "h0", dev, torch.float32, (bt, ch, n))
+    if reset is not None:
+        reset = _prep(reset, "reset", dev, None, (bt, L))
+        if reset.dtype == torch.bool:
+            reset = reset.view(torch.uint8)
+        elif reset.dtype != torch.uint8:
+            raise TypeError("reset must be bool or uint8")
+    if y is None:
+        y = torch.empty_like(x)
+    else:
+        y = _out(y, "y", dev, x.dtype, (bt, ch, L))
+    if h_last is None and return_last_state:
+        h_last = torch.empty(bt, ch, n, device=dev, dtype=torch.float32)
+    elif h_last is not None:
+        h_last = _out(h_last, "h_last", dev, torch.float32, (bt, ch, n))
+    flags = SS_DT_SOFTPLUS if dt_softplus else 0
+    lib = load_library()
+    if workspace is True:
+        workspace = scan_workspace(bt, ch, n, L, dev, stream)
+    elif workspace is False or workspace is None:
+        workspace = None
+    elif workspace.device != dev or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous uint8 tensor on the inputs' device")
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    st = lib.ss_scan_fwd(bt, ch, n, L, code, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
+                         _ptr(D), _ptr(z), _ptr(dt_bias), _ptr(reset), _ptr(h0), flags,
+                         _ptr(y), _ptr(h_last), _ptr(workspace), ws_bytes, _stream(stream, dev))
+    if st != 0:
+        raise SSError("ss_scan_fwd", st)
+    return y, h_last
+
+
+def ss_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, *, dt_softplus=True,
+                    y=None, stream=None):
+    """Decode step, ``state`` [batch, channels, state_dim] fp32 updated in place.
+    x, dt, z: [batch, channels]; B, C: [batch, state_dim].  Returns y [batch, channels]."""
+    if state.dim() != 3 or state.dtype != torch.float32:
+        raise ValueError("state must be a [batch, channels, state_dim] float32 tensor")
+    if not state.is_contiguous():
+        raise ValueError("state must be contiguous (it is updated in place)")
+    dev = state.device
+    if dev.type != "cuda":
+        raise ValueError("ss_state_update runs on CUDA tensors only")
+    bt, ch, n = state.shape
+    code = _dtype_code(x)
+    x = _prep(x, "x", dev, None, (bt, ch))
+    dt = _prep(dt, "dt", dev, x.dtype, (bt, ch))
+    z = _prep(z, "z", dev, x.dtype, (bt, ch))
+    B = _prep(B, "B", dev, x.dtype, (bt, n))
+    C = _prep(C, "C", dev, x.dtype, (bt, n))
+    A = _prep(A, "A", dev, torch.float32, (ch, n))
+    D = _prep(D, "D", dev, torch.float32, (ch,))
+    dt_bias = _prep(dt_bias, "dt_bias", dev, torch.float32, (ch,))
+    if y is None:
+        y = torch.empty(bt, ch, device=dev, dtype=x.dtype)
+    else:
+        y = _out(y, "y", dev, x.dtype, (bt, ch))
+    flags = SS_DT_SOFTPLUS if dt_softplus else 0
+    lib = load_library()
+    st = lib.ss_state_update(bt, ch, n, code, _ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
+                             _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias), flags, _ptr(y),
+                             _stream(stream, dev))
+    if st != 0:
+        raise SSError("ss_state_update", st)
+    return y
