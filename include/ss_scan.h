@@ -135,6 +135,14 @@ SS_API int ss_state_update(int64_t batch, int64_t channels, int64_t state_dim, s
                     const void *B, const void *C, const float *D, const void *z,
                     const float *dt_bias, uint32_t flags, void *y, ss_stream_t stream);
 
+/*
+ * Testing aid: cap every device-side wait of later calls on the current device at
+ * `microseconds` (0 restores the default of 2 s).  Used to make a wait that can never
+ * be satisfied end quickly with SS_ERR_TIMEOUT; waits for copies already in flight
+ * keep the default limit.  Synchronous; returns SS_OK or SS_ERR_CUDA.
+ */
+SS_API int ss_debug_set_wait_limit(uint32_t microseconds);
+
 /* Human-readable name of a status code (static string, never NULL). */
 SS_API const char *ss_status_string(int status);
 

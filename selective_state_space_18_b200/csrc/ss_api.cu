@@ -262,6 +262,13 @@ const char *ss_status_string(int status)
     }
 }
 
+int ss_debug_set_wait_limit(uint32_t microseconds)
+{
+    return cudaMemcpyToSymbol(ss::g_ss_wait_limit_us, &microseconds, sizeof(microseconds)) == cudaSuccess
+               ? SS_OK
+               : SS_ERR_CUDA;
+}
+
 int64_t ss_scan_workspace_bytes(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq)
 {
     if (batch <= 0 || channels <= 0 || seq <= 0)

@@ -15,12 +15,13 @@
 //  * Work split.  A scan lane owns TWO states of one channel and walks the tokens
 //    in order, so each exponential is computed once and the state never leaves
 //    registers.  A scan warp covers 32 / (N/2) channels (4 at N = 16).
-//  * Warp specialisation.  Each CTA has kScanWarps scan warps, one producer warp and
-//    one epilogue warp.  The producer streams x, dt_raw, z (16-byte loads), B and C
-//    (shared by every channel of a batch row) into a two-stage shared-memory ring,
-//    computing dt = softplus(dt_raw + dt_bias) and dt*x on the way.  The epilogue
-//    warp sums the scan lanes' partial outputs over the N/2 state pairs, applies D*x
-//    and the silu(z) gate and stores y.  The scan warps therefore run an
+//  * Warp specialisation.  Each CTA has four scan warps (one per SM sub-partition,
+//    so all four MUFU units work), two producer warps and two epilogue warps.  The
+//    producers stream x, dt_raw, z, B and C (B, C shared by every channel of a
+//    batch row) into a two-stage shared-memory ring -- as 2-D TMA tile loads several
+//    chunks ahead on aligned shapes -- computing dt = softplus(dt_raw + dt_bias) and
+//    dt*x on the way.  The epilogue warps sum the scan lanes' partial outputs over
+//    the N/2 state pairs, apply D*x and the silu(z) gate and store y.  The scan warps therefore run an
 //    uninterrupted stream of packed fp32x2 multiplies, MUFU ex2 and fused
 //    multiply-adds.  The roles hand chunks of 32 tokens over through mbarriers
 //    (bounded waits).
@@ -75,15 +76,21 @@ template <int N> struct ScanShape {
     static_assert(N == 4 || N == 8 || N == 16, "state_dim must be 4, 8 or 16");
     static constexpr int kPairs = N / 2;               // state pairs = lanes per channel
     static constexpr int kChanPerWarp = 32 / kPairs;
-    static constexpr int kScanWarps = 2;
-    static constexpr int kProducerWarp = kScanWarps, kEpilogueWarp = kScanWarps + 1;
-    static constexpr int kWarps = kScanWarps + 2;
+    // Roles: warps 0-3 scan, warps 4 and 6 produce, warps 5 and 7 run the epilogue,
+    // warp 8 issues the tile loads.  Warp w executes on sub-partition w % 4, so every
+    // sub-partition (and its MUFU unit) holds one scan warp and one IO warp of each CTA.
+    static constexpr int kScanWarps = 4;
+    static constexpr int kIssuerWarp = 8;
+    static constexpr int kWarps = 9;
     static constexpr int kThreads = 32 * kWarps;
+    static constexpr int kIoThreads = 64;              // threads per IO role (2 warps)
     static constexpr int kChanPerCta = kScanWarps * kChanPerWarp;
     static constexpr int kChunk = 32;                  // tokens per pipeline stage
     static constexpr int kBlocks = kChunk / 8;         // 8-token blocks per chunk
     static constexpr int kRow = kChunk + 4;            // padded row (floats)
-    static constexpr int kStages = 2, kYStages = 2;
+    // ring depths: the N = 16 layout (8 KB-scale stages) affords a deeper pipeline;
+    // N = 4 and 8 put 2-4x more channels in a CTA and keep the rings short to fit
+    static constexpr int kStages = N == 16 ? 3 : 2, kYStages = 2;
     // input stage (floats): meta | B,C rows | dt rows | dt*x rows | reset bias
     static constexpr int kMeta = 8;
     static constexpr int kBCOff = kMeta;
@@ -91,21 +98,26 @@ template <int N> struct ScanShape {
     static constexpr int kDXOff = kDTOff + kChanPerCta * kRow;
     static constexpr int kRBOff = kDXOff + kChanPerCta * kRow;
     static constexpr int kInStage = kRBOff + kChunk;
-    // output stage (floats): meta | partial outputs | raw x | raw z
+    // output stage (floats): meta | partial outputs
     static constexpr int kYChan = kPairs * kRow + 4;   // per-channel block, bank-skewed
     static constexpr int kYPOff = kMeta;
-    static constexpr int kXZOff = kYPOff + kChanPerCta * kYChan;
-    static constexpr int kXZFloats = (kChanPerCta * kChunk * 4) / 4; // room for fp32 x or z
-    static constexpr int kYStage = kXZOff + 2 * kXZFloats;
+    static constexpr int kYStage = kYPOff + kChanPerCta * kYChan;
     static constexpr int kFloats = kStages * kInStage + kYStages * kYStage;
     // IO work per chunk
     static constexpr int kTokTasks = kChanPerCta * kBlocks;       // (channel, 8 tokens)
-    static constexpr int kTokPerLane = kTokTasks / 32;
+    static constexpr int kTokPerLane = kTokTasks / kIoThreads;
     static constexpr int kBCTasks = 2 * N * kBlocks;              // (B/C row, 8 tokens)
-    static constexpr int kBCPerLane = (kBCTasks + 31) / 32;
-    // raw ring filled by TMA (aligned shapes): x, dt, z tiles [channels][chunk] and
-    // B, C tiles [N][chunk] in storage type, several chunks ahead of the producer
-    static constexpr int kRawStages = 4;
+    static constexpr int kBCPerLane = (kBCTasks + kIoThreads - 1) / kIoThreads;
+    // raw ring (TMA path): x, dt, z tiles [channels][chunk] and B, C tiles [N][chunk]
+    // in storage type; the issuer warp keeps every slot the producers have released
+    // loading, so up to kRawStages chunks are in flight ahead of them.
+    static constexpr int kRawStages = N == 16 ? 8 : 4;
+    // mbarriers: in_full, in_empty [kStages]; y_full, y_empty [kYStages]; raw_full,
+    // raw_empty [kRawStages]
+    static constexpr int kBarInFull = 0, kBarInEmpty = kStages;
+    static constexpr int kBarYFull = 2 * kStages, kBarYEmpty = 2 * kStages + kYStages;
+    static constexpr int kBarRawFull = 2 * (kStages + kYStages), kBarRawEmpty = kBarRawFull + kRawStages;
+    static constexpr int kBars = kBarRawEmpty + kRawStages;
     template <typename T> static constexpr int raw_x_off() { return 0; }
     template <typename T> static constexpr int raw_dt_off() { return kChanPerCta * kChunk * int(sizeof(T)); }
     template <typename T> static constexpr int raw_z_off() { return 2 * kChanPerCta * kChunk * int(sizeof(T)); }
@@ -119,9 +131,9 @@ template <int N> struct ScanShape {
     template <typename T, bool TMA> static constexpr size_t smem_bytes()
     {
         return size_t(TMA ? kRawStages * raw_stage_bytes<T>() : 0) + size_t(kFloats) * 4 +
-               8 * size_t(8 + kRawStages) + 32 * size_t(kRawStages);
+               8 * size_t(kBars) + 32 * size_t(kRawStages);
     }
-    static_assert(kTokTasks % 32 == 0, "token tasks fill whole IO lanes");
+    static_assert(kTokTasks % kIoThreads == 0, "token tasks fill whole IO lanes");
     static_assert(kInStage % 4 == 0 && kYStage % 4 == 0, "16-byte aligned stages");
 };
 
@@ -222,7 +234,22 @@ struct IoPrefetch {
     Raw8<T> bc[S::kBCPerLane];
     Raw8<T> xr[S::kTokPerLane], dr[S::kTokPerLane], zr[S::kTokPerLane];
     float bias[S::kTokPerLane];
+    int64_t bias_g = -1; // channel group whose dt_bias values `bias` holds
     uint32_t rbyte;
+
+    __device__ __forceinline__ void load_bias(const ScanArgs &p, int lane, int64_t g)
+    {
+        if (g == bias_g)
+            return;
+        bias_g = g;
+        const int64_t c0 = (g % p.groups_per_batch) * S::kChanPerCta;
+#pragma unroll
+        for (int m = 0; m < S::kTokPerLane; ++m) {
+            int64_t c = c0 + (lane + S::kIoThreads * m) / S::kBlocks;
+            c = c < p.channels ? c : p.channels - 1;
+            bias[m] = p.dt_bias ? __ldg(p.dt_bias + c) : 0.0f;
+        }
+    }
 
     __device__ __forceinline__ void load(const ScanArgs &p, int lane, int64_t g, int64_t t0)
     {
@@ -233,7 +260,7 @@ struct IoPrefetch {
         const T *Cb = static_cast<const T *>(p.C) + b * N * L;
 #pragma unroll
         for (int m = 0; m < S::kBCPerLane; ++m) {
-            const int q = lane + 32 * m;
+            const int q = lane + S::kIoThreads * m;
             if (q < S::kBCTasks) {
                 const int r = q % (2 * N), tb = q / (2 * N);
                 const T *src = r < N ? Bb + r * L : Cb + (r - N) * L;
@@ -245,7 +272,7 @@ struct IoPrefetch {
         }
 #pragma unroll
         for (int m = 0; m < S::kTokPerLane; ++m) {
-            const int q = lane + 32 * m;
+            const int q = lane + S::kIoThreads * m;
             const int cl = q / S::kBlocks, tb = q % S::kBlocks;
             int64_t c = c0 + cl;
             c = c < p.channels ? c : p.channels - 1;
@@ -264,8 +291,8 @@ struct IoPrefetch {
                 if (p.z)
                     zr[m].load_scalar(static_cast<const T *>(p.z) + row * L, t, L);
             }
-            bias[m] = p.dt_bias ? __ldg(p.dt_bias + c) : 0.0f;
         }
+        load_bias(p, lane, g);
         if (HAS_RESET)
             rbyte = (lane < S::kChunk && t0 + lane < L) ? uint32_t(__ldg(p.reset + b * L + t0 + lane)) : 0u;
     }
@@ -274,11 +301,10 @@ struct IoPrefetch {
     // the caller).
     __device__ __forceinline__ void load_smem(const ScanArgs &p, int lane, int64_t g, const unsigned char *raw)
     {
-        const int64_t c0 = (g % p.groups_per_batch) * S::kChanPerCta;
         const T *rbc = reinterpret_cast<const T *>(raw + S::template raw_b_off<T>());
 #pragma unroll
         for (int m = 0; m < S::kBCPerLane; ++m) {
-            const int q = lane + 32 * m;
+            const int q = lane + S::kIoThreads * m;
             if (q < S::kBCTasks) {
                 const int r = q % (2 * N), tb = q / (2 * N);
                 bc[m].load_smem(rbc + r * S::kChunk + tb * 8);
@@ -289,28 +315,26 @@ struct IoPrefetch {
         const T *rz = reinterpret_cast<const T *>(raw + S::template raw_z_off<T>());
 #pragma unroll
         for (int m = 0; m < S::kTokPerLane; ++m) {
-            const int q = lane + 32 * m;
+            const int q = lane + S::kIoThreads * m;
             const int cl = q / S::kBlocks, tb = q % S::kBlocks;
             xr[m].load_smem(rx + cl * S::kChunk + tb * 8);
             dr[m].load_smem(rd + cl * S::kChunk + tb * 8);
             if (p.z)
                 zr[m].load_smem(rz + cl * S::kChunk + tb * 8);
-            int64_t c = c0 + cl;
-            c = c < p.channels ? c : p.channels - 1;
-            bias[m] = p.dt_bias ? __ldg(p.dt_bias + c) : 0.0f;
         }
+        load_bias(p, lane, g);
     }
 };
 
 template <int N, typename T, bool HAS_RESET, bool VEC>
 __device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane, const IoPrefetch<N, T, HAS_RESET, VEC> &f,
-                                              float *stage, float *ystage, int64_t t0)
+                                              float *stage, int64_t t0)
 {
     using S = ScanShape<N>;
     const int64_t L = p.seq;
 #pragma unroll
     for (int m = 0; m < S::kBCPerLane; ++m) {
-        const int q = lane + 32 * m;
+        const int q = lane + S::kIoThreads * m;
         if (q < S::kBCTasks) {
             const int r = q % (2 * N), tb = q / (2 * N);
             const int srow = (r < N ? 0 : N) + bc_row<N>(r < N ? r : r - N);
@@ -324,7 +348,7 @@ __device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane, const
     const bool softplus_on = p.softplus != 0;
 #pragma unroll
     for (int m = 0; m < S::kTokPerLane; ++m) {
-        const int q = lane + 32 * m;
+        const int q = lane + S::kIoThreads * m;
         const int cl = q / S::kBlocks, tb = q % S::kBlocks;
         const int64_t tl = t0 + tb * 8;
         float2 dtv[4], dxv[4];
@@ -346,12 +370,6 @@ __device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane, const
         pd[1] = make_float4(dtv[2].x, dtv[2].y, dtv[3].x, dtv[3].y);
         px[0] = make_float4(dxv[0].x, dxv[0].y, dxv[1].x, dxv[1].y);
         px[1] = make_float4(dxv[2].x, dxv[2].y, dxv[3].x, dxv[3].y);
-        // raw x and z for the epilogue warp, in the output stage's side buffers
-        Raw8<T> *xs = reinterpret_cast<Raw8<T> *>(ystage + S::kXZOff) + cl * S::kBlocks + tb;
-        Raw8<T> *zs = reinterpret_cast<Raw8<T> *>(ystage + S::kXZOff + S::kXZFloats) + cl * S::kBlocks + tb;
-        *xs = f.xr[m];
-        if (p.z)
-            *zs = f.zr[m];
     }
 }
 
@@ -373,16 +391,46 @@ template <> __device__ __forceinline__ float2 gate2<__nv_bfloat16>(float2 v)
     return __ffma2_rn(h, t, h);
 }
 
+// D[c] of this thread's epilogue channels, reloaded only when the channel group changes.
+template <int N> struct DCache {
+    float d[ScanShape<N>::kTokPerLane];
+    int64_t g = -1;
+};
+
+// x and z are re-read from global memory (the producers' tile loads brought them into
+// L2 a few chunks earlier); the loads are issued first and their latency overlaps
+// the sum of the partial outputs.
 template <int N, typename T, bool VEC>
-__device__ __forceinline__ void epilogue_chunk(const ScanArgs &p, int lane, const float *ystage, int64_t g, int64_t t0)
+__device__ __forceinline__ void epilogue_chunk(const ScanArgs &p, int lane, const float *ystage, int64_t g, int64_t t0,
+                                               DCache<N> &dcache)
 {
     using S = ScanShape<N>;
     const int64_t L = p.seq;
     const int64_t b = g / p.groups_per_batch;
     const int64_t c0 = (g % p.groups_per_batch) * S::kChanPerCta;
+    Raw8<T> xs[S::kTokPerLane], zs[S::kTokPerLane];
+#pragma unroll
+    for (int m = 0; m < S::kTokPerLane; ++m) { // x and z first: their latency overlaps the sums
+        const int q = lane + S::kIoThreads * m;
+        const int cl = q / S::kBlocks, tb = q % S::kBlocks;
+        int64_t c = c0 + cl;
+        c = c < p.channels ? c : p.channels - 1;
+        const int64_t off = (b * p.channels + c) * L;
+        if (VEC) {
+            xs[m].load_vec(static_cast<const T *>(p.x) + off, t0 + tb * 8, L);
+            if (p.z)
+                zs[m].load_vec(static_cast<const T *>(p.z) + off, t0 + tb * 8, L);
+        } else {
+            xs[m].load_scalar(static_cast<const T *>(p.x) + off, t0 + tb * 8, L);
+            if (p.z)
+                zs[m].load_scalar(static_cast<const T *>(p.z) + off, t0 + tb * 8, L);
+        }
+        if (dcache.g != g)
+            dcache.d[m] = p.D ? __ldg(p.D + c) : 0.0f;
+    }
 #pragma unroll
     for (int m = 0; m < S::kTokPerLane; ++m) {
-        const int q = lane + 32 * m;
+        const int q = lane + S::kIoThreads * m;
         const int cl = q / S::kBlocks, tb = q % S::kBlocks;
         const int64_t c = c0 + cl;
         float2 o[4];
@@ -400,21 +448,20 @@ __device__ __forceinline__ void epilogue_chunk(const ScanArgs &p, int lane, cons
         }
         if (c >= p.channels)
             continue;
-        const Raw8<T> xs = reinterpret_cast<const Raw8<T> *>(ystage + S::kXZOff)[cl * S::kBlocks + tb];
-        const float Dc = p.D ? __ldg(p.D + c) : 0.0f;
+        const float Dc = dcache.d[m];
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-            o[k] = __ffma2_rn(make_float2(Dc, Dc), make_float2(xs.get(2 * k), xs.get(2 * k + 1)), o[k]);
+            o[k] = __ffma2_rn(make_float2(Dc, Dc), make_float2(xs[m].get(2 * k), xs[m].get(2 * k + 1)), o[k]);
         if (p.z) {
-            const Raw8<T> zs = reinterpret_cast<const Raw8<T> *>(ystage + S::kXZOff + S::kXZFloats)[cl * S::kBlocks + tb];
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-                o[k] = __fmul2_rn(o[k], gate2<T>(make_float2(zs.get(2 * k), zs.get(2 * k + 1))));
+                o[k] = __fmul2_rn(o[k], gate2<T>(make_float2(zs[m].get(2 * k), zs[m].get(2 * k + 1))));
         }
         const float out[8] = {o[0].x, o[0].y, o[1].x, o[1].y, o[2].x, o[2].y, o[3].x, o[3].y};
         T *yrow = static_cast<T *>(p.y) + (b * p.channels + c) * L;
         store8<T, VEC>(yrow, t0 + tb * 8, L, out);
     }
+    dcache.g = g;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -425,7 +472,7 @@ __device__ __forceinline__ void epilogue_chunk(const ScanArgs &p, int lane, cons
 struct CtaCtx {
     float *in_base, *y_base;
     unsigned char *raw_base;
-    uint64_t *in_full, *in_empty, *y_full, *y_empty, *raw_full;
+    uint64_t *in_full, *in_empty, *y_full, *y_empty, *raw_full, *raw_empty;
     int64_t *raw_meta; // per raw stage: t0, g, (s | flags << 32)
     WsHeader *ws;
     uint32_t *status;
@@ -450,154 +497,132 @@ template <int N> __device__ __forceinline__ int64_t unit_chunks(const ScanArgs &
     return (len + ScanShape<N>::kChunk - 1) / ScanShape<N>::kChunk;
 }
 
-// Register-prefetch producer (any shape and alignment): every lane walks the same
-// unit sequence; lane 0 takes units and broadcasts them.
-template <int N, typename T, bool HAS_RESET, bool VEC>
-__device__ __forceinline__ void producer_ldg(const ScanArgs &p, const CtaCtx &cx, int lane)
-{
-    using S = ScanShape<N>;
-    auto next = [&](bool first) -> uint32_t {
-        uint32_t u = 0;
-        if (lane == 0)
-            u = take_unit(p, cx.ws, first);
-        return __shfl_sync(0xffffffffu, u, 0);
-    };
-    uint32_t u = next(true);
-    int64_t k = 0, nck = u != kNoUnit ? unit_chunks<N>(p, u) : 0;
-    IoPrefetch<N, T, HAS_RESET, VEC> pf;
-    if (u != kNoUnit)
-        pf.load(p, lane, int64_t(u) % p.groups, (int64_t(u) / p.groups) * p.seg_len);
-    for (uint32_t i = 0;; ++i) {
-        const int st = int(i % S::kStages);
-        const uint32_t ph = ((i / S::kStages) & 1u) ^ 1u;
-        // the input stage is free once the scan warps are done with chunk i-2; the
-        // output stage's side buffers once the epilogue warp is
-        if (!mbar_wait(cx.in_empty + st, ph, cx.status) || !mbar_wait(cx.y_empty + st, ph, cx.status))
-            return;
-        float *stage = cx.in_base + st * S::kInStage;
-        float *ystage = cx.y_base + st * S::kYStage;
-        const bool end = (u == kNoUnit);
-        int64_t g = 0, s = 0, t0 = 0;
-        if (!end) {
-            g = int64_t(u) % p.groups;
-            s = int64_t(u) / p.groups;
-            t0 = s * p.seg_len + k * S::kChunk;
-            produce_chunk<N, T, HAS_RESET, VEC>(p, lane, pf, stage, ystage, t0);
-        }
-        if (lane == 0) {
-            const int32_t fl = end ? kEnd : ((k == 0 ? kFirst : 0) | (k + 1 == nck ? kLast : 0));
-            write_meta(stage, t0, g, int32_t(s), fl);
-            write_meta(ystage, t0, g, int32_t(s), fl);
-        }
-        mbar_arrive(cx.in_full + st);
-        if (end)
-            return;
-        if (++k == nck) {
-            u = next(false);
-            k = 0;
-            nck = u != kNoUnit ? unit_chunks<N>(p, u) : 0;
-        }
-        if (u != kNoUnit)
-            pf.load(p, lane, int64_t(u) % p.groups, (int64_t(u) / p.groups) * p.seg_len + k * S::kChunk);
-    }
-}
-
-// TMA producer (16-byte aligned tensors, seq a multiple of the vector width): lane 0
-// keeps kRawStages - 1 chunks of x, dt, z, B, C in flight as 2-D tile loads into
-// the raw ring; the warp converts each landed chunk into the input stage.
-template <int N, typename T, bool HAS_RESET>
-__device__ __forceinline__ void producer_tma(const ScanArgs &p, const TmaMaps &maps, const CtaCtx &cx, int lane)
+// The issuer warp (one lane works): takes work units, writes one chunk descriptor per
+// raw-ring slot as far ahead as the ring allows and, on the TMA path (VEC), starts the
+// chunk's 2-D tile loads of x, dt, z, B and C into the slot.  Every lane returns
+// normally, so the warp reaches the kernel's end-of-call accounting as a whole.
+template <int N, typename T, bool VEC>
+__device__ __forceinline__ bool issuer_warp(const ScanArgs &p, const TmaMaps &maps, const CtaCtx &cx, int lane)
 {
     using S = ScanShape<N>;
     constexpr int RS = S::kRawStages;
-    constexpr int kRawBytes = S::template raw_stage_bytes<T>();
+    if (lane != 0)
+        return true;
+    if constexpr (VEC) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.x)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.dt)) : "memory");
+        if (p.z)
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.z)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.B)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.C)) : "memory");
+    }
     const uint32_t tx_bytes = uint32_t(((p.z ? 3 : 2) * S::kChanPerCta + 2 * N) * S::kChunk * sizeof(T));
-    // issue cursor (lane 0 only)
-    uint32_t iu = kNoUnit;
-    int64_t ik = 0, ink = 0;
-    uint32_t issued = 0; // chunks whose loads were issued
-    auto issue = [&](int r) {
-        int64_t *m = cx.raw_meta + 3 * r;
-        if (iu == kNoUnit) {
-            m[2] = int64_t(kEnd) << 32;
-            return;
+    uint32_t u = take_unit(p, cx.ws, true);
+    int64_t k = 0, nck = u != kNoUnit ? unit_chunks<N>(p, u) : 0;
+    for (uint32_t j = 0;; ++j) {
+        const int r = int(j % RS);
+        if (j >= uint32_t(RS) && !mbar_wait(cx.raw_empty + r, ((j / RS) & 1u) ^ 1u, cx.status)) {
+            // the converters gave up: let the loads still in flight land, then leave
+            for (uint32_t c = j > uint32_t(RS) ? j - RS : 0; c < j; ++c)
+                mbar_wait(cx.raw_full + c % RS, (c / RS) & 1u, nullptr);
+            return false;
         }
-        const int64_t g = int64_t(iu) % p.groups, s = int64_t(iu) / p.groups;
-        const int64_t t0 = s * p.seg_len + ik * S::kChunk;
-        const int64_t b = g / p.groups_per_batch, c0 = (g % p.groups_per_batch) * S::kChanPerCta;
-        const int32_t fl = (ik == 0 ? kFirst : 0) | (ik + 1 == ink ? kLast : 0);
+        int64_t *m = cx.raw_meta + 3 * r;
+        if (u == kNoUnit) {
+            m[2] = int64_t(kEnd) << 32;
+            mbar_arrive(cx.raw_full + r);
+            return true;
+        }
+        const int64_t g = int64_t(u) % p.groups, s = int64_t(u) / p.groups;
+        const int64_t t0 = s * p.seg_len + k * S::kChunk;
+        const int32_t fl = (k == 0 ? kFirst : 0) | (k + 1 == nck ? kLast : 0);
         m[0] = t0;
         m[1] = g;
         m[2] = (int64_t(fl) << 32) | int64_t(s);
-        unsigned char *dst = cx.raw_base + r * kRawBytes;
-        uint64_t *bar = cx.raw_full + r;
-        mbar_arrive_expect_tx(bar, tx_bytes);
-        const int32_t tt = int32_t(t0), xrow = int32_t(b * p.channels + c0), brow = int32_t(b * N);
-        tma_load_2d(dst + S::template raw_x_off<T>(), &maps.x, tt, xrow, bar);
-        tma_load_2d(dst + S::template raw_dt_off<T>(), &maps.dt, tt, xrow, bar);
-        if (p.z)
-            tma_load_2d(dst + S::template raw_z_off<T>(), &maps.z, tt, xrow, bar);
-        tma_load_2d(dst + S::template raw_b_off<T>(), &maps.B, tt, brow, bar);
-        tma_load_2d(dst + S::template raw_c_off<T>(), &maps.C, tt, brow, bar);
-        ++issued;
-        if (++ik == ink) {
-            iu = take_unit(p, cx.ws, false);
-            ik = 0;
-            ink = iu != kNoUnit ? unit_chunks<N>(p, iu) : 0;
+        if constexpr (VEC) {
+            const int64_t b = g / p.groups_per_batch, c0 = (g % p.groups_per_batch) * S::kChanPerCta;
+            unsigned char *dst = cx.raw_base + r * S::template raw_stage_bytes<T>();
+            uint64_t *bar = cx.raw_full + r;
+            mbar_arrive_expect_tx(bar, tx_bytes);
+            const int32_t tt = int32_t(t0), xrow = int32_t(b * p.channels + c0), brow = int32_t(b * N);
+            tma_load_2d(dst + S::template raw_x_off<T>(), &maps.x, tt, xrow, bar);
+            tma_load_2d(dst + S::template raw_dt_off<T>(), &maps.dt, tt, xrow, bar);
+            if (p.z)
+                tma_load_2d(dst + S::template raw_z_off<T>(), &maps.z, tt, xrow, bar);
+            tma_load_2d(dst + S::template raw_b_off<T>(), &maps.B, tt, brow, bar);
+            tma_load_2d(dst + S::template raw_c_off<T>(), &maps.C, tt, brow, bar);
+        } else {
+            mbar_arrive(cx.raw_full + r);
         }
-    };
-    // on a timeout: let the loads still in flight land before the CTA can exit
-    auto drain = [&](uint32_t consumed) {
-        if (lane == 0)
-            for (uint32_t c = consumed; c < issued; ++c)
-                mbar_wait(cx.raw_full + c % RS, (c / RS) & 1u, nullptr);
-    };
-    if (lane == 0) {
-        iu = take_unit(p, cx.ws, true);
-        ink = iu != kNoUnit ? unit_chunks<N>(p, iu) : 0;
-        for (int r = 0; r < RS - 1; ++r)
-            issue(r);
+        if (++k == nck) {
+            u = take_unit(p, cx.ws, false);
+            k = 0;
+            nck = u != kNoUnit ? unit_chunks<N>(p, u) : 0;
+        }
     }
-    IoPrefetch<N, T, HAS_RESET, true> pf;
+}
+
+// The two producer warps: each thread converts its share of every chunk (from the
+// raw slot, or straight from global memory on the ragged path) into the input stage.
+template <int N, typename T, bool HAS_RESET, bool VEC>
+__device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, int pi, int lane)
+{
+    using S = ScanShape<N>;
+    constexpr int RS = S::kRawStages;
+    constexpr int kRawBytes = VEC ? S::template raw_stage_bytes<T>() : 0;
+    const int tl = pi * 32 + lane; // producer thread index
+    IoPrefetch<N, T, HAS_RESET, VEC> pf;
     for (uint32_t i = 0;; ++i) {
-        __syncwarp(); // every lane is done reading the raw stage refilled next
-        if (lane == 0) {
-            fence_proxy_async_smem();
-            issue(int((i + RS - 1) % RS));
-        }
-        __syncwarp();
         const int r = int(i % RS);
+        if (!mbar_wait(cx.raw_full + r, (i / RS) & 1u, cx.status))
+            return false;
         const int64_t *m = cx.raw_meta + 3 * r;
         const int64_t t0 = m[0], g = m[1];
         const int32_t s = int32_t(m[2] & 0xffffffff), fl = int32_t(m[2] >> 32);
         const bool end = (fl & kEnd) != 0;
-        if (HAS_RESET && !end) {
-            const int64_t b = g / p.groups_per_batch;
-            pf.rbyte = (lane < S::kChunk && t0 + lane < p.seq) ? uint32_t(__ldg(p.reset + b * p.seq + t0 + lane)) : 0u;
-        }
-        const int st = int(i % S::kStages);
-        const uint32_t ph = ((i / S::kStages) & 1u) ^ 1u;
-        if (!mbar_wait(cx.in_empty + st, ph, cx.status) || !mbar_wait(cx.y_empty + st, ph, cx.status)) {
-            drain(i);
-            return;
-        }
-        float *stage = cx.in_base + st * S::kInStage;
-        float *ystage = cx.y_base + st * S::kYStage;
         if (!end) {
-            if (!mbar_wait(cx.raw_full + r, (i / RS) & 1u, cx.status)) {
-                drain(i);
-                return;
+            if constexpr (VEC)
+                pf.load_smem(p, tl, g, cx.raw_base + r * kRawBytes);
+            else
+                pf.load(p, tl, g, t0);
+            if (HAS_RESET) {
+                const int64_t b = g / p.groups_per_batch;
+                pf.rbyte = (tl < S::kChunk && t0 + tl < p.seq) ? uint32_t(__ldg(p.reset + b * p.seq + t0 + tl)) : 0u;
             }
-            pf.load_smem(p, lane, g, cx.raw_base + r * kRawBytes);
-            produce_chunk<N, T, HAS_RESET, true>(p, lane, pf, stage, ystage, t0);
         }
-        if (lane == 0) {
-            write_meta(stage, t0, g, s, end ? kEnd : fl);
-            write_meta(ystage, t0, g, s, end ? kEnd : fl);
-        }
+        mbar_arrive(cx.raw_empty + r); // this thread's reads of slot r are done
+        const int st = int(i % S::kStages);
+        // the input stage is free once the scan warps are done with chunk i - kStages
+        if (!mbar_wait(cx.in_empty + st, ((i / S::kStages) & 1u) ^ 1u, cx.status))
+            return false;
+        float *stage = cx.in_base + st * S::kInStage;
+        if (!end)
+            produce_chunk<N, T, HAS_RESET, VEC>(p, tl, pf, stage, t0);
+        if (tl == 0)
+            write_meta(stage, t0, g, s, fl);
         mbar_arrive(cx.in_full + st);
         if (end)
-            return;
+            return true;
+    }
+}
+
+// The two epilogue warps: partial outputs of each chunk -> y.  False on a timeout.
+template <int N, typename T, bool VEC>
+__device__ __forceinline__ bool epilogue_role(const ScanArgs &p, const float *y_base, uint64_t *y_full,
+                                              uint64_t *y_empty, uint32_t *status, int tl)
+{
+    using S = ScanShape<N>;
+    DCache<N> dcache;
+    for (uint32_t j = 0;; ++j) {
+        const int ys = int(j % S::kYStages);
+        if (!mbar_wait(y_full + ys, (j / S::kYStages) & 1u, status))
+            return false;
+        const float *ystage = y_base + ys * S::kYStage;
+        const ChunkMeta meta = read_meta(ystage);
+        if (meta.flags & kEnd)
+            return true;
+        epilogue_chunk<N, T, VEC>(p, tl, ystage, meta.g, meta.t0, dcache);
+        mbar_arrive(y_empty + ys);
     }
 }
 
@@ -616,8 +641,8 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
     float *const in_base = reinterpret_cast<float *>(smem_bytes + kRawRing);
     float *const y_base = in_base + S::kStages * S::kInStage;
     uint64_t *const bars = reinterpret_cast<uint64_t *>(in_base + S::kFloats);
-    uint64_t *const in_full = bars, *const in_empty = bars + 2;
-    uint64_t *const y_full = bars + 4, *const y_empty = bars + 6;
+    uint64_t *const in_full = bars + S::kBarInFull, *const in_empty = bars + S::kBarInEmpty;
+    uint64_t *const y_full = bars + S::kBarYFull, *const y_empty = bars + S::kBarYEmpty;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     WsHeader *const ws = reinterpret_cast<WsHeader *>(p.workspace);
@@ -630,19 +655,24 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
         : nullptr;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(in_full + s, 32);
+        for (int s = 0; s < S::kStages; ++s) {
+            mbar_init(in_full + s, S::kIoThreads);          // both producer warps
             mbar_init(in_empty + s, 32 * S::kScanWarps);
-            mbar_init(y_full + s, 32 * S::kScanWarps);
-            mbar_init(y_empty + s, 32);
         }
-        for (int r = 0; r < S::kRawStages; ++r)
-            mbar_init(bars + 8 + r, 1);
+        for (int s = 0; s < S::kYStages; ++s) {
+            mbar_init(y_full + s, 32 * S::kScanWarps);
+            mbar_init(y_empty + s, S::kIoThreads);          // both epilogue warps
+        }
+        for (int r = 0; r < S::kRawStages; ++r) {
+            mbar_init(bars + S::kBarRawFull + r, 1);              // the issuer
+            mbar_init(bars + S::kBarRawEmpty + r, S::kIoThreads); // both producer warps
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
 
-    if (warp == S::kProducerWarp) {
+    if (warp >= S::kScanWarps) {
+        // ============================== IO warps ==============================
         CtaCtx cx;
         cx.in_base = in_base;
         cx.y_base = y_base;
@@ -651,27 +681,21 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
         cx.in_empty = in_empty;
         cx.y_full = y_full;
         cx.y_empty = y_empty;
-        cx.raw_full = bars + 8;
-        cx.raw_meta = reinterpret_cast<int64_t *>(bars + 8 + S::kRawStages);
+        cx.raw_full = bars + S::kBarRawFull;
+        cx.raw_empty = bars + S::kBarRawEmpty;
+        cx.raw_meta = reinterpret_cast<int64_t *>(bars + S::kBars);
         cx.ws = ws;
         cx.status = status;
-        if constexpr (kTma)
-            producer_tma<N, T, HAS_RESET>(p, maps, cx, lane);
+        bool ok;
+        if (warp == S::kIssuerWarp)
+            ok = issuer_warp<N, T, VEC>(p, maps, cx, lane);
+        else if (((warp - S::kScanWarps) & 1) == 0)
+            ok = producer<N, T, HAS_RESET, VEC>(p, cx, (warp - S::kScanWarps) >> 1, lane);
         else
-            producer_ldg<N, T, HAS_RESET, VEC>(p, cx, lane);
-    } else if (warp == S::kEpilogueWarp) {
-        // ============================== epilogue warp ============================
-        for (uint32_t j = 0;; ++j) {
-            const int ys = int(j % S::kYStages);
-            if (!mbar_wait(y_full + ys, (j / S::kYStages) & 1u, status))
-                return;
-            const float *ystage = y_base + ys * S::kYStage;
-            const ChunkMeta meta = read_meta(ystage);
-            if (meta.flags & kEnd)
-                break;
-            epilogue_chunk<N, T, VEC>(p, lane, ystage, meta.g, meta.t0);
-            mbar_arrive(y_empty + ys);
-        }
+            ok = epilogue_role<N, T, VEC>(p, y_base, y_full, y_empty, status,
+                                          ((warp - S::kScanWarps) >> 1) * 32 + lane);
+        if (!ok)
+            return; // gave up on a wait (SS_ERR_TIMEOUT recorded)
     } else {
         // =============================== scan warps ==============================
         const int cw = lane / S::kPairs;    // channel within the warp
@@ -691,6 +715,8 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
             const uint32_t ysi = j % S::kYStages;
             if (!mbar_wait(y_empty + ysi, ((j / S::kYStages) & 1u) ^ 1u, status))
                 return;
+            if (warp == 0 && lane == 0) // the epilogue warps learn the chunk from its output stage
+                write_meta(y_base + ysi * S::kYStage, meta.t0, meta.g, meta.s, meta.flags);
             if (meta.flags & kEnd) {
                 mbar_arrive(y_full + ysi); // lets the epilogue warp see the end marker
                 break;
@@ -794,7 +820,6 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
     // needed after the roles have diverged; a warp that gave up on a wait never gets
     // here, and then the workspace stays as it is and the status word says why.)
     if (chained) {
-        __syncwarp();
         if (lane == 0) {
             __threadfence();
             const uint32_t done = atomicAdd(&ws->done, 1u);

@@ -30,7 +30,7 @@ struct UpdateArgs {
 };
 
 constexpr int kUpdateThreads = 256;
-constexpr int kUpdateItems = 4; // row quarters per thread
+constexpr int kUpdateItems = 8; // row quarters per thread: 128 B of state in flight each
 
 template <typename T> struct Vec4;
 template <> struct Vec4<float> {
@@ -69,38 +69,42 @@ ss_state_update_kernel(const UpdateArgs p)
     const float4 bv = Vec4<T>::load(Bb + 4 * lane_q, VEC);
     const float4 cv = Vec4<T>::load(Cb + 4 * lane_q, VEC);
 
-    float4 s[kUpdateItems], a[kUpdateItems];
-    float xs[kUpdateItems], ds[kUpdateItems], zs[kUpdateItems], bias[kUpdateItems], dc[kUpdateItems];
-    int64_t rows[kUpdateItems];
-    bool valid[kUpdateItems];
+    // channel of item `it` (clamped: lanes past the end compute on a valid row and
+    // store nothing)
+    auto chan = [&](int it) -> int64_t {
+        const int64_t c = (j0 + it * kUpdateThreads) >> kQShift;
+        return c < p.channels ? c : p.channels - 1;
+    };
+    // all state loads first (the HBM stream), then the small per-row operands
+    float4 s[kUpdateItems];
 #pragma unroll
     for (int it = 0; it < kUpdateItems; ++it) {
-        const int64_t j = j0 + it * kUpdateThreads;
-        int64_t c = j >> kQShift;
-        valid[it] = c < p.channels;
-        c = valid[it] ? c : p.channels - 1;          // compute on a valid row, store nothing
-        const int64_t row = b * p.channels + c;
-        rows[it] = row;
-        const float *sp = p.state + row * N + 4 * lane_q;
+        const float *sp = p.state + (b * p.channels + chan(it)) * N + 4 * lane_q;
         s[it] = VEC ? __ldcs(reinterpret_cast<const float4 *>(sp)) : make_float4(sp[0], sp[1], sp[2], sp[3]);
-        a[it] = Vec4<float>::load(p.A + c * N + 4 * lane_q, VEC);
+    }
+    float xs[kUpdateItems], ds[kUpdateItems];
+#pragma unroll
+    for (int it = 0; it < kUpdateItems; ++it) {
+        const int64_t row = b * p.channels + chan(it);
         xs[it] = Elem<T>::load(static_cast<const T *>(p.x) + row);
         ds[it] = Elem<T>::load(static_cast<const T *>(p.dt) + row);
-        zs[it] = p.z ? Elem<T>::load(static_cast<const T *>(p.z) + row) : 0.0f;
-        bias[it] = p.dt_bias ? __ldg(p.dt_bias + c) : 0.0f;
-        dc[it] = p.D ? __ldg(p.D + c) : 0.0f;
     }
 #pragma unroll
     for (int it = 0; it < kUpdateItems; ++it) {
-        const float r = ds[it] + bias[it];
+        const int64_t c = chan(it);
+        const int64_t row = b * p.channels + c;
+        const bool valid = ((j0 + it * kUpdateThreads) >> kQShift) < p.channels;
+        const float4 a = Vec4<float>::load(p.A + c * N + 4 * lane_q, VEC);
+        const float bias = p.dt_bias ? __ldg(p.dt_bias + c) : 0.0f;
+        const float r = ds[it] + bias;
         const float d = p.softplus ? softplus(r) : r;
         const float dx = d * xs[it];
         const float dl = d * kLog2e;
         float4 st = s[it];
-        st.x = fmaf(ex2(dl * a[it].x), st.x, dx * bv.x);
-        st.y = fmaf(ex2(dl * a[it].y), st.y, dx * bv.y);
-        st.z = fmaf(ex2(dl * a[it].z), st.z, dx * bv.z);
-        st.w = fmaf(ex2(dl * a[it].w), st.w, dx * bv.w);
+        st.x = fmaf(ex2(dl * a.x), st.x, dx * bv.x);
+        st.y = fmaf(ex2(dl * a.y), st.y, dx * bv.y);
+        st.z = fmaf(ex2(dl * a.z), st.z, dx * bv.z);
+        st.w = fmaf(ex2(dl * a.w), st.w, dx * bv.w);
         float yp = cv.x * st.x;
         yp = fmaf(cv.y, st.y, yp);
         yp = fmaf(cv.z, st.z, yp);
@@ -108,8 +112,8 @@ ss_state_update_kernel(const UpdateArgs p)
 #pragma unroll
         for (int off = Q / 2; off >= 1; off >>= 1)
             yp += __shfl_xor_sync(0xffffffffu, yp, off);
-        if (valid[it]) {
-            float *sp = p.state + rows[it] * N + 4 * lane_q;
+        if (valid) {
+            float *sp = p.state + row * N + 4 * lane_q;
             if (VEC)
                 __stcs(reinterpret_cast<float4 *>(sp), st);
             else {
@@ -119,10 +123,10 @@ ss_state_update_kernel(const UpdateArgs p)
                 sp[3] = st.w;
             }
             if (lane_q == 0) {
-                float v = fmaf(dc[it], xs[it], yp);
+                float v = fmaf(p.D ? __ldg(p.D + c) : 0.0f, xs[it], yp);
                 if (p.z)
-                    v *= silu(zs[it]);
-                Elem<T>::store(static_cast<T *>(p.y) + rows[it], v);
+                    v *= silu(Elem<T>::load(static_cast<const T *>(p.z) + row));
+                Elem<T>::store(static_cast<T *>(p.y) + row, v);
             }
         }
     }

@@ -5,8 +5,9 @@
 //    sequence segment to the next (possibly on another SM);
 //  * a work counter in global memory handing out (channel group, segment) units.
 //
-// Every wait gives up after a fixed number of polls, records SS_ERR_TIMEOUT in the
-// workspace status word and lets the caller unwind; nothing here can spin forever.
+// Every wait gives up after a fixed time (2 s, measured with the global timer),
+// records SS_ERR_TIMEOUT in the status word and lets the caller unwind; nothing here
+// can spin forever.
 #pragma once
 
 #include <cuda.h> // CUtensorMap
@@ -15,9 +16,25 @@
 
 namespace ss {
 
-constexpr uint32_t kMaxBarrierPolls = 1u << 26;  // shared-memory barrier polls
-constexpr uint32_t kMaxFlagPolls = 1u << 24;     // global flag polls (with back-off)
+constexpr uint64_t kWaitLimitNs = 2000000000ull; // 2 s: far above any legitimate wait
 constexpr uint32_t kStatusTimeout = 7u;          // SS_ERR_TIMEOUT
+
+// Time limit override for the waits of later calls, in microseconds (0: kWaitLimitNs).
+// Lets a test make a wait run out quickly; set through ss_debug_set_wait_limit.
+__device__ uint32_t g_ss_wait_limit_us;
+
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint64_t wait_limit_ns(bool overridable)
+{
+    const uint32_t us = overridable ? *reinterpret_cast<volatile uint32_t *>(&g_ss_wait_limit_us) : 0u;
+    return us ? uint64_t(us) * 1000ull : kWaitLimitNs;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -62,25 +79,39 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// One test of the phase.  If it has not completed, the thread is suspended in
+// hardware until it completes or about kSuspendHintNs pass, so a waiting warp does
+// not take issue slots from the warps sharing its sub-partition.
+constexpr uint32_t kSuspendHintNs = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
                  "selp.u32 %0, 1, 0, p;\n\t}"
                  : "=r"(ok)
-                 : "r"(smem_u32(bar)), "r"(parity)
+                 : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
                  : "memory");
     return ok != 0;
 }
 
 // Wait until the phase of `bar` with the given parity has completed.  Returns false
-// (after recording a timeout in *status) if it did not within the poll budget.
+// (after recording a timeout in *status) if it did not within the time limit.  A NULL
+// status marks a drain wait (for copies in flight), which keeps the default limit
+// whatever the override says.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *status)
 {
-    for (uint32_t i = 0; i < kMaxBarrierPolls; ++i)
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t limit = wait_limit_ns(status != nullptr);
+    const uint64_t t0 = global_ns();
+    for (;;) {
         if (mbar_try_wait(bar, parity))
             return true;
+        if (global_ns() - t0 > limit)
+            break;
+    }
     if (status)
         atomicOr(status, 1u << kStatusTimeout);
     return false;
@@ -101,9 +132,13 @@ __device__ __forceinline__ void st_release_gpu(uint64_t *p, uint64_t v)
 // All lanes of a warp poll `flag` until it holds `want`.  Returns false on timeout.
 __device__ __forceinline__ bool flag_wait(const uint64_t *flag, uint64_t want, uint32_t *status)
 {
-    for (uint32_t i = 0; i < kMaxFlagPolls; ++i) {
+    const uint64_t limit = wait_limit_ns(true);
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 0;; ++i) {
         if (ld_acquire_gpu(flag) == want)
             return true;
+        if (global_ns() - t0 > limit)
+            break;
         __nanosleep(i < 64 ? 32 : 256);
     }
     if (status)

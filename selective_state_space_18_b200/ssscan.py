@@ -23,7 +23,7 @@ STATUS = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE", 4:
           5: "SS_ERR_UNSUPPORTED", 6: "SS_ERR_CUDA", 7: "SS_ERR_TIMEOUT", 8: "SS_ERR_ALIAS",
           9: "SS_ERR_WORKSPACE"}
 EXPORTS = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_scan_status", "ss_state_update",
-           "ss_status_string", "ss_abi_version")
+           "ss_debug_set_wait_limit", "ss_status_string", "ss_abi_version")
 ABI_MAJOR = 2
 
 _lock = threading.Lock()
@@ -62,6 +62,8 @@ def load_library(path: str = LIB_PATH):
             lib.ss_state_update.restype = ctypes.c_int
             lib.ss_status_string.argtypes = [ctypes.c_int]
             lib.ss_status_string.restype = ctypes.c_char_p
+            lib.ss_debug_set_wait_limit.argtypes = [ctypes.c_uint32]
+            lib.ss_debug_set_wait_limit.restype = ctypes.c_int
             lib.ss_abi_version.argtypes = []
             lib.ss_abi_version.restype = ctypes.c_int
             if lib.ss_abi_version() >> 16 != ABI_MAJOR:
@@ -135,6 +137,13 @@ def ss_scan_status(workspace=None, stream=None, device=None):
     if st != 0:
         raise SSError("ss_scan_status", st)
     return STATUS[out.value]
+
+
+def ss_debug_set_wait_limit(microseconds: int) -> None:
+    """Cap device-side waits of later calls at `microseconds` (0: the 2 s default)."""
+    st = load_library().ss_debug_set_wait_limit(int(microseconds))
+    if st != 0:
+        raise SSError("ss_debug_set_wait_limit", st)
 
 
 def _stream(stream, device):
