@@ -112,7 +112,7 @@ PFN_cuTensorMapEncodeTiled tensor_map_encoder()
 // 2-D map over `rows` rows of `inner` contiguous elements, box = chunk x box_rows.
 template <typename T>
 bool encode_rows(CUtensorMap *map, const void *base, int64_t inner, int64_t rows, uint32_t box_inner,
-                 uint32_t box_rows)
+                 uint32_t box_rows, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE)
 {
     PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
     if (!enc)
@@ -123,7 +123,7 @@ bool encode_rows(CUtensorMap *map, const void *base, int64_t inner, int64_t rows
     const cuuint32_t box[2] = {box_inner, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return enc(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -132,11 +132,14 @@ bool build_maps(const ss::ScanArgs &a, ss::TmaMaps *m)
 {
     using S = ss::ScanShape<N>;
     const int64_t rows = a.batch * a.channels, brows = a.batch * N;
+    // B and C tiles are read by the scan warps in place: their 16-byte chunks are
+    // swizzled across the banks (64-byte rows for bf16, 128-byte rows for fp32)
+    const CUtensorMapSwizzle bc_swizzle = sizeof(T) == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     return encode_rows<T>(&m->x, a.x, a.seq, rows, S::kChunk, S::kChanPerCta) &&
            encode_rows<T>(&m->dt, a.dt, a.seq, rows, S::kChunk, S::kChanPerCta) &&
            encode_rows<T>(&m->z, a.z ? a.z : a.x, a.seq, rows, S::kChunk, S::kChanPerCta) &&
-           encode_rows<T>(&m->B, a.B, a.seq, brows, S::kChunk, N) &&
-           encode_rows<T>(&m->C, a.C, a.seq, brows, S::kChunk, N);
+           encode_rows<T>(&m->B, a.B, a.seq, brows, S::kChunk, N, bc_swizzle) &&
+           encode_rows<T>(&m->C, a.C, a.seq, brows, S::kChunk, N, bc_swizzle);
 }
 
 template <int N, typename T, bool R, bool V>

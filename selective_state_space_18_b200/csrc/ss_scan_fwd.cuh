@@ -91,10 +91,9 @@ template <int N> struct ScanShape {
     // ring depths: the N = 16 layout (8 KB-scale stages) affords a deeper pipeline;
     // N = 4 and 8 put 2-4x more channels in a CTA and keep the rings short to fit
     static constexpr int kStages = N == 16 ? 3 : 2, kYStages = 2;
-    // input stage (floats): meta | B,C rows | dt rows | dt*x rows | reset bias
+    // input stage (floats): meta | dt rows | dt*x rows | reset bias
     static constexpr int kMeta = 8;
-    static constexpr int kBCOff = kMeta;
-    static constexpr int kDTOff = kBCOff + 2 * N * kRow;
+    static constexpr int kDTOff = kMeta;
     static constexpr int kDXOff = kDTOff + kChanPerCta * kRow;
     static constexpr int kRBOff = kDXOff + kChanPerCta * kRow;
     static constexpr int kInStage = kRBOff + kChunk;
@@ -108,9 +107,13 @@ template <int N> struct ScanShape {
     static constexpr int kTokPerLane = kTokTasks / kIoThreads;
     static constexpr int kBCTasks = 2 * N * kBlocks;              // (B/C row, 8 tokens)
     static constexpr int kBCPerLane = (kBCTasks + kIoThreads - 1) / kIoThreads;
-    // raw ring (TMA path): x, dt, z tiles [channels][chunk] and B, C tiles [N][chunk]
-    // in storage type; the issuer warp keeps every slot the producers have released
-    // loading, so up to kRawStages chunks are in flight ahead of them.
+    // raw ring: x, dt, z tiles [channels][chunk] and B, C tiles [N][chunk] in storage
+    // type.  On aligned shapes TMA fills whole slots; the issuer warp keeps every
+    // slot its readers have released loading, so up to kRawStages chunks are in
+    // flight.  The scan warps read B and C straight from the slot, in storage type
+    // (bf16 halves their shared-memory traffic), from tiles swizzled by TMA so the
+    // N/2 state rows a warp reads at once fall into distinct banks.  On the ragged
+    // path the producers write the B and C tiles themselves in the same layout.
     static constexpr int kRawStages = N == 16 ? 8 : 4;
     // mbarriers: in_full, in_empty [kStages]; y_full, y_empty [kYStages]; raw_full,
     // raw_empty [kRawStages]
@@ -118,20 +121,22 @@ template <int N> struct ScanShape {
     static constexpr int kBarYFull = 2 * kStages, kBarYEmpty = 2 * kStages + kYStages;
     static constexpr int kBarRawFull = 2 * (kStages + kYStages), kBarRawEmpty = kBarRawFull + kRawStages;
     static constexpr int kBars = kBarRawEmpty + kRawStages;
+    static constexpr int align1k(int b) { return (b + 1023) / 1024 * 1024; }
     template <typename T> static constexpr int raw_x_off() { return 0; }
     template <typename T> static constexpr int raw_dt_off() { return kChanPerCta * kChunk * int(sizeof(T)); }
     template <typename T> static constexpr int raw_z_off() { return 2 * kChanPerCta * kChunk * int(sizeof(T)); }
-    template <typename T> static constexpr int raw_b_off() { return 3 * kChanPerCta * kChunk * int(sizeof(T)); }
-    template <typename T> static constexpr int raw_c_off() { return raw_b_off<T>() + N * kChunk * int(sizeof(T)); }
+    // B and C tiles start on 1024-byte boundaries (the swizzle pattern's period)
+    template <typename T> static constexpr int raw_b_off() { return align1k(3 * kChanPerCta * kChunk * int(sizeof(T))); }
+    template <typename T> static constexpr int raw_c_off() { return raw_b_off<T>() + align1k(N * kChunk * int(sizeof(T))); }
     template <typename T> static constexpr int raw_stage_bytes()
     {
-        return ((raw_c_off<T>() + N * kChunk * int(sizeof(T))) + 127) / 128 * 128;
+        return raw_c_off<T>() + align1k(N * kChunk * int(sizeof(T)));
     }
     // shared memory: [raw ring] [input stages] [output stages] [barriers] [raw meta]
     template <typename T, bool TMA> static constexpr size_t smem_bytes()
     {
-        return size_t(TMA ? kRawStages * raw_stage_bytes<T>() : 0) + size_t(kFloats) * 4 +
-               8 * size_t(kBars) + 32 * size_t(kRawStages);
+        return size_t(kRawStages * raw_stage_bytes<T>()) + size_t(kFloats) * 4 + 8 * size_t(kBars) +
+               32 * size_t(kRawStages);
     }
     static_assert(kTokTasks % kIoThreads == 0, "token tasks fill whole IO lanes");
     static_assert(kInStage % 4 == 0 && kYStage % 4 == 0, "16-byte aligned stages");
@@ -168,11 +173,19 @@ __device__ __forceinline__ ChunkMeta read_meta(const float *stage)
     return m;
 }
 
-// Shared-memory row of state n of B (C rows follow at +N): even states first, then
-// odd ones, so the state pairs of a channel read distinct bank groups.
-template <int N> __device__ __forceinline__ int bc_row(int n)
+// Byte offset of 16-byte chunk `c16` of row `row` in a B or C tile of the raw ring.
+// The tile is a dense [N rows][chunk tokens] box written by TMA with the 64-byte
+// swizzle (bf16 rows of 64 bytes) or the 128-byte swizzle (fp32 rows of 128 bytes):
+// the chunk index is XORed with bits 7.. of the byte address, i.e. with row/2 mod 4
+// or row mod 8, so rows 0..7 of one chunk land in eight distinct bank groups.
+template <typename T> __device__ __forceinline__ int bc_offset(int row, int c16);
+template <> __device__ __forceinline__ int bc_offset<__nv_bfloat16>(int row, int c16)
 {
-    return (n & 1) * (N / 2) + (n >> 1);
+    return row * 64 + ((c16 ^ ((row >> 1) & 3)) << 4);
+}
+template <> __device__ __forceinline__ int bc_offset<float>(int row, int c16)
+{
+    return row * 128 + ((c16 ^ (row & 7)) << 4);
 }
 
 // silu on the output gate: the exact form for fp32 outputs; for bf16 outputs the
@@ -297,19 +310,10 @@ struct IoPrefetch {
             rbyte = (lane < S::kChunk && t0 + lane < L) ? uint32_t(__ldg(p.reset + b * L + t0 + lane)) : 0u;
     }
 
-    // The same registers filled from a raw TMA stage (the reset byte is loaded by
-    // the caller).
+    // x, dt_raw, z filled from a raw TMA stage (B and C stay in the stage for the
+    // scan warps; the reset byte is loaded by the caller).
     __device__ __forceinline__ void load_smem(const ScanArgs &p, int lane, int64_t g, const unsigned char *raw)
     {
-        const T *rbc = reinterpret_cast<const T *>(raw + S::template raw_b_off<T>());
-#pragma unroll
-        for (int m = 0; m < S::kBCPerLane; ++m) {
-            const int q = lane + S::kIoThreads * m;
-            if (q < S::kBCTasks) {
-                const int r = q % (2 * N), tb = q / (2 * N);
-                bc[m].load_smem(rbc + r * S::kChunk + tb * 8);
-            }
-        }
         const T *rx = reinterpret_cast<const T *>(raw + S::template raw_x_off<T>());
         const T *rd = reinterpret_cast<const T *>(raw + S::template raw_dt_off<T>());
         const T *rz = reinterpret_cast<const T *>(raw + S::template raw_z_off<T>());
@@ -328,19 +332,24 @@ struct IoPrefetch {
 
 template <int N, typename T, bool HAS_RESET, bool VEC>
 __device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane, const IoPrefetch<N, T, HAS_RESET, VEC> &f,
-                                              float *stage, int64_t t0)
+                                              float *stage, unsigned char *raw, int64_t t0)
 {
     using S = ScanShape<N>;
     const int64_t L = p.seq;
+    if constexpr (!VEC) { // ragged path: B and C tiles into the raw slot, as TMA would lay them out
 #pragma unroll
-    for (int m = 0; m < S::kBCPerLane; ++m) {
-        const int q = lane + S::kIoThreads * m;
-        if (q < S::kBCTasks) {
-            const int r = q % (2 * N), tb = q / (2 * N);
-            const int srow = (r < N ? 0 : N) + bc_row<N>(r < N ? r : r - N);
-            float4 *dst = reinterpret_cast<float4 *>(stage + S::kBCOff + srow * S::kRow + tb * 8);
-            dst[0] = make_float4(f.bc[m].get(0), f.bc[m].get(1), f.bc[m].get(2), f.bc[m].get(3));
-            dst[1] = make_float4(f.bc[m].get(4), f.bc[m].get(5), f.bc[m].get(6), f.bc[m].get(7));
+        for (int m = 0; m < S::kBCPerLane; ++m) {
+            const int q = lane + S::kIoThreads * m;
+            if (q < S::kBCTasks) {
+                const int r = q % (2 * N), tb = q / (2 * N);
+                unsigned char *tile = raw + (r < N ? S::template raw_b_off<T>() : S::template raw_c_off<T>());
+                const int row = r < N ? r : r - N;
+                constexpr int kChunksPer8 = int(sizeof(T)) / 2; // 16-byte chunks per 8 tokens
+#pragma unroll
+                for (int h = 0; h < kChunksPer8; ++h)
+                    *reinterpret_cast<uint4 *>(tile + bc_offset<T>(row, tb * kChunksPer8 + h)) =
+                        reinterpret_cast<const uint4 *>(&f.bc[m])[h];
+            }
         }
     }
     if (HAS_RESET && lane < S::kChunk)
@@ -497,6 +506,83 @@ template <int N> __device__ __forceinline__ int64_t unit_chunks(const ScanArgs &
     return (len + ScanShape<N>::kChunk - 1) / ScanShape<N>::kChunk;
 }
 
+// Token pair `pi` of a 16-byte chunk of a B or C row, widened to fp32: bf16 rows hold
+// 8 tokens (pairs are 32-bit words), fp32 rows 4.
+template <typename T> __device__ __forceinline__ float2 bc_pair(const uint4 &w, int pi);
+template <> __device__ __forceinline__ float2 bc_pair<__nv_bfloat16>(const uint4 &w, int pi)
+{
+    const uint32_t u = pi == 0 ? w.x : (pi == 1 ? w.y : (pi == 2 ? w.z : w.w));
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+template <> __device__ __forceinline__ float2 bc_pair<float>(const uint4 &w, int pi)
+{
+    return pi == 0 ? make_float2(__uint_as_float(w.x), __uint_as_float(w.y))
+                   : make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
+}
+
+// One chunk of the recurrence for this lane's two states n0, n1 of channel `cl`:
+// dt and dt*x from the input stage, B and C from the raw slot (storage type), the
+// partial outputs C.h over the two states to `ys`.  Per pair of tokens: two packed
+// multiplies for the exponent arguments, four MUFU ex2, two packed multiplies for
+// the increments, four FMAs along the sequence, two packed ops for the readout.
+template <int N, typename T, bool HAS_RESET>
+__device__ __forceinline__ void scan_chunk(const float *stage, const unsigned char *raw, float *ys, int cl, int n0,
+                                           int n1, float2 A0, float2 A1, float &hs0, float &hs1)
+{
+    using S = ScanShape<N>;
+    constexpr int kTok = 16 / int(sizeof(T)); // tokens per 16-byte chunk of a B/C row
+    const unsigned char *Bt = raw + S::template raw_b_off<T>();
+    const unsigned char *Ct = raw + S::template raw_c_off<T>();
+    const float *rbs = stage + S::kRBOff;
+    const float *dts = stage + S::kDTOff + cl * S::kRow;
+    const float *dxs = stage + S::kDXOff + cl * S::kRow;
+#pragma unroll
+    for (int c16 = 0; c16 < S::kChunk / kTok; ++c16) {
+        const uint4 wb0 = *reinterpret_cast<const uint4 *>(Bt + bc_offset<T>(n0, c16));
+        const uint4 wb1 = *reinterpret_cast<const uint4 *>(Bt + bc_offset<T>(n1, c16));
+        const uint4 wc0 = *reinterpret_cast<const uint4 *>(Ct + bc_offset<T>(n0, c16));
+        const uint4 wc1 = *reinterpret_cast<const uint4 *>(Ct + bc_offset<T>(n1, c16));
+#pragma unroll
+        for (int g4 = 0; g4 < kTok / 4; ++g4) {
+            const int t = c16 * kTok + g4 * 4;
+            const float4 d4 = *reinterpret_cast<const float4 *>(dts + t);
+            const float4 u4 = *reinterpret_cast<const float4 *>(dxs + t);
+            float4 r4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (HAS_RESET)
+                r4 = *reinterpret_cast<const float4 *>(rbs + t);
+            float2 yo[2];
+#pragma unroll
+            for (int pr = 0; pr < 2; ++pr) {
+                const int pi = g4 * 2 + pr;
+                const float2 dd = pr ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
+                const float2 uu = pr ? make_float2(u4.z, u4.w) : make_float2(u4.x, u4.y);
+                const float2 B0 = bc_pair<T>(wb0, pi), B1 = bc_pair<T>(wb1, pi);
+                const float2 C0 = bc_pair<T>(wc0, pi), C1 = bc_pair<T>(wc1, pi);
+                float2 g0, g1;
+                if (HAS_RESET) {
+                    const float2 rr = pr ? make_float2(r4.z, r4.w) : make_float2(r4.x, r4.y);
+                    g0 = __ffma2_rn(dd, A0, rr);
+                    g1 = __ffma2_rn(dd, A1, rr);
+                } else {
+                    g0 = __fmul2_rn(dd, A0);
+                    g1 = __fmul2_rn(dd, A1);
+                }
+                const float a0t = ex2(g0.x), a0u = ex2(g0.y);
+                const float a1t = ex2(g1.x), a1u = ex2(g1.y);
+                const float2 v0 = __fmul2_rn(uu, B0);
+                const float2 v1 = __fmul2_rn(uu, B1);
+                const float h0t = fmaf(a0t, hs0, v0.x);
+                hs0 = fmaf(a0u, h0t, v0.y);
+                const float h1t = fmaf(a1t, hs1, v1.x);
+                hs1 = fmaf(a1u, h1t, v1.y);
+                const float2 yy = __fmul2_rn(C0, make_float2(h0t, hs0));
+                yo[pr] = __ffma2_rn(C1, make_float2(h1t, hs1), yy);
+            }
+            *reinterpret_cast<float4 *>(ys + t) = make_float4(yo[0].x, yo[0].y, yo[1].x, yo[1].y);
+        }
+    }
+}
+
 // The issuer warp (one lane works): takes work units, writes one chunk descriptor per
 // raw-ring slot as far ahead as the ring allows and, on the TMA path (VEC), starts the
 // chunk's 2-D tile loads of x, dt, z, B and C into the slot.  Every lane returns
@@ -569,7 +655,7 @@ __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, in
 {
     using S = ScanShape<N>;
     constexpr int RS = S::kRawStages;
-    constexpr int kRawBytes = VEC ? S::template raw_stage_bytes<T>() : 0;
+    constexpr int kRawBytes = S::template raw_stage_bytes<T>();
     const int tl = pi * 32 + lane; // producer thread index
     IoPrefetch<N, T, HAS_RESET, VEC> pf;
     for (uint32_t i = 0;; ++i) {
@@ -597,7 +683,7 @@ __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, in
             return false;
         float *stage = cx.in_base + st * S::kInStage;
         if (!end)
-            produce_chunk<N, T, HAS_RESET, VEC>(p, tl, pf, stage, t0);
+            produce_chunk<N, T, HAS_RESET, VEC>(p, tl, pf, stage, cx.raw_base + r * kRawBytes, t0);
         if (tl == 0)
             write_meta(stage, t0, g, s, fl);
         mbar_arrive(cx.in_full + st);
@@ -635,9 +721,8 @@ __global__ void __launch_bounds__(ScanShape<N>::kThreads, 1)
 ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
 {
     using S = ScanShape<N>;
-    constexpr bool kTma = VEC;
-    constexpr int kRawRing = kTma ? S::kRawStages * S::template raw_stage_bytes<T>() : 0;
-    extern __shared__ __align__(128) unsigned char smem_bytes[];
+    constexpr int kRawRing = S::kRawStages * S::template raw_stage_bytes<T>();
+    extern __shared__ __align__(1024) unsigned char smem_bytes[];
     float *const in_base = reinterpret_cast<float *>(smem_bytes + kRawRing);
     float *const y_base = in_base + S::kStages * S::kInStage;
     uint64_t *const bars = reinterpret_cast<uint64_t *>(in_base + S::kFloats);
@@ -665,7 +750,7 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
         }
         for (int r = 0; r < S::kRawStages; ++r) {
             mbar_init(bars + S::kBarRawFull + r, 1);              // the issuer
-            mbar_init(bars + S::kBarRawEmpty + r, S::kIoThreads); // both producer warps
+            mbar_init(bars + S::kBarRawEmpty + r, S::kIoThreads + 32 * S::kScanWarps); // producers, scan
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -700,7 +785,7 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
         // =============================== scan warps ==============================
         const int cw = lane / S::kPairs;    // channel within the warp
         const int sub = lane % S::kPairs;   // state pair
-        const int n0 = 2 * sub, n1 = 2 * sub + 1;
+        const int n0 = sub, n1 = sub + S::kPairs;   // rows n0 < 8 and n1 >= N/2: distinct banks
         const int cl = warp * S::kChanPerWarp + cw;  // channel within the CTA
         float hs0 = 0.0f, hs1 = 0.0f;
         float2 A0 = make_float2(0.f, 0.f), A1 = make_float2(0.f, 0.f);
@@ -744,59 +829,15 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
                     hs1 = h.y;
                 }
             }
-            float *yst = y_base + ysi * S::kYStage;
-            {
-                const float *Bs0 = stage + S::kBCOff + bc_row<N>(n0) * S::kRow;
-                const float *Bs1 = stage + S::kBCOff + bc_row<N>(n1) * S::kRow;
-                const float *Cs0 = Bs0 + N * S::kRow;
-                const float *Cs1 = Bs1 + N * S::kRow;
-                const float *rbs = stage + S::kRBOff;
-                const float *dts = stage + S::kDTOff + cl * S::kRow;
-                const float *dxs = stage + S::kDXOff + cl * S::kRow;
-                float *ys = yst + S::kYPOff + cl * S::kYChan + sub * S::kRow;
-#pragma unroll
-                for (int t = 0; t < S::kChunk; t += 4) {
-                    const float4 d4 = *reinterpret_cast<const float4 *>(dts + t);
-                    const float4 u4 = *reinterpret_cast<const float4 *>(dxs + t);
-                    const float4 b0 = *reinterpret_cast<const float4 *>(Bs0 + t);
-                    const float4 b1 = *reinterpret_cast<const float4 *>(Bs1 + t);
-                    const float4 q0 = *reinterpret_cast<const float4 *>(Cs0 + t);
-                    const float4 q1 = *reinterpret_cast<const float4 *>(Cs1 + t);
-                    float4 r4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (HAS_RESET)
-                        r4 = *reinterpret_cast<const float4 *>(rbs + t);
-                    float2 yo[2];
-#pragma unroll
-                    for (int pr = 0; pr < 2; ++pr) {
-                        const float2 dd = pr ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
-                        const float2 uu = pr ? make_float2(u4.z, u4.w) : make_float2(u4.x, u4.y);
-                        const float2 B0 = pr ? make_float2(b0.z, b0.w) : make_float2(b0.x, b0.y);
-                        const float2 B1 = pr ? make_float2(b1.z, b1.w) : make_float2(b1.x, b1.y);
-                        const float2 C0 = pr ? make_float2(q0.z, q0.w) : make_float2(q0.x, q0.y);
-                        const float2 C1 = pr ? make_float2(q1.z, q1.w) : make_float2(q1.x, q1.y);
-                        float2 g0, g1;
-                        if (HAS_RESET) {
-                            const float2 rr = pr ? make_float2(r4.z, r4.w) : make_float2(r4.x, r4.y);
-                            g0 = __ffma2_rn(dd, A0, rr);
-                            g1 = __ffma2_rn(dd, A1, rr);
-                        } else {
-                            g0 = __fmul2_rn(dd, A0);
-                            g1 = __fmul2_rn(dd, A1);
-                        }
-                        const float a0t = ex2(g0.x), a0u = ex2(g0.y);
-                        const float a1t = ex2(g1.x), a1u = ex2(g1.y);
-                        const float2 v0 = __fmul2_rn(uu, B0);
-                        const float2 v1 = __fmul2_rn(uu, B1);
-                        const float h0t = fmaf(a0t, hs0, v0.x);
-                        hs0 = fmaf(a0u, h0t, v0.y);
-                        const float h1t = fmaf(a1t, hs1, v1.x);
-                        hs1 = fmaf(a1u, h1t, v1.y);
-                        const float2 yy = __fmul2_rn(C0, make_float2(h0t, hs0));
-                        yo[pr] = __ffma2_rn(C1, make_float2(h1t, hs1), yy);
-                    }
-                    *reinterpret_cast<float4 *>(ys + t) = make_float4(yo[0].x, yo[0].y, yo[1].x, yo[1].y);
-                }
-            }
+            // B and C of this chunk are in its raw slot (landed: the producers waited
+            // for it before releasing the input stage; the wait here is immediate)
+            const int rs = int(j % S::kRawStages);
+            if (!mbar_wait(bars + S::kBarRawFull + rs, (j / S::kRawStages) & 1u, status))
+                return;
+            scan_chunk<N, T, HAS_RESET>(stage, smem_bytes + rs * S::template raw_stage_bytes<T>(),
+                                        y_base + ysi * S::kYStage + S::kYPOff + cl * S::kYChan + sub * S::kRow,
+                                        cl, n0, n1, A0, A1, hs0, hs1);
+            mbar_arrive(bars + S::kBarRawEmpty + rs);
             mbar_arrive(in_empty + st);
             mbar_arrive(y_full + ysi);
             if (meta.flags & kLast) {
