@@ -67,7 +67,8 @@ enum {
     SS_ERR_CUDA = 6,        /* the CUDA runtime reported an error                  */
     SS_ERR_TIMEOUT = 7,     /* a bounded device-side wait gave up                  */
     SS_ERR_ALIAS = 8,       /* an output (or the workspace) overlaps an input      */
-    SS_ERR_WORKSPACE = 9    /* workspace smaller than ss_scan_workspace_bytes()    */
+    SS_ERR_WORKSPACE = 9,   /* workspace smaller than ss_scan_workspace_bytes()    */
+    SS_ERR_SCRATCH_LIMIT = 10 /* the shape needs more than SS_STATIC_SCRATCH_BYTES   */
 };
 
 /* flags bit 0: apply softplus to dt_raw + dt_bias (mamba's delta_softplus). */
@@ -116,6 +117,53 @@ SS_API int64_t ss_scan_workspace_bytes(int64_t batch, int64_t channels, int64_t 
  * SS_OK, or an error status if the query itself failed.
  */
 SS_API int ss_scan_status(const void *workspace, ss_stream_t stream, int *status);
+
+/*
+ * ss_scan_fwd without a caller-supplied workspace and without any allocation.
+ *
+ * The selective-scan method itself has no counterpart to this call: it is a
+ * convenience of this library for callers that cannot allocate or own device memory
+ * at the moment they scan -- a serving loop whose memory plan is fixed at start-up,
+ * or a host program that only receives device pointers from another framework and
+ * has no allocator of its own.  It runs the same segmented, balanced schedule as
+ * ss_scan_fwd with a workspace, using instead a fixed scratch of
+ * SS_STATIC_SCRATCH_BYTES (1 MiB) that the library holds in a static device array,
+ * one per device.  Neither this call nor anything it calls allocates memory.
+ *
+ * Arguments, layouts and results are those of ss_scan_fwd, except:
+ *   flags   : SS_DT_SOFTPLUS as for ss_scan_fwd, plus SS_SCRATCH_ZERO to clear the
+ *             scratch (an asynchronous memset on `stream`) before this scan.
+ *   scratch : nullable; receives the device address of this device's scratch, which
+ *             ss_scan_status(scratch, stream, &st) takes to read the device-side
+ *             status of these calls.
+ *
+ * Limit: the shape must need at most SS_STATIC_SCRATCH_BYTES of workspace
+ * (ss_scan_workspace_bytes); larger shapes are refused with SS_ERR_SCRATCH_LIMIT
+ * before anything is launched.  At state_dim 16 that is up to 992 channel groups of
+ * 16, i.e. batch * ceil(channels / 16) <= 992 (batch 1 at 5120 channels, or batch 8
+ * at 1536, fit).
+ *
+ * Zero state: the scratch is zero when the library is loaded, and every scan that
+ * completes leaves it ready for the next one.  After SS_ERR_TIMEOUT has been
+ * reported, pass SS_SCRATCH_ZERO on the next call.
+ *
+ * Set-up: the first call on each device, with that device current, looks up the
+ * scratch's address (which may load the library's device code) and configures the
+ * kernel; make that first call before any stream capture begins.
+ *
+ * Concurrency: all calls on one device share the one scratch.  Two calls whose
+ * executions overlap (different streams, not ordered by events) race on it and give
+ * wrong results; order them, or use ss_scan_fwd with a workspace per stream.
+ */
+#define SS_STATIC_SCRATCH_BYTES (1u << 20)
+enum { SS_SCRATCH_ZERO = 2u };
+SS_API int ss_scan_fwd_static_scratch(int64_t batch, int64_t channels, int64_t state_dim,
+                                      int64_t seq, ss_dtype_t dtype, const void *x,
+                                      const void *dt_raw, const float *A, const void *B,
+                                      const void *C, const float *D, const void *z,
+                                      const float *dt_bias, const uint8_t *reset,
+                                      const float *h0, uint32_t flags, void *y, float *h_last,
+                                      const void **scratch, ss_stream_t stream);
 
 /*
  * Decode step: one token of the same recurrence for every (b, c), updating `state`

@@ -242,6 +242,36 @@ int dispatch_update_n(const ss::UpdateArgs &a, ss_dtype_t dtype, bool vec, cudaS
     return vec ? launch_update<N, float, true>(a, s) : launch_update<N, float, false>(a, s);
 }
 
+// Scratch of ss_scan_fwd_static_scratch: a fixed workspace in device memory, one per
+// device that loads the library.  Zero at module load; every scan that completes
+// leaves it ready for the next.
+static_assert(SS_STATIC_SCRATCH_BYTES % 256 == 0, "scratch size");
+static __device__ __align__(256) uint8_t g_ss_static_scratch[SS_STATIC_SCRATCH_BYTES];
+
+// Device address of this device's scratch, looked up (with the device current) on
+// the first call and cached per device.
+int static_scratch_address(void **out)
+{
+    static std::atomic<uintptr_t> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return SS_ERR_CUDA;
+    if (dev < 64) {
+        const uintptr_t v = cache[dev].load(std::memory_order_acquire);
+        if (v) {
+            *out = reinterpret_cast<void *>(v);
+            return SS_OK;
+        }
+    }
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_ss_static_scratch) != cudaSuccess || !ptr)
+        return SS_ERR_CUDA;
+    if (dev < 64)
+        cache[dev].store(reinterpret_cast<uintptr_t>(ptr), std::memory_order_release);
+    *out = ptr;
+    return SS_OK;
+}
+
 } // namespace
 
 extern "C" {
@@ -261,6 +291,9 @@ const char *ss_status_string(int status)
     case SS_ERR_TIMEOUT: return "SS_ERR_TIMEOUT: a bounded device-side wait gave up";
     case SS_ERR_ALIAS: return "SS_ERR_ALIAS: an output overlaps an input";
     case SS_ERR_WORKSPACE: return "SS_ERR_WORKSPACE: the workspace is smaller than ss_scan_workspace_bytes()";
+    case SS_ERR_SCRATCH_LIMIT:
+        return "SS_ERR_SCRATCH_LIMIT: the shape needs more workspace than the static scratch holds "
+               "(SS_STATIC_SCRATCH_BYTES); use ss_scan_fwd with a workspace";
     default: return "unknown status";
     }
 }
@@ -446,6 +479,35 @@ int ss_state_update(int64_t batch, int64_t channels, int64_t state_dim, ss_dtype
     case 8: return dispatch_update_n<8>(a, dtype, vec, s);
     default: return dispatch_update_n<16>(a, dtype, vec, s);
     }
+}
+
+// The scratch stands in for the caller's workspace: the shape is checked against its
+// size first, then the scan is exactly ss_scan_fwd's segmented schedule.
+int ss_scan_fwd_static_scratch(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
+                               ss_dtype_t dtype, const void *x, const void *dt_raw, const float *A,
+                               const void *B, const void *C, const float *D, const void *z,
+                               const float *dt_bias, const uint8_t *reset, const float *h0,
+                               uint32_t flags, void *y, float *h_last, const void **scratch,
+                               ss_stream_t stream)
+{
+    if (!x || !dt_raw || !A || !B || !C || !y)
+        return SS_ERR_NULL;
+    if (flags & ~uint32_t(SS_DT_SOFTPLUS | SS_SCRATCH_ZERO))
+        return SS_ERR_UNSUPPORTED;
+    const int64_t need = ss_scan_workspace_bytes(batch, channels, state_dim, seq);
+    if (need > int64_t(SS_STATIC_SCRATCH_BYTES))
+        return SS_ERR_SCRATCH_LIMIT;
+    // (need == 0: an invalid shape, which ss_scan_fwd reports with its own status)
+    void *ws = nullptr;
+    if (static_scratch_address(&ws) != SS_OK)
+        return SS_ERR_CUDA;
+    if (scratch)
+        *scratch = ws;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (need > 0 && (flags & SS_SCRATCH_ZERO) && cudaMemsetAsync(ws, 0, size_t(need), s) != cudaSuccess)
+        return SS_ERR_CUDA;
+    return ss_scan_fwd(batch, channels, state_dim, seq, dtype, x, dt_raw, A, B, C, D, z, dt_bias, reset, h0,
+                       flags & uint32_t(SS_DT_SOFTPLUS), y, h_last, ws, SS_STATIC_SCRATCH_BYTES, stream);
 }
 
 } // extern "C"

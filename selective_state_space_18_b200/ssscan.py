@@ -19,11 +19,14 @@ LIB_PATH = os.path.join(_PKG, "libssscan.so")
 
 SS_F32, SS_BF16 = 0, 1
 SS_DT_SOFTPLUS = 1
+SS_SCRATCH_ZERO = 2
+SS_STATIC_SCRATCH_BYTES = 1 << 20
 STATUS = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE", 4: "SS_ERR_ALIGN",
           5: "SS_ERR_UNSUPPORTED", 6: "SS_ERR_CUDA", 7: "SS_ERR_TIMEOUT", 8: "SS_ERR_ALIAS",
-          9: "SS_ERR_WORKSPACE"}
+          9: "SS_ERR_WORKSPACE", 10: "SS_ERR_SCRATCH_LIMIT"}
 EXPORTS = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_scan_status", "ss_state_update",
-           "ss_debug_set_wait_limit", "ss_status_string", "ss_abi_version")
+           "ss_debug_set_wait_limit", "ss_status_string", "ss_abi_version",
+           "ss_scan_fwd_static_scratch")
 ABI_MAJOR = 2
 
 _lock = threading.Lock()
@@ -53,6 +56,9 @@ def load_library(path: str = LIB_PATH):
             lib.ss_scan_fwd.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 10 + [
                 ctypes.c_uint32, _vp, _vp, _vp, ctypes.c_size_t, _vp]
             lib.ss_scan_fwd.restype = ctypes.c_int
+            lib.ss_scan_fwd_static_scratch.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 10 + [
+                ctypes.c_uint32, _vp, _vp, ctypes.POINTER(_vp), _vp]
+            lib.ss_scan_fwd_static_scratch.restype = ctypes.c_int
             lib.ss_scan_workspace_bytes.argtypes = [_i64, _i64, _i64, _i64]
             lib.ss_scan_workspace_bytes.restype = _i64
             lib.ss_scan_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_int)]
@@ -242,3 +248,70 @@ def ss_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, *, dt_s
     if st != 0:
         raise SSError("ss_state_update", st)
     return y
+
+
+_scratch_addr = {}
+
+
+def ss_scan_fwd_static_scratch(x, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h0=None, *,
+                               dt_softplus=True, y=None, h_last=None, return_last_state=True,
+                               stream=None, zero_scratch=False):
+    """Prompt scan through the library's fixed per-device scratch instead of a
+    workspace (for callers that cannot allocate device memory when they scan; the
+    library call allocates nothing -- outputs not supplied here are allocated by
+    torch before it).  Same tensors and results as ``ss_scan_fwd``; shapes that need
+    more than SS_STATIC_SCRATCH_BYTES of workspace raise SS_ERR_SCRATCH_LIMIT.
+    Calls on one device share the scratch, so they must not overlap in time."""
+    if x.dim() != 3:
+        raise ValueError("x must be [batch, channels, seq]")
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("ss_scan_fwd_static_scratch runs on CUDA tensors only")
+    bt, ch, L = x.shape
+    n = A.shape[-1]
+    code = _dtype_code(x)
+    x = _prep(x, "x", dev)
+    dt = _prep(dt, "dt", dev, x.dtype, (bt, ch, L))
+    z = _prep(z, "z", dev, x.dtype, (bt, ch, L))
+    B = _prep(B, "B", dev, x.dtype, (bt, n, L))
+    C = _prep(C, "C", dev, x.dtype, (bt, n, L))
+    A = _prep(A, "A", dev, torch.float32, (ch, n))
+    D = _prep(D, "D", dev, torch.float32, (ch,))
+    dt_bias = _prep(dt_bias, "dt_bias", dev, torch.float32, (ch,))
+    h0 = _prep(h0, "h0", dev, torch.float32, (bt, ch, n))
+    if reset is not None:
+        reset = _prep(reset, "reset", dev, None, (bt, L))
+        if reset.dtype == torch.bool:
+            reset = reset.view(torch.uint8)
+        elif reset.dtype != torch.uint8:
+            raise TypeError("reset must be bool or uint8")
+    y = torch.empty_like(x) if y is None else _out(y, "y", dev, x.dtype, (bt, ch, L))
+    if h_last is None and return_last_state:
+        h_last = torch.empty(bt, ch, n, device=dev, dtype=torch.float32)
+    elif h_last is not None:
+        h_last = _out(h_last, "h_last", dev, torch.float32, (bt, ch, n))
+    flags = (SS_DT_SOFTPLUS if dt_softplus else 0) | (SS_SCRATCH_ZERO if zero_scratch else 0)
+    addr = _vp()
+    st = load_library().ss_scan_fwd_static_scratch(
+        bt, ch, n, L, code, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(dt_bias), _ptr(reset), _ptr(h0), flags, _ptr(y), _ptr(h_last), ctypes.byref(addr),
+        _stream(stream, dev))
+    if st != 0:
+        raise SSError("ss_scan_fwd_static_scratch", st)
+    _scratch_addr[dev.index] = addr.value
+    return y, h_last
+
+
+def static_scratch_status(stream=None, device=None):
+    """Read and clear the device status word of ss_scan_fwd_static_scratch calls on
+    `device` (synchronises the stream): 'SS_OK' or 'SS_ERR_TIMEOUT'."""
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    addr = _scratch_addr.get(device.index)
+    if addr is None:
+        raise RuntimeError("no ss_scan_fwd_static_scratch call has run on this device")
+    out = ctypes.c_int(-1)
+    st = load_library().ss_scan_status(_vp(addr), _stream(stream, device), ctypes.byref(out))
+    if st != 0:
+        raise SSError("ss_scan_status", st)
+    return STATUS[out.value]
