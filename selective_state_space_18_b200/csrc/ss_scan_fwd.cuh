@@ -520,66 +520,92 @@ template <> __device__ __forceinline__ float2 bc_pair<float>(const uint4 &w, int
                    : make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
 }
 
+// Decays and increments of one group of four tokens for the lane's two states:
+// [token pair][state] as (token t, token t + 1).
+struct GroupTerms {
+    float2 a0[2], a1[2], v0[2], v1[2];
+};
+
 // One chunk of the recurrence for this lane's two states n0, n1 of channel `cl`:
 // dt and dt*x from the input stage, B and C from the raw slot (storage type), the
 // partial outputs C.h over the two states to `ys`.  Per pair of tokens: two packed
 // multiplies for the exponent arguments, four MUFU ex2, two packed multiplies for
 // the increments, four FMAs along the sequence, two packed ops for the readout.
+//
+// Software pipelined over groups of four tokens: the exponentials and increments of
+// group k + 1 are issued before the sequential FMA chain of group k, so the MUFU
+// latency of one group hides behind the chain of the previous one (with only about
+// two scan warps per sub-partition there is little other work to switch to).
 template <int N, typename T, bool HAS_RESET>
 __device__ __forceinline__ void scan_chunk(const float *stage, const unsigned char *raw, float *ys, int cl, int n0,
                                            int n1, float2 A0, float2 A1, float &hs0, float &hs1)
 {
     using S = ScanShape<N>;
     constexpr int kTok = 16 / int(sizeof(T)); // tokens per 16-byte chunk of a B/C row
+    constexpr int kGroups = S::kChunk / 4;
     const unsigned char *Bt = raw + S::template raw_b_off<T>();
     const unsigned char *Ct = raw + S::template raw_c_off<T>();
     const float *rbs = stage + S::kRBOff;
     const float *dts = stage + S::kDTOff + cl * S::kRow;
     const float *dxs = stage + S::kDXOff + cl * S::kRow;
-#pragma unroll
-    for (int c16 = 0; c16 < S::kChunk / kTok; ++c16) {
-        const uint4 wb0 = *reinterpret_cast<const uint4 *>(Bt + bc_offset<T>(n0, c16));
-        const uint4 wb1 = *reinterpret_cast<const uint4 *>(Bt + bc_offset<T>(n1, c16));
-        const uint4 wc0 = *reinterpret_cast<const uint4 *>(Ct + bc_offset<T>(n0, c16));
-        const uint4 wc1 = *reinterpret_cast<const uint4 *>(Ct + bc_offset<T>(n1, c16));
-#pragma unroll
-        for (int g4 = 0; g4 < kTok / 4; ++g4) {
-            const int t = c16 * kTok + g4 * 4;
-            const float4 d4 = *reinterpret_cast<const float4 *>(dts + t);
-            const float4 u4 = *reinterpret_cast<const float4 *>(dxs + t);
-            float4 r4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (HAS_RESET)
-                r4 = *reinterpret_cast<const float4 *>(rbs + t);
-            float2 yo[2];
-#pragma unroll
-            for (int pr = 0; pr < 2; ++pr) {
-                const int pi = g4 * 2 + pr;
-                const float2 dd = pr ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
-                const float2 uu = pr ? make_float2(u4.z, u4.w) : make_float2(u4.x, u4.y);
-                const float2 B0 = bc_pair<T>(wb0, pi), B1 = bc_pair<T>(wb1, pi);
-                const float2 C0 = bc_pair<T>(wc0, pi), C1 = bc_pair<T>(wc1, pi);
-                float2 g0, g1;
-                if (HAS_RESET) {
-                    const float2 rr = pr ? make_float2(r4.z, r4.w) : make_float2(r4.x, r4.y);
-                    g0 = __ffma2_rn(dd, A0, rr);
-                    g1 = __ffma2_rn(dd, A1, rr);
-                } else {
-                    g0 = __fmul2_rn(dd, A0);
-                    g1 = __fmul2_rn(dd, A1);
-                }
-                const float a0t = ex2(g0.x), a0u = ex2(g0.y);
-                const float a1t = ex2(g1.x), a1u = ex2(g1.y);
-                const float2 v0 = __fmul2_rn(uu, B0);
-                const float2 v1 = __fmul2_rn(uu, B1);
-                const float h0t = fmaf(a0t, hs0, v0.x);
-                hs0 = fmaf(a0u, h0t, v0.y);
-                const float h1t = fmaf(a1t, hs1, v1.x);
-                hs1 = fmaf(a1u, h1t, v1.y);
-                const float2 yy = __fmul2_rn(C0, make_float2(h0t, hs0));
-                yo[pr] = __ffma2_rn(C1, make_float2(h1t, hs1), yy);
-            }
-            *reinterpret_cast<float4 *>(ys + t) = make_float4(yo[0].x, yo[0].y, yo[1].x, yo[1].y);
+    uint4 wb0 = make_uint4(0, 0, 0, 0), wb1 = wb0, wc0 = wb0, wc1 = wb0;
+    GroupTerms gt[2];
+    // decays and increments of group k into `f`
+    auto front = [&](int k, GroupTerms &f) {
+        const int t = 4 * k;
+        if (t % kTok == 0) {
+            wb0 = *reinterpret_cast<const uint4 *>(Bt + bc_offset<T>(n0, t / kTok));
+            wb1 = *reinterpret_cast<const uint4 *>(Bt + bc_offset<T>(n1, t / kTok));
         }
+        const float4 d4 = *reinterpret_cast<const float4 *>(dts + t);
+        const float4 u4 = *reinterpret_cast<const float4 *>(dxs + t);
+        float4 r4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (HAS_RESET)
+            r4 = *reinterpret_cast<const float4 *>(rbs + t);
+#pragma unroll
+        for (int pr = 0; pr < 2; ++pr) {
+            const int pi = (t % kTok) / 2 + pr;
+            const float2 dd = pr ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
+            const float2 uu = pr ? make_float2(u4.z, u4.w) : make_float2(u4.x, u4.y);
+            float2 g0, g1;
+            if (HAS_RESET) {
+                const float2 rr = pr ? make_float2(r4.z, r4.w) : make_float2(r4.x, r4.y);
+                g0 = __ffma2_rn(dd, A0, rr);
+                g1 = __ffma2_rn(dd, A1, rr);
+            } else {
+                g0 = __fmul2_rn(dd, A0);
+                g1 = __fmul2_rn(dd, A1);
+            }
+            f.a0[pr] = make_float2(ex2(g0.x), ex2(g0.y));
+            f.a1[pr] = make_float2(ex2(g1.x), ex2(g1.y));
+            f.v0[pr] = __fmul2_rn(uu, bc_pair<T>(wb0, pi));
+            f.v1[pr] = __fmul2_rn(uu, bc_pair<T>(wb1, pi));
+        }
+    };
+    front(0, gt[0]);
+#pragma unroll
+    for (int k = 0; k < kGroups; ++k) {
+        const int t = 4 * k;
+        if (t % kTok == 0) {
+            wc0 = *reinterpret_cast<const uint4 *>(Ct + bc_offset<T>(n0, t / kTok));
+            wc1 = *reinterpret_cast<const uint4 *>(Ct + bc_offset<T>(n1, t / kTok));
+        }
+        const uint4 cc0 = wc0, cc1 = wc1;
+        if (k + 1 < kGroups)
+            front(k + 1, gt[(k + 1) & 1]);
+        const GroupTerms &f = gt[k & 1];
+        float2 yo[2];
+#pragma unroll
+        for (int pr = 0; pr < 2; ++pr) {
+            const int pi = (t % kTok) / 2 + pr;
+            const float h0t = fmaf(f.a0[pr].x, hs0, f.v0[pr].x);
+            hs0 = fmaf(f.a0[pr].y, h0t, f.v0[pr].y);
+            const float h1t = fmaf(f.a1[pr].x, hs1, f.v1[pr].x);
+            hs1 = fmaf(f.a1[pr].y, h1t, f.v1[pr].y);
+            const float2 yy = __fmul2_rn(bc_pair<T>(cc0, pi), make_float2(h0t, hs0));
+            yo[pr] = __ffma2_rn(bc_pair<T>(cc1, pi), make_float2(h1t, hs1), yy);
+        }
+        *reinterpret_cast<float4 *>(ys + t) = make_float4(yo[0].x, yo[0].y, yo[1].x, yo[1].y);
     }
 }
 
