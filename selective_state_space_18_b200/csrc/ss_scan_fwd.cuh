@@ -55,10 +55,10 @@ struct ScanArgs {
     uint32_t *status;         // status word when there is no workspace
 };
 
-// Tensor maps of the TMA path: x, dt, z as [batch * channels rows][seq] and B, C as
+// Tensor maps of the TMA path: x, dt as [batch * channels rows][seq] and B, C as
 // [batch * state_dim rows][seq], boxes of one chunk of tokens.
 struct TmaMaps {
-    CUtensorMap x, dt, z, B, C;
+    CUtensorMap x, dt, B, C;
 };
 
 // Workspace layout (bytes): the caller zeroes it once; every complete call leaves
@@ -107,8 +107,8 @@ template <int N> struct ScanShape {
     static constexpr int kTokPerLane = kTokTasks / kIoThreads;
     static constexpr int kBCTasks = 2 * N * kBlocks;              // (B/C row, 8 tokens)
     static constexpr int kBCPerLane = (kBCTasks + kIoThreads - 1) / kIoThreads;
-    // raw ring: x, dt, z tiles [channels][chunk] and B, C tiles [N][chunk] in storage
-    // type.  On aligned shapes TMA fills whole slots; the issuer warp keeps every
+    // raw ring: x, dt tiles [channels][chunk] and B, C tiles [N][chunk] in storage
+    // type (z is only needed by the epilogue, which reads it from global memory).  On aligned shapes TMA fills whole slots; the issuer warp keeps every
     // slot its readers have released loading, so up to kRawStages chunks are in
     // flight.  The scan warps read B and C straight from the slot, in storage type
     // (bf16 halves their shared-memory traffic), from tiles swizzled by TMA so the
@@ -124,9 +124,8 @@ template <int N> struct ScanShape {
     static constexpr int align1k(int b) { return (b + 1023) / 1024 * 1024; }
     template <typename T> static constexpr int raw_x_off() { return 0; }
     template <typename T> static constexpr int raw_dt_off() { return kChanPerCta * kChunk * int(sizeof(T)); }
-    template <typename T> static constexpr int raw_z_off() { return 2 * kChanPerCta * kChunk * int(sizeof(T)); }
     // B and C tiles start on 1024-byte boundaries (the swizzle pattern's period)
-    template <typename T> static constexpr int raw_b_off() { return align1k(3 * kChanPerCta * kChunk * int(sizeof(T))); }
+    template <typename T> static constexpr int raw_b_off() { return align1k(2 * kChanPerCta * kChunk * int(sizeof(T))); }
     template <typename T> static constexpr int raw_c_off() { return raw_b_off<T>() + align1k(N * kChunk * int(sizeof(T))); }
     template <typename T> static constexpr int raw_stage_bytes()
     {
@@ -245,7 +244,7 @@ template <int N, typename T, bool HAS_RESET, bool VEC>
 struct IoPrefetch {
     using S = ScanShape<N>;
     Raw8<T> bc[S::kBCPerLane];
-    Raw8<T> xr[S::kTokPerLane], dr[S::kTokPerLane], zr[S::kTokPerLane];
+    Raw8<T> xr[S::kTokPerLane], dr[S::kTokPerLane];
     float bias[S::kTokPerLane];
     int64_t bias_g = -1; // channel group whose dt_bias values `bias` holds
     uint32_t rbyte;
@@ -267,8 +266,9 @@ struct IoPrefetch {
     __device__ __forceinline__ void load(const ScanArgs &p, int lane, int64_t g, int64_t t0)
     {
         const int64_t L = p.seq;
-        const int64_t b = g / p.groups_per_batch;
-        const int64_t c0 = (g % p.groups_per_batch) * S::kChanPerCta;
+        const uint32_t gpb = uint32_t(p.groups_per_batch), b32 = uint32_t(g) / gpb;
+        const int64_t b = b32;
+        const int64_t c0 = int64_t(uint32_t(g) - b32 * gpb) * S::kChanPerCta;
         const T *Bb = static_cast<const T *>(p.B) + b * N * L;
         const T *Cb = static_cast<const T *>(p.C) + b * N * L;
 #pragma unroll
@@ -296,13 +296,9 @@ struct IoPrefetch {
             if (VEC) {
                 xr[m].load_vec_stream(xrow, t, L);
                 dr[m].load_vec_stream(drow, t, L);
-                if (p.z)
-                    zr[m].load_vec_stream(static_cast<const T *>(p.z) + row * L, t, L);
             } else {
                 xr[m].load_scalar(xrow, t, L);
                 dr[m].load_scalar(drow, t, L);
-                if (p.z)
-                    zr[m].load_scalar(static_cast<const T *>(p.z) + row * L, t, L);
             }
         }
         load_bias(p, lane, g);
@@ -310,21 +306,18 @@ struct IoPrefetch {
             rbyte = (lane < S::kChunk && t0 + lane < L) ? uint32_t(__ldg(p.reset + b * L + t0 + lane)) : 0u;
     }
 
-    // x, dt_raw, z filled from a raw TMA stage (B and C stay in the stage for the
-    // scan warps; the reset byte is loaded by the caller).
+    // x and dt_raw from a raw TMA stage (B and C stay in the stage for the scan
+    // warps; the reset byte is loaded by the caller).
     __device__ __forceinline__ void load_smem(const ScanArgs &p, int lane, int64_t g, const unsigned char *raw)
     {
         const T *rx = reinterpret_cast<const T *>(raw + S::template raw_x_off<T>());
         const T *rd = reinterpret_cast<const T *>(raw + S::template raw_dt_off<T>());
-        const T *rz = reinterpret_cast<const T *>(raw + S::template raw_z_off<T>());
 #pragma unroll
         for (int m = 0; m < S::kTokPerLane; ++m) {
             const int q = lane + S::kIoThreads * m;
             const int cl = q / S::kBlocks, tb = q % S::kBlocks;
             xr[m].load_smem(rx + cl * S::kChunk + tb * 8);
             dr[m].load_smem(rd + cl * S::kChunk + tb * 8);
-            if (p.z)
-                zr[m].load_smem(rz + cl * S::kChunk + tb * 8);
         }
         load_bias(p, lane, g);
     }
@@ -400,48 +393,60 @@ template <> __device__ __forceinline__ float2 gate2<__nv_bfloat16>(float2 v)
     return __ffma2_rn(h, t, h);
 }
 
-// D[c] of this thread's epilogue channels, reloaded only when the channel group changes.
-template <int N> struct DCache {
+// Per-thread state of the epilogue that depends only on the channel group: the rows
+// of x, z and y of this thread's channels and their D values.  Refreshed when the
+// group changes (once per work unit), so a chunk costs no index arithmetic.
+template <int N, typename T> struct EpiCache {
+    const T *x[ScanShape<N>::kTokPerLane];
+    const T *z[ScanShape<N>::kTokPerLane];
+    T *y[ScanShape<N>::kTokPerLane];
     float d[ScanShape<N>::kTokPerLane];
     int64_t g = -1;
 };
 
 // x and z are re-read from global memory (the producers' tile loads brought them into
-// L2 a few chunks earlier); the loads are issued first and their latency overlaps
-// the sum of the partial outputs.
+// L2 a few chunks earlier), issued first so their latency overlaps the partial sums.
 template <int N, typename T, bool VEC>
 __device__ __forceinline__ void epilogue_chunk(const ScanArgs &p, int lane, const float *ystage, int64_t g, int64_t t0,
-                                               DCache<N> &dcache)
+                                               EpiCache<N, T> &ec)
 {
     using S = ScanShape<N>;
     const int64_t L = p.seq;
-    const int64_t b = g / p.groups_per_batch;
-    const int64_t c0 = (g % p.groups_per_batch) * S::kChanPerCta;
+    if (ec.g != g) {
+        const int64_t b = g / p.groups_per_batch;
+        const int64_t c0 = (g - b * p.groups_per_batch) * S::kChanPerCta;
+#pragma unroll
+        for (int m = 0; m < S::kTokPerLane; ++m) {
+            const int cl = (lane + S::kIoThreads * m) / S::kBlocks;
+            const int64_t c_raw = c0 + cl;
+            const bool valid = c_raw < p.channels;
+            const int64_t c = valid ? c_raw : p.channels - 1;
+            const int64_t off = (b * p.channels + c) * L;
+            ec.x[m] = static_cast<const T *>(p.x) + off;
+            ec.z[m] = p.z ? static_cast<const T *>(p.z) + off : nullptr;
+            ec.y[m] = valid ? static_cast<T *>(p.y) + off : nullptr;
+            ec.d[m] = p.D ? __ldg(p.D + c) : 0.0f;
+        }
+        ec.g = g;
+    }
     Raw8<T> xs[S::kTokPerLane], zs[S::kTokPerLane];
 #pragma unroll
-    for (int m = 0; m < S::kTokPerLane; ++m) { // x and z first: their latency overlaps the sums
-        const int q = lane + S::kIoThreads * m;
-        const int cl = q / S::kBlocks, tb = q % S::kBlocks;
-        int64_t c = c0 + cl;
-        c = c < p.channels ? c : p.channels - 1;
-        const int64_t off = (b * p.channels + c) * L;
+    for (int m = 0; m < S::kTokPerLane; ++m) {
+        const int tb = (lane + S::kIoThreads * m) % S::kBlocks;
         if (VEC) {
-            xs[m].load_vec(static_cast<const T *>(p.x) + off, t0 + tb * 8, L);
+            xs[m].load_vec(ec.x[m], t0 + tb * 8, L);
             if (p.z)
-                zs[m].load_vec(static_cast<const T *>(p.z) + off, t0 + tb * 8, L);
+                zs[m].load_vec(ec.z[m], t0 + tb * 8, L);
         } else {
-            xs[m].load_scalar(static_cast<const T *>(p.x) + off, t0 + tb * 8, L);
+            xs[m].load_scalar(ec.x[m], t0 + tb * 8, L);
             if (p.z)
-                zs[m].load_scalar(static_cast<const T *>(p.z) + off, t0 + tb * 8, L);
+                zs[m].load_scalar(ec.z[m], t0 + tb * 8, L);
         }
-        if (dcache.g != g)
-            dcache.d[m] = p.D ? __ldg(p.D + c) : 0.0f;
     }
 #pragma unroll
     for (int m = 0; m < S::kTokPerLane; ++m) {
         const int q = lane + S::kIoThreads * m;
         const int cl = q / S::kBlocks, tb = q % S::kBlocks;
-        const int64_t c = c0 + cl;
         float2 o[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k)
@@ -455,9 +460,9 @@ __device__ __forceinline__ void epilogue_chunk(const ScanArgs &p, int lane, cons
             o[2] = __fadd2_rn(o[2], make_float2(v1.x, v1.y));
             o[3] = __fadd2_rn(o[3], make_float2(v1.z, v1.w));
         }
-        if (c >= p.channels)
+        if (!ec.y[m])
             continue;
-        const float Dc = dcache.d[m];
+        const float Dc = ec.d[m];
 #pragma unroll
         for (int k = 0; k < 4; ++k)
             o[k] = __ffma2_rn(make_float2(Dc, Dc), make_float2(xs[m].get(2 * k), xs[m].get(2 * k + 1)), o[k]);
@@ -467,10 +472,8 @@ __device__ __forceinline__ void epilogue_chunk(const ScanArgs &p, int lane, cons
                 o[k] = __fmul2_rn(o[k], gate2<T>(make_float2(zs[m].get(2 * k), zs[m].get(2 * k + 1))));
         }
         const float out[8] = {o[0].x, o[0].y, o[1].x, o[1].y, o[2].x, o[2].y, o[3].x, o[3].y};
-        T *yrow = static_cast<T *>(p.y) + (b * p.channels + c) * L;
-        store8<T, VEC>(yrow, t0 + tb * 8, L, out);
+        store8<T, VEC>(ec.y[m], t0 + tb * 8, L, out);
     }
-    dcache.g = g;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -498,12 +501,29 @@ __device__ __forceinline__ uint32_t take_unit(const ScanArgs &p, WsHeader *ws, b
     return int64_t(u) >= p.groups * p.segments ? kNoUnit : u;
 }
 
-template <int N> __device__ __forceinline__ int64_t unit_chunks(const ScanArgs &p, uint32_t u)
+// Where work unit u = segment * groups + group lies: computed once per unit (the
+// divisions are not cheap), then advanced chunk by chunk.
+struct UnitPos {
+    int64_t g, s, t_begin; // channel group, segment, first token
+    int64_t nck;           // chunks in the unit
+    int32_t xrow, brow;    // first x / dt row and first B / C row of the group
+};
+
+template <int N> __device__ __forceinline__ UnitPos unit_pos(const ScanArgs &p, uint32_t u)
 {
-    const int64_t s = int64_t(u) / p.groups;
-    const int64_t rest = p.seq - s * p.seg_len;
+    UnitPos up;
+    // units, groups and rows all fit in 32 bits (checked on the host)
+    const uint32_t groups = uint32_t(p.groups), gpb = uint32_t(p.groups_per_batch);
+    const uint32_t g = u % groups, s = u / groups, b = g / gpb;
+    up.g = g;
+    up.s = s;
+    up.t_begin = int64_t(s) * p.seg_len;
+    const int64_t rest = p.seq - up.t_begin;
     const int64_t len = rest < p.seg_len ? rest : p.seg_len;
-    return (len + ScanShape<N>::kChunk - 1) / ScanShape<N>::kChunk;
+    up.nck = (len + ScanShape<N>::kChunk - 1) / ScanShape<N>::kChunk;
+    up.xrow = int32_t(int64_t(b) * p.channels + int64_t(g - b * gpb) * ScanShape<N>::kChanPerCta);
+    up.brow = int32_t(b * N);
+    return up;
 }
 
 // Token pair `pi` of a 16-byte chunk of a B or C row, widened to fp32: bf16 rows hold
@@ -623,14 +643,15 @@ __device__ __forceinline__ bool issuer_warp(const ScanArgs &p, const TmaMaps &ma
     if constexpr (VEC) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.x)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.dt)) : "memory");
-        if (p.z)
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.z)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.B)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.C)) : "memory");
     }
-    const uint32_t tx_bytes = uint32_t(((p.z ? 3 : 2) * S::kChanPerCta + 2 * N) * S::kChunk * sizeof(T));
+    constexpr uint32_t tx_bytes = uint32_t((2 * S::kChanPerCta + 2 * N) * S::kChunk * sizeof(T));
     uint32_t u = take_unit(p, cx.ws, true);
-    int64_t k = 0, nck = u != kNoUnit ? unit_chunks<N>(p, u) : 0;
+    UnitPos up;
+    if (u != kNoUnit)
+        up = unit_pos<N>(p, u);
+    int64_t k = 0;
     for (uint32_t j = 0;; ++j) {
         const int r = int(j % RS);
         if (j >= uint32_t(RS) && !mbar_wait(cx.raw_empty + r, ((j / RS) & 1u) ^ 1u, cx.status)) {
@@ -645,31 +666,28 @@ __device__ __forceinline__ bool issuer_warp(const ScanArgs &p, const TmaMaps &ma
             mbar_arrive(cx.raw_full + r);
             return true;
         }
-        const int64_t g = int64_t(u) % p.groups, s = int64_t(u) / p.groups;
-        const int64_t t0 = s * p.seg_len + k * S::kChunk;
-        const int32_t fl = (k == 0 ? kFirst : 0) | (k + 1 == nck ? kLast : 0);
+        const int64_t t0 = up.t_begin + k * S::kChunk;
+        const int32_t fl = (k == 0 ? kFirst : 0) | (k + 1 == up.nck ? kLast : 0);
         m[0] = t0;
-        m[1] = g;
-        m[2] = (int64_t(fl) << 32) | int64_t(s);
+        m[1] = up.g;
+        m[2] = (int64_t(fl) << 32) | int64_t(up.s);
         if constexpr (VEC) {
-            const int64_t b = g / p.groups_per_batch, c0 = (g % p.groups_per_batch) * S::kChanPerCta;
             unsigned char *dst = cx.raw_base + r * S::template raw_stage_bytes<T>();
             uint64_t *bar = cx.raw_full + r;
             mbar_arrive_expect_tx(bar, tx_bytes);
-            const int32_t tt = int32_t(t0), xrow = int32_t(b * p.channels + c0), brow = int32_t(b * N);
+            const int32_t tt = int32_t(t0), xrow = up.xrow, brow = up.brow;
             tma_load_2d(dst + S::template raw_x_off<T>(), &maps.x, tt, xrow, bar);
             tma_load_2d(dst + S::template raw_dt_off<T>(), &maps.dt, tt, xrow, bar);
-            if (p.z)
-                tma_load_2d(dst + S::template raw_z_off<T>(), &maps.z, tt, xrow, bar);
             tma_load_2d(dst + S::template raw_b_off<T>(), &maps.B, tt, brow, bar);
             tma_load_2d(dst + S::template raw_c_off<T>(), &maps.C, tt, brow, bar);
         } else {
             mbar_arrive(cx.raw_full + r);
         }
-        if (++k == nck) {
+        if (++k == up.nck) {
             u = take_unit(p, cx.ws, false);
             k = 0;
-            nck = u != kNoUnit ? unit_chunks<N>(p, u) : 0;
+            if (u != kNoUnit)
+                up = unit_pos<N>(p, u);
         }
     }
 }
@@ -684,6 +702,8 @@ __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, in
     constexpr int kRawBytes = S::template raw_stage_bytes<T>();
     const int tl = pi * 32 + lane; // producer thread index
     IoPrefetch<N, T, HAS_RESET, VEC> pf;
+    int64_t reset_g = -1;
+    const uint8_t *reset_row = p.reset;
     for (uint32_t i = 0;; ++i) {
         const int r = int(i % RS);
         if (!mbar_wait(cx.raw_full + r, (i / RS) & 1u, cx.status))
@@ -698,8 +718,11 @@ __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, in
             else
                 pf.load(p, tl, g, t0);
             if (HAS_RESET) {
-                const int64_t b = g / p.groups_per_batch;
-                pf.rbyte = (tl < S::kChunk && t0 + tl < p.seq) ? uint32_t(__ldg(p.reset + b * p.seq + t0 + tl)) : 0u;
+                if (g != reset_g) { // the reset row of the batch entry, once per unit
+                    reset_g = g;
+                    reset_row = p.reset + int64_t(uint32_t(g) / uint32_t(p.groups_per_batch)) * p.seq;
+                }
+                pf.rbyte = (tl < S::kChunk && t0 + tl < p.seq) ? uint32_t(__ldg(reset_row + t0 + tl)) : 0u;
             }
         }
         mbar_arrive(cx.raw_empty + r); // this thread's reads of slot r are done
@@ -724,7 +747,7 @@ __device__ __forceinline__ bool epilogue_role(const ScanArgs &p, const float *y_
                                               uint64_t *y_empty, uint32_t *status, int tl)
 {
     using S = ScanShape<N>;
-    DCache<N> dcache;
+    EpiCache<N, T> ec;
     for (uint32_t j = 0;; ++j) {
         const int ys = int(j % S::kYStages);
         if (!mbar_wait(y_full + ys, (j / S::kYStages) & 1u, status))
@@ -733,7 +756,7 @@ __device__ __forceinline__ bool epilogue_role(const ScanArgs &p, const float *y_
         const ChunkMeta meta = read_meta(ystage);
         if (meta.flags & kEnd)
             return true;
-        epilogue_chunk<N, T, VEC>(p, tl, ystage, meta.g, meta.t0, dcache);
+        epilogue_chunk<N, T, VEC>(p, tl, ystage, meta.g, meta.t0, ec);
         mbar_arrive(y_empty + ys);
     }
 }
