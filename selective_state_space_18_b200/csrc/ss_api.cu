@@ -223,6 +223,36 @@ int dispatch_scan_n(ss::ScanArgs a, ss_dtype_t dtype, bool vec, size_t ws_bytes,
 template <int N, typename T, bool V>
 int launch_update(ss::UpdateArgs a, cudaStream_t stream)
 {
+    if constexpr (V) {
+        // aligned state: persistent CTAs streaming the state through shared memory
+        constexpr int kChanPerTile = ss::kDecQuarters / (N / 4);
+        auto kernel = ss::ss_state_update_stream_kernel<N, T>;
+        static std::atomic<uint64_t> smem_done{0};
+        static std::atomic<int> occ_cache[64];
+        int st = ensure_smem(kernel, ss::kDecSmem, smem_done);
+        if (st != SS_OK)
+            return st;
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || device_sm_count(&sms) != SS_OK)
+            return SS_ERR_CUDA;
+        int occ = dev < 64 ? occ_cache[dev].load(std::memory_order_acquire) : 0;
+        if (!occ) {
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, ss::kDecThreads, ss::kDecSmem) !=
+                cudaSuccess)
+                return SS_ERR_CUDA;
+            occ = occ > 0 ? occ : 1;
+            if (dev < 64)
+                occ_cache[dev].store(occ, std::memory_order_release);
+        }
+        const int64_t tiles = a.batch * ((a.channels + kChanPerTile - 1) / kChanPerTile);
+        const int64_t resident = int64_t(sms) * occ;
+        const int64_t grid = tiles < resident ? tiles : resident;
+        uint32_t *status = nullptr;
+        if (status_word_address(&status) != SS_OK)
+            return SS_ERR_CUDA;
+        kernel<<<unsigned(grid), ss::kDecThreads, ss::kDecSmem, stream>>>(a, tiles, status);
+        return launch_status();
+    }
     const int64_t per_block = int64_t(ss::kUpdateThreads) * ss::kUpdateItems; // row quarters
     const int64_t quarters = a.channels * (N / 4);
     a.blocks_per_row = int((quarters + per_block - 1) / per_block);
