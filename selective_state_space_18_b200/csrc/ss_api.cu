@@ -225,11 +225,11 @@ int launch_update(ss::UpdateArgs a, cudaStream_t stream)
 {
     if constexpr (V) {
         // aligned state: persistent CTAs streaming the state through shared memory
-        constexpr int kChanPerTile = ss::kDecQuarters / (N / 4);
+        using D = ss::DecShape<N, T>;
         auto kernel = ss::ss_state_update_stream_kernel<N, T>;
         static std::atomic<uint64_t> smem_done{0};
         static std::atomic<int> occ_cache[64];
-        int st = ensure_smem(kernel, ss::kDecSmem, smem_done);
+        int st = ensure_smem(kernel, D::kSmem, smem_done);
         if (st != SS_OK)
             return st;
         int dev = 0, sms = 0;
@@ -237,20 +237,34 @@ int launch_update(ss::UpdateArgs a, cudaStream_t stream)
             return SS_ERR_CUDA;
         int occ = dev < 64 ? occ_cache[dev].load(std::memory_order_acquire) : 0;
         if (!occ) {
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, ss::kDecThreads, ss::kDecSmem) !=
-                cudaSuccess)
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, ss::kDecThreads, D::kSmem) != cudaSuccess)
                 return SS_ERR_CUDA;
             occ = occ > 0 ? occ : 1;
             if (dev < 64)
                 occ_cache[dev].store(occ, std::memory_order_release);
         }
-        const int64_t tiles = a.batch * ((a.channels + kChanPerTile - 1) / kChanPerTile);
+        ss::DecArgs da{};
+        da.u = a;
+        da.ncb = (a.channels + D::kChanPerTile - 1) / D::kChanPerTile;
+        const int64_t tiles = a.batch * da.ncb;
         const int64_t resident = int64_t(sms) * occ;
-        const int64_t grid = tiles < resident ? tiles : resident;
+        int64_t grid = tiles < resident ? tiles : resident;
+        // with more tiles than CTAs, a grid that is a multiple of the channel blocks
+        // lets every CTA keep one channel block (A, dt_bias, D loaded once)
+        if (tiles > resident && resident >= da.ncb) {
+            grid = resident / da.ncb * da.ncb;
+            da.fixed_cb = 1;
+        }
+        // x, dt_raw, z rows ride along with the state when every tile's rows are
+        // 16-byte aligned
+        const size_t es = sizeof(T);
+        da.bulk_xdz = aligned(a.x, 16) && aligned(a.dt, 16) && (!a.z || aligned(a.z, 16)) &&
+                      (size_t(a.channels) * es) % 16 == 0;
+        da.bulk_bc = aligned(a.B, 16) && aligned(a.C, 16) && (N * es) % 16 == 0;
         uint32_t *status = nullptr;
         if (status_word_address(&status) != SS_OK)
             return SS_ERR_CUDA;
-        kernel<<<unsigned(grid), ss::kDecThreads, ss::kDecSmem, stream>>>(a, tiles, status);
+        kernel<<<unsigned(grid), ss::kDecThreads, D::kSmem, stream>>>(da, status);
         return launch_status();
     }
     const int64_t per_block = int64_t(ss::kUpdateThreads) * ss::kUpdateItems; // row quarters

@@ -60,6 +60,7 @@ template <typename T> struct Elem;
 template <> struct Elem<float> {
     static constexpr int kBytes = 4;
     static __device__ __forceinline__ float load(const float *p) { return __ldg(p); }
+    static __device__ __forceinline__ float load_smem(const float *p) { return *p; }
     static __device__ __forceinline__ void store(float *p, float v) { *p = v; }
 };
 
@@ -68,6 +69,10 @@ template <> struct Elem<__nv_bfloat16> {
     static __device__ __forceinline__ float load(const __nv_bfloat16 *p)
     {
         return __bfloat162float(__ldg(p));
+    }
+    static __device__ __forceinline__ float load_smem(const __nv_bfloat16 *p)
+    {
+        return __uint_as_float(uint32_t(*reinterpret_cast<const unsigned short *>(p)) << 16);
     }
     static __device__ __forceinline__ void store(__nv_bfloat16 *p, float v)
     {

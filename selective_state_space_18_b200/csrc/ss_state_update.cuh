@@ -35,6 +35,7 @@ constexpr int kUpdateItems = 8; // row quarters per thread: 128 B of state in fl
 
 template <typename T> struct Vec4;
 template <> struct Vec4<float> {
+    static __device__ __forceinline__ float4 load_smem(const float *p) { return *reinterpret_cast<const float4 *>(p); }
     static __device__ __forceinline__ float4 load(const float *p, bool vec)
     {
         if (vec)
@@ -43,6 +44,12 @@ template <> struct Vec4<float> {
     }
 };
 template <> struct Vec4<__nv_bfloat16> {
+    static __device__ __forceinline__ float4 load_smem(const __nv_bfloat16 *p)
+    {
+        const uint2 w = *reinterpret_cast<const uint2 *>(p);
+        return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                           __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+    }
     static __device__ __forceinline__ float4 load(const __nv_bfloat16 *p, bool vec)
     {
         if (vec) {
@@ -140,17 +147,30 @@ ss_state_update_kernel(const UpdateArgs p)
 // The state is the only large operand, and the kernel above keeps at most its
 // registers' worth of it in flight (about 64 KB per SM at its occupancy), below what
 // HBM needs to run at full rate.  Here persistent CTAs stream the state through a
-// ring of shared-memory stages filled by bulk asynchronous copies (one per tile, no
-// multicast), so kDecStages tiles of every CTA are always on their way regardless of
-// the registers the arithmetic needs.  A tile is 1024 row quarters (16 KB of state)
-// of one batch row; thread t owns quarters t, t + 256, t + 512, t + 768 of it.  The
-// updated state goes straight back to global memory with streaming stores.
+// ring of shared-memory stages filled by bulk asynchronous copies (no multicast), so
+// kDecStages tiles of every CTA are always on their way regardless of the registers
+// the arithmetic needs.  A tile is 1024 row quarters (16 KB of state) of one batch
+// row, plus -- when their rows are 16-byte aligned -- the tile's x, dt_raw and z and
+// the row's B and C in the same stage, so a tile's arithmetic waits on nothing but
+// its stage.  Thread t owns quarters t, t + 256, t + 512, t + 768 of a tile.
+// When the grid is a multiple of the channel blocks per row, every CTA keeps one
+// channel block and walks batch rows, so A, dt_bias and D are loaded once per CTA.
+// The updated state goes straight back to global memory with streaming stores.
 constexpr int kDecThreads = 256;
 constexpr int kDecItems = 4;                              // quarters per thread per tile
 constexpr int kDecQuarters = kDecThreads * kDecItems;     // 1024 quarters = 16 KB
-constexpr int kDecStages = 5;
+constexpr int kDecStages = 4;
 constexpr int kDecTileBytes = kDecQuarters * 16;
-constexpr size_t kDecSmem = size_t(kDecStages) * kDecTileBytes + 8 * kDecStages;
+
+template <int N, typename T> struct DecShape {
+    static constexpr int kQ = N / 4;                           // quarters per (b, c) row
+    static constexpr int kChanPerTile = kDecQuarters / kQ;
+    static constexpr int kVecBytes = kChanPerTile * int(sizeof(T)); // x, dt or z of a tile
+    static constexpr int kBCOff = kDecTileBytes + 3 * kVecBytes;  // B then C of the row
+    static constexpr int kStageBytes = kBCOff + 2 * 64;
+    static constexpr size_t kSmem = size_t(kDecStages) * kStageBytes + 8 * kDecStages;
+    static_assert(kStageBytes % 16 == 0, "16-byte aligned stages");
+};
 
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
 {
@@ -160,29 +180,64 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
                  : "memory");
 }
 
+struct DecArgs {
+    UpdateArgs u;
+    int64_t ncb;     // channel blocks per batch row
+    int fixed_cb;    // grid is a multiple of ncb: CTA i keeps channel block i % ncb
+    int bulk_xdz;    // x, dt_raw (and z) rows are copied with the state
+    int bulk_bc;     // B and C rows are copied with the state
+};
+
 template <int N, typename T>
 __global__ void __launch_bounds__(kDecThreads)
-ss_state_update_stream_kernel(const UpdateArgs p, int64_t ntiles, uint32_t *status)
+ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
 {
-    constexpr int Q = N / 4;                  // quarters per (b, c) row
-    constexpr int kChanPerTile = kDecQuarters / Q;
+    using D = DecShape<N, T>;
+    constexpr int Q = D::kQ;
+    const UpdateArgs &p = da.u;
     extern __shared__ __align__(128) unsigned char dsm[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(dsm + size_t(kDecStages) * kDecTileBytes);
-    const int tid = threadIdx.x;
-    const int64_t tiles_per_row = (p.channels + kChanPerTile - 1) / kChanPerTile;
+    uint64_t *full = reinterpret_cast<uint64_t *>(dsm + size_t(kDecStages) * D::kStageBytes);
+    const int tid = threadIdx.x, lane_q = tid & (Q - 1);
 
-    // bytes of tile `tile` and where its state starts
-    auto tile_span = [&](int64_t tile, int64_t &b, int64_t &c0) -> uint32_t {
-        b = tile / tiles_per_row;
-        c0 = (tile - b * tiles_per_row) * kChanPerTile;
-        const int64_t nch = p.channels - c0 < kChanPerTile ? p.channels - c0 : kChanPerTile;
-        return uint32_t(nch * N * 4);
+    // the k-th tile of this CTA: batch row b, channel block cb (false past the end)
+    auto tile_of = [&](int64_t k, int64_t &b, int64_t &cb) -> bool {
+        if (da.fixed_cb) {
+            cb = blockIdx.x % da.ncb;
+            b = blockIdx.x / da.ncb + k * (gridDim.x / da.ncb);
+        } else {
+            const int64_t t = blockIdx.x + k * gridDim.x;
+            b = t / da.ncb;
+            cb = t - b * da.ncb;
+        }
+        return b < p.batch;
     };
-    auto issue = [&](int64_t tile, int stage) {
-        int64_t b, c0;
-        const uint32_t bytes = tile_span(tile, b, c0);
-        mbar_arrive_expect_tx(full + stage, bytes);
-        bulk_load(dsm + size_t(stage) * kDecTileBytes, p.state + (b * p.channels + c0) * N, bytes, full + stage);
+    auto nchan = [&](int64_t cb) -> int64_t {
+        const int64_t rest = p.channels - cb * D::kChanPerTile;
+        return rest < D::kChanPerTile ? rest : D::kChanPerTile;
+    };
+    auto issue = [&](int64_t k, int stage) -> bool {
+        int64_t b, cb;
+        if (!tile_of(k, b, cb))
+            return false;
+        const int64_t nch = nchan(cb), row0 = b * p.channels + cb * D::kChanPerTile;
+        const uint32_t sbytes = uint32_t(nch * N * 4), vbytes = uint32_t(nch * int64_t(sizeof(T)));
+        const int nvec = da.bulk_xdz ? (p.z ? 3 : 2) : 0;
+        const uint32_t bcbytes = da.bulk_bc ? uint32_t(2 * N * sizeof(T)) : 0u;
+        unsigned char *dst = dsm + size_t(stage) * D::kStageBytes;
+        mbar_arrive_expect_tx(full + stage, sbytes + nvec * vbytes + bcbytes);
+        bulk_load(dst, p.state + row0 * N, sbytes, full + stage);
+        if (nvec) {
+            bulk_load(dst + kDecTileBytes, static_cast<const T *>(p.x) + row0, vbytes, full + stage);
+            bulk_load(dst + kDecTileBytes + D::kVecBytes, static_cast<const T *>(p.dt) + row0, vbytes, full + stage);
+            if (p.z)
+                bulk_load(dst + kDecTileBytes + 2 * D::kVecBytes, static_cast<const T *>(p.z) + row0, vbytes,
+                          full + stage);
+        }
+        if (bcbytes) {
+            bulk_load(dst + D::kBCOff, static_cast<const T *>(p.B) + b * N, bcbytes / 2, full + stage);
+            bulk_load(dst + D::kBCOff + 64, static_cast<const T *>(p.C) + b * N, bcbytes / 2, full + stage);
+        }
+        return true;
     };
 
     if (tid == 0) {
@@ -192,70 +247,111 @@ ss_state_update_stream_kernel(const UpdateArgs p, int64_t ntiles, uint32_t *stat
     }
     __syncthreads();
     int64_t issued = 0; // tiles of this CTA handed to the copy engine (thread 0's count)
-    if (tid == 0) {
-        for (int s = 0; s < kDecStages - 1; ++s) {
-            const int64_t tile = blockIdx.x + int64_t(s) * gridDim.x;
-            if (tile < ntiles) {
-                issue(tile, s);
-                ++issued;
-            }
-        }
-    }
+    if (tid == 0)
+        for (int s = 0; s < kDecStages - 1; ++s)
+            issued += issue(s, s) ? 1 : 0;
+
+    float4 av[kDecItems];
+    float bias[kDecItems], dco[kDecItems];
+    int64_t cached_cb = -1;
     bool ok = true;
-    int64_t it = 0;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-        // every thread is done with the stage of tile it - 1: refill it with tile
-        // it + kDecStages - 1
+    int64_t k = 0;
+    for (;; ++k) {
+        int64_t b, cb;
+        if (!tile_of(k, b, cb))
+            break;
+        // every thread is done with the stage of tile k - 1: refill it
         __syncthreads();
-        if (tid == 0) {
-            const int64_t nt = tile + int64_t(kDecStages - 1) * gridDim.x;
-            if (nt < ntiles) {
-                issue(nt, int((it + kDecStages - 1) % kDecStages));
-                ++issued;
+        if (tid == 0)
+            issued += issue(k + kDecStages - 1, int((k + kDecStages - 1) % kDecStages)) ? 1 : 0;
+        const int64_t c0 = cb * D::kChanPerTile;
+        const int nq = int(nchan(cb) * Q); // valid quarters in this tile
+        if (cb != cached_cb) {
+            cached_cb = cb;
+#pragma unroll
+            for (int it = 0; it < kDecItems; ++it) {
+                const int q = tid + it * kDecThreads;
+                const int64_t c = c0 + (q < nq ? q : nq - 1) / Q;
+                av[it] = __ldg(reinterpret_cast<const float4 *>(p.A + c * N) + lane_q);
+                bias[it] = p.dt_bias ? __ldg(p.dt_bias + c) : 0.0f;
+                dco[it] = p.D ? __ldg(p.D + c) : 0.0f;
             }
         }
-        int64_t b, c0;
-        const uint32_t bytes = tile_span(tile, b, c0);
-        const int nq = int(bytes / 16); // valid quarters in this tile
         // the small operands first: their latency overlaps the wait for the state
-        const int lane_q = tid & (Q - 1);
-        const float4 bv = Vec4<T>::load(static_cast<const T *>(p.B) + b * N + 4 * lane_q, false);
-        const float4 cv = Vec4<T>::load(static_cast<const T *>(p.C) + b * N + 4 * lane_q, false);
-        float xs[kDecItems], ds[kDecItems], zs[kDecItems], bias[kDecItems], dd[kDecItems];
-        float4 av[kDecItems];
-#pragma unroll
-        for (int k = 0; k < kDecItems; ++k) {
-            const int q = tid + k * kDecThreads;
-            const int qq = q < nq ? q : nq - 1;
-            const int64_t c = c0 + qq / Q;
-            const int64_t row = b * p.channels + c;
-            xs[k] = Elem<T>::load(static_cast<const T *>(p.x) + row);
-            ds[k] = Elem<T>::load(static_cast<const T *>(p.dt) + row);
-            zs[k] = p.z ? Elem<T>::load(static_cast<const T *>(p.z) + row) : 0.0f;
-            bias[k] = p.dt_bias ? __ldg(p.dt_bias + c) : 0.0f;
-            dd[k] = p.D ? __ldg(p.D + c) : 0.0f;
-            av[k] = __ldg(reinterpret_cast<const float4 *>(p.A + c * N) + lane_q);
+        float4 bv = make_float4(0.f, 0.f, 0.f, 0.f), cv = bv;
+        if (!da.bulk_bc) {
+            bv = Vec4<T>::load(static_cast<const T *>(p.B) + b * N + 4 * lane_q, true);
+            cv = Vec4<T>::load(static_cast<const T *>(p.C) + b * N + 4 * lane_q, true);
         }
-        const int stage = int(it % kDecStages);
-        if (!mbar_wait(full + stage, uint32_t(it / kDecStages) & 1u, status)) {
+        float xs[kDecItems], ds[kDecItems], zs[kDecItems];
+        if (!da.bulk_xdz) {
+#pragma unroll
+            for (int it = 0; it < kDecItems; ++it) {
+                const int q = tid + it * kDecThreads;
+                const int64_t row = b * p.channels + c0 + (q < nq ? q : nq - 1) / Q;
+                xs[it] = Elem<T>::load(static_cast<const T *>(p.x) + row);
+                ds[it] = Elem<T>::load(static_cast<const T *>(p.dt) + row);
+                zs[it] = p.z ? Elem<T>::load(static_cast<const T *>(p.z) + row) : 0.0f;
+            }
+        }
+        const int stage = int(k % kDecStages);
+        if (!mbar_wait(full + stage, uint32_t(k / kDecStages) & 1u, status)) {
             ok = false;
             break;
         }
-        const float4 *sv = reinterpret_cast<const float4 *>(dsm + size_t(stage) * kDecTileBytes);
+        const unsigned char *sb = dsm + size_t(stage) * D::kStageBytes;
+        const float4 *sv = reinterpret_cast<const float4 *>(sb);
+        if (da.bulk_bc) {
+            bv = Vec4<T>::load_smem(reinterpret_cast<const T *>(sb + D::kBCOff) + 4 * lane_q);
+            cv = Vec4<T>::load_smem(reinterpret_cast<const T *>(sb + D::kBCOff + 64) + 4 * lane_q);
+        }
+        if (da.bulk_xdz) {
+            const T *sx = reinterpret_cast<const T *>(sb + kDecTileBytes);
+            const T *sd = reinterpret_cast<const T *>(sb + kDecTileBytes + D::kVecBytes);
+            const T *sz = reinterpret_cast<const T *>(sb + kDecTileBytes + 2 * D::kVecBytes);
 #pragma unroll
-        for (int k = 0; k < kDecItems; ++k) {
-            const int q = tid + k * kDecThreads;
+            for (int it = 0; it < kDecItems; ++it) {
+                const int q = tid + it * kDecThreads;
+                const int cl = (q < nq ? q : nq - 1) / Q;
+                xs[it] = Elem<T>::load_smem(sx + cl);
+                ds[it] = Elem<T>::load_smem(sd + cl);
+                zs[it] = p.z ? Elem<T>::load_smem(sz + cl) : 0.0f;
+            }
+        }
+        // dt of the four items: the Q lanes of a row share them, so lane j computes
+        // the softplus of the items it with it % Q == j and the row's lanes exchange
+        float dsp[kDecItems];
+        if (p.softplus) {
+            float mine[kDecItems / Q];
+#pragma unroll
+            for (int u = 0; u < kDecItems / Q; ++u) {
+                float r = ds[u * Q] + bias[u * Q];
+#pragma unroll
+                for (int j = 1; j < Q; ++j)
+                    r = lane_q == j ? ds[u * Q + j] + bias[u * Q + j] : r;
+                mine[u] = softplus(r);
+            }
+            const int base = (tid & 31) & ~(Q - 1);
+#pragma unroll
+            for (int it = 0; it < kDecItems; ++it)
+                dsp[it] = Q == 1 ? mine[it] : __shfl_sync(0xffffffffu, mine[it / Q], base | (it % Q));
+        } else {
+#pragma unroll
+            for (int it = 0; it < kDecItems; ++it)
+                dsp[it] = ds[it] + bias[it];
+        }
+#pragma unroll
+        for (int it = 0; it < kDecItems; ++it) {
+            const int q = tid + it * kDecThreads;
             const bool valid = q < nq;
-            const int qq = valid ? q : nq - 1;
-            float4 st = sv[qq];
-            const float r = ds[k] + bias[k];
-            const float d = p.softplus ? softplus(r) : r;
-            const float dx = d * xs[k];
+            float4 st = sv[valid ? q : nq - 1];
+            const float d = dsp[it];
+            const float dx = d * xs[it];
             const float dl = d * kLog2e;
-            st.x = fmaf(ex2(dl * av[k].x), st.x, dx * bv.x);
-            st.y = fmaf(ex2(dl * av[k].y), st.y, dx * bv.y);
-            st.z = fmaf(ex2(dl * av[k].z), st.z, dx * bv.z);
-            st.w = fmaf(ex2(dl * av[k].w), st.w, dx * bv.w);
+            st.x = fmaf(ex2(dl * av[it].x), st.x, dx * bv.x);
+            st.y = fmaf(ex2(dl * av[it].y), st.y, dx * bv.y);
+            st.z = fmaf(ex2(dl * av[it].z), st.z, dx * bv.z);
+            st.w = fmaf(ex2(dl * av[it].w), st.w, dx * bv.w);
             float yp = cv.x * st.x;
             yp = fmaf(cv.y, st.y, yp);
             yp = fmaf(cv.z, st.z, yp);
@@ -264,13 +360,12 @@ ss_state_update_stream_kernel(const UpdateArgs p, int64_t ntiles, uint32_t *stat
             for (int off = Q / 2; off >= 1; off >>= 1)
                 yp += __shfl_xor_sync(0xffffffffu, yp, off);
             if (valid) {
-                const int64_t c = c0 + q / Q;
-                const int64_t row = b * p.channels + c;
+                const int64_t row = b * p.channels + c0 + q / Q;
                 __stcs(reinterpret_cast<float4 *>(p.state + row * N) + lane_q, st);
                 if (lane_q == 0) {
-                    float v = fmaf(dd[k], xs[k], yp);
+                    float v = fmaf(dco[it], xs[it], yp);
                     if (p.z)
-                        v *= silu(zs[k]);
+                        v *= silu(zs[it]);
                     Elem<T>::store(static_cast<T *>(p.y) + row, v);
                 }
             }
@@ -278,8 +373,8 @@ ss_state_update_stream_kernel(const UpdateArgs p, int64_t ntiles, uint32_t *stat
     }
     if (!ok && tid == 0) {
         // gave up (SS_ERR_TIMEOUT recorded): let the copies still in flight land
-        for (int64_t k = it; k < issued; ++k)
-            mbar_wait(full + int(k % kDecStages), uint32_t(k / kDecStages) & 1u, nullptr);
+        for (int64_t j = k; j < issued; ++j)
+            mbar_wait(full + int(j % kDecStages), uint32_t(j / kDecStages) & 1u, nullptr);
     }
 }
 

@@ -143,6 +143,35 @@ def test_decode_shapes(orc, n, dtype, extras):
     assert_close(st, ref["state"], 1e-4, "state")
 
 
+@pytest.mark.parametrize("batch,ch,n,dtype", [
+    (600, 1000, 16, "bf16"),   # several tiles per CTA, one channel block per CTA, partial tiles
+    (300, 1001, 8, "f32"),     # x/dt/z rows not 16-byte aligned: loaded per channel
+    (97, 3000, 4, "bf16"),     # 4 states: 1024 channels per tile
+])
+def test_decode_streaming_tiles(orc, batch, ch, n, dtype):
+    inp = make_update_inputs(batch, ch, n, dtype, seed=310 + n)
+    y, st = gpu_update(inp)
+    ref = orc.update(**inp)
+    assert_close(y, ref["y"], TOL[inp["x"].dtype], "y")
+    assert_close(st, ref["state"], 1e-4, "state")
+
+
+def test_decode_unaligned_state(orc):
+    """A state that is not 16-byte aligned takes the per-thread kernel; same results."""
+    from selective_state_space_18_b200 import ssscan
+    inp = make_update_inputs(5, 70, 16, "bf16", seed=320)
+    d = {k: (None if v is None else v.cuda()) for k, v in inp.items()}
+    buf = torch.empty(d["state"].numel() + 1, dtype=torch.float32, device="cuda")
+    state = buf[1:].view(d["state"].shape)
+    state.copy_(d["state"])
+    assert state.data_ptr() % 16 != 0
+    y = ssscan.ss_state_update(state, d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["z"], d["dt_bias"])
+    torch.cuda.synchronize()
+    ref = orc.update(**inp)
+    assert_close(y.cpu(), ref["y"], TOL[torch.bfloat16], "y")
+    assert_close(state.cpu(), ref["state"], 1e-4, "state")
+
+
 # ---- properties the pages fix, on the GPU path ---------------------------------------------
 
 def test_decode_equals_last_scan_step():
