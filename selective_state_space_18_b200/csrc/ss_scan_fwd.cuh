@@ -735,6 +735,15 @@ __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, in
             produce_chunk<N, T, HAS_RESET, VEC>(p, tl, pf, stage, cx.raw_base + r * kRawBytes, t0);
         if (tl == 0)
             write_meta(stage, t0, g, s, fl);
+        // The chunk's output stage must be free as well (the epilogue is done with
+        // chunk i - kYStages).  Waiting for it here, and for the raw slot above, makes
+        // in_full the one barrier the scan warps wait on per chunk: a satisfied wait
+        // still costs on the order of a hundred cycles, on the critical warps.
+        const int ys = int(i % S::kYStages);
+        if (!mbar_wait(cx.y_empty + ys, ((i / S::kYStages) & 1u) ^ 1u, cx.status))
+            return false;
+        if (tl == 0) // the epilogue warps learn the chunk from its output stage
+            write_meta(cx.y_base + ys * S::kYStage, t0, g, s, fl);
         mbar_arrive(cx.in_full + st);
         if (end)
             return true;
@@ -844,13 +853,11 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
             const int st = int(j % S::kStages);
             if (!mbar_wait(in_full + st, (j / S::kStages) & 1u, status))
                 return;
+            // (in_full also means: the chunk's raw slot has landed and its output
+            // stage is free -- the producers waited for both before arriving)
             const float *stage = in_base + st * S::kInStage;
             const ChunkMeta meta = read_meta(stage);
             const uint32_t ysi = j % S::kYStages;
-            if (!mbar_wait(y_empty + ysi, ((j / S::kYStages) & 1u) ^ 1u, status))
-                return;
-            if (warp == 0 && lane == 0) // the epilogue warps learn the chunk from its output stage
-                write_meta(y_base + ysi * S::kYStage, meta.t0, meta.g, meta.s, meta.flags);
             if (meta.flags & kEnd) {
                 mbar_arrive(y_full + ysi); // lets the epilogue warp see the end marker
                 break;
@@ -878,11 +885,7 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
                     hs1 = h.y;
                 }
             }
-            // B and C of this chunk are in its raw slot (landed: the producers waited
-            // for it before releasing the input stage; the wait here is immediate)
             const int rs = int(j % S::kRawStages);
-            if (!mbar_wait(bars + S::kBarRawFull + rs, (j / S::kRawStages) & 1u, status))
-                return;
             scan_chunk<N, T, HAS_RESET>(stage, smem_bytes + rs * S::template raw_stage_bytes<T>(),
                                         y_base + ysi * S::kYStage + S::kYPOff + cl * S::kYChan + sub * S::kRow,
                                         cl, n0, n1, A0, A1, hs0, hs1);

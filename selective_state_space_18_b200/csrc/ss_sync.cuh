@@ -79,19 +79,17 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// One test of the phase.  If it has not completed, the thread is suspended in
-// hardware until it completes or about kSuspendHintNs pass, so a waiting warp does
-// not take issue slots from the warps sharing its sub-partition.
-constexpr uint32_t kSuspendHintNs = 20000;
-
+// One test of the phase.  If it has not completed, the thread may wait in hardware
+// for a short, system-defined time before the test returns false.  (An explicit
+// suspend-time hint was measured to resume waiting warps later than this form.)
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
                  "selp.u32 %0, 1, 0, p;\n\t}"
                  : "=r"(ok)
-                 : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+                 : "r"(smem_u32(bar)), "r"(parity)
                  : "memory");
     return ok != 0;
 }
