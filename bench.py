@@ -319,12 +319,13 @@ def run_ours(args):
         "scan": {"ms": round(scan_ms, 5), "elems_per_s": pw["elems"] / scan_s,
                  "hbm_gbs": round(scan_hbm, 1), "roofline_frac": round(t_roof_scan / scan_s, 4),
                  "t_roof_ms": round(t_roof_scan * 1e3, 5)},
-        "decode": {"ms": round(dec_ms, 5), "elems_per_s": dw["elems"] / dec_s,
+        "decode": {"kernel": "ss_state_update_stream_kernel (decode update)",
+                   "ms": round(dec_ms, 5), "elems_per_s": dw["elems"] / dec_s,
                    "hbm_gbs": round(dw["bytes"] / dec_s / 1e9, 1),
                    "hbm_frac": round(dw["bytes"] / dec_s / 1e9 / hbm_gbs, 4),
                    "roofline_frac": round(t_roof_dec / dec_s, 4),
                    "t_roof_ms": round(t_roof_dec * 1e3, 5),
-                   "traffic": _measured_traffic("ss_state_update_kernel")},
+                   "traffic": _measured_traffic("ss_state_update_stream_kernel")},
     }
 
     cpu = None
