@@ -167,9 +167,10 @@ int launch_scan(ss::ScanArgs a, cudaStream_t stream)
                 occ_cache[dev].store(occ, std::memory_order_release);
         }
         const int64_t resident = int64_t(sms) * occ;
-        // about eight units per resident CTA, segments of at least eight chunks
-        int64_t segs = (8 * resident + a.groups - 1) / a.groups;
-        const int64_t max_segs = nchunks / 8 > 1 ? nchunks / 8 : 1;
+        // about sixteen units per resident CTA (finer units balance the tail), segments
+        // of at least sixteen chunks (each unit start costs a carry hand-off)
+        int64_t segs = (16 * resident + a.groups - 1) / a.groups;
+        const int64_t max_segs = nchunks / 16 > 1 ? nchunks / 16 : 1;
         segs = segs < 1 ? 1 : (segs > max_segs ? max_segs : segs);
         const int64_t seg_chunks = (nchunks + segs - 1) / segs;
         a.seg_len = seg_chunks * S::kChunk;
@@ -237,7 +238,7 @@ int launch_update(ss::UpdateArgs a, cudaStream_t stream)
             return SS_ERR_CUDA;
         int occ = dev < 64 ? occ_cache[dev].load(std::memory_order_acquire) : 0;
         if (!occ) {
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, ss::kDecThreads, D::kSmem) != cudaSuccess)
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, ss::kDecBlock, D::kSmem) != cudaSuccess)
                 return SS_ERR_CUDA;
             occ = occ > 0 ? occ : 1;
             if (dev < 64)
@@ -264,7 +265,7 @@ int launch_update(ss::UpdateArgs a, cudaStream_t stream)
         uint32_t *status = nullptr;
         if (status_word_address(&status) != SS_OK)
             return SS_ERR_CUDA;
-        kernel<<<unsigned(grid), ss::kDecThreads, D::kSmem, stream>>>(da, status);
+        kernel<<<unsigned(grid), ss::kDecBlock, D::kSmem, stream>>>(da, status);
         return launch_status();
     }
     const int64_t per_block = int64_t(ss::kUpdateThreads) * ss::kUpdateItems; // row quarters

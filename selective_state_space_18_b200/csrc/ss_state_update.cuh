@@ -155,8 +155,12 @@ ss_state_update_kernel(const UpdateArgs p)
 // its stage.  Thread t owns quarters t, t + 256, t + 512, t + 768 of a tile.
 // When the grid is a multiple of the channel blocks per row, every CTA keeps one
 // channel block and walks batch rows, so A, dt_bias and D are loaded once per CTA.
+// One extra warp issues the copies: it refills a stage as soon as the eight consumer
+// warps have each released it (an "empty" mbarrier per stage), so consumer warps never
+// wait for one another.
 // The updated state goes straight back to global memory with streaming stores.
-constexpr int kDecThreads = 256;
+constexpr int kDecThreads = 256;                          // consumer threads (8 warps)
+constexpr int kDecBlock = kDecThreads + 32;               // + one copy-issuing warp
 constexpr int kDecItems = 4;                              // quarters per thread per tile
 constexpr int kDecQuarters = kDecThreads * kDecItems;     // 1024 quarters = 16 KB
 constexpr int kDecStages = 4;
@@ -168,7 +172,7 @@ template <int N, typename T> struct DecShape {
     static constexpr int kVecBytes = kChanPerTile * int(sizeof(T)); // x, dt or z of a tile
     static constexpr int kBCOff = kDecTileBytes + 3 * kVecBytes;  // B then C of the row
     static constexpr int kStageBytes = kBCOff + 2 * 64;
-    static constexpr size_t kSmem = size_t(kDecStages) * kStageBytes + 8 * kDecStages;
+    static constexpr size_t kSmem = size_t(kDecStages) * kStageBytes + 16 * kDecStages; // + full, empty
     static_assert(kStageBytes % 16 == 0, "16-byte aligned stages");
 };
 
@@ -189,7 +193,7 @@ struct DecArgs {
 };
 
 template <int N, typename T>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecBlock)
 ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
 {
     using D = DecShape<N, T>;
@@ -197,6 +201,7 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
     const UpdateArgs &p = da.u;
     extern __shared__ __align__(128) unsigned char dsm[];
     uint64_t *full = reinterpret_cast<uint64_t *>(dsm + size_t(kDecStages) * D::kStageBytes);
+    uint64_t *empty = full + kDecStages;
     const int tid = threadIdx.x, lane_q = tid & (Q - 1);
 
     // the k-th tile of this CTA: batch row b, channel block cb (false past the end)
@@ -241,29 +246,42 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
     };
 
     if (tid == 0) {
-        for (int s = 0; s < kDecStages; ++s)
+        for (int s = 0; s < kDecStages; ++s) {
             mbar_init(full + s, 1);
+            mbar_init(empty + s, kDecThreads / 32); // one arrival per consumer warp
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
-    int64_t issued = 0; // tiles of this CTA handed to the copy engine (thread 0's count)
-    if (tid == 0)
-        for (int s = 0; s < kDecStages - 1; ++s)
-            issued += issue(s, s) ? 1 : 0;
+    if (tid >= kDecThreads) {
+        // the copy-issuing warp: tile k goes into stage k % kDecStages once the
+        // consumers have released tile k - kDecStages
+        if (tid == kDecThreads) {
+            for (int64_t k = 0;; ++k) {
+                const int s = int(k % kDecStages);
+                if (k >= kDecStages &&
+                    !mbar_wait(empty + s, (uint32_t(k / kDecStages) & 1u) ^ 1u, status)) {
+                    // the consumers gave up (SS_ERR_TIMEOUT recorded): let the copies
+                    // still in flight land, then leave
+                    for (int64_t j = k - kDecStages + 1; j < k; ++j)
+                        mbar_wait(full + int(j % kDecStages), uint32_t(j / kDecStages) & 1u, nullptr);
+                    break;
+                }
+                if (!issue(k, s))
+                    break;
+            }
+        }
+        return;
+    }
 
     float4 av[kDecItems];
     float bias[kDecItems], dco[kDecItems];
     int64_t cached_cb = -1;
     bool ok = true;
-    int64_t k = 0;
-    for (;; ++k) {
+    for (int64_t k = 0;; ++k) {
         int64_t b, cb;
         if (!tile_of(k, b, cb))
             break;
-        // every thread is done with the stage of tile k - 1: refill it
-        __syncthreads();
-        if (tid == 0)
-            issued += issue(k + kDecStages - 1, int((k + kDecStages - 1) % kDecStages)) ? 1 : 0;
         const int64_t c0 = cb * D::kChanPerTile;
         const int nq = int(nchan(cb) * Q); // valid quarters in this tile
         if (cb != cached_cb) {
@@ -370,12 +388,12 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
                 }
             }
         }
+        // this warp is done reading the stage
+        __syncwarp();
+        if ((tid & 31) == 0)
+            mbar_arrive(empty + stage);
     }
-    if (!ok && tid == 0) {
-        // gave up (SS_ERR_TIMEOUT recorded): let the copies still in flight land
-        for (int64_t j = k; j < issued; ++j)
-            mbar_wait(full + int(j % kDecStages), uint32_t(j / kDecStages) & 1u, nullptr);
-    }
+    (void)ok;
 }
 
 } // namespace ss
