@@ -105,6 +105,26 @@ SS_API int ss_scan_fwd(int64_t batch, int64_t channels, int64_t state_dim, int64
                        uint32_t flags, void *y, float *h_last, void *workspace,
                        size_t workspace_bytes, ss_stream_t stream);
 
+/*
+ * ss_scan_fwd that also returns the state after every token (nnterp selective_scan:
+ * the interpretability readers ask for the state after each token; TransformerLens
+ * ssm_mixer: the unrolled state S_t at every position):
+ *
+ *   h_all : [batch, channels, seq, state_dim] float32 output, required;
+ *           h_all[b,c,t,:] = h_t of row (b, c), resets and h0 included.
+ *
+ * Everything else is as for ss_scan_fwd (same outputs, bit-identical y and h_last).
+ * h_all must not overlap any other buffer (SS_ERR_ALIAS).  The extra traffic is
+ * 4 * state_dim bytes per (b, t, c) written once, so this form is bound by HBM
+ * bandwidth rather than by the exponentials.
+ */
+SS_API int ss_scan_fwd_states(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
+                              ss_dtype_t dtype, const void *x, const void *dt_raw, const float *A,
+                              const void *B, const void *C, const float *D, const void *z,
+                              const float *dt_bias, const uint8_t *reset, const float *h0,
+                              uint32_t flags, void *y, float *h_last, float *h_all,
+                              void *workspace, size_t workspace_bytes, ss_stream_t stream);
+
 /* Workspace bytes ss_scan_fwd needs for this shape (0 for an invalid shape). */
 SS_API int64_t ss_scan_workspace_bytes(int64_t batch, int64_t channels, int64_t state_dim,
                                        int64_t seq);

@@ -14,7 +14,7 @@
 
 namespace {
 
-constexpr int kAbiMajor = 2, kAbiMinor = 0;
+constexpr int kAbiMajor = 2, kAbiMinor = 1;
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -141,12 +141,12 @@ bool build_maps(const ss::ScanArgs &a, ss::TmaMaps *m)
            encode_rows<T>(&m->C, a.C, a.seq, brows, S::kChunk, N, bc_swizzle);
 }
 
-template <int N, typename T, bool R, bool V>
+template <int N, typename T, bool R, bool V, bool E>
 int launch_scan(ss::ScanArgs a, cudaStream_t stream)
 {
     using S = ss::ScanShape<N>;
     constexpr size_t kSmem = S::template smem_bytes<T, V>();
-    auto kernel = ss::ss_scan_fwd_kernel<N, T, R, V>;
+    auto kernel = ss::ss_scan_fwd_kernel<N, T, R, V, E>;
     static std::atomic<uint64_t> smem_done{0};
     static std::atomic<int> occ_cache[64];
     int st = ensure_smem(kernel, kSmem, smem_done);
@@ -193,13 +193,19 @@ int launch_scan(ss::ScanArgs a, cudaStream_t stream)
     return launch_status();
 }
 
-template <int N, typename T>
-int dispatch_scan_t(const ss::ScanArgs &a, bool vec, cudaStream_t s)
+template <int N, typename T, bool E>
+int dispatch_scan_e(const ss::ScanArgs &a, bool vec, cudaStream_t s)
 {
     const bool r = a.reset != nullptr;
     if (r)
-        return vec ? launch_scan<N, T, true, true>(a, s) : launch_scan<N, T, true, false>(a, s);
-    return vec ? launch_scan<N, T, false, true>(a, s) : launch_scan<N, T, false, false>(a, s);
+        return vec ? launch_scan<N, T, true, true, E>(a, s) : launch_scan<N, T, true, false, E>(a, s);
+    return vec ? launch_scan<N, T, false, true, E>(a, s) : launch_scan<N, T, false, false, E>(a, s);
+}
+
+template <int N, typename T>
+int dispatch_scan_t(const ss::ScanArgs &a, bool vec, cudaStream_t s)
+{
+    return a.h_all ? dispatch_scan_e<N, T, true>(a, vec, s) : dispatch_scan_e<N, T, false>(a, vec, s);
 }
 
 template <int N> int64_t scan_groups(int64_t batch, int64_t channels)
@@ -385,11 +391,17 @@ int ss_scan_status(const void *workspace, ss_stream_t stream, int *status)
     return SS_OK;
 }
 
-int ss_scan_fwd(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, ss_dtype_t dtype,
-                const void *x, const void *dt_raw, const float *A, const void *B, const void *C,
-                const float *D, const void *z, const float *dt_bias, const uint8_t *reset,
-                const float *h0, uint32_t flags, void *y, float *h_last, void *workspace,
-                size_t workspace_bytes, ss_stream_t stream)
+} // extern "C"
+
+namespace {
+
+// ss_scan_fwd and ss_scan_fwd_states: validation, then the launch.  h_all (nullable)
+// receives the state after every token.
+int scan_impl(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, ss_dtype_t dtype,
+              const void *x, const void *dt_raw, const float *A, const void *B, const void *C,
+              const float *D, const void *z, const float *dt_bias, const uint8_t *reset,
+              const float *h0, uint32_t flags, void *y, float *h_last, float *h_all, void *workspace,
+              size_t workspace_bytes, ss_stream_t stream)
 {
     if (!x || !dt_raw || !A || !B || !C || !y)
         return SS_ERR_NULL;
@@ -431,6 +443,20 @@ int ss_scan_fwd(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
     }
     if (h_last && overlaps(h_last, hbytes, y, ybytes))
         return SS_ERR_ALIAS;
+    size_t abytes = 0; // h_all
+    if (h_all) {
+        int64_t ael = 0;
+        if (!mul_ok(elems, state_dim, &ael) || ael > (INT64_MAX / 8))
+            return SS_ERR_SHAPE;
+        abytes = size_t(ael) * 4;
+        if (!aligned(h_all, 4))
+            return SS_ERR_ALIGN;
+        for (int i = 0; i < 10; ++i)
+            if (overlaps(h_all, abytes, in_p[i], in_n[i]))
+                return SS_ERR_ALIAS;
+        if (overlaps(h_all, abytes, y, ybytes) || (h_last && overlaps(h_all, abytes, h_last, hbytes)))
+            return SS_ERR_ALIAS;
+    }
     if (workspace) {
         if (!aligned(workspace, 16))
             return SS_ERR_ALIGN;
@@ -438,7 +464,8 @@ int ss_scan_fwd(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
             if (overlaps(workspace, workspace_bytes, in_p[i], in_n[i]))
                 return SS_ERR_ALIAS;
         if (overlaps(workspace, workspace_bytes, y, ybytes) ||
-            (h_last && overlaps(workspace, workspace_bytes, h_last, hbytes)))
+            (h_last && overlaps(workspace, workspace_bytes, h_last, hbytes)) ||
+            (h_all && overlaps(workspace, workspace_bytes, h_all, abytes)))
             return SS_ERR_ALIAS;
     }
 
@@ -459,6 +486,7 @@ int ss_scan_fwd(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
     a.reset = reset;
     a.y = y;
     a.h_last = h_last;
+    a.h_all = h_all;
     a.softplus = (flags & SS_DT_SOFTPLUS) ? 1 : 0;
     a.workspace = static_cast<uint8_t *>(workspace);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -467,6 +495,32 @@ int ss_scan_fwd(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
     case 8: return dispatch_scan_n<8>(a, dtype, vec, workspace_bytes, s);
     default: return dispatch_scan_n<16>(a, dtype, vec, workspace_bytes, s);
     }
+}
+
+} // namespace
+
+extern "C" {
+
+int ss_scan_fwd(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, ss_dtype_t dtype,
+                const void *x, const void *dt_raw, const float *A, const void *B, const void *C,
+                const float *D, const void *z, const float *dt_bias, const uint8_t *reset,
+                const float *h0, uint32_t flags, void *y, float *h_last, void *workspace,
+                size_t workspace_bytes, ss_stream_t stream)
+{
+    return scan_impl(batch, channels, state_dim, seq, dtype, x, dt_raw, A, B, C, D, z, dt_bias, reset, h0, flags, y,
+                     h_last, nullptr, workspace, workspace_bytes, stream);
+}
+
+int ss_scan_fwd_states(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, ss_dtype_t dtype,
+                       const void *x, const void *dt_raw, const float *A, const void *B, const void *C,
+                       const float *D, const void *z, const float *dt_bias, const uint8_t *reset,
+                       const float *h0, uint32_t flags, void *y, float *h_last, float *h_all, void *workspace,
+                       size_t workspace_bytes, ss_stream_t stream)
+{
+    if (!h_all)
+        return SS_ERR_NULL;
+    return scan_impl(batch, channels, state_dim, seq, dtype, x, dt_raw, A, B, C, D, z, dt_bias, reset, h0, flags, y,
+                     h_last, h_all, workspace, workspace_bytes, stream);
 }
 
 int ss_state_update(int64_t batch, int64_t channels, int64_t state_dim, ss_dtype_t dtype,

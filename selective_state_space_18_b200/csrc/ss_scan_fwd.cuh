@@ -46,6 +46,7 @@ struct ScanArgs {
     const uint8_t *reset;
     void *y;
     float *h_last;
+    float *h_all;             // nullable: the state after every token [b, c, L, N] fp32
     int softplus;
     int64_t groups_per_batch; // channel groups per batch row
     int64_t groups;           // batch * groups_per_batch
@@ -556,9 +557,13 @@ struct GroupTerms {
 // group k + 1 are issued before the sequential FMA chain of group k, so the MUFU
 // latency of one group hides behind the chain of the previous one (with only about
 // two scan warps per sub-partition there is little other work to switch to).
-template <int N, typename T, bool HAS_RESET>
+//
+// EMIT: also store the state after every token to `hrow` (this channel's row of h_all
+// at the chunk's first token, N floats per token), for the first `valid` tokens.
+template <int N, typename T, bool HAS_RESET, bool EMIT>
 __device__ __forceinline__ void scan_chunk(const float *stage, const unsigned char *raw, float *ys, int cl, int n0,
-                                           int n1, float2 A0, float2 A1, float &hs0, float &hs1)
+                                           int n1, float2 A0, float2 A1, float &hs0, float &hs1, float *hrow,
+                                           int64_t valid)
 {
     using S = ScanShape<N>;
     constexpr int kTok = 16 / int(sizeof(T)); // tokens per 16-byte chunk of a B/C row
@@ -624,6 +629,17 @@ __device__ __forceinline__ void scan_chunk(const float *stage, const unsigned ch
             hs1 = fmaf(f.a1[pr].y, h1t, f.v1[pr].y);
             const float2 yy = __fmul2_rn(bc_pair<T>(cc0, pi), make_float2(h0t, hs0));
             yo[pr] = __ffma2_rn(bc_pair<T>(cc1, pi), make_float2(h1t, hs1), yy);
+            if (EMIT) {
+                const int tt = t + 2 * pr;
+                if (tt < valid) {
+                    __stcs(hrow + tt * N + n0, h0t);
+                    __stcs(hrow + tt * N + n1, h1t);
+                }
+                if (tt + 1 < valid) {
+                    __stcs(hrow + (tt + 1) * N + n0, hs0);
+                    __stcs(hrow + (tt + 1) * N + n1, hs1);
+                }
+            }
         }
         *reinterpret_cast<float4 *>(ys + t) = make_float4(yo[0].x, yo[0].y, yo[1].x, yo[1].y);
     }
@@ -774,7 +790,7 @@ __device__ __forceinline__ bool epilogue_role(const ScanArgs &p, const float *y_
 // the kernel
 // ---------------------------------------------------------------------------------------
 
-template <int N, typename T, bool HAS_RESET, bool VEC>
+template <int N, typename T, bool HAS_RESET, bool VEC, bool EMIT>
 __global__ void __launch_bounds__(ScanShape<N>::kThreads, 1)
 ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
 {
@@ -886,9 +902,13 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
                 }
             }
             const int rs = int(j % S::kRawStages);
-            scan_chunk<N, T, HAS_RESET>(stage, smem_bytes + rs * S::template raw_stage_bytes<T>(),
-                                        y_base + ysi * S::kYStage + S::kYPOff + cl * S::kYChan + sub * S::kRow,
-                                        cl, n0, n1, A0, A1, hs0, hs1);
+            float *hrow = nullptr;
+            if (EMIT)
+                hrow = p.h_all + (row * p.seq + meta.t0) * N;
+            scan_chunk<N, T, HAS_RESET, EMIT>(stage, smem_bytes + rs * S::template raw_stage_bytes<T>(),
+                                              y_base + ysi * S::kYStage + S::kYPOff + cl * S::kYChan + sub * S::kRow,
+                                              cl, n0, n1, A0, A1, hs0, hs1, hrow,
+                                              cvalid ? p.seq - meta.t0 : int64_t(0));
             mbar_arrive(bars + S::kBarRawEmpty + rs);
             mbar_arrive(in_empty + st);
             mbar_arrive(y_full + ysi);

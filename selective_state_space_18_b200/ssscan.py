@@ -26,7 +26,7 @@ STATUS = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE", 4:
           9: "SS_ERR_WORKSPACE", 10: "SS_ERR_SCRATCH_LIMIT"}
 EXPORTS = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_scan_status", "ss_state_update",
            "ss_debug_set_wait_limit", "ss_status_string", "ss_abi_version",
-           "ss_scan_fwd_static_scratch")
+           "ss_scan_fwd_static_scratch", "ss_scan_fwd_states")
 ABI_MAJOR = 2
 
 _lock = threading.Lock()
@@ -56,6 +56,9 @@ def load_library(path: str = LIB_PATH):
             lib.ss_scan_fwd.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 10 + [
                 ctypes.c_uint32, _vp, _vp, _vp, ctypes.c_size_t, _vp]
             lib.ss_scan_fwd.restype = ctypes.c_int
+            lib.ss_scan_fwd_states.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 10 + [
+                ctypes.c_uint32, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+            lib.ss_scan_fwd_states.restype = ctypes.c_int
             lib.ss_scan_fwd_static_scratch.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 10 + [
                 ctypes.c_uint32, _vp, _vp, ctypes.POINTER(_vp), _vp]
             lib.ss_scan_fwd_static_scratch.restype = ctypes.c_int
@@ -160,10 +163,12 @@ def _stream(stream, device):
 
 def ss_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h0=None, *,
                 dt_softplus=True, y=None, h_last=None, return_last_state=True, stream=None,
-                workspace=True):
+                workspace=True, h_all=None, return_states=False):
     """Prompt scan.  x, dt, z: [batch, channels, seq]; B, C: [batch, state_dim, seq];
     A: [channels, state_dim] fp32; D, dt_bias: [channels] fp32; reset: [batch, seq]
-    bool/uint8; h0: [batch, channels, state_dim] fp32.  Returns (y, h_last).
+    bool/uint8; h0: [batch, channels, state_dim] fp32.  Returns (y, h_last), or
+    (y, h_last, h_all) with the state after every token [batch, channels, seq,
+    state_dim] fp32 when return_states is set or h_all is given (ss_scan_fwd_states).
 
     workspace: True (a cached per-stream workspace: segmented, balanced schedule),
     False (none: one CTA per channel group) or a zero-initialised uint8 tensor."""
@@ -200,6 +205,11 @@ def ss_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h0=Non
         h_last = _out(h_last, "h_last", dev, torch.float32, (bt, ch, n))
     flags = SS_DT_SOFTPLUS if dt_softplus else 0
     lib = load_library()
+    states = return_states or h_all is not None
+    if h_all is None and states:
+        h_all = torch.empty(bt, ch, L, n, device=dev, dtype=torch.float32)
+    elif h_all is not None:
+        h_all = _out(h_all, "h_all", dev, torch.float32, (bt, ch, L, n))
     if workspace is True:
         workspace = scan_workspace(bt, ch, n, L, dev, stream)
     elif workspace is False or workspace is None:
@@ -207,6 +217,14 @@ def ss_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h0=Non
     elif workspace.device != dev or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous uint8 tensor on the inputs' device")
     ws_bytes = 0 if workspace is None else workspace.numel()
+    if states:
+        st = lib.ss_scan_fwd_states(bt, ch, n, L, code, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
+                                    _ptr(D), _ptr(z), _ptr(dt_bias), _ptr(reset), _ptr(h0), flags,
+                                    _ptr(y), _ptr(h_last), _ptr(h_all), _ptr(workspace), ws_bytes,
+                                    _stream(stream, dev))
+        if st != 0:
+            raise SSError("ss_scan_fwd_states", st)
+        return y, h_last, h_all
     st = lib.ss_scan_fwd(bt, ch, n, L, code, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
                          _ptr(D), _ptr(z), _ptr(dt_bias), _ptr(reset), _ptr(h0), flags,
                          _ptr(y), _ptr(h_last), _ptr(workspace), ws_bytes, _stream(stream, dev))

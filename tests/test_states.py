@@ -1,0 +1,80 @@
+"""The state after every token (ss_scan_fwd_states) against the oracle's per-token
+states (nnterp selective_scan: the state after each token, for the interpretability
+readers; TransformerLens ssm_mixer: the unrolled state S_t at every position)."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import SCAN_KEYS, TOL, assert_close, dev
+from selective_state_space_18_b200 import ssscan
+from selective_state_space_18_b200.inputs import make_scan_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+
+
+def _gpu(inp, **kw):
+    y, h, hall = ssscan.ss_scan_fwd(**dev(inp, SCAN_KEYS), return_states=True, **kw)
+    torch.cuda.synchronize()
+    return y.cpu(), h.cpu(), hall.cpu()
+
+
+@pytest.mark.parametrize("n", [4, 8, 16])
+@pytest.mark.parametrize("dtype,L", [("f32", 100), ("bf16", 264), ("bf16", 77)])
+@pytest.mark.parametrize("resets", [False, True])
+def test_states_match_oracle(orc, n, dtype, L, resets):
+    inp = make_scan_inputs(2, 40, n, L, dtype, seed=400 + n + L, h0=True, reset_mean_doc=30 if resets else 0)
+    y, h, hall = _gpu(inp)
+    ref = orc.scan(**inp, return_states=True)
+    tol = TOL[inp["x"].dtype]
+    assert_close(y, ref["y"], tol, "y")
+    # states are fp32 whatever the storage type: the fp32 state tolerance
+    assert_close(hall, ref["h_all"], 1e-4, "h_all")
+    assert torch.equal(hall[:, :, -1, :], h)  # the last state is h_last, bit for bit
+
+
+def test_states_leave_y_and_h_last_unchanged():
+    """Emitting the states changes nothing else, bit for bit, in either schedule."""
+    inp = make_scan_inputs(3, 96, 16, 1500, "bf16", seed=420, h0=True, reset_mean_doc=200)
+    d = dev(inp, SCAN_KEYS)
+    for ws in (True, False):
+        y0, h0 = ssscan.ss_scan_fwd(**d, workspace=ws)
+        y1, h1, hall = ssscan.ss_scan_fwd(**d, workspace=ws, return_states=True)
+        torch.cuda.synchronize()
+        assert torch.equal(y0, y1) and torch.equal(h0, h1)
+        assert torch.equal(hall[:, :, -1, :], h1)
+
+
+def test_states_segmented_equals_static():
+    inp = make_scan_inputs(1, 320, 16, 4096, "bf16", seed=421)
+    d = dev(inp, SCAN_KEYS)
+    _, _, a = ssscan.ss_scan_fwd(**d, workspace=True, return_states=True)
+    _, _, b = ssscan.ss_scan_fwd(**d, workspace=False, return_states=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_states_sampled_rows_medium(orc):
+    """A shape with many channel groups and a ragged tail: sampled rows, every token."""
+    inp = make_scan_inputs(2, 512, 16, 3001, "bf16", seed=422, reset_mean_doc=300)
+    y, h, hall = _gpu(inp)
+    rows = [(0, 0), (0, 17), (1, 255), (1, 511), (0, 300)]
+    sub = {k: v for k, v in inp.items()}
+    for b, c in rows:
+        one = dict(sub)
+        for k in ("x", "dt", "z"):
+            one[k] = inp[k][b:b + 1, c:c + 1]
+        for k in ("B", "C", "reset"):
+            one[k] = inp[k][b:b + 1] if inp[k] is not None else None
+        one["A"] = inp["A"][c:c + 1]
+        for k in ("D", "dt_bias"):
+            one[k] = inp[k][c:c + 1] if inp[k] is not None else None
+        one["h0"] = None
+        ref = orc.scan(**one, return_states=True)
+        assert_close(hall[b, c], ref["h_all"][0, 0], 1e-4, f"h_all row {(b, c)}")
+        assert_close(y[b, c], ref["y"][0, 0], TOL[torch.bfloat16], f"y row {(b, c)}")
