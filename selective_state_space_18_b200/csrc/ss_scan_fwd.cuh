@@ -791,7 +791,7 @@ __device__ __forceinline__ bool epilogue_role(const ScanArgs &p, const float *y_
 // ---------------------------------------------------------------------------------------
 
 template <int N, typename T, bool HAS_RESET, bool VEC, bool EMIT>
-__global__ void __launch_bounds__(ScanShape<N>::kThreads, 1)
+__global__ void __launch_bounds__(ScanShape<N>::kThreads, EMIT ? 2 : 1)
 ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
 {
     using S = ScanShape<N>;
@@ -859,7 +859,9 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
         // =============================== scan warps ==============================
         const int cw = lane / S::kPairs;    // channel within the warp
         const int sub = lane % S::kPairs;   // state pair
-        const int n0 = sub, n1 = sub + S::kPairs;   // rows n0 < 8 and n1 >= N/2: distinct banks
+        // rows n0 < N/2 and n1 >= N/2: distinct banks of the B/C tiles (and the same
+        // lane-to-state map in every form, so outputs are bit-identical across forms)
+        const int n0 = sub, n1 = sub + S::kPairs;
         const int cl = warp * S::kChanPerWarp + cw;  // channel within the CTA
         float hs0 = 0.0f, hs1 = 0.0f;
         float2 A0 = make_float2(0.f, 0.f), A1 = make_float2(0.f, 0.f);
