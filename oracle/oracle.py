@@ -55,6 +55,8 @@ def _load():
             lib.ss_oracle_update.argtypes = [_i64, _i64, _i64, _dp] + [_dp] * 8 + [
                 ctypes.c_int, _dp, ctypes.c_int]
             lib.ss_oracle_update.restype = ctypes.c_int
+            lib.ss_oracle_gated_scan.argtypes = [_i64, _i64, _i64, _i64] + [_dp] * 7 + [ctypes.c_int]
+            lib.ss_oracle_gated_scan.restype = ctypes.c_int
             lib.ss_oracle_num_threads.argtypes = []
             lib.ss_oracle_num_threads.restype = ctypes.c_int
             _lib = lib
@@ -168,6 +170,26 @@ def update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, *, dt_softplus=T
                               int(bool(dt_softplus)), _ptr(y), int(nthreads or num_threads()))
     _check(rc, "ss_oracle_update")
     return {"y": y, "state": st_arr}
+
+
+def gated_scan(q, k, v, gamma, h0=None, *, nthreads=None):
+    """Gated state scan oracle ("Mamba 2 Gated State Scan": S_t = gamma_t S_{t-1} +
+    k_t v_t^T, y_t = q_t^T S_t).  q, k [B, S, Dk]; v [B, S, Dv]; gamma [B, S];
+    h0 [B, Dk, Dv] or None.  Returns dict(outputs [B, S, Dv], final_state [B, Dk, Dv])."""
+    q, k, v, gamma = (_f64(a) for a in (q, k, v, gamma))
+    h0 = _f64(h0)
+    bt, sl, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != (bt, sl, dk) or v.shape != (bt, sl, dv) or gamma.shape != (bt, sl):
+        raise ValueError("inconsistent shapes")
+    if h0 is not None and h0.shape != (bt, dk, dv):
+        raise ValueError("h0 must be [B, Dk, Dv]")
+    y = np.empty((bt, sl, dv))
+    fs = np.empty((bt, dk, dv))
+    rc = _load().ss_oracle_gated_scan(bt, sl, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(h0),
+                                      _ptr(y), _ptr(fs), int(nthreads or num_threads()))
+    _check(rc, "ss_oracle_gated_scan")
+    return {"outputs": y, "final_state": fs}
 
 
 def scan_rows(inputs: dict, rows, *, dt_softplus=True, nthreads=1):

@@ -287,3 +287,56 @@ int ss_oracle_update(int64_t batch, int64_t channels, int64_t state_dim, double 
     }
     return ORC_OK;
 }
+
+/*
+ * Mamba-2 gated state scan ("Mamba 2 Gated State Scan" exercise page): per batch item
+ * b, with S_{-1} = h0[b] (zeros when h0 is NULL),
+ *
+ *   S_t = gamma[b,t] * S_{t-1} + k[b,t,:] v[b,t,:]^T      (Dk x Dv)
+ *   y[b,t,:] = q[b,t,:]^T S_t                             (the updated state is read)
+ *
+ * and final_state[b] = S_{seq-1}.  Layouts: q, k [batch, seq, dk]; v, y
+ * [batch, seq, dv]; gamma [batch, seq]; h0, final_state [batch, dk, dv].  The token
+ * loop in sequence order, every sum in index order; OpenMP over batch items only.
+ */
+int ss_oracle_gated_scan(int64_t batch, int64_t seq, int64_t dk, int64_t dv, const double *q,
+                         const double *k, const double *v, const double *gamma, const double *h0,
+                         double *y, double *final_state, int nthreads)
+{
+    if (!q || !k || !v || !gamma || !y || !final_state)
+        return ORC_ERR_NULL;
+    if (batch <= 0 || seq <= 0 || dk <= 0 || dv <= 0)
+        return ORC_ERR_SHAPE;
+    int failed = 0;
+#ifdef _OPENMP
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+#endif
+    for (int64_t b = 0; b < batch; ++b) {
+        double *S = (double *)malloc(sizeof(double) * (size_t)(dk * dv));
+        if (!S) {
+            failed = 1;
+            continue;
+        }
+        for (int64_t i = 0; i < dk * dv; ++i)
+            S[i] = h0 ? h0[b * dk * dv + i] : 0.0;
+        for (int64_t t = 0; t < seq; ++t) {
+            const double g = gamma[b * seq + t];
+            const double *kt = k + (b * seq + t) * dk, *qt = q + (b * seq + t) * dk;
+            const double *vt = v + (b * seq + t) * dv;
+            for (int64_t i = 0; i < dk; ++i)
+                for (int64_t j = 0; j < dv; ++j)
+                    S[i * dv + j] = g * S[i * dv + j] + kt[i] * vt[j];
+            for (int64_t j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int64_t i = 0; i < dk; ++i)
+                    acc += qt[i] * S[i * dv + j];
+                y[(b * seq + t) * dv + j] = acc;
+            }
+        }
+        for (int64_t i = 0; i < dk * dv; ++i)
+            final_state[b * dk * dv + i] = S[i];
+        free(S);
+    }
+    (void)nthreads;
+    return failed ? ORC_ERR_NOMEM : ORC_OK;
+}
