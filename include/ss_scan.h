@@ -211,6 +211,30 @@ SS_API int ss_state_update(int64_t batch, int64_t channels, int64_t state_dim, s
  */
 SS_API int ss_debug_set_wait_limit(uint32_t microseconds);
 
+/*
+ * Gated state scan (the "Mamba 2 Gated State Scan" exercise page): per batch item b,
+ *
+ *   S_t = gamma[b,t] * S_{t-1} + k[b,t,:] v[b,t,:]^T      (Dk x Dv state, fp32)
+ *   outputs[b,t,:] = q[b,t,:]^T S_t                        (the updated state is read)
+ *
+ * with S_{-1} = h0[b] (zeros when h0 is NULL) and final_state[b] = S_{seq-1}.
+ *
+ *   q, k        : [batch, seq, dk]  dtype (SS_F32 or SS_BF16)
+ *   v           : [batch, seq, dv]  dtype
+ *   gamma       : [batch, seq]      float32, in [0, 1]
+ *   h0          : [batch, dk, dv]   float32, nullable
+ *   outputs     : [batch, seq, dv]  dtype (output)
+ *   final_state : [batch, dk, dv]   dtype (output)
+ *
+ * All arithmetic is fp32; results are rounded to the dtype of q, as the page asks.
+ * dk must be at most 128 (SS_ERR_UNSUPPORTED otherwise); dv is unrestricted.  Inputs
+ * are not modified; outputs must not overlap inputs or each other (SS_ERR_ALIAS).
+ * Asynchronous on `stream`; returns SS_OK or an error status.
+ */
+SS_API int ss_gated_scan(int64_t batch, int64_t seq, int64_t dk, int64_t dv, ss_dtype_t dtype,
+                         const void *q, const void *k, const void *v, const float *gamma,
+                         const float *h0, void *outputs, void *final_state, ss_stream_t stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 SS_API const char *ss_status_string(int status);
 

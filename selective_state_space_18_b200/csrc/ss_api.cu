@@ -11,6 +11,7 @@
 
 #include "ss_scan_fwd.cuh"
 #include "ss_state_update.cuh"
+#include "ss_gated_scan.cuh"
 
 namespace {
 
@@ -497,9 +498,80 @@ int scan_impl(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, s
     }
 }
 
+template <int RG, typename T> int launch_gated(ss::GatedArgs a, cudaStream_t stream)
+{
+    using G = ss::GatedShape<RG>;
+    auto kernel = ss::ss_gated_scan_kernel<RG, T>;
+    static std::atomic<uint64_t> smem_done{0};
+    const int st = ensure_smem(kernel, G::kSmem, smem_done);
+    if (st != SS_OK)
+        return st;
+    a.col_tiles = int((a.dv + G::kCols - 1) / G::kCols);
+    int64_t grid = 0;
+    if (!mul_ok(a.batch, a.col_tiles, &grid) || grid > 0x7fffffffLL)
+        return SS_ERR_SHAPE;
+    kernel<<<unsigned(grid), ss::kGThreads, G::kSmem, stream>>>(a);
+    return launch_status();
+}
+
+template <typename T> int dispatch_gated(const ss::GatedArgs &a, cudaStream_t s)
+{
+    if (a.dk <= 32)
+        return launch_gated<4, T>(a, s);
+    if (a.dk <= 64)
+        return launch_gated<8, T>(a, s);
+    return launch_gated<16, T>(a, s);
+}
+
 } // namespace
 
 extern "C" {
+
+int ss_gated_scan(int64_t batch, int64_t seq, int64_t dk, int64_t dv, ss_dtype_t dtype, const void *q,
+                  const void *k, const void *v, const float *gamma, const float *h0, void *outputs,
+                  void *final_state, ss_stream_t stream)
+{
+    if (!q || !k || !v || !gamma || !outputs || !final_state)
+        return SS_ERR_NULL;
+    if (batch <= 0 || seq <= 0 || dk <= 0 || dv <= 0)
+        return SS_ERR_SHAPE;
+    if (dtype != SS_F32 && dtype != SS_BF16)
+        return SS_ERR_DTYPE;
+    if (dk > 128)
+        return SS_ERR_UNSUPPORTED;
+    const size_t es = dtype == SS_BF16 ? 2 : 4;
+    int64_t bs = 0, qel = 0, vel = 0, sel = 0;
+    if (!mul_ok(batch, seq, &bs) || !mul_ok(bs, dk, &qel) || !mul_ok(bs, dv, &vel) ||
+        !mul_ok(batch * dk, dv, &sel) || qel > (INT64_MAX / 8) || vel > (INT64_MAX / 8))
+        return SS_ERR_SHAPE;
+    const void *typed[] = {q, k, v, outputs, final_state};
+    for (const void *p : typed)
+        if (!aligned(p, es))
+            return SS_ERR_ALIGN;
+    if (!aligned(gamma, 4) || (h0 && !aligned(h0, 4)))
+        return SS_ERR_ALIGN;
+    const void *in_p[] = {q, k, v, gamma, h0};
+    const size_t in_n[] = {size_t(qel) * es, size_t(qel) * es, size_t(vel) * es, size_t(bs) * 4,
+                           h0 ? size_t(sel) * 4 : 0};
+    const size_t ybytes = size_t(vel) * es, fbytes = size_t(sel) * es;
+    for (int i = 0; i < 5; ++i)
+        if (overlaps(outputs, ybytes, in_p[i], in_n[i]) || overlaps(final_state, fbytes, in_p[i], in_n[i]))
+            return SS_ERR_ALIAS;
+    if (overlaps(outputs, ybytes, final_state, fbytes))
+        return SS_ERR_ALIAS;
+    ss::GatedArgs a{};
+    a.batch = batch;
+    a.seq = seq;
+    a.dk = dk;
+    a.dv = dv;
+    a.q = q; a.k = k; a.v = v;
+    a.gamma = gamma;
+    a.h0 = h0;
+    a.y = outputs;
+    a.final_state = final_state;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return dtype == SS_BF16 ? dispatch_gated<__nv_bfloat16>(a, s) : dispatch_gated<float>(a, s);
+}
 
 int ss_scan_fwd(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, ss_dtype_t dtype,
                 const void *x, const void *dt_raw, const float *A, const void *B, const void *C,

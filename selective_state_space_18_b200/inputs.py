@@ -142,6 +142,23 @@ def make_update_inputs(batch, channels, state_dim, dtype="bf16", *, seed=0, z=Tr
     return out
 
 
+def make_gated_inputs(batch, seq, dk, dv, dtype="bf16", *, seed=0, h0=False):
+    """Seeded gated-state-scan inputs: q, k [B, S, Dk] scaled by 1/sqrt(Dk), v [B, S, Dv]
+    in ``dtype``; gamma [B, S] fp32 in [0, 1] -- mostly in [0.5, 1), with about 1% exact
+    zeros (the state is discarded) and 1% exact ones (kept whole)."""
+    g = _gen(seed)
+    sc = 1.0 / math.sqrt(dk)
+    q = (torch.randn(batch, seq, dk, generator=g) * sc).to(DTYPES[dtype])
+    k = (torch.randn(batch, seq, dk, generator=g) * sc).to(DTYPES[dtype])
+    v = _randn(g, (batch, seq, dv), dtype)
+    gamma = 0.5 + 0.5 * torch.rand(batch, seq, generator=g)
+    u = torch.rand(batch, seq, generator=g)
+    gamma = torch.where(u < 0.01, torch.zeros_like(gamma), torch.where(u > 0.99, torch.ones_like(gamma), gamma))
+    out = {"q": q, "k": k, "v": v, "gamma": gamma.float().contiguous()}
+    out["h0"] = torch.randn(batch, dk, dv, generator=g) if h0 else None
+    return out
+
+
 def make_workload(name_or_workload, **overrides):
     """Inputs for a named workload (prompt scan or decode update)."""
     w = WORKLOADS[name_or_workload] if isinstance(name_or_workload, str) else name_or_workload

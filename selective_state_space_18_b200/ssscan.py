@@ -26,7 +26,7 @@ STATUS = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE", 4:
           9: "SS_ERR_WORKSPACE", 10: "SS_ERR_SCRATCH_LIMIT"}
 EXPORTS = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_scan_status", "ss_state_update",
            "ss_debug_set_wait_limit", "ss_status_string", "ss_abi_version",
-           "ss_scan_fwd_static_scratch", "ss_scan_fwd_states")
+           "ss_scan_fwd_static_scratch", "ss_scan_fwd_states", "ss_gated_scan")
 ABI_MAJOR = 2
 
 _lock = threading.Lock()
@@ -62,6 +62,8 @@ def load_library(path: str = LIB_PATH):
             lib.ss_scan_fwd_static_scratch.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 10 + [
                 ctypes.c_uint32, _vp, _vp, ctypes.POINTER(_vp), _vp]
             lib.ss_scan_fwd_static_scratch.restype = ctypes.c_int
+            lib.ss_gated_scan.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 7 + [_vp]
+            lib.ss_gated_scan.restype = ctypes.c_int
             lib.ss_scan_workspace_bytes.argtypes = [_i64, _i64, _i64, _i64]
             lib.ss_scan_workspace_bytes.restype = _i64
             lib.ss_scan_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_int)]
@@ -333,3 +335,30 @@ def static_scratch_status(stream=None, device=None):
     if st != 0:
         raise SSError("ss_scan_status", st)
     return STATUS[out.value]
+
+
+def ss_gated_scan(q, k, v, gamma, h0=None, *, stream=None):
+    """Gated state scan S_t = gamma_t S_{t-1} + k_t v_t^T, y_t = q_t^T S_t.  q, k:
+    [B, S, Dk]; v: [B, S, Dv] (float32 or bfloat16, same dtype); gamma: [B, S] float32;
+    h0: [B, Dk, Dv] float32 or None.  Non-contiguous inputs are copied, never modified.
+    Returns {"outputs": [B, S, Dv], "final_state": [B, Dk, Dv]} in the dtype of q."""
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("ss_gated_scan runs on CUDA tensors only")
+    if q.dim() != 3:
+        raise ValueError("q must be [B, S, Dk]")
+    bt, sl, dk = q.shape
+    dv = v.shape[-1]
+    code = _dtype_code(q)
+    q = _prep(q, "q", dev)
+    k = _prep(k, "k", dev, q.dtype, (bt, sl, dk))
+    v = _prep(v, "v", dev, q.dtype, (bt, sl, dv))
+    gamma = _prep(gamma, "gamma", dev, torch.float32, (bt, sl))
+    h0 = _prep(h0, "h0", dev, torch.float32, (bt, dk, dv))
+    y = torch.empty(bt, sl, dv, device=dev, dtype=q.dtype)
+    fs = torch.empty(bt, dk, dv, device=dev, dtype=q.dtype)
+    st = load_library().ss_gated_scan(bt, sl, dk, dv, code, _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(h0),
+                                      _ptr(y), _ptr(fs), _stream(stream, dev))
+    if st != 0:
+        raise SSError("ss_gated_scan", st)
+    return {"outputs": y, "final_state": fs}

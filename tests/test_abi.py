@@ -193,3 +193,20 @@ def test_scan_states_checks(lib):
     assert ssscan.STATUS[_scan_states(lib, ctypes.c_void_p(P[5].value))] == "SS_ERR_ALIAS"
     assert ssscan.STATUS[_scan_states(lib, P[9], state_dim=5)] == "SS_ERR_UNSUPPORTED"
     assert ssscan.STATUS[_scan_states(lib, P[9], x=None)] == "SS_ERR_NULL"
+
+
+def test_gated_scan_checks(lib):
+    def call(**kw):
+        a = dict(batch=2, seq=16, dk=64, dv=32, dtype=ssscan.SS_BF16, q=P[0], k=P[1], v=P[2], gamma=P[3],
+                 h0=None, y=P[4], fs=P[5])
+        a.update(kw)
+        return ssscan.STATUS[lib.ss_gated_scan(a["batch"], a["seq"], a["dk"], a["dv"], a["dtype"], a["q"], a["k"],
+                                               a["v"], a["gamma"], a["h0"], a["y"], a["fs"], None)]
+    assert call(q=None) == "SS_ERR_NULL"
+    assert call(fs=None) == "SS_ERR_NULL"
+    assert call(seq=0) == "SS_ERR_SHAPE"
+    assert call(dtype=9) == "SS_ERR_DTYPE"
+    assert call(dk=129) == "SS_ERR_UNSUPPORTED"
+    assert call(q=ctypes.c_void_p(P[0].value + 1)) == "SS_ERR_ALIGN"
+    assert call(y=ctypes.c_void_p(P[1].value + 64)) == "SS_ERR_ALIAS"
+    assert call(fs=ctypes.c_void_p(P[4].value)) == "SS_ERR_ALIAS"
