@@ -498,10 +498,10 @@ int scan_impl(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, s
     }
 }
 
-template <int RG, typename T> int launch_gated(ss::GatedArgs a, cudaStream_t stream)
+template <int RG, typename T, bool VEC> int launch_gated(ss::GatedArgs a, cudaStream_t stream)
 {
     using G = ss::GatedShape<RG>;
-    auto kernel = ss::ss_gated_scan_kernel<RG, T>;
+    auto kernel = ss::ss_gated_scan_kernel<RG, T, VEC>;
     static std::atomic<uint64_t> smem_done{0};
     const int st = ensure_smem(kernel, G::kSmem, smem_done);
     if (st != SS_OK)
@@ -514,13 +514,21 @@ template <int RG, typename T> int launch_gated(ss::GatedArgs a, cudaStream_t str
     return launch_status();
 }
 
+template <int RG, typename T> int dispatch_gated_v(const ss::GatedArgs &a, cudaStream_t s)
+{
+    // 8-element vector staging: whole rows (dk equals the padded row count), dv a
+    // multiple of 8, rows 16-byte aligned
+    const bool vec = a.dk == 8 * RG && a.dv % 8 == 0 && aligned(a.q, 16) && aligned(a.k, 16) && aligned(a.v, 16);
+    return vec ? launch_gated<RG, T, true>(a, s) : launch_gated<RG, T, false>(a, s);
+}
+
 template <typename T> int dispatch_gated(const ss::GatedArgs &a, cudaStream_t s)
 {
     if (a.dk <= 32)
-        return launch_gated<4, T>(a, s);
+        return dispatch_gated_v<4, T>(a, s);
     if (a.dk <= 64)
-        return launch_gated<8, T>(a, s);
-    return launch_gated<16, T>(a, s);
+        return dispatch_gated_v<8, T>(a, s);
+    return dispatch_gated_v<16, T>(a, s);
 }
 
 } // namespace

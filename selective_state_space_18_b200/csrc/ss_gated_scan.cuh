@@ -59,8 +59,31 @@ template <> __device__ __forceinline__ float gload<__nv_bfloat16>(const __nv_bfl
     return __bfloat162float(__ldg(p + i));
 }
 
-template <int RG, typename T>
-__global__ void __launch_bounds__(kGThreads) ss_gated_scan_kernel(const GatedArgs p)
+// Eight consecutive elements of a q, k or v row as fp32, from one 16-byte load (bf16)
+// or two (fp32).
+template <typename T> __device__ __forceinline__ void load8(const T *src, float (&o)[8]);
+template <> __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *src, float (&o)[8])
+{
+    const uint4 w = __ldg(reinterpret_cast<const uint4 *>(src));
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        o[2 * h] = __uint_as_float(u[h] << 16);
+        o[2 * h + 1] = __uint_as_float(u[h] & 0xffff0000u);
+    }
+}
+template <> __device__ __forceinline__ void load8<float>(const float *src, float (&o)[8])
+{
+    const float4 a = __ldg(reinterpret_cast<const float4 *>(src)), b = __ldg(reinterpret_cast<const float4 *>(src) + 1);
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+    o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+
+// VEC: dk equals the padded row count and dv is a multiple of 8, with 16-byte aligned
+// rows, so a chunk is staged with 8-element vector loads (a few per thread) instead
+// of one scalar load per element.
+template <int RG, typename T, bool VEC>
+__global__ void __launch_bounds__(kGThreads, 4) ss_gated_scan_kernel(const GatedArgs p)
 {
     using G = GatedShape<RG>;
     extern __shared__ __align__(16) float gsm[];
@@ -91,7 +114,42 @@ __global__ void __launch_bounds__(kGThreads) ss_gated_scan_kernel(const GatedArg
     for (int64_t t0 = 0; t0 < p.seq; t0 += kGChunk) {
         const int nt = p.seq - t0 < kGChunk ? int(p.seq - t0) : kGChunk;
         __syncthreads(); // the previous chunk's staging and partials are consumed
-        for (int e = tid; e < kGChunk * G::kRows; e += kGThreads) {
+        if constexpr (VEC) {
+            for (int e8 = tid; e8 < kGChunk * G::kRows / 8; e8 += kGThreads) {
+                const int t = (8 * e8) / G::kRows, i = (8 * e8) % G::kRows;
+                const int pos = t * G::kRowStride + G::row_pos(i);
+                float a[8], c[8];
+                if (t < nt) {
+                    load8<T>(q + (t0 + t) * p.dk + i, a);
+                    load8<T>(k + (t0 + t) * p.dk + i, c);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        a[u] = c[u] = 0.f;
+                }
+                float4 *dq = reinterpret_cast<float4 *>(gsm + G::kQOff + pos);
+                float4 *dk4 = reinterpret_cast<float4 *>(gsm + G::kKOff + pos);
+                dq[0] = make_float4(a[0], a[1], a[2], a[3]);
+                dq[1] = make_float4(a[4], a[5], a[6], a[7]);
+                dk4[0] = make_float4(c[0], c[1], c[2], c[3]);
+                dk4[1] = make_float4(c[4], c[5], c[6], c[7]);
+            }
+            for (int e8 = tid; e8 < kGChunk * G::kCols / 8; e8 += kGThreads) {
+                const int t = (8 * e8) / G::kCols, cc = (8 * e8) % G::kCols;
+                float a[8];
+                if (t < nt && j0 + cc < p.dv) {
+                    load8<T>(v + (t0 + t) * p.dv + j0 + cc, a);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        a[u] = 0.f;
+                }
+                float4 *dv4 = reinterpret_cast<float4 *>(gsm + G::kVOff + 8 * e8);
+                dv4[0] = make_float4(a[0], a[1], a[2], a[3]);
+                dv4[1] = make_float4(a[4], a[5], a[6], a[7]);
+            }
+        }
+        for (int e = tid; e < (VEC ? 0 : kGChunk * G::kRows); e += kGThreads) {
             const int t = e / G::kRows, i = e % G::kRows;
             const bool in = t < nt && i < p.dk;
             const int64_t off = (t0 + t) * p.dk + i;
@@ -99,7 +157,7 @@ __global__ void __launch_bounds__(kGThreads) ss_gated_scan_kernel(const GatedArg
             gsm[G::kQOff + pos] = in ? gload<T>(q, off) : 0.f;
             gsm[G::kKOff + pos] = in ? gload<T>(k, off) : 0.f;
         }
-        for (int e = tid; e < kGChunk * G::kCols; e += kGThreads) {
+        for (int e = tid; e < (VEC ? 0 : kGChunk * G::kCols); e += kGThreads) {
             const int t = e / G::kCols, c = e % G::kCols;
             const bool in = t < nt && j0 + c < p.dv;
             gsm[G::kVOff + e] = in ? gload<T>(v, (t0 + t) * p.dv + j0 + c) : 0.f;
@@ -134,16 +192,24 @@ __global__ void __launch_bounds__(kGThreads) ss_gated_scan_kernel(const GatedArg
             pp[1] = make_float4(acc[2].x, acc[2].y, acc[3].x, acc[3].y);
         }
         __syncthreads();
-        // outputs of the chunk: the sum over row groups, in index order
-        for (int e = tid; e < nt * G::kCols; e += kGThreads) {
-            const int t = e / G::kCols, c = e % G::kCols;
-            if (j0 + c >= p.dv)
-                continue;
-            float s = 0.f;
+        // outputs of the chunk, four columns per thread: the sum over row groups
+        for (int e = tid; e < nt * (G::kCols / 4); e += kGThreads) {
+            const int t = e / (G::kCols / 4), c4 = 4 * (e % (G::kCols / 4));
+            float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int g2 = 0; g2 < RG; ++g2)
-                s += gsm[G::kPOff + (t * RG + g2) * G::kPStride + c];
-            Elem<T>::store(static_cast<T *>(p.y) + (b * p.seq + t0 + t) * p.dv + j0 + c, s);
+            for (int g2 = 0; g2 < RG; ++g2) {
+                const float4 v4 = *reinterpret_cast<const float4 *>(gsm + G::kPOff + (t * RG + g2) * G::kPStride + c4);
+                s4.x += v4.x;
+                s4.y += v4.y;
+                s4.z += v4.z;
+                s4.w += v4.w;
+            }
+            T *yr = static_cast<T *>(p.y) + (b * p.seq + t0 + t) * p.dv + j0 + c4;
+            const float o[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (j0 + c4 + u < p.dv)
+                    Elem<T>::store(yr + u, o[u]);
         }
     }
     // the final state, in the dtype of q
