@@ -510,7 +510,7 @@ template <int RG, typename T, bool VEC> int launch_gated(ss::GatedArgs a, cudaSt
     int64_t grid = 0;
     if (!mul_ok(a.batch, a.col_tiles, &grid) || grid > 0x7fffffffLL)
         return SS_ERR_SHAPE;
-    kernel<<<unsigned(grid), ss::kGThreads, G::kSmem, stream>>>(a);
+    kernel<<<unsigned(grid), G::kThreads, G::kSmem, stream>>>(a);
     return launch_status();
 }
 

@@ -6,7 +6,7 @@
 // each state starting at zero (or at an optional h0), outputs and the final state
 // cast to the dtype of q, all intermediate arithmetic in fp32.
 //
-// Work split.  A CTA owns one batch item and a tile of value columns; thread
+// Work split.  A CTA owns one batch item and a tile of 64 value columns; thread
 // (rg, cg) keeps the 8 x 8 block S[8 rg .. 8 rg + 8, 8 cg .. 8 cg + 8] in registers
 // for the whole sequence.  Tokens are staged in chunks of kGChunk through shared
 // memory as fp32 (q and k rows, the tile's v columns, gamma).  Per token a thread
@@ -30,14 +30,15 @@ struct GatedArgs {
     int col_tiles;           // value-column tiles per batch item
 };
 
-constexpr int kGChunk = 8;       // tokens staged per round
-constexpr int kGThreads = 128;
+constexpr int kGChunk = 8; // tokens staged per round
+constexpr int kGCols = 64; // value columns per CTA
 
-// RG row groups of 8 rows (Dk <= 8 RG) and 128 / RG column groups of 8 columns.
+// RG row groups of 8 rows (Dk <= 8 RG) and 8 column groups of 8 columns: 8 RG threads.
 template <int RG> struct GatedShape {
     static constexpr int kRows = 8 * RG;                 // padded Dk
-    static constexpr int kCG = kGThreads / RG;
-    static constexpr int kCols = 8 * kCG;                // value columns per CTA
+    static constexpr int kCG = kGCols / 8;
+    static constexpr int kCols = kGCols;
+    static constexpr int kThreads = RG * kCG;
     // shared memory (floats): q, k [chunk][kRowStride]; v [chunk][kCols]; gamma
     // [chunk]; partial readouts [chunk][RG][kPStride].  Rows are padded by 4 floats
     // every 32 (and partial rows by 4) so the row groups a warp reads or writes at once
@@ -83,7 +84,8 @@ template <> __device__ __forceinline__ void load8<float>(const float *src, float
 // rows, so a chunk is staged with 8-element vector loads (a few per thread) instead
 // of one scalar load per element.
 template <int RG, typename T, bool VEC>
-__global__ void __launch_bounds__(kGThreads, 4) ss_gated_scan_kernel(const GatedArgs p)
+__global__ void __launch_bounds__(GatedShape<RG>::kThreads, 512 / GatedShape<RG>::kThreads)
+ss_gated_scan_kernel(const GatedArgs p)
 {
     using G = GatedShape<RG>;
     extern __shared__ __align__(16) float gsm[];
@@ -115,7 +117,7 @@ __global__ void __launch_bounds__(kGThreads, 4) ss_gated_scan_kernel(const Gated
         const int nt = p.seq - t0 < kGChunk ? int(p.seq - t0) : kGChunk;
         __syncthreads(); // the previous chunk's staging and partials are consumed
         if constexpr (VEC) {
-            for (int e8 = tid; e8 < kGChunk * G::kRows / 8; e8 += kGThreads) {
+            for (int e8 = tid; e8 < kGChunk * G::kRows / 8; e8 += G::kThreads) {
                 const int t = (8 * e8) / G::kRows, i = (8 * e8) % G::kRows;
                 const int pos = t * G::kRowStride + G::row_pos(i);
                 float a[8], c[8];
@@ -134,7 +136,7 @@ __global__ void __launch_bounds__(kGThreads, 4) ss_gated_scan_kernel(const Gated
                 dk4[0] = make_float4(c[0], c[1], c[2], c[3]);
                 dk4[1] = make_float4(c[4], c[5], c[6], c[7]);
             }
-            for (int e8 = tid; e8 < kGChunk * G::kCols / 8; e8 += kGThreads) {
+            for (int e8 = tid; e8 < kGChunk * G::kCols / 8; e8 += G::kThreads) {
                 const int t = (8 * e8) / G::kCols, cc = (8 * e8) % G::kCols;
                 float a[8];
                 if (t < nt && j0 + cc < p.dv) {
@@ -149,7 +151,7 @@ __global__ void __launch_bounds__(kGThreads, 4) ss_gated_scan_kernel(const Gated
                 dv4[1] = make_float4(a[4], a[5], a[6], a[7]);
             }
         }
-        for (int e = tid; e < (VEC ? 0 : kGChunk * G::kRows); e += kGThreads) {
+        for (int e = tid; e < (VEC ? 0 : kGChunk * G::kRows); e += G::kThreads) {
             const int t = e / G::kRows, i = e % G::kRows;
             const bool in = t < nt && i < p.dk;
             const int64_t off = (t0 + t) * p.dk + i;
@@ -157,7 +159,7 @@ __global__ void __launch_bounds__(kGThreads, 4) ss_gated_scan_kernel(const Gated
             gsm[G::kQOff + pos] = in ? gload<T>(q, off) : 0.f;
             gsm[G::kKOff + pos] = in ? gload<T>(k, off) : 0.f;
         }
-        for (int e = tid; e < (VEC ? 0 : kGChunk * G::kCols); e += kGThreads) {
+        for (int e = tid; e < (VEC ? 0 : kGChunk * G::kCols); e += G::kThreads) {
             const int t = e / G::kCols, c = e % G::kCols;
             const bool in = t < nt && j0 + c < p.dv;
             gsm[G::kVOff + e] = in ? gload<T>(v, (t0 + t) * p.dv + j0 + c) : 0.f;
@@ -193,7 +195,7 @@ __global__ void __launch_bounds__(kGThreads, 4) ss_gated_scan_kernel(const Gated
         }
         __syncthreads();
         // outputs of the chunk, four columns per thread: the sum over row groups
-        for (int e = tid; e < nt * (G::kCols / 4); e += kGThreads) {
+        for (int e = tid; e < nt * (G::kCols / 4); e += G::kThreads) {
             const int t = e / (G::kCols / 4), c4 = 4 * (e % (G::kCols / 4));
             float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
