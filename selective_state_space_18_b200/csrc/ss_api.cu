@@ -415,10 +415,10 @@ int scan_impl(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, s
     if (flags & ~uint32_t(SS_DT_SOFTPLUS))
         return SS_ERR_UNSUPPORTED;
     const size_t es = dtype == SS_BF16 ? 2 : 4;
-    int64_t rows = 0, elems = 0, bcel = 0, stel = 0, rsel = 0;
-    if (!mul_ok(batch, channels, &rows) || !mul_ok(rows, seq, &elems) ||
-        !mul_ok(batch * state_dim, seq, &bcel) || !mul_ok(rows, state_dim, &stel) ||
-        !mul_ok(batch, seq, &rsel) || elems > (INT64_MAX / 8))
+    int64_t rows = 0, elems = 0, bn = 0, bcel = 0, stel = 0, rsel = 0;
+    if (!mul_ok(batch, channels, &rows) || !mul_ok(rows, seq, &elems) || !mul_ok(batch, state_dim, &bn) ||
+        !mul_ok(bn, seq, &bcel) || !mul_ok(rows, state_dim, &stel) || !mul_ok(batch, seq, &rsel) ||
+        elems > (INT64_MAX / 8) || bcel > (INT64_MAX / 8) || stel > (INT64_MAX / 8))
         return SS_ERR_SHAPE;
     const void *typed[] = {x, dt_raw, B, C, z, y};
     for (const void *p : typed)
@@ -548,9 +548,9 @@ int ss_gated_scan(int64_t batch, int64_t seq, int64_t dk, int64_t dv, ss_dtype_t
     if (dk > 128)
         return SS_ERR_UNSUPPORTED;
     const size_t es = dtype == SS_BF16 ? 2 : 4;
-    int64_t bs = 0, qel = 0, vel = 0, sel = 0;
-    if (!mul_ok(batch, seq, &bs) || !mul_ok(bs, dk, &qel) || !mul_ok(bs, dv, &vel) ||
-        !mul_ok(batch * dk, dv, &sel) || qel > (INT64_MAX / 8) || vel > (INT64_MAX / 8))
+    int64_t bs = 0, qel = 0, vel = 0, bk = 0, sel = 0;
+    if (!mul_ok(batch, seq, &bs) || !mul_ok(bs, dk, &qel) || !mul_ok(bs, dv, &vel) || !mul_ok(batch, dk, &bk) ||
+        !mul_ok(bk, dv, &sel) || qel > (INT64_MAX / 8) || vel > (INT64_MAX / 8) || sel > (INT64_MAX / 8))
         return SS_ERR_SHAPE;
     const void *typed[] = {q, k, v, outputs, final_state};
     for (const void *p : typed)

@@ -210,3 +210,13 @@ def test_gated_scan_checks(lib):
     assert call(q=ctypes.c_void_p(P[0].value + 1)) == "SS_ERR_ALIGN"
     assert call(y=ctypes.c_void_p(P[1].value + 64)) == "SS_ERR_ALIAS"
     assert call(fs=ctypes.c_void_p(P[4].value)) == "SS_ERR_ALIAS"
+
+
+def test_huge_shapes_are_refused_without_overflow(lib):
+    """Products of sizes that overflow 64 bits are refused before any pointer is used."""
+    assert _scan(lib, batch=1 << 60, channels=1, seq=64) == 2
+    assert _scan(lib, batch=1 << 59, channels=2, seq=1) == 2
+    st = lib.ss_gated_scan(1 << 58, 1, 128, 64, ssscan.SS_BF16, P[0], P[1], P[2], P[3], None, P[4], P[5], None)
+    assert ssscan.STATUS[st] == "SS_ERR_SHAPE"
+    st = lib.ss_gated_scan(1, 1 << 60, 64, 64, ssscan.SS_BF16, P[0], P[1], P[2], P[3], None, P[4], P[5], None)
+    assert ssscan.STATUS[st] == "SS_ERR_SHAPE"
