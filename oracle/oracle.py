@@ -55,6 +55,8 @@ def _load():
             lib.ss_oracle_update.argtypes = [_i64, _i64, _i64, _dp] + [_dp] * 8 + [
                 ctypes.c_int, _dp, ctypes.c_int]
             lib.ss_oracle_update.restype = ctypes.c_int
+            lib.ss_oracle_conv_silu.argtypes = [_i64, _i64, _i64, _i64] + [_dp] * 6 + [ctypes.c_int]
+            lib.ss_oracle_conv_silu.restype = ctypes.c_int
             lib.ss_oracle_gated_scan.argtypes = [_i64, _i64, _i64, _i64] + [_dp] * 7 + [ctypes.c_int]
             lib.ss_oracle_gated_scan.restype = ctypes.c_int
             lib.ss_oracle_num_threads.argtypes = []
@@ -170,6 +172,26 @@ def update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, *, dt_softplus=T
                               int(bool(dt_softplus)), _ptr(y), int(nthreads or num_threads()))
     _check(rc, "ss_oracle_update")
     return {"y": y, "state": st_arr}
+
+
+def conv_silu(u, w, cb=None, state=None, *, nthreads=None):
+    """Causal depthwise conv + SiLU oracle (TransformerLens ssm_mixer: the scan's x is
+    SiLU of the conv1d output).  u [b, c, L]; w [c, K]; cb [c] or None; state [b, c, K-1]
+    (the inputs before u, oldest first) or None.  Returns dict(x [b, c, L],
+    state [b, c, K-1] = the last K-1 inputs of state ++ u)."""
+    u, w, cb, state = _f64(u), _f64(w), _f64(cb), _f64(state)
+    bt, ch, L = u.shape
+    K = w.shape[1]
+    if w.shape != (ch, K) or (cb is not None and cb.shape != (ch,)):
+        raise ValueError("inconsistent conv shapes")
+    if state is not None and state.shape != (bt, ch, K - 1):
+        raise ValueError("state must be [b, c, K-1]")
+    x = np.empty((bt, ch, L))
+    so = np.empty((bt, ch, K - 1))
+    rc = _load().ss_oracle_conv_silu(bt, ch, L, K, _ptr(u), _ptr(w), _ptr(cb), _ptr(state), _ptr(x), _ptr(so),
+                                     int(nthreads or num_threads()))
+    _check(rc, "ss_oracle_conv_silu")
+    return {"x": x, "state": so}
 
 
 def gated_scan(q, k, v, gamma, h0=None, *, nthreads=None):

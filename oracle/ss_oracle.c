@@ -340,3 +340,48 @@ int ss_oracle_gated_scan(int64_t batch, int64_t seq, int64_t dk, int64_t dv, con
     (void)nthreads;
     return failed ? ORC_ERR_NOMEM : ORC_OK;
 }
+
+/*
+ * Causal depthwise convolution followed by SiLU, the step that produces the scan's x
+ * (TransformerLens docs, ssm_mixer: "x is the post-conv SiLU input", SiLU(conv1d
+ * output)).  Per row (b, c) with K taps w[c, 0..K-1] and bias cb[c]:
+ *
+ *   x[b,c,t] = silu( cb[c] + sum_{k<K} w[c,k] * u[b,c,t-K+1+k] )
+ *
+ * where u at t < 0 is taken from state_in[b,c,K-1+t] (the K-1 inputs that preceded
+ * this call, oldest first; zeros when state_in is NULL).  state_out[b,c,:] receives
+ * the last K-1 inputs of the concatenation state_in ++ u (oldest first).  Layouts:
+ * u, x [batch, channels, seq]; w [channels, K]; cb [channels]; state_in, state_out
+ * [batch, channels, K-1].  The sum runs over k in index order.
+ */
+int ss_oracle_conv_silu(int64_t batch, int64_t channels, int64_t seq, int64_t K, const double *u,
+                        const double *w, const double *cb, const double *state_in, double *x,
+                        double *state_out, int nthreads)
+{
+    if (!u || !w || !x)
+        return ORC_ERR_NULL;
+    if (batch <= 0 || channels <= 0 || seq <= 0 || K <= 0)
+        return ORC_ERR_SHAPE;
+    const int64_t rows = batch * channels, H = K - 1;
+#ifdef _OPENMP
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+#endif
+    for (int64_t r = 0; r < rows; ++r) {
+        const int64_t c = r % channels;
+        const double *ur = u + r * seq;
+        /* input at position t of the concatenation: t < 0 reads the state */
+#define ORC_IN(t) ((t) >= 0 ? ur[(t)] : (state_in ? state_in[r * H + H + (t)] : 0.0))
+        for (int64_t t = 0; t < seq; ++t) {
+            double acc = cb ? cb[c] : 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += w[c * K + k] * ORC_IN(t - K + 1 + k);
+            x[r * seq + t] = orc_silu(acc);
+        }
+        if (state_out)
+            for (int64_t j = 0; j < H; ++j)
+                state_out[r * H + j] = ORC_IN(seq - H + j);
+#undef ORC_IN
+    }
+    (void)nthreads;
+    return ORC_OK;
+}
