@@ -125,6 +125,38 @@ SS_API int ss_scan_fwd_states(int64_t batch, int64_t channels, int64_t state_dim
                               uint32_t flags, void *y, float *h_last, float *h_all,
                               void *workspace, size_t workspace_bytes, ss_stream_t stream);
 
+/*
+ * ss_scan_fwd with the causal depthwise convolution and SiLU that produce its input
+ * fused in front (TransformerLens ssm_mixer: the scan's x is SiLU of the conv1d
+ * output; a decode step carries the conv's recent inputs as its state):
+ *
+ *   x[b,c,t] = silu( conv_b[c] + sum_{k<conv_k} conv_w[c,k] * u[b,c,t-conv_k+1+k] )
+ *
+ * with u before t = 0 read from conv_state, and then the scan of ss_scan_fwd on x.
+ *
+ *   u              : [batch, channels, seq] dtype (the conv input; takes x's place)
+ *   conv_w         : [channels, conv_k] float32, conv_k in 1..4
+ *   conv_b         : [channels] float32 (nullable: 0)
+ *   conv_state     : [batch, channels, conv_k-1] float32 (nullable: zeros), the inputs
+ *                    that preceded u, oldest first
+ *   conv_state_out : [batch, channels, conv_k-1] float32 (nullable output), the last
+ *                    conv_k-1 inputs of conv_state ++ u, for the next call
+ *   x_out          : [batch, channels, seq] dtype (nullable output), x itself
+ *
+ * The other arguments are those of ss_scan_fwd.  SiLU of x is evaluated like the
+ * output gate (exact for float32 storage; the MUFU tanh form for bfloat16, within the
+ * bfloat16 tolerance).  No output may overlap an input or another output
+ * (SS_ERR_ALIAS).
+ */
+SS_API int ss_scan_fwd_conv(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
+                            ss_dtype_t dtype, const void *u, const float *conv_w,
+                            const float *conv_b, int64_t conv_k, const float *conv_state,
+                            float *conv_state_out, void *x_out, const void *dt_raw,
+                            const float *A, const void *B, const void *C, const float *D,
+                            const void *z, const float *dt_bias, const uint8_t *reset,
+                            const float *h0, uint32_t flags, void *y, float *h_last,
+                            void *workspace, size_t workspace_bytes, ss_stream_t stream);
+
 /* Workspace bytes ss_scan_fwd needs for this shape (0 for an invalid shape). */
 SS_API int64_t ss_scan_workspace_bytes(int64_t batch, int64_t channels, int64_t state_dim,
                                        int64_t seq);

@@ -142,12 +142,12 @@ bool build_maps(const ss::ScanArgs &a, ss::TmaMaps *m)
            encode_rows<T>(&m->C, a.C, a.seq, brows, S::kChunk, N, bc_swizzle);
 }
 
-template <int N, typename T, bool R, bool V, bool E>
+template <int N, typename T, bool R, bool V, bool E, bool C>
 int launch_scan(ss::ScanArgs a, cudaStream_t stream)
 {
     using S = ss::ScanShape<N>;
     constexpr size_t kSmem = S::template smem_bytes<T, V>();
-    auto kernel = ss::ss_scan_fwd_kernel<N, T, R, V, E>;
+    auto kernel = ss::ss_scan_fwd_kernel<N, T, R, V, E, C>;
     static std::atomic<uint64_t> smem_done{0};
     static std::atomic<int> occ_cache[64];
     int st = ensure_smem(kernel, kSmem, smem_done);
@@ -194,19 +194,22 @@ int launch_scan(ss::ScanArgs a, cudaStream_t stream)
     return launch_status();
 }
 
-template <int N, typename T, bool E>
+template <int N, typename T, bool E, bool C>
 int dispatch_scan_e(const ss::ScanArgs &a, bool vec, cudaStream_t s)
 {
     const bool r = a.reset != nullptr;
     if (r)
-        return vec ? launch_scan<N, T, true, true, E>(a, s) : launch_scan<N, T, true, false, E>(a, s);
-    return vec ? launch_scan<N, T, false, true, E>(a, s) : launch_scan<N, T, false, false, E>(a, s);
+        return vec ? launch_scan<N, T, true, true, E, C>(a, s) : launch_scan<N, T, true, false, E, C>(a, s);
+    return vec ? launch_scan<N, T, false, true, E, C>(a, s) : launch_scan<N, T, false, false, E, C>(a, s);
 }
 
+// forms: plain; with per-token states (E); with the fused conv prologue (C)
 template <int N, typename T>
 int dispatch_scan_t(const ss::ScanArgs &a, bool vec, cudaStream_t s)
 {
-    return a.h_all ? dispatch_scan_e<N, T, true>(a, vec, s) : dispatch_scan_e<N, T, false>(a, vec, s);
+    if (a.conv_w)
+        return dispatch_scan_e<N, T, false, true>(a, vec, s);
+    return a.h_all ? dispatch_scan_e<N, T, true, false>(a, vec, s) : dispatch_scan_e<N, T, false, false>(a, vec, s);
 }
 
 template <int N> int64_t scan_groups(int64_t batch, int64_t channels)
@@ -398,11 +401,19 @@ namespace {
 
 // ss_scan_fwd and ss_scan_fwd_states: validation, then the launch.  h_all (nullable)
 // receives the state after every token.
+// Fused conv prologue of ss_scan_fwd_conv (w NULL: none); x is then the conv input.
+struct ConvArgs {
+    const float *w = nullptr, *b = nullptr, *state = nullptr;
+    float *state_out = nullptr;
+    void *x_out = nullptr;
+    int k = 0;
+};
+
 int scan_impl(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, ss_dtype_t dtype,
               const void *x, const void *dt_raw, const float *A, const void *B, const void *C,
               const float *D, const void *z, const float *dt_bias, const uint8_t *reset,
               const float *h0, uint32_t flags, void *y, float *h_last, float *h_all, void *workspace,
-              size_t workspace_bytes, ss_stream_t stream)
+              size_t workspace_bytes, ss_stream_t stream, const ConvArgs &cv = ConvArgs())
 {
     if (!x || !dt_raw || !A || !B || !C || !y)
         return SS_ERR_NULL;
@@ -458,6 +469,35 @@ int scan_impl(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, s
         if (overlaps(h_all, abytes, y, ybytes) || (h_last && overlaps(h_all, abytes, h_last, hbytes)))
             return SS_ERR_ALIAS;
     }
+    size_t cbytes = 0; // conv state
+    if (cv.w) {
+        if (cv.k < 1 || cv.k > 4 || h_all)
+            return SS_ERR_UNSUPPORTED;
+        const float *f32c[] = {cv.w, cv.b, cv.state, cv.state_out};
+        for (const float *q : f32c)
+            if (q && !aligned(q, 4))
+                return SS_ERR_ALIGN;
+        if (cv.x_out && !aligned(cv.x_out, es))
+            return SS_ERR_ALIGN;
+        cbytes = size_t(rows) * size_t(cv.k - 1) * 4;
+        const size_t wbytes = size_t(channels) * size_t(cv.k) * 4;
+        const void *cin[] = {cv.w, cv.b, cv.state};
+        const size_t cin_n[] = {wbytes, cv.b ? size_t(channels) * 4 : 0, cv.state ? cbytes : 0};
+        // the outputs (y, h_last, x_out, state_out) overlap no input and no other output
+        const void *outs[] = {y, h_last, cv.x_out, cv.state_out};
+        const size_t out_n[] = {ybytes, h_last ? hbytes : 0, cv.x_out ? ybytes : 0, cv.state_out ? cbytes : 0};
+        for (int o = 0; o < 4; ++o) {
+            for (int i = 0; i < 10; ++i)
+                if (!(o == 1 && i == 9 && in_p[i] == h_last) && overlaps(outs[o], out_n[o], in_p[i], in_n[i]))
+                    return SS_ERR_ALIAS;
+            for (int i = 0; i < 3; ++i)
+                if (overlaps(outs[o], out_n[o], cin[i], cin_n[i]))
+                    return SS_ERR_ALIAS;
+            for (int o2 = o + 1; o2 < 4; ++o2)
+                if (overlaps(outs[o], out_n[o], outs[o2], out_n[o2]))
+                    return SS_ERR_ALIAS;
+        }
+    }
     if (workspace) {
         if (!aligned(workspace, 16))
             return SS_ERR_ALIGN;
@@ -466,7 +506,9 @@ int scan_impl(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, s
                 return SS_ERR_ALIAS;
         if (overlaps(workspace, workspace_bytes, y, ybytes) ||
             (h_last && overlaps(workspace, workspace_bytes, h_last, hbytes)) ||
-            (h_all && overlaps(workspace, workspace_bytes, h_all, abytes)))
+            (h_all && overlaps(workspace, workspace_bytes, h_all, abytes)) ||
+            (cv.x_out && overlaps(workspace, workspace_bytes, cv.x_out, ybytes)) ||
+            (cv.state_out && overlaps(workspace, workspace_bytes, cv.state_out, cbytes)))
             return SS_ERR_ALIAS;
     }
 
@@ -477,6 +519,8 @@ int scan_impl(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, s
     for (const void *p : typed)
         if (p && !aligned(p, 16))
             vec = false;
+    if (cv.x_out && !aligned(cv.x_out, 16))
+        vec = false;
 
     ss::ScanArgs a{};
     a.batch = batch;
@@ -488,6 +532,12 @@ int scan_impl(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, s
     a.y = y;
     a.h_last = h_last;
     a.h_all = h_all;
+    a.conv_w = cv.w;
+    a.conv_b = cv.b;
+    a.conv_state = cv.state;
+    a.conv_state_out = cv.state_out;
+    a.x_out = cv.x_out;
+    a.conv_k = cv.k;
     a.softplus = (flags & SS_DT_SOFTPLUS) ? 1 : 0;
     a.workspace = static_cast<uint8_t *>(workspace);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -589,6 +639,28 @@ int ss_scan_fwd(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
 {
     return scan_impl(batch, channels, state_dim, seq, dtype, x, dt_raw, A, B, C, D, z, dt_bias, reset, h0, flags, y,
                      h_last, nullptr, workspace, workspace_bytes, stream);
+}
+
+int ss_scan_fwd_conv(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, ss_dtype_t dtype,
+                     const void *u, const float *conv_w, const float *conv_b, int64_t conv_k,
+                     const float *conv_state, float *conv_state_out, void *x_out, const void *dt_raw,
+                     const float *A, const void *B, const void *C, const float *D, const void *z,
+                     const float *dt_bias, const uint8_t *reset, const float *h0, uint32_t flags, void *y,
+                     float *h_last, void *workspace, size_t workspace_bytes, ss_stream_t stream)
+{
+    if (!conv_w)
+        return SS_ERR_NULL;
+    if (conv_k < 1 || conv_k > 4)
+        return SS_ERR_UNSUPPORTED;
+    ConvArgs cv;
+    cv.w = conv_w;
+    cv.b = conv_b;
+    cv.state = conv_state;
+    cv.state_out = conv_state_out;
+    cv.x_out = x_out;
+    cv.k = int(conv_k);
+    return scan_impl(batch, channels, state_dim, seq, dtype, u, dt_raw, A, B, C, D, z, dt_bias, reset, h0, flags, y,
+                     h_last, nullptr, workspace, workspace_bytes, stream, cv);
 }
 
 int ss_scan_fwd_states(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, ss_dtype_t dtype,

@@ -47,6 +47,13 @@ struct ScanArgs {
     void *y;
     float *h_last;
     float *h_all;             // nullable: the state after every token [b, c, L, N] fp32
+    // fused causal conv + SiLU prologue (x above is then the conv's input u):
+    const float *conv_w;      // [channels, conv_k] taps
+    const float *conv_b;      // [channels] bias (nullable)
+    const float *conv_state;  // [b, c, conv_k - 1] inputs before the sequence (nullable: 0)
+    float *conv_state_out;    // [b, c, conv_k - 1] the last conv_k - 1 inputs (nullable)
+    void *x_out;              // [b, c, L] the scan input x = silu(conv) (nullable)
+    int conv_k;               // taps, 1..4
     int softplus;
     int64_t groups_per_batch; // channel groups per batch row
     int64_t groups;           // batch * groups_per_batch
@@ -102,8 +109,11 @@ template <int N> struct ScanShape {
     // output stage (floats): meta | partial outputs
     static constexpr int kYChan = kPairs * kRow + 4;   // per-channel block, bank-skewed
     static constexpr int kYPOff = kMeta;
-    static constexpr int kYStage = kYPOff + kChanPerCta * kYChan;
-    static constexpr int kFloats = kStages * kInStage + kYStages * kYStage;
+    // then x of the chunk in storage type [channels][chunk] (the fused conv form hands
+    // it from the producers to the epilogue here)
+    static constexpr int kYXOff = kYPOff + kChanPerCta * kYChan;
+    template <typename T> static constexpr int y_stage() { return kYXOff + kChanPerCta * kChunk * int(sizeof(T)) / 4; }
+    template <typename T> static constexpr int floats() { return kStages * kInStage + kYStages * y_stage<T>(); }
     // IO work per chunk
     static constexpr int kTokTasks = kChanPerCta * kBlocks;       // (channel, 8 tokens)
     static constexpr int kTokPerLane = kTokTasks / kIoThreads;
@@ -136,11 +146,11 @@ template <int N> struct ScanShape {
     // shared memory: [raw ring] [input stages] [output stages] [barriers] [raw meta]
     template <typename T, bool TMA> static constexpr size_t smem_bytes()
     {
-        return size_t(kRawStages * raw_stage_bytes<T>()) + size_t(kFloats) * 4 + 8 * size_t(kBars) +
+        return size_t(kRawStages * raw_stage_bytes<T>()) + size_t(floats<T>()) * 4 + 8 * size_t(kBars) +
                32 * size_t(kRawStages);
     }
     static_assert(kTokTasks % kIoThreads == 0, "token tasks fill whole IO lanes");
-    static_assert(kInStage % 4 == 0 && kYStage % 4 == 0, "16-byte aligned stages");
+    static_assert(kInStage % 4 == 0 && kYXOff % 4 == 0, "16-byte aligned stages");
 };
 
 struct ChunkMeta {
@@ -242,7 +252,7 @@ __device__ __forceinline__ float2 softplus_poly2(float2 r)
 // producer warp: global -> registers (one chunk ahead) -> shared-memory stage
 // ---------------------------------------------------------------------------------------
 
-template <int N, typename T, bool HAS_RESET, bool VEC>
+template <int N, typename T, bool HAS_RESET, bool VEC, bool CONV>
 struct IoPrefetch {
     using S = ScanShape<N>;
     Raw8<T> bc[S::kBCPerLane];
@@ -250,6 +260,10 @@ struct IoPrefetch {
     float bias[S::kTokPerLane];
     int64_t bias_g = -1; // channel group whose dt_bias values `bias` holds
     uint32_t rbyte;
+    // fused conv: taps and bias of each task's channel (cached with dt_bias), and the
+    // three conv inputs before each task's first token
+    float cw[CONV ? S::kTokPerLane : 1][4], cb[CONV ? S::kTokPerLane : 1];
+    float halo[CONV ? S::kTokPerLane : 1][3];
 
     __device__ __forceinline__ void load_bias(const ScanArgs &p, int lane, int64_t g)
     {
@@ -262,6 +276,15 @@ struct IoPrefetch {
             int64_t c = c0 + (lane + S::kIoThreads * m) / S::kBlocks;
             c = c < p.channels ? c : p.channels - 1;
             bias[m] = p.dt_bias ? __ldg(p.dt_bias + c) : 0.0f;
+            if constexpr (CONV) {
+                // taps aligned to the newest input: cw[m][3] multiplies u_t
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int kk = k - (4 - p.conv_k);
+                    cw[m][k] = kk >= 0 ? __ldg(p.conv_w + c * p.conv_k + kk) : 0.0f;
+                }
+                cb[m] = p.conv_b ? __ldg(p.conv_b + c) : 0.0f;
+            }
         }
     }
 
@@ -304,13 +327,45 @@ struct IoPrefetch {
             }
         }
         load_bias(p, lane, g);
+        if constexpr (CONV)
+            load_halo(p, lane, g, t0);
         if (HAS_RESET)
             rbyte = (lane < S::kChunk && t0 + lane < L) ? uint32_t(__ldg(p.reset + b * L + t0 + lane)) : 0u;
     }
 
+    // The three conv inputs before each task's first token t: u[t-3 .. t-1] from global
+    // memory (L2 hits: the same rows are being tiled in), or from the caller's conv
+    // state before the sequence start (zeros without one).
+    __device__ __forceinline__ void load_halo(const ScanArgs &p, int lane, int64_t g, int64_t t0)
+    {
+        const uint32_t gpb = uint32_t(p.groups_per_batch), b32 = uint32_t(g) / gpb;
+        const int64_t c0 = int64_t(uint32_t(g) - b32 * gpb) * S::kChanPerCta;
+        const int64_t H = p.conv_k - 1;
+#pragma unroll
+        for (int m = 0; m < S::kTokPerLane; ++m) {
+            const int q = lane + S::kIoThreads * m;
+            const int cl = q / S::kBlocks, tb = q % S::kBlocks;
+            int64_t c = c0 + cl;
+            c = c < p.channels ? c : p.channels - 1;
+            const int64_t row = int64_t(b32) * p.channels + c;
+            const int64_t t = t0 + tb * 8;
+#pragma unroll
+            for (int k = 0; k < 3; ++k) {
+                const int64_t pos = t - 3 + k;
+                float v = 0.0f;
+                if (pos >= 0)
+                    v = Elem<T>::load(static_cast<const T *>(p.x) + row * p.seq + pos);
+                else if (p.conv_state && H + pos >= 0)
+                    v = __ldg(p.conv_state + row * H + H + pos);
+                halo[m][k] = v;
+            }
+        }
+    }
+
     // x and dt_raw from a raw TMA stage (B and C stay in the stage for the scan
     // warps; the reset byte is loaded by the caller).
-    __device__ __forceinline__ void load_smem(const ScanArgs &p, int lane, int64_t g, const unsigned char *raw)
+    __device__ __forceinline__ void load_smem(const ScanArgs &p, int lane, int64_t g, const unsigned char *raw,
+                                              int64_t t0)
     {
         const T *rx = reinterpret_cast<const T *>(raw + S::template raw_x_off<T>());
         const T *rd = reinterpret_cast<const T *>(raw + S::template raw_dt_off<T>());
@@ -322,12 +377,32 @@ struct IoPrefetch {
             dr[m].load_smem(rd + cl * S::kChunk + tb * 8);
         }
         load_bias(p, lane, g);
+        if constexpr (CONV)
+            load_halo(p, lane, g, t0);
     }
 };
 
-template <int N, typename T, bool HAS_RESET, bool VEC>
-__device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane, const IoPrefetch<N, T, HAS_RESET, VEC> &f,
-                                              float *stage, unsigned char *raw, int64_t t0)
+// Eight values to shared memory in storage type (one 16-byte store for bf16).
+template <typename T> __device__ __forceinline__ void smem_store8(T *dst, const float (&o)[8]);
+template <> __device__ __forceinline__ void smem_store8<__nv_bfloat16>(__nv_bfloat16 *dst, const float (&o)[8])
+{
+    *reinterpret_cast<uint4 *>(dst) = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                                                 pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+}
+template <> __device__ __forceinline__ void smem_store8<float>(float *dst, const float (&o)[8])
+{
+    reinterpret_cast<float4 *>(dst)[0] = make_float4(o[0], o[1], o[2], o[3]);
+    reinterpret_cast<float4 *>(dst)[1] = make_float4(o[4], o[5], o[6], o[7]);
+}
+
+// CONV (fused causal conv + SiLU): x of each token is silu(cb + sum_k w_k u_{t-3+k})
+// from the task's eight inputs u (the raw x tile) and the three before them; x also
+// goes to the chunk's output stage (`ystage`, already free) for the epilogue, and the
+// last conv_k - 1 inputs of each row to conv_state_out.
+template <int N, typename T, bool HAS_RESET, bool VEC, bool CONV>
+__device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane,
+                                              const IoPrefetch<N, T, HAS_RESET, VEC, CONV> &f, float *stage,
+                                              unsigned char *raw, int64_t t0, int64_t g, float *ystage)
 {
     using S = ScanShape<N>;
     const int64_t L = p.seq;
@@ -355,6 +430,49 @@ __device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane, const
         const int q = lane + S::kIoThreads * m;
         const int cl = q / S::kBlocks, tb = q % S::kBlocks;
         const int64_t tl = t0 + tb * 8;
+        float xv[8];
+        if constexpr (CONV) {
+            float U[11];
+#pragma unroll
+            for (int k = 0; k < 3; ++k)
+                U[k] = f.halo[m][k];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                U[3 + j] = f.xr[m].get(j);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float acc = f.cb[m];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    acc = fmaf(f.cw[m][k], U[j + k], acc);
+                xv[j] = tl + j < L ? gate<T>(acc) : 0.0f;
+            }
+            smem_store8<T>(reinterpret_cast<T *>(ystage + S::kYXOff) + cl * S::kChunk + tb * 8, xv);
+            // the last conv_k - 1 inputs of the row (before the sequence start: from the
+            // conv state, for sequences shorter than the window)
+            const int64_t H = p.conv_k - 1;
+            if (p.conv_state_out && H > 0 && tl + 8 > L - H && tl <= L) {
+                const uint32_t gpb = uint32_t(p.groups_per_batch), b32 = uint32_t(g) / gpb;
+                const int64_t c = int64_t(uint32_t(g) - b32 * gpb) * S::kChanPerCta + cl;
+                if (c < p.channels) {
+                    const int64_t row = int64_t(b32) * p.channels + c;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int64_t pos = tl + j;
+                        if (pos >= L - H && pos < L)
+                            p.conv_state_out[row * H + (pos - (L - H))] = U[3 + j];
+                    }
+                    if (tl == 0)
+                        for (int64_t pos = L - H; pos < 0; ++pos)
+                            p.conv_state_out[row * H + (pos - (L - H))] =
+                                p.conv_state ? __ldg(p.conv_state + row * H + H + pos) : 0.0f;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                xv[j] = f.xr[m].get(j);
+        }
         float2 dtv[4], dxv[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -366,7 +484,7 @@ __device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane, const
                 d.y = (tl + 2 * k + 1 < L) ? d.y : 0.0f;
             }
             dtv[k] = d;
-            dxv[k] = __fmul2_rn(d, make_float2(f.xr[m].get(2 * k), f.xr[m].get(2 * k + 1)));
+            dxv[k] = __fmul2_rn(d, make_float2(xv[2 * k], xv[2 * k + 1]));
         }
         float4 *pd = reinterpret_cast<float4 *>(stage + S::kDTOff + cl * S::kRow + tb * 8);
         float4 *px = reinterpret_cast<float4 *>(stage + S::kDXOff + cl * S::kRow + tb * 8);
@@ -402,13 +520,16 @@ template <int N, typename T> struct EpiCache {
     const T *x[ScanShape<N>::kTokPerLane];
     const T *z[ScanShape<N>::kTokPerLane];
     T *y[ScanShape<N>::kTokPerLane];
+    T *xo[ScanShape<N>::kTokPerLane]; // fused conv form: rows of x_out (or null)
     float d[ScanShape<N>::kTokPerLane];
     int64_t g = -1;
 };
 
 // x and z are re-read from global memory (the producers' tile loads brought them into
 // L2 a few chunks earlier), issued first so their latency overlaps the partial sums.
-template <int N, typename T, bool VEC>
+// In the fused conv form x is not an input: the producers left it in the output
+// stage, and it is also stored to x_out when the caller asks for it.
+template <int N, typename T, bool VEC, bool CONV>
 __device__ __forceinline__ void epilogue_chunk(const ScanArgs &p, int lane, const float *ystage, int64_t g, int64_t t0,
                                                EpiCache<N, T> &ec)
 {
@@ -427,6 +548,7 @@ __device__ __forceinline__ void epilogue_chunk(const ScanArgs &p, int lane, cons
             ec.x[m] = static_cast<const T *>(p.x) + off;
             ec.z[m] = p.z ? static_cast<const T *>(p.z) + off : nullptr;
             ec.y[m] = valid ? static_cast<T *>(p.y) + off : nullptr;
+            ec.xo[m] = (CONV && valid && p.x_out) ? static_cast<T *>(p.x_out) + off : nullptr;
             ec.d[m] = p.D ? __ldg(p.D + c) : 0.0f;
         }
         ec.g = g;
@@ -434,8 +556,17 @@ __device__ __forceinline__ void epilogue_chunk(const ScanArgs &p, int lane, cons
     Raw8<T> xs[S::kTokPerLane], zs[S::kTokPerLane];
 #pragma unroll
     for (int m = 0; m < S::kTokPerLane; ++m) {
-        const int tb = (lane + S::kIoThreads * m) % S::kBlocks;
-        if (VEC) {
+        const int q = lane + S::kIoThreads * m;
+        const int tb = q % S::kBlocks;
+        if constexpr (CONV) {
+            xs[m].load_smem(reinterpret_cast<const T *>(ystage + S::kYXOff) + (q / S::kBlocks) * S::kChunk + tb * 8);
+            if (p.z) {
+                if (VEC)
+                    zs[m].load_vec(ec.z[m], t0 + tb * 8, L);
+                else
+                    zs[m].load_scalar(ec.z[m], t0 + tb * 8, L);
+            }
+        } else if (VEC) {
             xs[m].load_vec(ec.x[m], t0 + tb * 8, L);
             if (p.z)
                 zs[m].load_vec(ec.z[m], t0 + tb * 8, L);
@@ -475,6 +606,13 @@ __device__ __forceinline__ void epilogue_chunk(const ScanArgs &p, int lane, cons
         }
         const float out[8] = {o[0].x, o[0].y, o[1].x, o[1].y, o[2].x, o[2].y, o[3].x, o[3].y};
         store8<T, VEC>(ec.y[m], t0 + tb * 8, L, out);
+        if (CONV && ec.xo[m]) {
+            float xo[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                xo[j] = xs[m].get(j);
+            store8<T, VEC>(ec.xo[m], t0 + tb * 8, L, xo);
+        }
     }
 }
 
@@ -711,14 +849,14 @@ __device__ __forceinline__ bool issuer_warp(const ScanArgs &p, const TmaMaps &ma
 
 // The two producer warps: each thread converts its share of every chunk (from the
 // raw slot, or straight from global memory on the ragged path) into the input stage.
-template <int N, typename T, bool HAS_RESET, bool VEC>
+template <int N, typename T, bool HAS_RESET, bool VEC, bool CONV>
 __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, int pi, int lane)
 {
     using S = ScanShape<N>;
     constexpr int RS = S::kRawStages;
     constexpr int kRawBytes = S::template raw_stage_bytes<T>();
     const int tl = pi * 32 + lane; // producer thread index
-    IoPrefetch<N, T, HAS_RESET, VEC> pf;
+    IoPrefetch<N, T, HAS_RESET, VEC, CONV> pf;
     int64_t reset_g = -1;
     const uint8_t *reset_row = p.reset;
     for (uint32_t i = 0;; ++i) {
@@ -731,7 +869,7 @@ __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, in
         const bool end = (fl & kEnd) != 0;
         if (!end) {
             if constexpr (VEC)
-                pf.load_smem(p, tl, g, cx.raw_base + r * kRawBytes);
+                pf.load_smem(p, tl, g, cx.raw_base + r * kRawBytes, t0);
             else
                 pf.load(p, tl, g, t0);
             if (HAS_RESET) {
@@ -748,19 +886,23 @@ __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, in
         if (!mbar_wait(cx.in_empty + st, ((i / S::kStages) & 1u) ^ 1u, cx.status))
             return false;
         float *stage = cx.in_base + st * S::kInStage;
-        if (!end)
-            produce_chunk<N, T, HAS_RESET, VEC>(p, tl, pf, stage, cx.raw_base + r * kRawBytes, t0);
-        if (tl == 0)
-            write_meta(stage, t0, g, s, fl);
         // The chunk's output stage must be free as well (the epilogue is done with
         // chunk i - kYStages).  Waiting for it here, and for the raw slot above, makes
         // in_full the one barrier the scan warps wait on per chunk: a satisfied wait
-        // still costs on the order of a hundred cycles, on the critical warps.
+        // still costs on the order of a hundred cycles, on the critical warps.  (The
+        // fused conv form writes x into the output stage, so it waits first.)
         const int ys = int(i % S::kYStages);
-        if (!mbar_wait(cx.y_empty + ys, ((i / S::kYStages) & 1u) ^ 1u, cx.status))
+        float *ystage = cx.y_base + ys * S::template y_stage<T>();
+        if (CONV && !mbar_wait(cx.y_empty + ys, ((i / S::kYStages) & 1u) ^ 1u, cx.status))
+            return false;
+        if (!end)
+            produce_chunk<N, T, HAS_RESET, VEC, CONV>(p, tl, pf, stage, cx.raw_base + r * kRawBytes, t0, g, ystage);
+        if (tl == 0)
+            write_meta(stage, t0, g, s, fl);
+        if (!CONV && !mbar_wait(cx.y_empty + ys, ((i / S::kYStages) & 1u) ^ 1u, cx.status))
             return false;
         if (tl == 0) // the epilogue warps learn the chunk from its output stage
-            write_meta(cx.y_base + ys * S::kYStage, t0, g, s, fl);
+            write_meta(ystage, t0, g, s, fl);
         mbar_arrive(cx.in_full + st);
         if (end)
             return true;
@@ -768,7 +910,7 @@ __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, in
 }
 
 // The two epilogue warps: partial outputs of each chunk -> y.  False on a timeout.
-template <int N, typename T, bool VEC>
+template <int N, typename T, bool VEC, bool CONV>
 __device__ __forceinline__ bool epilogue_role(const ScanArgs &p, const float *y_base, uint64_t *y_full,
                                               uint64_t *y_empty, uint32_t *status, int tl)
 {
@@ -778,11 +920,11 @@ __device__ __forceinline__ bool epilogue_role(const ScanArgs &p, const float *y_
         const int ys = int(j % S::kYStages);
         if (!mbar_wait(y_full + ys, (j / S::kYStages) & 1u, status))
             return false;
-        const float *ystage = y_base + ys * S::kYStage;
+        const float *ystage = y_base + ys * S::template y_stage<T>();
         const ChunkMeta meta = read_meta(ystage);
         if (meta.flags & kEnd)
             return true;
-        epilogue_chunk<N, T, VEC>(p, tl, ystage, meta.g, meta.t0, ec);
+        epilogue_chunk<N, T, VEC, CONV>(p, tl, ystage, meta.g, meta.t0, ec);
         mbar_arrive(y_empty + ys);
     }
 }
@@ -791,8 +933,16 @@ __device__ __forceinline__ bool epilogue_role(const ScanArgs &p, const float *y_
 // the kernel
 // ---------------------------------------------------------------------------------------
 
-template <int N, typename T, bool HAS_RESET, bool VEC, bool EMIT>
-__global__ void __launch_bounds__(ScanShape<N>::kThreads, EMIT ? 2 : 1)
+// CTAs per SM to plan registers for: the states and conv forms need more registers
+// than the plain form and are bounded to two CTAs per SM wherever shared memory fits
+// two (about 113 KB each); the plain form gets there at its natural allocation.
+template <int N, typename T, bool EMIT, bool CONV> constexpr int scan_min_ctas()
+{
+    return (EMIT || CONV) && ScanShape<N>::template smem_bytes<T, true>() <= 113 * 1024 ? 2 : 1;
+}
+
+template <int N, typename T, bool HAS_RESET, bool VEC, bool EMIT, bool CONV>
+__global__ void __launch_bounds__(ScanShape<N>::kThreads, (scan_min_ctas<N, T, EMIT, CONV>()))
 ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
 {
     using S = ScanShape<N>;
@@ -800,7 +950,7 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
     extern __shared__ __align__(1024) unsigned char smem_bytes[];
     float *const in_base = reinterpret_cast<float *>(smem_bytes + kRawRing);
     float *const y_base = in_base + S::kStages * S::kInStage;
-    uint64_t *const bars = reinterpret_cast<uint64_t *>(in_base + S::kFloats);
+    uint64_t *const bars = reinterpret_cast<uint64_t *>(in_base + S::template floats<T>());
     uint64_t *const in_full = bars + S::kBarInFull, *const in_empty = bars + S::kBarInEmpty;
     uint64_t *const y_full = bars + S::kBarYFull, *const y_empty = bars + S::kBarYEmpty;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -850,9 +1000,9 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
         if (warp == S::kIssuerWarp)
             ok = issuer_warp<N, T, VEC>(p, maps, cx, lane);
         else if (((warp - S::kScanWarps) & 1) == 0)
-            ok = producer<N, T, HAS_RESET, VEC>(p, cx, (warp - S::kScanWarps) >> 1, lane);
+            ok = producer<N, T, HAS_RESET, VEC, CONV>(p, cx, (warp - S::kScanWarps) >> 1, lane);
         else
-            ok = epilogue_role<N, T, VEC>(p, y_base, y_full, y_empty, status,
+            ok = epilogue_role<N, T, VEC, CONV>(p, y_base, y_full, y_empty, status,
                                           ((warp - S::kScanWarps) >> 1) * 32 + lane);
         if (!ok)
             return; // gave up on a wait (SS_ERR_TIMEOUT recorded)
@@ -909,7 +1059,7 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
             if (EMIT)
                 hrow = p.h_all + (row * p.seq + meta.t0) * N;
             scan_chunk<N, T, HAS_RESET, EMIT>(stage, smem_bytes + rs * S::template raw_stage_bytes<T>(),
-                                              y_base + ysi * S::kYStage + S::kYPOff + cl * S::kYChan + sub * S::kRow,
+                                              y_base + ysi * S::template y_stage<T>() + S::kYPOff + cl * S::kYChan + sub * S::kRow,
                                               cl, n0, n1, A0, A1, hs0, hs1, hrow,
                                               cvalid ? p.seq - meta.t0 : int64_t(0));
             mbar_arrive(bars + S::kBarRawEmpty + rs);

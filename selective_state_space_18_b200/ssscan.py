@@ -26,7 +26,7 @@ STATUS = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE", 4:
           9: "SS_ERR_WORKSPACE", 10: "SS_ERR_SCRATCH_LIMIT"}
 EXPORTS = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_scan_status", "ss_state_update",
            "ss_debug_set_wait_limit", "ss_status_string", "ss_abi_version",
-           "ss_scan_fwd_static_scratch", "ss_scan_fwd_states", "ss_gated_scan")
+           "ss_scan_fwd_static_scratch", "ss_scan_fwd_states", "ss_gated_scan", "ss_scan_fwd_conv")
 ABI_MAJOR = 2
 
 _lock = threading.Lock()
@@ -62,6 +62,9 @@ def load_library(path: str = LIB_PATH):
             lib.ss_scan_fwd_static_scratch.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 10 + [
                 ctypes.c_uint32, _vp, _vp, ctypes.POINTER(_vp), _vp]
             lib.ss_scan_fwd_static_scratch.restype = ctypes.c_int
+            lib.ss_scan_fwd_conv.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 3 + [_i64] + [_vp] * 12 + [
+                ctypes.c_uint32, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+            lib.ss_scan_fwd_conv.restype = ctypes.c_int
             lib.ss_gated_scan.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 7 + [_vp]
             lib.ss_gated_scan.restype = ctypes.c_int
             lib.ss_scan_workspace_bytes.argtypes = [_i64, _i64, _i64, _i64]
@@ -362,3 +365,57 @@ def ss_gated_scan(q, k, v, gamma, h0=None, *, stream=None):
     if st != 0:
         raise SSError("ss_gated_scan", st)
     return {"outputs": y, "final_state": fs}
+
+
+def ss_scan_fwd_conv(u, conv_w, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h0=None, *,
+                     conv_b=None, conv_state=None, dt_softplus=True, return_conv_state=True,
+                     return_x=False, stream=None, workspace=True):
+    """Prompt scan with the causal depthwise conv + SiLU fused in front: u is the conv
+    input [batch, channels, seq] (the scan's x = silu(conv(u))); conv_w [channels, K]
+    fp32 (K <= 4); conv_b [channels] fp32; conv_state [batch, channels, K-1] fp32 (the
+    inputs before u).  Returns dict(y, h_last, conv_state (the last K-1 inputs, for the
+    next call), x (when return_x))."""
+    dev = u.device
+    if dev.type != "cuda":
+        raise ValueError("ss_scan_fwd_conv runs on CUDA tensors only")
+    if u.dim() != 3:
+        raise ValueError("u must be [batch, channels, seq]")
+    bt, ch, L = u.shape
+    n = A.shape[-1]
+    K = conv_w.shape[-1]
+    code = _dtype_code(u)
+    u = _prep(u, "u", dev)
+    conv_w = _prep(conv_w, "conv_w", dev, torch.float32, (ch, K))
+    conv_b = _prep(conv_b, "conv_b", dev, torch.float32, (ch,))
+    conv_state = _prep(conv_state, "conv_state", dev, torch.float32, (bt, ch, K - 1))
+    dt = _prep(dt, "dt", dev, u.dtype, (bt, ch, L))
+    z = _prep(z, "z", dev, u.dtype, (bt, ch, L))
+    B = _prep(B, "B", dev, u.dtype, (bt, n, L))
+    C = _prep(C, "C", dev, u.dtype, (bt, n, L))
+    A = _prep(A, "A", dev, torch.float32, (ch, n))
+    D = _prep(D, "D", dev, torch.float32, (ch,))
+    dt_bias = _prep(dt_bias, "dt_bias", dev, torch.float32, (ch,))
+    h0 = _prep(h0, "h0", dev, torch.float32, (bt, ch, n))
+    if reset is not None:
+        reset = _prep(reset, "reset", dev, None, (bt, L))
+        reset = reset.view(torch.uint8) if reset.dtype == torch.bool else reset
+    y = torch.empty_like(u)
+    h_last = torch.empty(bt, ch, n, device=dev, dtype=torch.float32)
+    cs_out = torch.empty(bt, ch, K - 1, device=dev, dtype=torch.float32) if return_conv_state and K > 1 else None
+    x_out = torch.empty_like(u) if return_x else None
+    if workspace is True:
+        workspace = scan_workspace(bt, ch, n, L, dev, stream)
+    elif workspace is False or workspace is None:
+        workspace = None
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    flags = SS_DT_SOFTPLUS if dt_softplus else 0
+    st = load_library().ss_scan_fwd_conv(
+        bt, ch, n, L, code, _ptr(u), _ptr(conv_w), _ptr(conv_b), K, _ptr(conv_state), _ptr(cs_out), _ptr(x_out),
+        _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias), _ptr(reset), _ptr(h0), flags,
+        _ptr(y), _ptr(h_last), _ptr(workspace), ws_bytes, _stream(stream, dev))
+    if st != 0:
+        raise SSError("ss_scan_fwd_conv", st)
+    out = {"y": y, "h_last": h_last, "conv_state": cs_out}
+    if return_x:
+        out["x"] = x_out
+    return out

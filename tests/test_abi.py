@@ -220,3 +220,20 @@ def test_huge_shapes_are_refused_without_overflow(lib):
     assert ssscan.STATUS[st] == "SS_ERR_SHAPE"
     st = lib.ss_gated_scan(1, 1 << 60, 64, 64, ssscan.SS_BF16, P[0], P[1], P[2], P[3], None, P[4], P[5], None)
     assert ssscan.STATUS[st] == "SS_ERR_SHAPE"
+
+
+def test_scan_conv_checks(lib):
+    def call(**kw):
+        a = dict(u=P[0], w=P[6], cb=None, K=4, cs=None, cso=None, xo=None, dt=P[1], A=P[2], B=P[3], C=P[4], y=P[5])
+        a.update(kw)
+        return ssscan.STATUS[lib.ss_scan_fwd_conv(2, 16, 16, 64, ssscan.SS_BF16, a["u"], a["w"], a["cb"], a["K"],
+                                                  a["cs"], a["cso"], a["xo"], a["dt"], a["A"], a["B"], a["C"], None,
+                                                  None, None, None, None, 1, a["y"], None, None, 0, None)]
+    assert call(w=None) == "SS_ERR_NULL"
+    assert call(K=5) == "SS_ERR_UNSUPPORTED"
+    assert call(K=0) == "SS_ERR_UNSUPPORTED"
+    assert call(u=None) == "SS_ERR_NULL"
+    assert call(xo=ctypes.c_void_p(P[0].value + 64)) == "SS_ERR_ALIAS"      # x_out over u
+    assert call(cs=P[7], cso=ctypes.c_void_p(P[7].value + 4)) == "SS_ERR_ALIAS"  # state out over state in
+    assert call(xo=P[5]) == "SS_ERR_ALIAS"                                  # x_out over y
+    assert call(cso=ctypes.c_void_p(P[6].value + 2)) == "SS_ERR_ALIGN"

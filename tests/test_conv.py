@@ -1,0 +1,83 @@
+"""The scan with the causal depthwise conv + SiLU fused in front (ss_scan_fwd_conv)
+against the oracle composition: conv + SiLU (TransformerLens ssm_mixer: the scan's x is
+SiLU of the conv1d output), then the selective scan."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import TOL, assert_close
+from selective_state_space_18_b200 import ssscan
+from selective_state_space_18_b200.inputs import make_scan_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+
+
+def _inputs(bt, ch, n, L, dtype, K, seed, state=True, bias=True, resets=False):
+    inp = make_scan_inputs(bt, ch, n, L, dtype, seed=seed, reset_mean_doc=25 if resets else 0, h0=True)
+    g = torch.Generator().manual_seed(seed + 1)
+    inp["u"] = inp.pop("x")
+    inp["conv_w"] = torch.randn(ch, K, generator=g) * 0.5
+    inp["conv_b"] = torch.randn(ch, generator=g) * 0.1 if bias else None
+    inp["conv_state"] = torch.randn(bt, ch, K - 1, generator=g) if state and K > 1 else None
+    return inp
+
+
+def _gpu(inp, **kw):
+    d = {k: (None if v is None else v.cuda()) for k, v in inp.items()}
+    out = ssscan.ss_scan_fwd_conv(d["u"], d["conv_w"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["z"], d["dt_bias"],
+                                  d["reset"], d["h0"], conv_b=d["conv_b"], conv_state=d["conv_state"], return_x=True,
+                                  **kw)
+    torch.cuda.synchronize()
+    return {k: (None if v is None else v.cpu()) for k, v in out.items()}
+
+
+def _oracle(orc, inp):
+    cv = orc.conv_silu(inp["u"], inp["conv_w"], inp["conv_b"], inp["conv_state"])
+    sc = orc.scan(x=cv["x"], dt=inp["dt"], A=inp["A"], B=inp["B"], C=inp["C"], D=inp["D"], z=inp["z"],
+                  dt_bias=inp["dt_bias"], reset=inp["reset"], h0=inp["h0"])
+    return cv, sc
+
+
+@pytest.mark.parametrize("case", [
+    (2, 40, 16, 264, "bf16", 4, True, True, False),   # tile-load path
+    (2, 40, 16, 77, "bf16", 4, True, True, True),     # ragged path, resets
+    (1, 24, 8, 100, "f32", 3, False, True, False),
+    (3, 20, 4, 50, "f32", 2, True, False, True),
+    (2, 16, 16, 40, "f32", 1, False, False, False),
+    (1, 8, 16, 2, "f32", 4, True, True, False),       # shorter than the conv window
+    (1, 320, 16, 2048, "bf16", 4, True, True, False), # many channel groups, segmented schedule
+], ids=lambda c: "x".join(str(v) for v in c))
+def test_matches_oracle_composition(orc, case):
+    bt, ch, n, L, dtype, K, state, bias, resets = case
+    inp = _inputs(bt, ch, n, L, dtype, K, seed=600 + L + K, state=state, bias=bias, resets=resets)
+    out = _gpu(inp)
+    cv, sc = _oracle(orc, inp)
+    tol = TOL[inp["u"].dtype]
+    assert_close(out["y"], sc["y"], tol, "y")
+    assert_close(out["h_last"], sc["h_last"], tol, "h_last")
+    assert_close(out["x"], cv["x"], tol, "x")
+    if K > 1:  # a copy of inputs: exact
+        np.testing.assert_array_equal(out["conv_state"].double().numpy(), cv["state"])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_two_calls_chained_through_both_states(dtype):
+    """A prompt split in two calls (conv state and scan state handed over) equals one call."""
+    inp = _inputs(2, 48, 16, 640, dtype, 4, seed=650, state=False)
+    full = _gpu(inp)
+    a, b = dict(inp), dict(inp)
+    for k in ("u", "dt", "z", "B", "C"):
+        a[k] = inp[k][:, :, :296].contiguous()
+        b[k] = inp[k][:, :, 296:].contiguous()
+    oa = _gpu(a)
+    b["conv_state"], b["h0"] = oa["conv_state"], oa["h_last"]
+    ob = _gpu(b)
+    assert_close(torch.cat([oa["y"], ob["y"]], -1), full["y"].double().numpy(), 1e-6, "y")
+    assert_close(ob["h_last"], full["h_last"].double().numpy(), 1e-6, "h_last")
+    assert torch.equal(ob["conv_state"], full["conv_state"])
