@@ -236,6 +236,28 @@ SS_API int ss_state_update(int64_t batch, int64_t channels, int64_t state_dim, s
                     const float *dt_bias, uint32_t flags, void *y, ss_stream_t stream);
 
 /*
+ * Decode step of the fused conv form: the new token's scan input x comes from the
+ * causal conv over the row's conv state and the new input u, and the conv state
+ * advances by one input (TransformerLens ssm_mixer: SiLU of the conv1d output; a decode
+ * step carries the conv's recent inputs as its state):
+ *
+ *   x[b,c]          = silu( conv_b[c] + sum_{k<conv_k-1} conv_w[c,k] * conv_state[b,c,k]
+ *                           + conv_w[c,conv_k-1] * u[b,c] )
+ *   conv_state[b,c] = (conv_state[b,c,1:], u[b,c])          (in place)
+ *
+ * then the update of ss_state_update with x.  conv_state: [batch, channels, conv_k-1]
+ * float32, required when conv_k > 1, overlapping no other buffer; conv_w [channels,
+ * conv_k], conv_b [channels] (nullable) float32; conv_k in 1..4.  The state must be
+ * 16-byte aligned (SS_ERR_ALIGN otherwise).  SiLU of x is the exact form here.
+ */
+SS_API int ss_state_update_conv(int64_t batch, int64_t channels, int64_t state_dim,
+                                ss_dtype_t dtype, float *state, float *conv_state,
+                                const float *conv_w, const float *conv_b, int64_t conv_k,
+                                const void *u, const void *dt_raw, const float *A, const void *B,
+                                const void *C, const float *D, const void *z,
+                                const float *dt_bias, uint32_t flags, void *y, ss_stream_t stream);
+
+/*
  * Testing aid: cap every device-side wait of later calls on the current device at
  * `microseconds` (0 restores the default of 2 s).  Used to make a wait that can never
  * be satisfied end quickly with SS_ERR_TIMEOUT; waits for copies already in flight

@@ -231,13 +231,20 @@ int dispatch_scan_n(ss::ScanArgs a, ss_dtype_t dtype, bool vec, size_t ws_bytes,
     return dispatch_scan_t<N, float>(a, vec, s);
 }
 
-template <int N, typename T, bool V>
-int launch_update(ss::UpdateArgs a, cudaStream_t stream)
+// The conv form of the decode step (w NULL: none).
+struct UpdConv {
+    const float *w = nullptr, *b = nullptr;
+    float *state = nullptr;
+    int k = 0;
+};
+
+template <int N, typename T, bool V, bool CV>
+int launch_update(ss::UpdateArgs a, cudaStream_t stream, const UpdConv &cv)
 {
     if constexpr (V) {
         // aligned state: persistent CTAs streaming the state through shared memory
         using D = ss::DecShape<N, T>;
-        auto kernel = ss::ss_state_update_stream_kernel<N, T>;
+        auto kernel = ss::ss_state_update_stream_kernel<N, T, CV>;
         static std::atomic<uint64_t> smem_done{0};
         static std::atomic<int> occ_cache[64];
         int st = ensure_smem(kernel, D::kSmem, smem_done);
@@ -272,12 +279,18 @@ int launch_update(ss::UpdateArgs a, cudaStream_t stream)
         da.bulk_xdz = aligned(a.x, 16) && aligned(a.dt, 16) && (!a.z || aligned(a.z, 16)) &&
                       (size_t(a.channels) * es) % 16 == 0;
         da.bulk_bc = aligned(a.B, 16) && aligned(a.C, 16) && (N * es) % 16 == 0;
+        da.conv_w = cv.w;
+        da.conv_b = cv.b;
+        da.conv_state = cv.state;
+        da.conv_k = cv.k;
         uint32_t *status = nullptr;
         if (status_word_address(&status) != SS_OK)
             return SS_ERR_CUDA;
         kernel<<<unsigned(grid), ss::kDecBlock, D::kSmem, stream>>>(da, status);
         return launch_status();
     }
+    if constexpr (CV)
+        return SS_ERR_ALIGN; // the conv form runs on the streaming kernel only
     const int64_t per_block = int64_t(ss::kUpdateThreads) * ss::kUpdateItems; // row quarters
     const int64_t quarters = a.channels * (N / 4);
     a.blocks_per_row = int((quarters + per_block - 1) / per_block);
@@ -288,12 +301,19 @@ int launch_update(ss::UpdateArgs a, cudaStream_t stream)
     return launch_status();
 }
 
-template <int N>
-int dispatch_update_n(const ss::UpdateArgs &a, ss_dtype_t dtype, bool vec, cudaStream_t s)
+template <int N, bool CV>
+int dispatch_update_c(const ss::UpdateArgs &a, ss_dtype_t dtype, bool vec, cudaStream_t s, const UpdConv &cv)
 {
     if (dtype == SS_BF16)
-        return vec ? launch_update<N, __nv_bfloat16, true>(a, s) : launch_update<N, __nv_bfloat16, false>(a, s);
-    return vec ? launch_update<N, float, true>(a, s) : launch_update<N, float, false>(a, s);
+        return vec ? launch_update<N, __nv_bfloat16, true, CV>(a, s, cv)
+                   : launch_update<N, __nv_bfloat16, false, CV>(a, s, cv);
+    return vec ? launch_update<N, float, true, CV>(a, s, cv) : launch_update<N, float, false, CV>(a, s, cv);
+}
+
+template <int N>
+int dispatch_update_n(const ss::UpdateArgs &a, ss_dtype_t dtype, bool vec, cudaStream_t s, const UpdConv &cv)
+{
+    return cv.w ? dispatch_update_c<N, true>(a, dtype, vec, s, cv) : dispatch_update_c<N, false>(a, dtype, vec, s, cv);
 }
 
 // Scratch of ss_scan_fwd_static_scratch: a fixed workspace in device memory, one per
@@ -675,10 +695,14 @@ int ss_scan_fwd_states(int64_t batch, int64_t channels, int64_t state_dim, int64
                      h_last, h_all, workspace, workspace_bytes, stream);
 }
 
-int ss_state_update(int64_t batch, int64_t channels, int64_t state_dim, ss_dtype_t dtype,
-                    float *state, const void *x, const void *dt_raw, const float *A,
-                    const void *B, const void *C, const float *D, const void *z,
-                    const float *dt_bias, uint32_t flags, void *y, ss_stream_t stream)
+} // extern "C"
+
+namespace {
+
+int update_impl(int64_t batch, int64_t channels, int64_t state_dim, ss_dtype_t dtype, float *state,
+                const void *x, const void *dt_raw, const float *A, const void *B, const void *C, const float *D,
+                const void *z, const float *dt_bias, uint32_t flags, void *y, ss_stream_t stream,
+                const UpdConv &cv = UpdConv())
 {
     if (!state || !x || !dt_raw || !A || !B || !C || !y)
         return SS_ERR_NULL;
@@ -713,6 +737,26 @@ int ss_state_update(int64_t batch, int64_t channels, int64_t state_dim, ss_dtype
             return SS_ERR_ALIAS;
     if (overlaps(y, ybytes, state, sbytes))
         return SS_ERR_ALIAS;
+    if (cv.w) {
+        if (cv.k < 1 || cv.k > 4)
+            return SS_ERR_UNSUPPORTED;
+        if (cv.k > 1 && !cv.state)
+            return SS_ERR_NULL;
+        const float *f32c[] = {cv.w, cv.b, cv.state};
+        for (const float *q : f32c)
+            if (q && !aligned(q, 4))
+                return SS_ERR_ALIGN;
+        // the conv state is updated in place: it overlaps no other buffer
+        const size_t cbytes = size_t(rows) * size_t(cv.k - 1) * 4;
+        const void *oth[] = {x, dt_raw, z, B, C, A, D, dt_bias, y, state, cv.w, cv.b};
+        const size_t oth_n[] = {ybytes, ybytes, z ? ybytes : 0, size_t(bnel) * es, size_t(bnel) * es,
+                                size_t(channels * state_dim) * 4, D ? size_t(channels) * 4 : 0,
+                                dt_bias ? size_t(channels) * 4 : 0, ybytes, sbytes, size_t(channels) * cv.k * 4,
+                                cv.b ? size_t(channels) * 4 : 0};
+        for (int i = 0; i < 12; ++i)
+            if (overlaps(cv.state, cbytes, oth[i], oth_n[i]))
+                return SS_ERR_ALIAS;
+    }
 
     const bool vec = aligned(state, 16) && aligned(A, 16) && aligned(B, 4 * es) && aligned(C, 4 * es);
     ss::UpdateArgs a{};
@@ -725,10 +769,41 @@ int ss_state_update(int64_t batch, int64_t channels, int64_t state_dim, ss_dtype
     a.softplus = (flags & SS_DT_SOFTPLUS) ? 1 : 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     switch (state_dim) {
-    case 4: return dispatch_update_n<4>(a, dtype, vec, s);
-    case 8: return dispatch_update_n<8>(a, dtype, vec, s);
-    default: return dispatch_update_n<16>(a, dtype, vec, s);
+    case 4: return dispatch_update_n<4>(a, dtype, vec, s, cv);
+    case 8: return dispatch_update_n<8>(a, dtype, vec, s, cv);
+    default: return dispatch_update_n<16>(a, dtype, vec, s, cv);
     }
+}
+
+} // namespace
+
+extern "C" {
+
+int ss_state_update(int64_t batch, int64_t channels, int64_t state_dim, ss_dtype_t dtype,
+                    float *state, const void *x, const void *dt_raw, const float *A,
+                    const void *B, const void *C, const float *D, const void *z,
+                    const float *dt_bias, uint32_t flags, void *y, ss_stream_t stream)
+{
+    return update_impl(batch, channels, state_dim, dtype, state, x, dt_raw, A, B, C, D, z, dt_bias, flags, y, stream);
+}
+
+int ss_state_update_conv(int64_t batch, int64_t channels, int64_t state_dim, ss_dtype_t dtype, float *state,
+                         float *conv_state, const float *conv_w, const float *conv_b, int64_t conv_k,
+                         const void *u, const void *dt_raw, const float *A, const void *B, const void *C,
+                         const float *D, const void *z, const float *dt_bias, uint32_t flags, void *y,
+                         ss_stream_t stream)
+{
+    if (!conv_w)
+        return SS_ERR_NULL;
+    if (conv_k < 1 || conv_k > 4)
+        return SS_ERR_UNSUPPORTED;
+    UpdConv cv;
+    cv.w = conv_w;
+    cv.b = conv_b;
+    cv.state = conv_state;
+    cv.k = int(conv_k);
+    return update_impl(batch, channels, state_dim, dtype, state, u, dt_raw, A, B, C, D, z, dt_bias, flags, y, stream,
+                       cv);
 }
 
 // The scratch stands in for the caller's workspace: the shape is checked against its

@@ -190,10 +190,16 @@ struct DecArgs {
     int fixed_cb;    // grid is a multiple of ncb: CTA i keeps channel block i % ncb
     int bulk_xdz;    // x, dt_raw (and z) rows are copied with the state
     int bulk_bc;     // B and C rows are copied with the state
+    // conv form: x above is the conv input u; x = silu(conv_b + conv_w . [state, u])
+    const float *conv_w, *conv_b; // [channels, conv_k], [channels] (nullable)
+    float *conv_state;            // [batch, channels, conv_k - 1] in/out
+    int conv_k;
 };
 
-template <int N, typename T>
-__global__ void __launch_bounds__(kDecBlock)
+// CONV: the decode step of the fused conv form -- x is silu of the causal conv over the
+// row's conv state and the new input u, and the conv state shifts by one input.
+template <int N, typename T, bool CONV>
+__global__ void __launch_bounds__(kDecBlock, 2)
 ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
 {
     using D = DecShape<N, T>;
@@ -276,6 +282,8 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
 
     float4 av[kDecItems];
     float bias[kDecItems], dco[kDecItems];
+    float cw[CONV ? kDecItems : 1][4], cbi[CONV ? kDecItems : 1]; // taps aligned: cw[3] multiplies u
+    const int H = CONV ? da.conv_k - 1 : 0;
     int64_t cached_cb = -1;
     bool ok = true;
     for (int64_t k = 0;; ++k) {
@@ -293,6 +301,27 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
                 av[it] = __ldg(reinterpret_cast<const float4 *>(p.A + c * N) + lane_q);
                 bias[it] = p.dt_bias ? __ldg(p.dt_bias + c) : 0.0f;
                 dco[it] = p.D ? __ldg(p.D + c) : 0.0f;
+                if constexpr (CONV) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int kk = k - (4 - da.conv_k);
+                        cw[it][k] = kk >= 0 ? __ldg(da.conv_w + c * da.conv_k + kk) : 0.0f;
+                    }
+                    cbi[it] = da.conv_b ? __ldg(da.conv_b + c) : 0.0f;
+                }
+            }
+        }
+        // the conv state of each item's row (read by the row's lanes before its first
+        // lane writes the shifted state back, below)
+        float cs[CONV ? kDecItems : 1][3];
+        if constexpr (CONV) {
+#pragma unroll
+            for (int it = 0; it < kDecItems; ++it) {
+                const int q = tid + it * kDecThreads;
+                const int64_t row = b * p.channels + c0 + (q < nq ? q : nq - 1) / Q;
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+                    cs[it][j] = j < H ? __ldg(da.conv_state + row * H + j) : 0.0f;
             }
         }
         // the small operands first: their latency overlaps the wait for the state
@@ -336,6 +365,19 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
                 zs[it] = p.z ? Elem<T>::load_smem(sz + cl) : 0.0f;
             }
         }
+        if constexpr (CONV) { // x = silu(conv over [state, u]); xs held u until here
+#pragma unroll
+            for (int it = 0; it < kDecItems; ++it) {
+                float acc = fmaf(cw[it][3], xs[it], cbi[it]);
+#pragma unroll
+                for (int j = 0; j < 3; ++j) // state entry j is the input 3 - H + j back
+                    if (j < H)
+                        acc = fmaf(cw[it][3 - H + j], cs[it][j], acc);
+                const float u = xs[it];
+                xs[it] = silu(acc);
+                cs[it][0] = u; // keep u for the state shift below
+            }
+        }
         // dt of the four items: the Q lanes of a row share them, so lane j computes
         // the softplus of the items it with it % Q == j and the row's lanes exchange
         float dsp[kDecItems];
@@ -377,6 +419,20 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
 #pragma unroll
             for (int off = Q / 2; off >= 1; off >>= 1)
                 yp += __shfl_xor_sync(0xffffffffu, yp, off);
+            if constexpr (CONV) {
+                __syncwarp(); // every lane of the row has read the conv state
+                if (valid && lane_q == 0 && H > 0) {
+                    const int64_t row = b * p.channels + c0 + q / Q;
+                    float *csr = da.conv_state + row * H;
+                    // shift: drop the oldest input (entry 0, whose register now holds u),
+                    // keep entries 1 .. H-1 from registers, append u
+#pragma unroll
+                    for (int j = 0; j < 2; ++j)
+                        if (j + 1 < H)
+                            csr[j] = cs[it][j + 1];
+                    csr[H - 1] = cs[it][0];
+                }
+            }
             if (valid) {
                 const int64_t row = b * p.channels + c0 + q / Q;
                 __stcs(reinterpret_cast<float4 *>(p.state + row * N) + lane_q, st);

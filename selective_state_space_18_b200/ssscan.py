@@ -26,7 +26,8 @@ STATUS = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE", 4:
           9: "SS_ERR_WORKSPACE", 10: "SS_ERR_SCRATCH_LIMIT"}
 EXPORTS = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_scan_status", "ss_state_update",
            "ss_debug_set_wait_limit", "ss_status_string", "ss_abi_version",
-           "ss_scan_fwd_static_scratch", "ss_scan_fwd_states", "ss_gated_scan", "ss_scan_fwd_conv")
+           "ss_scan_fwd_static_scratch", "ss_scan_fwd_states", "ss_gated_scan", "ss_scan_fwd_conv",
+           "ss_state_update_conv")
 ABI_MAJOR = 2
 
 _lock = threading.Lock()
@@ -65,6 +66,9 @@ def load_library(path: str = LIB_PATH):
             lib.ss_scan_fwd_conv.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 3 + [_i64] + [_vp] * 12 + [
                 ctypes.c_uint32, _vp, _vp, _vp, ctypes.c_size_t, _vp]
             lib.ss_scan_fwd_conv.restype = ctypes.c_int
+            lib.ss_state_update_conv.argtypes = [_i64, _i64, _i64, ctypes.c_int] + [_vp] * 4 + [_i64] + [_vp] * 8 + [
+                ctypes.c_uint32, _vp, _vp]
+            lib.ss_state_update_conv.restype = ctypes.c_int
             lib.ss_gated_scan.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 7 + [_vp]
             lib.ss_gated_scan.restype = ctypes.c_int
             lib.ss_scan_workspace_bytes.argtypes = [_i64, _i64, _i64, _i64]
@@ -419,3 +423,40 @@ def ss_scan_fwd_conv(u, conv_w, dt, A, B, C, D=None, z=None, dt_bias=None, reset
     if return_x:
         out["x"] = x_out
     return out
+
+
+def ss_state_update_conv(state, conv_state, conv_w, u, dt, A, B, C, D=None, z=None, dt_bias=None, *,
+                         conv_b=None, dt_softplus=True, stream=None):
+    """Decode step of the fused conv form: ``state`` [batch, channels, state_dim] fp32 and
+    ``conv_state`` [batch, channels, K-1] fp32 are updated in place; u is the new conv
+    input [batch, channels].  Returns y [batch, channels]."""
+    dev = state.device
+    if dev.type != "cuda":
+        raise ValueError("ss_state_update_conv runs on CUDA tensors only")
+    bt, ch, n = state.shape
+    K = conv_w.shape[-1]
+    code = _dtype_code(u)
+    if state.dtype != torch.float32 or not state.is_contiguous():
+        raise ValueError("state must be a contiguous float32 tensor (updated in place)")
+    if K > 1 and (conv_state is None or conv_state.dtype != torch.float32 or not conv_state.is_contiguous()
+                  or tuple(conv_state.shape) != (bt, ch, K - 1)):
+        raise ValueError("conv_state must be a contiguous float32 [batch, channels, K-1] tensor (updated in place)")
+    u = _prep(u, "u", dev, None, (bt, ch))
+    dt = _prep(dt, "dt", dev, u.dtype, (bt, ch))
+    z = _prep(z, "z", dev, u.dtype, (bt, ch))
+    B = _prep(B, "B", dev, u.dtype, (bt, n))
+    C = _prep(C, "C", dev, u.dtype, (bt, n))
+    A = _prep(A, "A", dev, torch.float32, (ch, n))
+    D = _prep(D, "D", dev, torch.float32, (ch,))
+    dt_bias = _prep(dt_bias, "dt_bias", dev, torch.float32, (ch,))
+    conv_w = _prep(conv_w, "conv_w", dev, torch.float32, (ch, K))
+    conv_b = _prep(conv_b, "conv_b", dev, torch.float32, (ch,))
+    y = torch.empty(bt, ch, device=dev, dtype=u.dtype)
+    flags = SS_DT_SOFTPLUS if dt_softplus else 0
+    st = load_library().ss_state_update_conv(bt, ch, n, code, _ptr(state), _ptr(conv_state if K > 1 else None),
+                                             _ptr(conv_w), _ptr(conv_b), K, _ptr(u), _ptr(dt), _ptr(A), _ptr(B),
+                                             _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias), flags, _ptr(y),
+                                             _stream(stream, dev))
+    if st != 0:
+        raise SSError("ss_state_update_conv", st)
+    return y

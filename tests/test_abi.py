@@ -237,3 +237,17 @@ def test_scan_conv_checks(lib):
     assert call(cs=P[7], cso=ctypes.c_void_p(P[7].value + 4)) == "SS_ERR_ALIAS"  # state out over state in
     assert call(xo=P[5]) == "SS_ERR_ALIAS"                                  # x_out over y
     assert call(cso=ctypes.c_void_p(P[6].value + 2)) == "SS_ERR_ALIGN"
+
+
+def test_decode_conv_checks(lib):
+    def call(**kw):
+        a = dict(state=P[0], cs=P[7], w=P[6], K=4, u=P[1], dt=P[2], A=P[3], B=P[4], C=P[5], y=P[8])
+        a.update(kw)
+        return ssscan.STATUS[lib.ss_state_update_conv(4, 32, 16, ssscan.SS_F32, a["state"], a["cs"], a["w"], None,
+                                                      a["K"], a["u"], a["dt"], a["A"], a["B"], a["C"], None, None,
+                                                      None, 1, a["y"], None)]
+    assert call(w=None) == "SS_ERR_NULL"
+    assert call(K=5) == "SS_ERR_UNSUPPORTED"
+    assert call(cs=None) == "SS_ERR_NULL"
+    assert call(cs=ctypes.c_void_p(P[0].value + 64)) == "SS_ERR_ALIAS"   # conv state over the state
+    assert call(cs=ctypes.c_void_p(P[7].value + 2)) == "SS_ERR_ALIGN"

@@ -81,3 +81,54 @@ def test_two_calls_chained_through_both_states(dtype):
     assert_close(torch.cat([oa["y"], ob["y"]], -1), full["y"].double().numpy(), 1e-6, "y")
     assert_close(ob["h_last"], full["h_last"].double().numpy(), 1e-6, "h_last")
     assert torch.equal(ob["conv_state"], full["conv_state"])
+
+
+def _upd_inputs(bt, ch, n, dtype, K, seed):
+    from selective_state_space_18_b200.inputs import make_update_inputs
+    inp = make_update_inputs(bt, ch, n, dtype, seed=seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    inp["u"] = inp.pop("x")
+    inp["conv_w"] = torch.randn(ch, K, generator=g) * 0.5
+    inp["conv_b"] = torch.randn(ch, generator=g) * 0.1
+    inp["conv_state"] = torch.randn(bt, ch, K - 1, generator=g)
+    return inp
+
+
+@pytest.mark.parametrize("case", [(256, 5120, 16, "bf16", 4), (3, 37, 8, "f32", 3), (5, 64, 4, "f32", 2),
+                                  (4, 100, 16, "bf16", 1)], ids=lambda c: "x".join(str(v) for v in c))
+def test_decode_conv_matches_oracle(orc, case):
+    bt, ch, n, dtype, K = case
+    inp = _upd_inputs(bt, ch, n, dtype, K, seed=700 + K)
+    d = {k: (None if v is None else v.cuda()) for k, v in inp.items()}
+    y = ssscan.ss_state_update_conv(d["state"], d["conv_state"] if K > 1 else None, d["conv_w"], d["u"], d["dt"],
+                                    d["A"], d["B"], d["C"], d["D"], d["z"], d["dt_bias"], conv_b=d["conv_b"])
+    torch.cuda.synchronize()
+    cv = orc.conv_silu(inp["u"][:, :, None], inp["conv_w"], inp["conv_b"], inp["conv_state"] if K > 1 else None)
+    ref = orc.update(state=inp["state"], x=cv["x"][:, :, 0], dt=inp["dt"], A=inp["A"], B=inp["B"], C=inp["C"],
+                     D=inp["D"], z=inp["z"], dt_bias=inp["dt_bias"])
+    assert_close(y.cpu(), ref["y"], TOL[inp["u"].dtype], "y")
+    assert_close(d["state"].cpu(), ref["state"], 1e-4, "state")
+    if K > 1:  # the shifted inputs: exact
+        np.testing.assert_array_equal(d["conv_state"].cpu().double().numpy(), cv["state"])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_conv_continues_the_fused_prompt(dtype):
+    """Prompt over L-1 tokens, then one decode step from its two states, equals the
+    prompt over L tokens at the last token."""
+    inp = _inputs(2, 64, 16, 97, dtype, 4, seed=710, state=True)
+    full = _gpu(inp)
+    head = dict(inp)
+    for k in ("u", "dt", "z", "B", "C"):
+        head[k] = inp[k][:, :, :-1].contiguous()
+    oh = _gpu(head)
+    st, cs = oh["h_last"].cuda(), oh["conv_state"].cuda()
+    last = {k: inp[k][:, :, -1].contiguous().cuda() for k in ("u", "dt", "z", "B", "C")}
+    y = ssscan.ss_state_update_conv(st, cs, inp["conv_w"].cuda(), last["u"], last["dt"], inp["A"].cuda(), last["B"],
+                                    last["C"], inp["D"].cuda(), last["z"], inp["dt_bias"].cuda(),
+                                    conv_b=inp["conv_b"].cuda())
+    torch.cuda.synchronize()
+    tol = 1e-5 if dtype == "f32" else TOL[torch.bfloat16]
+    assert_close(y.cpu(), full["y"][:, :, -1].double().numpy(), tol, "y")
+    assert_close(st.cpu(), full["h_last"].double().numpy(), max(tol, 1e-5), "state")
+    assert torch.equal(cs.cpu(), full["conv_state"])
