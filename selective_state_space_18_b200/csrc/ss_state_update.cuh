@@ -365,16 +365,31 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
                 zs[it] = p.z ? Elem<T>::load_smem(sz + cl) : 0.0f;
             }
         }
-        if constexpr (CONV) { // x = silu(conv over [state, u]); xs held u until here
+        if constexpr (CONV) {
+            // x = silu(conv over [state, u]); xs held u until here.  The Q lanes of a row
+            // share each item's x: lane j evaluates the items it with it % Q == j and the
+            // row's lanes exchange (as for the softplus below)
+            float xm[kDecItems / Q];
+#pragma unroll
+            for (int v = 0; v < kDecItems / Q; ++v) {
+                float acc = 0.0f;
+#pragma unroll
+                for (int j = 0; j < Q; ++j) {
+                    const int it = v * Q + j;
+                    float a = fmaf(cw[it][3], xs[it], cbi[it]);
+#pragma unroll
+                    for (int e = 0; e < 3; ++e) // state entry e is the input 3 - H + e back
+                        if (e < H)
+                            a = fmaf(cw[it][3 - H + e], cs[it][e], a);
+                    acc = lane_q == j ? a : acc;
+                }
+                xm[v] = silu(acc);
+            }
+            const int xbase = (tid & 31) & ~(Q - 1);
 #pragma unroll
             for (int it = 0; it < kDecItems; ++it) {
-                float acc = fmaf(cw[it][3], xs[it], cbi[it]);
-#pragma unroll
-                for (int j = 0; j < 3; ++j) // state entry j is the input 3 - H + j back
-                    if (j < H)
-                        acc = fmaf(cw[it][3 - H + j], cs[it][j], acc);
                 const float u = xs[it];
-                xs[it] = silu(acc);
+                xs[it] = Q == 1 ? xm[it] : __shfl_sync(0xffffffffu, xm[it / Q], xbase | (it % Q));
                 cs[it][0] = u; // keep u for the state shift below
             }
         }
