@@ -59,6 +59,9 @@ def _load():
             lib.ss_oracle_conv_silu.restype = ctypes.c_int
             lib.ss_oracle_gated_scan.argtypes = [_i64, _i64, _i64, _i64] + [_dp] * 7 + [ctypes.c_int]
             lib.ss_oracle_gated_scan.restype = ctypes.c_int
+            lib.ss_oracle_segment.argtypes = [_i64, _i64, _i64, _i64] + [_dp] * 5 + [
+                _u8p, ctypes.c_int, _dp, _dp, ctypes.c_int]
+            lib.ss_oracle_segment.restype = ctypes.c_int
             lib.ss_oracle_num_threads.argtypes = []
             lib.ss_oracle_num_threads.restype = ctypes.c_int
             _lib = lib
@@ -212,6 +215,43 @@ def gated_scan(q, k, v, gamma, h0=None, *, nthreads=None):
                                       _ptr(y), _ptr(fs), int(nthreads or num_threads()))
     _check(rc, "ss_oracle_gated_scan")
     return {"outputs": y, "final_state": fs}
+
+
+def segment(x, dt, A, B, dt_bias=None, reset=None, *, dt_softplus=True, nthreads=None):
+    """Composite of one segment ("s6_reset", Associative Boundary Resetting: the
+    segment's maps folded with the resettable operator).  Returns dict(decay
+    [b,c,n] = the product of the segment's decays, 0 when it holds a reset;
+    state [b,c,n] = its end state entered from zero)."""
+    x, dt, A, B, dt_bias = (_f64(v) for v in (x, dt, A, B, dt_bias))
+    reset = _u8(reset)
+    bt, ch, L = x.shape
+    n = A.shape[1]
+    if dt.shape != x.shape or A.shape != (ch, n) or B.shape != (bt, n, L):
+        raise ValueError("inconsistent shapes")
+    if dt_bias is not None and dt_bias.shape != (ch,):
+        raise ValueError("dt_bias must be [channels]")
+    if reset is not None and reset.shape != (bt, L):
+        raise ValueError("reset must be [batch, seq]")
+    decay = np.empty((bt, ch, n))
+    state = np.empty((bt, ch, n))
+    rc = _load().ss_oracle_segment(bt, ch, n, L, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(dt_bias),
+                                   _ptr(reset, _u8p), int(bool(dt_softplus)), _ptr(decay), _ptr(state),
+                                   int(nthreads or num_threads()))
+    _check(rc, "ss_oracle_segment")
+    return {"decay": decay, "state": state}
+
+
+def join_segments(decays, states, h0=None):
+    """Apply the composites of consecutive segments in order, starting from h0 (zeros
+    when None): carry_0 = h0, carry_{s+1} = decay_s * carry_s + state_s.  Returns
+    (carries, final): carries[s] is the state entering segment s, final the state
+    after the last one."""
+    carry = np.zeros_like(_f64(states[0])) if h0 is None else _f64(h0).copy()
+    carries = []
+    for d, st in zip(decays, states):
+        carries.append(carry.copy())
+        carry = _f64(d) * carry + _f64(st)
+    return carries, carry
 
 
 def scan_rows(inputs: dict, rows, *, dt_softplus=True, nthreads=1):

@@ -32,6 +32,8 @@
  *   ss_oracle_tree_scan -- an inclusive associative scan (recursive doubling) of
  *                          the affine maps h -> a*h + u with an explicit reset
  *                          flag ("s6_reset", "Associative Boundary Resetting").
+ * ss_oracle_segment folds one segment's maps with the same operator into a single
+ * composite (decay, end state), the unit a sequence cut into segments is joined by.
  * The test suite pins each against closed forms and against the other.
  *
  * Parallelism: OpenMP over independent (batch, channel) rows only, so that the
@@ -247,6 +249,54 @@ int ss_oracle_tree_scan(int64_t batch, int64_t channels, int64_t state_dim, int6
         free(steps);
     }
     return status;
+}
+
+/*
+ * Composite of one segment of the sequence (the affine map a whole segment applies
+ * to the state that enters it): the segment's elements h -> (r ? u : a*h + u) folded
+ * left to right with the operator above ("s6_reset", Associative Boundary
+ * Resetting).  The result, per (b, c, n), is written as the map h -> decay*h + state:
+ *
+ *   decay[b,c,n] = product over the segment of exp(dt_t * A[c,n]), or 0 when the
+ *                  segment holds a reset (the entering state is then discarded);
+ *   state[b,c,n] = the segment's end state when it is entered with h = 0.
+ *
+ * Applying the composites of consecutive segments in order to h0 gives the state
+ * at the end of their concatenation, which is what lets a sequence be cut into
+ * segments that are scanned independently and then joined.
+ */
+int ss_oracle_segment(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
+                      const double *x, const double *dt, const double *A, const double *B,
+                      const double *dt_bias, const uint8_t *reset, int dt_softplus,
+                      double *decay, double *state, int nthreads)
+{
+    if (!x || !dt || !A || !B || !decay || !state)
+        return ORC_ERR_NULL;
+    if (batch <= 0 || channels <= 0 || state_dim <= 0 || seq <= 0)
+        return ORC_ERR_SHAPE;
+    if (nthreads <= 0)
+        nthreads = 1;
+    const int64_t rows = batch * channels;
+
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1)
+    for (int64_t row = 0; row < rows; ++row) {
+        const int64_t b = row / channels;
+        const int64_t c = row % channels;
+        for (int64_t n = 0; n < state_dim; ++n) {
+            orc_elem acc = {1.0, 0.0, 0}; /* the identity map */
+            for (int64_t t = 0; t < seq; ++t) {
+                const double d = orc_step(dt, dt_bias, dt_softplus, row * seq + t, c);
+                orc_elem e;
+                e.a = exp(d * A[c * state_dim + n]);
+                e.u = d * B[(b * state_dim + n) * seq + t] * x[row * seq + t];
+                e.r = reset ? (reset[b * seq + t] != 0) : 0;
+                acc = orc_combine(acc, e);
+            }
+            decay[row * state_dim + n] = acc.r ? 0.0 : acc.a;
+            state[row * state_dim + n] = acc.u;
+        }
+    }
+    return ORC_OK;
 }
 
 /*
