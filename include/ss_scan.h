@@ -289,6 +289,58 @@ SS_API int ss_gated_scan(int64_t batch, int64_t seq, int64_t dk, int64_t dv, ss_
                          const void *q, const void *k, const void *v, const float *gamma,
                          const float *h0, void *outputs, void *final_state, ss_stream_t stream);
 
+/*
+ * Sequence cut into segments (one per GPU, say) -- the two joining steps.
+ *
+ * The scan's recurrence composes associatively ("s6_reset" blog draft, Associative
+ * Boundary Resetting: that is what lets a long sequence be scanned in parallel).  A
+ * segment acts on the state that enters it as the map h -> decay * h + state, with
+ *
+ *   decay[b,c,n] = prod over the segment of exp(dt_t * A[c,n])
+ *                = exp(A[c,n] * sum_t dt_t), and exactly 0 when reset[b,t] != 0 for
+ *                  some t of the segment (the entering state is then discarded);
+ *   state[b,c,n] = the segment's end state when it is entered from zero, i.e. the
+ *                  h_last of ss_scan_fwd on the segment with h0 = NULL.
+ *
+ * Joining: segment 0 is scanned from the real h0 and is final.  Every other segment
+ * s is scanned once from zero to get its composite; the composites of all segments
+ * are gathered (in segment order) on every GPU; ss_join_segments folds those before
+ * s into the state entering s; and ss_scan_fwd on segment s with that state as h0
+ * gives its final outputs.
+ *
+ * ss_segment_decay -- the decay of one segment.
+ *   dt_raw      : [batch, channels, seq] dtype
+ *   A           : [channels, state_dim] float32
+ *   dt_bias     : [channels] float32, nullable
+ *   reset       : [batch, seq] uint8, nullable (the segment's slice of the mask)
+ *   flags       : SS_DT_SOFTPLUS as for ss_scan_fwd (other bits: SS_ERR_UNSUPPORTED)
+ *   decay       : [batch, channels, state_dim] float32 (output)
+ * The step sizes are summed in float32; decay uses the same flush-to-zero exp2 as
+ * the scan.  state_dim must be 4, 8 or 16.  decay must not overlap an input
+ * (SS_ERR_ALIAS).  Asynchronous on `stream`; reads dt_raw once.
+ */
+SS_API int ss_segment_decay(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, ss_dtype_t dtype,
+                            const void *dt_raw, const float *A, const float *dt_bias, const uint8_t *reset,
+                            uint32_t flags, float *decay, ss_stream_t stream);
+
+/*
+ * ss_join_segments -- fold gathered composites in segment order.
+ *   composites  : [segments][2][count] float32: for segment s, decay at
+ *                 composites[(2s) * count ...] and end state at
+ *                 composites[(2s + 1) * count ...] (count = batch*channels*state_dim).
+ *                 Segment 0's entry holds its end state from the real h0; its decay
+ *                 is never read.
+ *   rank        : the segment whose entering state `carry` receives; 1 <= rank <
+ *                 segments when carry is not NULL (SS_ERR_SHAPE otherwise).
+ *   carry       : [count] float32, nullable: the state entering segment `rank`.
+ *   final_state : [count] float32, nullable: the state after the last segment.
+ * At least one of carry, final_state must be given (SS_ERR_NULL).  Outputs must not
+ * overlap composites or each other (SS_ERR_ALIAS).  float32 arithmetic, one fused
+ * multiply-add per segment and element.  Asynchronous on `stream`.
+ */
+SS_API int ss_join_segments(int64_t segments, int64_t count, const float *composites, int64_t rank,
+                            float *carry, float *final_state, ss_stream_t stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 SS_API const char *ss_status_string(int status);
 

@@ -12,10 +12,11 @@
 #include "ss_scan_fwd.cuh"
 #include "ss_state_update.cuh"
 #include "ss_gated_scan.cuh"
+#include "ss_segment.cuh"
 
 namespace {
 
-constexpr int kAbiMajor = 2, kAbiMinor = 1;
+constexpr int kAbiMajor = 2, kAbiMinor = 2;
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -833,6 +834,101 @@ int ss_scan_fwd_static_scratch(int64_t batch, int64_t channels, int64_t state_di
         return SS_ERR_CUDA;
     return ss_scan_fwd(batch, channels, state_dim, seq, dtype, x, dt_raw, A, B, C, D, z, dt_bias, reset, h0,
                        flags & uint32_t(SS_DT_SOFTPLUS), y, h_last, ws, SS_STATIC_SCRATCH_BYTES, stream);
+}
+
+
+int ss_segment_decay(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, ss_dtype_t dtype,
+                     const void *dt_raw, const float *A, const float *dt_bias, const uint8_t *reset,
+                     uint32_t flags, float *decay, ss_stream_t stream)
+{
+    if (!dt_raw || !A || !decay)
+        return SS_ERR_NULL;
+    if (batch <= 0 || channels <= 0 || state_dim <= 0 || seq <= 0)
+        return SS_ERR_SHAPE;
+    if (dtype != SS_F32 && dtype != SS_BF16)
+        return SS_ERR_DTYPE;
+    if ((state_dim != 4 && state_dim != 8 && state_dim != 16) || (flags & ~uint32_t(SS_DT_SOFTPLUS)))
+        return SS_ERR_UNSUPPORTED;
+    const size_t es = dtype == SS_BF16 ? 2 : 4;
+    int64_t rows = 0, el = 0, st = 0, bs = 0, an = 0;
+    if (!mul_ok(batch, channels, &rows) || !mul_ok(rows, seq, &el) || !mul_ok(rows, state_dim, &st) ||
+        !mul_ok(batch, seq, &bs) || !mul_ok(channels, state_dim, &an) || el > INT64_MAX / 8 ||
+        st > INT64_MAX / 8)
+        return SS_ERR_SHAPE;
+    if (!aligned(dt_raw, es) || !aligned(A, 4) || !aligned(decay, 4) || (dt_bias && !aligned(dt_bias, 4)))
+        return SS_ERR_ALIGN;
+    const void *in_p[] = {dt_raw, A, dt_bias, reset};
+    const size_t in_n[] = {size_t(el) * es, size_t(an) * 4, dt_bias ? size_t(channels) * 4 : 0,
+                           reset ? size_t(bs) : 0};
+    for (int i = 0; i < 4; ++i)
+        if (overlaps(decay, size_t(st) * 4, in_p[i], in_n[i]))
+            return SS_ERR_ALIAS;
+    ss::SegDecayArgs a{};
+    a.dt = dt_raw;
+    a.A = A;
+    a.dt_bias = dt_bias;
+    a.reset = reset;
+    a.decay = decay;
+    a.batch = batch;
+    a.channels = channels;
+    a.seq = seq;
+    a.state_dim = int(state_dim);
+    a.softplus = (flags & SS_DT_SOFTPLUS) ? 1 : 0;
+    a.reset_vec = reset && aligned(reset, 16) && seq % 16 == 0;
+    int sms = 0;
+    if (device_sm_count(&sms) != SS_OK)
+        return SS_ERR_CUDA;
+    // one warp per row; at most 8 blocks of 8 warps per SM, grid-strided beyond that
+    const int64_t blocks = (rows + ss::kSegWarps - 1) / ss::kSegWarps;
+    const unsigned grid = unsigned(blocks < int64_t(sms) * 8 ? blocks : int64_t(sms) * 8);
+    const bool vec = seq % 8 == 0 && aligned(dt_raw, 16);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == SS_BF16) {
+        if (vec)
+            ss::ss_segment_decay_kernel<__nv_bfloat16, true><<<grid, ss::kSegWarps * 32, 0, s>>>(a);
+        else
+            ss::ss_segment_decay_kernel<__nv_bfloat16, false><<<grid, ss::kSegWarps * 32, 0, s>>>(a);
+    } else {
+        if (vec)
+            ss::ss_segment_decay_kernel<float, true><<<grid, ss::kSegWarps * 32, 0, s>>>(a);
+        else
+            ss::ss_segment_decay_kernel<float, false><<<grid, ss::kSegWarps * 32, 0, s>>>(a);
+    }
+    return launch_status();
+}
+
+int ss_join_segments(int64_t segments, int64_t count, const float *composites, int64_t rank, float *carry,
+                     float *final_state, ss_stream_t stream)
+{
+    if (!composites || (!carry && !final_state))
+        return SS_ERR_NULL;
+    if (segments <= 0 || count <= 0 || segments > 0x7fffffffLL)
+        return SS_ERR_SHAPE;
+    if (carry && (rank < 1 || rank >= segments))
+        return SS_ERR_SHAPE;
+    int64_t per = 0, total = 0;
+    if (!mul_ok(count, 2, &per) || !mul_ok(per, segments, &total) || total > INT64_MAX / 4)
+        return SS_ERR_SHAPE;
+    if (!aligned(composites, 4) || (carry && !aligned(carry, 4)) || (final_state && !aligned(final_state, 4)))
+        return SS_ERR_ALIGN;
+    const size_t cb = size_t(total) * 4, ob = size_t(count) * 4;
+    if (overlaps(carry, ob, composites, cb) || overlaps(final_state, ob, composites, cb) ||
+        overlaps(carry, ob, final_state, ob))
+        return SS_ERR_ALIAS;
+    ss::JoinArgs a{};
+    a.comp = composites;
+    a.carry = carry;
+    a.final_state = final_state;
+    a.count = count;
+    a.segments = int(segments);
+    a.rank = carry ? int(rank) : 0;
+    int sms = 0;
+    if (device_sm_count(&sms) != SS_OK)
+        return SS_ERR_CUDA;
+    const int64_t blocks = (count + 255) / 256;
+    const unsigned grid = unsigned(blocks < int64_t(sms) * 8 ? blocks : int64_t(sms) * 8);
+    ss::ss_join_segments_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
 }
 
 } // extern "C"

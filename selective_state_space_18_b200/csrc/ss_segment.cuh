@@ -1,0 +1,119 @@
+// ss_segment.cuh -- joining a sequence that was cut into segments scanned apart.
+//
+// The recurrence h_t = a_t * h_{t-1} + u_t composes associatively ("s6_reset" blog
+// draft, Associative Boundary Resetting: pairs (a, u) combine as
+// (a_i, u_i) o (a_j, u_j) = (a_i a_j, a_j u_i + u_j), and a reset inside a segment
+// makes it discard the state that enters it).  A whole segment therefore acts on
+// its entering state as one map h -> decay * h + state, where
+//
+//   decay = prod_t exp(dt_t * A[c,n]) = exp(A[c,n] * sum_t dt_t), or 0 when the
+//           segment holds a reset for its batch row;
+//   state = the segment's end state entered from zero (a plain scan's h_last).
+//
+// Two kernels live here: the decay of one segment (the state comes from the scan
+// kernel itself), and the join of gathered composites into the state that enters
+// a given segment.  Both are small next to the scan: the first reads dt once (HBM
+// bound, 2 or 4 bytes per (b, c, t)), the second touches 2 floats per segment and
+// state element.
+#pragma once
+
+#include "ss_device.cuh"
+
+namespace ss {
+
+struct SegDecayArgs {
+    const void *dt;          // [batch, channels, seq] T
+    const float *A;          // [channels, state_dim]
+    const float *dt_bias;    // [channels] or null
+    const uint8_t *reset;    // [batch, seq] or null
+    float *decay;            // [batch, channels, state_dim]
+    int64_t batch, channels, seq;
+    int state_dim;
+    int softplus;            // apply softplus to dt_raw + dt_bias
+    int reset_vec;           // reset rows are 16-byte aligned and seq % 16 == 0
+};
+
+constexpr int kSegWarps = 8;
+
+// One warp per (b, c) row, grid-strided: the lanes sum the row's step sizes
+// (8 elements per 16-byte vector when VEC), OR the batch row's reset flags,
+// reduce across the warp, and lanes n < state_dim write exp2(A log2(e) sum).
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(kSegWarps * 32) ss_segment_decay_kernel(SegDecayArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t rows = a.batch * a.channels;
+    const int64_t stride = int64_t(gridDim.x) * kSegWarps;
+    for (int64_t row = int64_t(blockIdx.x) * kSegWarps + (threadIdx.x >> 5); row < rows; row += stride) {
+        const int64_t b = row / a.channels, c = row - b * a.channels;
+        const T *dr = static_cast<const T *>(a.dt) + row * a.seq;
+        const float bias = a.dt_bias ? __ldg(a.dt_bias + c) : 0.0f;
+        float sum = 0.0f;
+        if (VEC) {
+            // seq % 8 == 0: every vector the loop touches lies wholly inside the row
+            for (int64_t t = int64_t(lane) * 8; t < a.seq; t += 256) {
+                Raw8<T> v;
+                v.load_vec_stream(dr, t, a.seq);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float r = v.get(j) + bias;
+                    sum += a.softplus ? softplus(r) : r;
+                }
+            }
+        } else {
+            for (int64_t t = lane; t < a.seq; t += 32) {
+                const float r = Elem<T>::load(dr + t) + bias;
+                sum += a.softplus ? softplus(r) : r;
+            }
+        }
+        uint32_t any = 0;
+        if (a.reset) {
+            const uint8_t *rr = a.reset + b * a.seq;
+            if (a.reset_vec) {
+                for (int64_t t = int64_t(lane) * 16; t < a.seq; t += 512) {
+                    const uint4 w = __ldg(reinterpret_cast<const uint4 *>(rr + t));
+                    any |= w.x | w.y | w.z | w.w;
+                }
+            } else {
+                for (int64_t t = lane; t < a.seq; t += 32)
+                    any |= __ldg(rr + t);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        const bool discard = __any_sync(0xffffffffu, any != 0);
+        if (lane < a.state_dim) {
+            const float An = __ldg(a.A + c * a.state_dim + lane);
+            a.decay[row * a.state_dim + lane] = discard ? 0.0f : ex2(An * kLog2e * sum);
+        }
+    }
+}
+
+struct JoinArgs {
+    const float *comp;  // [segments][2][count]: decay then end state of each segment
+    float *carry;       // [count] or null: the state entering segment `rank`
+    float *final_state; // [count] or null: the state after the last segment
+    int64_t count;
+    int segments, rank;
+};
+
+// Element-wise fold of the composites in segment order.  Segment 0 was scanned from
+// the true initial state, so its end state starts the fold and its decay is unread.
+__global__ void __launch_bounds__(256) ss_join_segments_kernel(JoinArgs a)
+{
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < a.count; i += stride) {
+        float h = __ldg(a.comp + a.count + i);
+        for (int s = 1; s < a.segments; ++s) {
+            if (s == a.rank && a.carry)
+                a.carry[i] = h;
+            const float *cs = a.comp + int64_t(2 * s) * a.count;
+            h = fmaf(__ldg(cs + i), h, __ldg(cs + a.count + i));
+        }
+        if (a.final_state)
+            a.final_state[i] = h;
+    }
+}
+
+} // namespace ss

@@ -27,7 +27,7 @@ STATUS = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE", 4:
 EXPORTS = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_scan_status", "ss_state_update",
            "ss_debug_set_wait_limit", "ss_status_string", "ss_abi_version",
            "ss_scan_fwd_static_scratch", "ss_scan_fwd_states", "ss_gated_scan", "ss_scan_fwd_conv",
-           "ss_state_update_conv")
+           "ss_state_update_conv", "ss_segment_decay", "ss_join_segments")
 ABI_MAJOR = 2
 
 _lock = threading.Lock()
@@ -71,6 +71,11 @@ def load_library(path: str = LIB_PATH):
             lib.ss_state_update_conv.restype = ctypes.c_int
             lib.ss_gated_scan.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 7 + [_vp]
             lib.ss_gated_scan.restype = ctypes.c_int
+            lib.ss_segment_decay.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 4 + [
+                ctypes.c_uint32, _vp, _vp]
+            lib.ss_segment_decay.restype = ctypes.c_int
+            lib.ss_join_segments.argtypes = [_i64, _i64, _vp, _i64, _vp, _vp, _vp]
+            lib.ss_join_segments.restype = ctypes.c_int
             lib.ss_scan_workspace_bytes.argtypes = [_i64, _i64, _i64, _i64]
             lib.ss_scan_workspace_bytes.restype = _i64
             lib.ss_scan_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_int)]
@@ -460,3 +465,67 @@ def ss_state_update_conv(state, conv_state, conv_w, u, dt, A, B, C, D=None, z=No
     if st != 0:
         raise SSError("ss_state_update_conv", st)
     return y
+
+
+def ss_segment_decay(dt, A, dt_bias=None, reset=None, *, dt_softplus=True, out=None, stream=None):
+    """Decay of one segment of a sequence: [batch, channels, state_dim] fp32 =
+    exp(A * sum of the segment's step sizes), 0 where the segment holds a reset.
+    dt: [batch, channels, seq] (the segment's slice); reset: [batch, seq] or None.
+    ``out`` (contiguous fp32) is written in place when given."""
+    if dt.dim() != 3:
+        raise ValueError("dt must be [batch, channels, seq]")
+    dev = dt.device
+    if dev.type != "cuda":
+        raise ValueError("ss_segment_decay runs on CUDA tensors only")
+    bt, ch, L = dt.shape
+    n = A.shape[-1]
+    code = _dtype_code(dt)
+    dt = _prep(dt, "dt", dev)
+    A = _prep(A, "A", dev, torch.float32, (ch, n))
+    dt_bias = _prep(dt_bias, "dt_bias", dev, torch.float32, (ch,))
+    if reset is not None:
+        reset = _prep(reset, "reset", dev, None, (bt, L))
+        if reset.dtype == torch.bool:
+            reset = reset.view(torch.uint8)
+        elif reset.dtype != torch.uint8:
+            raise TypeError("reset must be bool or uint8")
+    if out is None:
+        out = torch.empty(bt, ch, n, device=dev, dtype=torch.float32)
+    else:
+        out = _out(out, "out", dev, torch.float32, (bt, ch, n))
+    flags = SS_DT_SOFTPLUS if dt_softplus else 0
+    st = load_library().ss_segment_decay(bt, ch, n, L, code, _ptr(dt), _ptr(A), _ptr(dt_bias), _ptr(reset),
+                                         flags, _ptr(out), _stream(stream, dev))
+    if st != 0:
+        raise SSError("ss_segment_decay", st)
+    return out
+
+
+def ss_join_segments(composites, rank=None, *, carry=None, final_state=None, want_final=True, stream=None):
+    """Fold gathered segment composites [segments, 2, ...] (decay, end state; fp32,
+    contiguous) in segment order.  Returns (carry, final_state): the state entering
+    segment ``rank`` (None when rank is None) and, when ``want_final``, the state
+    after the last segment; both have the composites' trailing shape."""
+    if composites.dim() < 3 or composites.shape[1] != 2:
+        raise ValueError("composites must be [segments, 2, ...]")
+    dev = composites.device
+    if dev.type != "cuda":
+        raise ValueError("ss_join_segments runs on CUDA tensors only")
+    if composites.dtype != torch.float32 or not composites.is_contiguous():
+        raise ValueError("composites must be a contiguous float32 tensor")
+    segs = composites.shape[0]
+    shape = tuple(composites.shape[2:])
+    count = composites[0, 0].numel()
+    if rank is not None and carry is None:
+        carry = torch.empty(shape, device=dev, dtype=torch.float32)
+    elif carry is not None:
+        carry = _out(carry, "carry", dev, torch.float32, shape)
+    if want_final and final_state is None:
+        final_state = torch.empty(shape, device=dev, dtype=torch.float32)
+    elif final_state is not None:
+        final_state = _out(final_state, "final_state", dev, torch.float32, shape)
+    st = load_library().ss_join_segments(segs, count, _ptr(composites), -1 if rank is None else int(rank),
+                                         _ptr(carry), _ptr(final_state), _stream(stream, dev))
+    if st != 0:
+        raise SSError("ss_join_segments", st)
+    return carry, final_state

@@ -251,3 +251,42 @@ def test_decode_conv_checks(lib):
     assert call(cs=None) == "SS_ERR_NULL"
     assert call(cs=ctypes.c_void_p(P[0].value + 64)) == "SS_ERR_ALIAS"   # conv state over the state
     assert call(cs=ctypes.c_void_p(P[7].value + 2)) == "SS_ERR_ALIGN"
+
+
+def test_segment_decay_checks(lib):
+    E = ssscan.STATUS
+
+    def call(**kw):
+        a = dict(batch=1, channels=16, state_dim=16, seq=64, dtype=ssscan.SS_BF16, dt=P[0], A=P[1],
+                 dt_bias=None, reset=None, flags=1, decay=P[2])
+        a.update(kw)
+        return E[lib.ss_segment_decay(a["batch"], a["channels"], a["state_dim"], a["seq"], a["dtype"], a["dt"],
+                                      a["A"], a["dt_bias"], a["reset"], a["flags"], a["decay"], None)]
+
+    assert call(dt=None) == "SS_ERR_NULL"
+    assert call(decay=None) == "SS_ERR_NULL"
+    assert call(seq=0) == "SS_ERR_SHAPE"
+    assert call(dtype=7) == "SS_ERR_DTYPE"
+    assert call(state_dim=5) == "SS_ERR_UNSUPPORTED"
+    assert call(flags=2) == "SS_ERR_UNSUPPORTED"
+    assert call(A=ctypes.c_void_p(P[1].value + 2)) == "SS_ERR_ALIGN"
+    assert call(decay=ctypes.c_void_p(P[0].value + 64)) == "SS_ERR_ALIAS"   # inside dt
+    assert call(batch=1 << 40, channels=1 << 40) == "SS_ERR_SHAPE"
+
+
+def test_join_segments_checks(lib):
+    E = ssscan.STATUS
+
+    def call(segments=4, count=256, comp=P[0], rank=1, carry=P[1], final=P[2]):
+        return E[lib.ss_join_segments(segments, count, comp, rank, carry, final, None)]
+
+    assert call(comp=None) == "SS_ERR_NULL"
+    assert call(carry=None, final=None) == "SS_ERR_NULL"
+    assert call(segments=0) == "SS_ERR_SHAPE"
+    assert call(count=0) == "SS_ERR_SHAPE"
+    assert call(rank=0) == "SS_ERR_SHAPE"          # segment 0's entering state is h0 itself
+    assert call(rank=4) == "SS_ERR_SHAPE"
+    assert call(carry=ctypes.c_void_p(P[1].value + 1)) == "SS_ERR_ALIGN"
+    assert call(carry=ctypes.c_void_p(P[0].value + 1024)) == "SS_ERR_ALIAS"  # inside the composites
+    assert call(final=ctypes.c_void_p(P[1].value + 512)) == "SS_ERR_ALIAS"   # overlaps carry
+    assert call(count=1 << 62) == "SS_ERR_SHAPE"
