@@ -178,6 +178,7 @@ def test_segment_decay_without_softplus():
     d = _cuda()
     inp = make_scan_inputs(1, 24, 16, 513, "f32", seed=2)
     inp["dt"] = inp["dt"].abs() * 0.01       # positive steps, no bias: decays in (0, 1]
+    inp["A"] = inp["A"] * 0.05
     ref = oracle.segment(inp["x"], inp["dt"], inp["A"], inp["B"], None, dt_softplus=False)["decay"]
     got = seqshard.ssscan.ss_segment_decay(inp["dt"].to(d), inp["A"].to(d), None,
                                            dt_softplus=False).cpu().double().numpy()
@@ -194,7 +195,9 @@ def test_join_matches_oracle(segments):
     comp[:, 0] = torch.rand(segments, 3, 33, 16, generator=g)
     comp[:, 1] = torch.randn(segments, 3, 33, 16, generator=g)
     comp[0, 0] = float("nan")        # segment 0's decay is never read
-    carries, final = oracle.join_segments(comp[:, 0].double().numpy(), comp[:, 1].double().numpy())
+    ref_decay = comp[:, 0].double().numpy().copy()
+    ref_decay[0] = 0.0               # the oracle's join starts from zeros, so any finite value does
+    carries, final = oracle.join_segments(ref_decay, comp[:, 1].double().numpy())
     for rank in range(1, segments):
         carry, fin = seqshard.ssscan.ss_join_segments(comp.to(d), rank)
         e = np.abs(carry.cpu().double().numpy() - carries[rank]) / (1 + np.abs(carries[rank]))
