@@ -12,6 +12,11 @@ channels 5120, state_dim 16, fp32 state in place).  The metric is scan elements
 With N > 1 (launched by torch.distributed.run) every rank runs the same per-GPU
 workload on its own problems (weak scaling, no data-path collective); the time is
 the maximum over ranks of the device-timed region.  Rank 0 prints one JSON line.
+
+    python bench.py --seq-shard [--emulate-ranks R] ...
+
+times the prompt scan alone with its one sequence cut into a segment per rank
+(strong scaling; one NCCL all-gather of segment composites per step).
 """
 from __future__ import annotations
 
@@ -513,6 +518,146 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_seq_shard(args):
+    """The 2.8B-layer prompt cut into sequence segments, one per rank (strong scaling):
+    each rank scans its segment, the segments' composites are all-gathered (NCCL), and
+    every rank but 0 rescans from its joined entering state.  With one process and
+    --emulate-ranks R, the R segments run one after another on this GPU and each
+    emulated rank's own work is timed separately (the all-gather is not emulated)."""
+    from selective_state_space_18_b200 import seqshard, ssscan
+
+    world, rank, local = _dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    ssscan.load_library()
+    emulate = args.emulate_ranks if world == 1 else 1
+    segs = max(world, emulate)
+    full = make_workload(PROMPT, seed=PROMPT.seed)
+    L = full["x"].shape[-1]
+    bounds = seqshard.shard_bounds(L, segs)
+    seq_keys = ("x", "dt", "z", "B", "C")
+
+    def part(r):
+        a, b = bounds[r]
+        q = {k: (None if v is None else (v[..., a:b].contiguous() if k in seq_keys else v).to(dev))
+             for k, v in full.items() if k not in ("reset", "h0")}
+        q["dt_softplus"] = True
+        return q
+
+    mine = [part(r) for r in range(segs)] if emulate > 1 else [part(rank)]
+    del full
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 256 MB > L2
+
+    if emulate > 1:
+        K = args.steps
+        ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+                torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(segs)] for _ in range(K + args.warmup)]
+
+        def step(i):
+            ys, comps = [], []
+            for r, q in enumerate(mine):
+                ev[i][r][0].record(stream)
+                y, comp = seqshard.local_pass(q, r)
+                ev[i][r][1].record(stream)
+                ys.append(y)
+                comps.append(comp)
+            gathered = torch.stack(comps)
+            for r, q in enumerate(mine):
+                ev[i][r][2].record(stream)
+                seqshard.finish_pass(q, r, gathered, ys[r])
+                ev[i][r][3].record(stream)
+
+        for i in range(args.warmup):
+            step(i)
+        torch.cuda.synchronize(dev)
+        sampler = ClockSampler(local)
+        sampler.start()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(args.warmup, args.warmup + K):
+            step(i)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        clocks = sampler.stop()
+        serial_ms = start.elapsed_time(end) / K
+        per_rank = []
+        for r in range(segs):
+            loc = sum(ev[i][r][0].elapsed_time(ev[i][r][1]) for i in range(args.warmup, args.warmup + K)) / K
+            fin = sum(ev[i][r][2].elapsed_time(ev[i][r][3]) for i in range(args.warmup, args.warmup + K)) / K
+            per_rank.append({"rank": r, "tokens": bounds[r][1] - bounds[r][0], "local_pass_ms": round(loc, 5),
+                             "finish_pass_ms": round(fin, 5)})
+        worst = max(p["local_pass_ms"] + p["finish_pass_ms"] for p in per_rank)
+        ms = serial_ms
+        launches = K * (1 + 4 * (segs - 1))
+        extra = {"emulated": {"ranks": segs, "per_rank": per_rank, "max_rank_compute_ms": round(worst, 5),
+                              "note": "all segments on one GPU in turn; the value is that serial time. "
+                                      "max_rank_compute_ms is the slowest emulated rank's own kernels, "
+                                      "without the all-gather of composites"}}
+    else:
+        q = mine[0]
+        K = args.steps
+        for _ in range(args.warmup):
+            seqshard.seq_sharded_scan(q["x"], q["dt"], q["A"], q["B"], q["C"], q["D"], q["z"], q["dt_bias"])
+        torch.cuda.synchronize(dev)
+        sampler = ClockSampler(local)
+        sampler.start()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        _barrier(world)
+        torch.cuda.synchronize(dev)
+        for i in range(K):
+            flush.zero_()                      # L2 flushed between steps, outside the timed events
+            ev[i][0].record(stream)
+            seqshard.seq_sharded_scan(q["x"], q["dt"], q["A"], q["B"], q["C"], q["D"], q["z"], q["dt_bias"])
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        _barrier(world)
+        clocks = sampler.stop()
+        ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev) / K, world, dev)
+        launches = K * (1 if world == 1 else 4)
+        extra = {}
+
+    elems = PROMPT.batch * PROMPT.channels * PROMPT.state_dim * L
+    line = {
+        "metric": "scan elems/s (B·L·D·N), 2.8B-shape prompt cut into sequence segments",
+        "value": elems / (ms * 1e-3),
+        "unit": "elems/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "strong",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": "mamba2p8b_layer_long prompt scan (batch 1, channels 5120, state_dim 16, seq 16384, "
+                        "bf16 x/dt/z/B/C/y, z gate, dt_bias, fp32 state), one sequence cut into segments",
+            "segments": bounds,
+            "parallelism": (f"sequence segments x{world}: NCCL all-gather of segment composites" if world > 1
+                            else f"{segs} segments emulated on one GPU" if segs > 1 else "one segment"),
+            "l2": ("all segments' inputs (673 MB) per step" if emulate > 1
+                   else "256 MB buffer written between steps, outside the timed events"),
+        },
+        **extra,
+        "clocks": clocks,
+        "gpu_launches": launches,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -525,11 +670,17 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--sets", type=int, default=2, choices=[1, 2],
                     help="rotating input sets (1 for small profiler captures)")
+    ap.add_argument("--seq-shard", action="store_true",
+                    help="time the prompt scan with its sequence cut into one segment per rank (strong scaling)")
+    ap.add_argument("--emulate-ranks", type=int, default=1,
+                    help="with --seq-shard on one process: run this many segments on the one GPU")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.seq_shard:
+        run_seq_shard(args)
     else:
         run_ours(args)
 

@@ -50,7 +50,9 @@ __global__ void __launch_bounds__(kSegWarps * 32) ss_segment_decay_kernel(SegDec
         const float bias = a.dt_bias ? __ldg(a.dt_bias + c) : 0.0f;
         float sum = 0.0f;
         if (VEC) {
-            // seq % 8 == 0: every vector the loop touches lies wholly inside the row
+            // seq % 8 == 0: every vector the loop touches lies wholly inside the row;
+            // unrolled so that several 16-byte loads per lane are in flight at once
+#pragma unroll 4
             for (int64_t t = int64_t(lane) * 8; t < a.seq; t += 256) {
                 Raw8<T> v;
                 v.load_vec_stream(dr, t, a.seq);
@@ -61,6 +63,7 @@ __global__ void __launch_bounds__(kSegWarps * 32) ss_segment_decay_kernel(SegDec
                 }
             }
         } else {
+#pragma unroll 8
             for (int64_t t = lane; t < a.seq; t += 32) {
                 const float r = Elem<T>::load(dr + t) + bias;
                 sum += a.softplus ? softplus(r) : r;
