@@ -602,6 +602,20 @@ template <typename T> int dispatch_gated(const ss::GatedArgs &a, cudaStream_t s)
     return dispatch_gated_v<16, T>(a, s);
 }
 
+template <typename T>
+void launch_segment_decay(bool vec, bool sp, unsigned grid, const ss::SegDecayArgs &a, cudaStream_t s)
+{
+    const unsigned threads = ss::kSegWarps * 32;
+    if (vec && sp)
+        ss::ss_segment_decay_kernel<T, true, true><<<grid, threads, 0, s>>>(a);
+    else if (vec)
+        ss::ss_segment_decay_kernel<T, true, false><<<grid, threads, 0, s>>>(a);
+    else if (sp)
+        ss::ss_segment_decay_kernel<T, false, true><<<grid, threads, 0, s>>>(a);
+    else
+        ss::ss_segment_decay_kernel<T, false, false><<<grid, threads, 0, s>>>(a);
+}
+
 } // namespace
 
 extern "C" {
@@ -873,7 +887,6 @@ int ss_segment_decay(int64_t batch, int64_t channels, int64_t state_dim, int64_t
     a.channels = channels;
     a.seq = seq;
     a.state_dim = int(state_dim);
-    a.softplus = (flags & SS_DT_SOFTPLUS) ? 1 : 0;
     a.reset_vec = reset && aligned(reset, 16) && seq % 16 == 0;
     int sms = 0;
     if (device_sm_count(&sms) != SS_OK)
@@ -882,18 +895,12 @@ int ss_segment_decay(int64_t batch, int64_t channels, int64_t state_dim, int64_t
     const int64_t blocks = (rows + ss::kSegWarps - 1) / ss::kSegWarps;
     const unsigned grid = unsigned(blocks < int64_t(sms) * 8 ? blocks : int64_t(sms) * 8);
     const bool vec = seq % 8 == 0 && aligned(dt_raw, 16);
+    const bool sp = (flags & SS_DT_SOFTPLUS) != 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (dtype == SS_BF16) {
-        if (vec)
-            ss::ss_segment_decay_kernel<__nv_bfloat16, true><<<grid, ss::kSegWarps * 32, 0, s>>>(a);
-        else
-            ss::ss_segment_decay_kernel<__nv_bfloat16, false><<<grid, ss::kSegWarps * 32, 0, s>>>(a);
-    } else {
-        if (vec)
-            ss::ss_segment_decay_kernel<float, true><<<grid, ss::kSegWarps * 32, 0, s>>>(a);
-        else
-            ss::ss_segment_decay_kernel<float, false><<<grid, ss::kSegWarps * 32, 0, s>>>(a);
-    }
+    if (dtype == SS_BF16)
+        launch_segment_decay<__nv_bfloat16>(vec, sp, grid, a, s);
+    else
+        launch_segment_decay<float>(vec, sp, grid, a, s);
     return launch_status();
 }
 

@@ -2,8 +2,10 @@
 //
 // Element access for the two storage types (fp32, bf16), the MUFU base-2
 // exponential, and the two pointwise functions of the S6 step: softplus for the
-// step size and silu for the output gate (nnterp "selective_scan" component:
-// dt = softplus(dt_proj(x) + dt_bias); the output is y gated by silu(z)).
+// step size (a series form, and the polynomial form that the prompt scan and the
+// segment decay share, scalar and packed) and silu for the output gate (nnterp
+// "selective_scan" component: dt = softplus(dt_proj(x) + dt_bias); the output is y
+// gated by silu(z)).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -45,6 +47,42 @@ __device__ __forceinline__ float log1p_unit(float e)
 __device__ __forceinline__ float softplus(float r)
 {
     return fmaxf(r, 0.0f) + log1p_unit(ex2(-fabsf(r) * kLog2e));
+}
+
+// softplus(r) = max(r, 0) + log(1 + e), e = exp(-|r|) in (0, 1].  log(1 + e) = e Q(e)
+// with Q a degree-8 polynomial fitted to log1p(e)/e on [0, 1] for relative error
+// (1.5e-7 in fp32 Horner form): no division, one MUFU op.
+__device__ __forceinline__ float softplus_poly(float r)
+{
+    const float e = ex2(-fabsf(r) * kLog2e);
+    float q = 5.232690697e-03f;
+    q = fmaf(q, e, -2.950522892e-02f);
+    q = fmaf(q, e, 7.822594434e-02f);
+    q = fmaf(q, e, -1.366324604e-01f);
+    q = fmaf(q, e, 1.910600743e-01f);
+    q = fmaf(q, e, -2.484298259e-01f);
+    q = fmaf(q, e, 3.331909690e-01f);
+    q = fmaf(q, e, -4.999949315e-01f);
+    q = fmaf(q, e, 9.999999699e-01f);
+    return fmaxf(r, 0.0f) + e * q;
+}
+
+// The same for two tokens at once with packed fp32x2 arithmetic; the polynomial
+// and the final e Q(e) + max(r, 0) run as fp32x2 fused multiply-adds.
+__device__ __forceinline__ float2 softplus_poly2(float2 r)
+{
+    const float2 t = __fmul2_rn(make_float2(-fabsf(r.x), -fabsf(r.y)), make_float2(kLog2e, kLog2e));
+    const float2 e = make_float2(ex2(t.x), ex2(t.y));
+    float2 q = make_float2(5.232690697e-03f, 5.232690697e-03f);
+    q = __ffma2_rn(q, e, make_float2(-2.950522892e-02f, -2.950522892e-02f));
+    q = __ffma2_rn(q, e, make_float2(7.822594434e-02f, 7.822594434e-02f));
+    q = __ffma2_rn(q, e, make_float2(-1.366324604e-01f, -1.366324604e-01f));
+    q = __ffma2_rn(q, e, make_float2(1.910600743e-01f, 1.910600743e-01f));
+    q = __ffma2_rn(q, e, make_float2(-2.484298259e-01f, -2.484298259e-01f));
+    q = __ffma2_rn(q, e, make_float2(3.331909690e-01f, 3.331909690e-01f));
+    q = __ffma2_rn(q, e, make_float2(-4.999949315e-01f, -4.999949315e-01f));
+    q = __ffma2_rn(q, e, make_float2(9.999999699e-01f, 9.999999699e-01f));
+    return __ffma2_rn(e, q, make_float2(fmaxf(r.x, 0.0f), fmaxf(r.y, 0.0f)));
 }
 
 // silu(v) = v / (1 + e^{-v}).

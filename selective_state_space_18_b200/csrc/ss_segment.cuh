@@ -29,7 +29,6 @@ struct SegDecayArgs {
     float *decay;            // [batch, channels, state_dim]
     int64_t batch, channels, seq;
     int state_dim;
-    int softplus;            // apply softplus to dt_raw + dt_bias
     int reset_vec;           // reset rows are 16-byte aligned and seq % 16 == 0
 };
 
@@ -37,8 +36,10 @@ constexpr int kSegWarps = 8;
 
 // One warp per (b, c) row, grid-strided: the lanes sum the row's step sizes
 // (8 elements per 16-byte vector when VEC), OR the batch row's reset flags,
-// reduce across the warp, and lanes n < state_dim write exp2(A log2(e) sum).
-template <typename T, bool VEC>
+// reduce across the warp, and lanes n < state_dim write exp2(A log2(e) sum).  SP:
+// the step is softplus(dt_raw + dt_bias), computed exactly as the prompt scan's
+// producers compute it (the same polynomial, packed two tokens at a time).
+template <typename T, bool VEC, bool SP>
 __global__ void __launch_bounds__(kSegWarps * 32) ss_segment_decay_kernel(SegDecayArgs a)
 {
     const int lane = threadIdx.x & 31;
@@ -52,21 +53,23 @@ __global__ void __launch_bounds__(kSegWarps * 32) ss_segment_decay_kernel(SegDec
         if (VEC) {
             // seq % 8 == 0: every vector the loop touches lies wholly inside the row;
             // unrolled so that several 16-byte loads per lane are in flight at once
+            float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll 4
             for (int64_t t = int64_t(lane) * 8; t < a.seq; t += 256) {
                 Raw8<T> v;
                 v.load_vec_stream(dr, t, a.seq);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float r = v.get(j) + bias;
-                    sum += a.softplus ? softplus(r) : r;
+                for (int k = 0; k < 4; ++k) {
+                    const float2 r = __fadd2_rn(make_float2(v.get(2 * k), v.get(2 * k + 1)), make_float2(bias, bias));
+                    acc = __fadd2_rn(acc, SP ? softplus_poly2(r) : r);
                 }
             }
+            sum = acc.x + acc.y;
         } else {
 #pragma unroll 8
             for (int64_t t = lane; t < a.seq; t += 32) {
                 const float r = Elem<T>::load(dr + t) + bias;
-                sum += a.softplus ? softplus(r) : r;
+                sum += SP ? softplus_poly(r) : r;
             }
         }
         uint32_t any = 0;
