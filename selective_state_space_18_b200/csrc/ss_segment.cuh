@@ -33,6 +33,7 @@ struct SegDecayArgs {
 };
 
 constexpr int kSegWarps = 8;
+constexpr int kSegBatch = 4; // 16-byte loads in flight per lane
 
 // One warp per (b, c) row, grid-strided: the lanes sum the row's step sizes
 // (8 elements per 16-byte vector when VEC), OR the batch row's reset flags,
@@ -51,17 +52,25 @@ __global__ void __launch_bounds__(kSegWarps * 32) ss_segment_decay_kernel(SegDec
         const float bias = a.dt_bias ? __ldg(a.dt_bias + c) : 0.0f;
         float sum = 0.0f;
         if (VEC) {
-            // seq % 8 == 0: every vector the loop touches lies wholly inside the row;
-            // unrolled so that several 16-byte loads per lane are in flight at once
+            // seq % 8 == 0, so each vector lies wholly inside the row or wholly past it.
+            // The loads of a batch are all issued before any of them is used, so each
+            // lane keeps kSegBatch 16-byte loads in flight.
             float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll 4
-            for (int64_t t = int64_t(lane) * 8; t < a.seq; t += 256) {
-                Raw8<T> v;
-                v.load_vec_stream(dr, t, a.seq);
+            for (int64_t t0 = int64_t(lane) * 8; t0 < a.seq; t0 += 256 * kSegBatch) {
+                Raw8<T> v[kSegBatch];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float2 r = __fadd2_rn(make_float2(v.get(2 * k), v.get(2 * k + 1)), make_float2(bias, bias));
-                    acc = __fadd2_rn(acc, SP ? softplus_poly2(r) : r);
+                for (int i = 0; i < kSegBatch; ++i)
+                    v[i].load_vec_stream(dr, t0 + 256 * i, a.seq);
+#pragma unroll
+                for (int i = 0; i < kSegBatch; ++i) {
+                    if (t0 + 256 * i >= a.seq)
+                        break;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 r = __fadd2_rn(make_float2(v[i].get(2 * k), v[i].get(2 * k + 1)),
+                                                    make_float2(bias, bias));
+                        acc = __fadd2_rn(acc, SP ? softplus_poly2(r) : r);
+                    }
                 }
             }
             sum = acc.x + acc.y;
