@@ -248,7 +248,8 @@ int launch_update(ss::UpdateArgs a, cudaStream_t stream, const UpdConv &cv)
         auto kernel = ss::ss_state_update_stream_kernel<N, T, CV>;
         static std::atomic<uint64_t> smem_done{0};
         static std::atomic<int> occ_cache[64];
-        int st = ensure_smem(kernel, D::kSmem, smem_done);
+        constexpr size_t kSmem = D::template smem<CV>();
+        int st = ensure_smem(kernel, kSmem, smem_done);
         if (st != SS_OK)
             return st;
         int dev = 0, sms = 0;
@@ -256,7 +257,7 @@ int launch_update(ss::UpdateArgs a, cudaStream_t stream, const UpdConv &cv)
             return SS_ERR_CUDA;
         int occ = dev < 64 ? occ_cache[dev].load(std::memory_order_acquire) : 0;
         if (!occ) {
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, ss::kDecBlock, D::kSmem) != cudaSuccess)
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, ss::kDecBlock, kSmem) != cudaSuccess)
                 return SS_ERR_CUDA;
             occ = occ > 0 ? occ : 1;
             if (dev < 64)
@@ -284,10 +285,12 @@ int launch_update(ss::UpdateArgs a, cudaStream_t stream, const UpdConv &cv)
         da.conv_b = cv.b;
         da.conv_state = cv.state;
         da.conv_k = cv.k;
+        // conv-state rows ride along too when every tile's rows start and end on 16 bytes
+        da.bulk_cs = CV && cv.k > 1 && aligned(cv.state, 16) && a.channels % 4 == 0;
         uint32_t *status = nullptr;
         if (status_word_address(&status) != SS_OK)
             return SS_ERR_CUDA;
-        kernel<<<unsigned(grid), ss::kDecBlock, D::kSmem, stream>>>(da, status);
+        kernel<<<unsigned(grid), ss::kDecBlock, kSmem, stream>>>(da, status);
         return launch_status();
     }
     if constexpr (CV)

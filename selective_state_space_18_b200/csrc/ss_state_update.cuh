@@ -173,7 +173,15 @@ template <int N, typename T> struct DecShape {
     static constexpr int kBCOff = kDecTileBytes + 3 * kVecBytes;  // B then C of the row
     static constexpr int kStageBytes = kBCOff + 2 * 64;
     static constexpr size_t kSmem = size_t(kDecStages) * kStageBytes + 16 * kDecStages; // + full, empty
-    static_assert(kStageBytes % 16 == 0, "16-byte aligned stages");
+    // the fused conv form also copies the tile's conv-state rows (up to 3 inputs each)
+    static constexpr int kCSOff = kStageBytes;
+    static constexpr int kStageBytesConv = kCSOff + kChanPerTile * 3 * 4;
+    template <bool CONV> static constexpr int stage_bytes() { return CONV ? kStageBytesConv : kStageBytes; }
+    template <bool CONV> static constexpr size_t smem()
+    {
+        return size_t(kDecStages) * stage_bytes<CONV>() + 16 * kDecStages;
+    }
+    static_assert(kStageBytes % 16 == 0 && kStageBytesConv % 16 == 0, "16-byte aligned stages");
 };
 
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
@@ -190,6 +198,7 @@ struct DecArgs {
     int fixed_cb;    // grid is a multiple of ncb: CTA i keeps channel block i % ncb
     int bulk_xdz;    // x, dt_raw (and z) rows are copied with the state
     int bulk_bc;     // B and C rows are copied with the state
+    int bulk_cs;     // conv form: the tile's conv-state rows are copied with the state
     // conv form: x above is the conv input u; x = silu(conv_b + conv_w . [state, u])
     const float *conv_w, *conv_b; // [channels, conv_k], [channels] (nullable)
     float *conv_state;            // [batch, channels, conv_k - 1] in/out
@@ -204,9 +213,10 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
 {
     using D = DecShape<N, T>;
     constexpr int Q = D::kQ;
+    constexpr int kStage = D::template stage_bytes<CONV>();
     const UpdateArgs &p = da.u;
     extern __shared__ __align__(128) unsigned char dsm[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(dsm + size_t(kDecStages) * D::kStageBytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(dsm + size_t(kDecStages) * kStage);
     uint64_t *empty = full + kDecStages;
     const int tid = threadIdx.x, lane_q = tid & (Q - 1);
 
@@ -234,8 +244,10 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
         const uint32_t sbytes = uint32_t(nch * N * 4), vbytes = uint32_t(nch * int64_t(sizeof(T)));
         const int nvec = da.bulk_xdz ? (p.z ? 3 : 2) : 0;
         const uint32_t bcbytes = da.bulk_bc ? uint32_t(2 * N * sizeof(T)) : 0u;
-        unsigned char *dst = dsm + size_t(stage) * D::kStageBytes;
-        mbar_arrive_expect_tx(full + stage, sbytes + nvec * vbytes + bcbytes);
+        // (bulk_cs: channels % 4 == 0, so row0 * H * 4 and nch * H * 4 are multiples of 16)
+        const uint32_t csbytes = (CONV && da.bulk_cs) ? uint32_t(nch * (da.conv_k - 1) * 4) : 0u;
+        unsigned char *dst = dsm + size_t(stage) * kStage;
+        mbar_arrive_expect_tx(full + stage, sbytes + nvec * vbytes + bcbytes + csbytes);
         bulk_load(dst, p.state + row0 * N, sbytes, full + stage);
         if (nvec) {
             bulk_load(dst + kDecTileBytes, static_cast<const T *>(p.x) + row0, vbytes, full + stage);
@@ -248,6 +260,8 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
             bulk_load(dst + D::kBCOff, static_cast<const T *>(p.B) + b * N, bcbytes / 2, full + stage);
             bulk_load(dst + D::kBCOff + 64, static_cast<const T *>(p.C) + b * N, bcbytes / 2, full + stage);
         }
+        if (csbytes)
+            bulk_load(dst + D::kCSOff, da.conv_state + row0 * (da.conv_k - 1), csbytes, full + stage);
         return true;
     };
 
@@ -314,7 +328,7 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
         // the conv state of each item's row (read by the row's lanes before its first
         // lane writes the shifted state back, below)
         float cs[CONV ? kDecItems : 1][3];
-        if constexpr (CONV) {
+        if (CONV && !da.bulk_cs) {
 #pragma unroll
             for (int it = 0; it < kDecItems; ++it) {
                 const int q = tid + it * kDecThreads;
@@ -346,7 +360,7 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
             ok = false;
             break;
         }
-        const unsigned char *sb = dsm + size_t(stage) * D::kStageBytes;
+        const unsigned char *sb = dsm + size_t(stage) * kStage;
         const float4 *sv = reinterpret_cast<const float4 *>(sb);
         if (da.bulk_bc) {
             bv = Vec4<T>::load_smem(reinterpret_cast<const T *>(sb + D::kBCOff) + 4 * lane_q);
@@ -363,6 +377,17 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
                 xs[it] = Elem<T>::load_smem(sx + cl);
                 ds[it] = Elem<T>::load_smem(sd + cl);
                 zs[it] = p.z ? Elem<T>::load_smem(sz + cl) : 0.0f;
+            }
+        }
+        if (CONV && da.bulk_cs) { // the conv state arrived with the tile
+            const float *scs = reinterpret_cast<const float *>(sb + D::kCSOff);
+#pragma unroll
+            for (int it = 0; it < kDecItems; ++it) {
+                const int q = tid + it * kDecThreads;
+                const int cl = (q < nq ? q : nq - 1) / Q;
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+                    cs[it][j] = j < H ? scs[cl * H + j] : 0.0f;
             }
         }
         if constexpr (CONV) {

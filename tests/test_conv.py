@@ -95,7 +95,8 @@ def _upd_inputs(bt, ch, n, dtype, K, seed):
 
 
 @pytest.mark.parametrize("case", [(256, 5120, 16, "bf16", 4), (3, 37, 8, "f32", 3), (5, 64, 4, "f32", 2),
-                                  (4, 100, 16, "bf16", 1)], ids=lambda c: "x".join(str(v) for v in c))
+                                  (4, 100, 16, "bf16", 1), (3, 1000, 16, "bf16", 4), (2, 1000, 16, "f32", 3)],
+                         ids=lambda c: "x".join(str(v) for v in c))
 def test_decode_conv_matches_oracle(orc, case):
     bt, ch, n, dtype, K = case
     inp = _upd_inputs(bt, ch, n, dtype, K, seed=700 + K)
