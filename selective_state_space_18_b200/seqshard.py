@@ -113,7 +113,9 @@ def seq_sharded_scan(x, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h
     A, D, dt_bias are the same on every rank; h0 (the state before the sequence's
     first token) is read on rank 0 only.  Returns dict(y, h_last = the state after
     this segment, final_state = the state after the whole sequence, on every rank,
-    when return_final_state).  Every rank must call it (it holds one collective)."""
+    when return_final_state).  Every rank must call it (it holds one collective), with
+    the same batch, channels and state_dim and the same dtype; only the segment length
+    may differ between ranks."""
     if dist.is_available() and dist.is_initialized():
         world, rank = dist.get_world_size(group), dist.get_rank(group)
     else:

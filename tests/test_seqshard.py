@@ -166,7 +166,7 @@ def test_segment_decay_matches_oracle(dtype, n, L, resets):
     got = out.cpu().double().numpy()
     assert np.all(np.isfinite(got))
     assert np.all(got[ref == 0.0] == 0.0)
-    assert np.median(ref[ref > 0]) > 1e-6 if (ref > 0).any() else resets
+    assert np.median(ref[1]) > 1e-6          # batch row 1 has no reset: its decays are far from 0
     if resets:
         assert np.all(got[0] == 0.0)     # the row with a reset discards the entering state
     err = np.abs(got - ref) - 1e-4 * np.abs(ref)
