@@ -296,7 +296,11 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
 
     float4 av[kDecItems];
     float bias[kDecItems], dco[kDecItems];
-    float cw[CONV ? kDecItems : 1][4], cbi[CONV ? kDecItems : 1]; // taps aligned: cw[3] multiplies u
+    // conv taps of the items this lane evaluates (item v * Q + lane_q, see below):
+    // cs_w[e] multiplies conv-state entry e (the input H - e back; 0 for e >= H), cu_w
+    // the new input u.  Every index is a compile-time constant, so they stay in registers.
+    constexpr int kMine = CONV ? kDecItems / Q : 1;
+    float cs_w[kMine][3], cu_w[kMine], cbi[kMine];
     const int H = CONV ? da.conv_k - 1 : 0;
     int64_t cached_cb = -1;
     bool ok = true;
@@ -315,13 +319,19 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
                 av[it] = __ldg(reinterpret_cast<const float4 *>(p.A + c * N) + lane_q);
                 bias[it] = p.dt_bias ? __ldg(p.dt_bias + c) : 0.0f;
                 dco[it] = p.D ? __ldg(p.D + c) : 0.0f;
-                if constexpr (CONV) {
+            }
+            if constexpr (CONV) {
+                // tap k of a row multiplies the input K-1-k back: taps 0..H-1 the conv
+                // state (oldest first), tap H = K-1 the new input
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int kk = k - (4 - da.conv_k);
-                        cw[it][k] = kk >= 0 ? __ldg(da.conv_w + c * da.conv_k + kk) : 0.0f;
-                    }
-                    cbi[it] = da.conv_b ? __ldg(da.conv_b + c) : 0.0f;
+                for (int v = 0; v < kMine; ++v) {
+                    const int q = tid + (v * Q + lane_q) * kDecThreads;
+                    const int64_t c = c0 + (q < nq ? q : nq - 1) / Q;
+#pragma unroll
+                    for (int e = 0; e < 3; ++e)
+                        cs_w[v][e] = e < H ? __ldg(da.conv_w + c * da.conv_k + e) : 0.0f;
+                    cu_w[v] = __ldg(da.conv_w + c * da.conv_k + H);
+                    cbi[v] = da.conv_b ? __ldg(da.conv_b + c) : 0.0f;
                 }
             }
         }
@@ -394,21 +404,25 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
             // x = silu(conv over [state, u]); xs held u until here.  The Q lanes of a row
             // share each item's x: lane j evaluates the items it with it % Q == j and the
             // row's lanes exchange (as for the softplus below)
-            float xm[kDecItems / Q];
+            float xm[kMine];
 #pragma unroll
-            for (int v = 0; v < kDecItems / Q; ++v) {
-                float acc = 0.0f;
+            for (int v = 0; v < kMine; ++v) {
+                // this lane's item v * Q + lane_q: its input and conv state, selected
+                // with compile-time indices
+                float uu = xs[v * Q], s0 = cs[v * Q][0], s1 = cs[v * Q][1], s2 = cs[v * Q][2];
 #pragma unroll
-                for (int j = 0; j < Q; ++j) {
-                    const int it = v * Q + j;
-                    float a = fmaf(cw[it][3], xs[it], cbi[it]);
-#pragma unroll
-                    for (int e = 0; e < 3; ++e) // state entry e is the input 3 - H + e back
-                        if (e < H)
-                            a = fmaf(cw[it][3 - H + e], cs[it][e], a);
-                    acc = lane_q == j ? a : acc;
-                }
-                xm[v] = silu(acc);
+                for (int j = 1; j < Q; ++j)
+                    if (lane_q == j) {
+                        uu = xs[v * Q + j];
+                        s0 = cs[v * Q + j][0];
+                        s1 = cs[v * Q + j][1];
+                        s2 = cs[v * Q + j][2];
+                    }
+                float a = fmaf(cu_w[v], uu, cbi[v]); // entries e >= H hold 0, and so do their taps
+                a = fmaf(cs_w[v][0], s0, a);
+                a = fmaf(cs_w[v][1], s1, a);
+                a = fmaf(cs_w[v][2], s2, a);
+                xm[v] = silu(a);
             }
             const int xbase = (tid & 31) & ~(Q - 1);
 #pragma unroll
