@@ -553,7 +553,6 @@ def run_seq_shard(args):
     mine = [part(r) for r in range(segs)] if emulate > 1 else [part(rank)]
     del full
     stream = torch.cuda.current_stream(dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 256 MB > L2
 
     if emulate > 1:
         K = args.steps
@@ -604,6 +603,7 @@ def run_seq_shard(args):
     else:
         q = mine[0]
         K = args.steps
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 256 MB > L2
         for _ in range(args.warmup):
             seqshard.seq_sharded_scan(q["x"], q["dt"], q["A"], q["B"], q["C"], q["D"], q["z"], q["dt_bias"])
         torch.cuda.synchronize(dev)
