@@ -72,18 +72,27 @@ class OracleSteps:
                 torch.from_numpy(final) if want_final else None)
 
 
-def _problem(L=480):
-    inp = make_scan_inputs(2, 8, 4, L, "f32", seed=31, reset_mean_doc=90, h0=True)
+def _problem(L=480, variant="h0"):
+    """variant "h0": initial state, softplus, resets (two of them on segment starts);
+    "plain": no initial state, no softplus (positive raw steps, no bias), no resets."""
+    if variant == "h0":
+        inp = make_scan_inputs(2, 8, 4, L, "f32", seed=31, reset_mean_doc=90, h0=True)
+    else:
+        inp = make_scan_inputs(2, 8, 4, L, "f32", seed=32, dt_bias=False)
+        inp["dt"] = inp["dt"].abs() * 0.05
     out = {k: (v.double() if torch.is_tensor(v) and v.is_floating_point() else v) for k, v in inp.items()}
-    out["reset"][1, 240] = 1     # resets on the first token of a segment: the cut at 240 (three
-    out["reset"][0, 320] = 1     # ranks) and at 320 (two ranks)
+    if variant == "h0":
+        out["reset"][1, 240] = 1     # resets on the first token of a segment: the cut at 240 (three
+        out["reset"][0, 320] = 1     # ranks) and at 320 (two ranks)
     return out
 
 
 def _slice(p, a, b):
     q = {}
     for k, v in p.items():
-        if k in ("x", "dt", "z", "B", "C"):
+        if v is None:
+            q[k] = None
+        elif k in ("x", "dt", "z", "B", "C"):
             q[k] = v[..., a:b].contiguous()
         elif k == "reset":
             q[k] = v[:, a:b].contiguous()
@@ -98,29 +107,29 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank_worker(rank, world, port, out):
+def _rank_worker(rank, world, port, variant, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        p = _problem()
+        p = _problem(variant=variant)
         a, b = seqshard.shard_bounds(p["x"].shape[-1], world)[rank]
         q = _slice(p, a, b)
         res = seqshard.seq_sharded_scan(q["x"], q["dt"], q["A"], q["B"], q["C"], q["D"], q["z"], q["dt_bias"],
                                         q["reset"], q["h0"] if rank == 0 else None, return_final_state=True,
-                                        steps=OracleSteps)
+                                        dt_softplus=variant == "h0", steps=OracleSteps)
         out[rank] = (a, b, res["y"].numpy(), res["h_last"].numpy(), res["final_state"].numpy())
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_gloo_ranks_join_to_the_whole_scan(world):
+@pytest.mark.parametrize("world,variant", [(2, "h0"), (3, "h0"), (4, "plain")])
+def test_gloo_ranks_join_to_the_whole_scan(world, variant):
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
-    mp.spawn(_rank_worker, args=(world, _free_port(), out), nprocs=world, join=True)
-    p = _problem()
+    mp.spawn(_rank_worker, args=(world, _free_port(), variant, out), nprocs=world, join=True)
+    p = _problem(variant=variant)
     whole = oracle.scan(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], p["z"], p["dt_bias"], p["reset"],
-                        p["h0"], return_states=True)
+                        p["h0"], dt_softplus=variant == "h0", return_states=True)
     y = np.concatenate([out[r][2] for r in range(world)], axis=-1)
     scale = 1.0 + np.abs(whole["y"]).max()
     assert np.abs(y - whole["y"]).max() <= 1e-12 * scale
