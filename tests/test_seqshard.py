@@ -292,3 +292,40 @@ def test_one_segment_is_the_plain_scan_bit_for_bit(dtype):
     y, h = seqshard.ssscan.ss_scan_fwd(*(dd[k] for k in keys))
     torch.cuda.synchronize()
     assert torch.equal(res["y"], y) and torch.equal(res["h_last"], h) and torch.equal(res["final_state"], h)
+
+
+def _leaving_worker(rank, world, port, out):
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        out[rank] = "left before the exchange"
+        return  # the process ends without joining the all-gather
+    p = _problem()
+    a, b = seqshard.shard_bounds(p["x"].shape[-1], world)[rank]
+    q = _slice(p, a, b)
+    try:
+        seqshard.seq_sharded_scan(q["x"], q["dt"], q["A"], q["B"], q["C"], q["D"], q["z"], q["dt_bias"],
+                                  q["reset"], q["h0"], steps=OracleSteps)
+        out[rank] = "returned"
+    except Exception as e:  # the collective fails: the peer is gone or the timeout ran out
+        out[rank] = f"error: {type(e).__name__}"
+
+
+def test_a_rank_that_leaves_surfaces_as_an_error_not_a_hang():
+    """Failure made on the host: rank 1 exits before the exchange step.  Rank 0's
+    all-gather must end with an error (peer gone, or the 5 s process-group timeout)."""
+    ctx = mp.get_context("spawn")
+    out = ctx.Manager().dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_leaving_worker, args=(r, 2, port, out)) for r in range(2)]
+    for pr in procs:
+        pr.start()
+    for pr in procs:
+        pr.join(timeout=90)
+    alive = [pr for pr in procs if pr.is_alive()]
+    for pr in alive:
+        pr.kill()
+    assert not alive, "a rank hung"
+    assert out[1] == "left before the exchange"
+    assert out[0].startswith("error"), out[0]
