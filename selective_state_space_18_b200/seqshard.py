@@ -115,7 +115,9 @@ def seq_sharded_scan(x, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h
     this segment, final_state = the state after the whole sequence, on every rank,
     when return_final_state).  Every rank must call it (it holds one collective), with
     the same batch, channels and state_dim and the same dtype; only the segment length
-    may differ between ranks."""
+    may differ between ranks.  `steps` carries out the scan, decay and join: the
+    library's kernels (CudaSteps); the tests put float64 stand-ins there to check the
+    exchange on CPU ranks."""
     if dist.is_available() and dist.is_initialized():
         world, rank = dist.get_world_size(group), dist.get_rank(group)
     else:
