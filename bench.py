@@ -116,58 +116,99 @@ def _peaks():
 # ---------------------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons of one GPU, sampled every `period` seconds by a
+    background thread over NVML (nvidia-smi polling if NVML is unavailable), each
+    sample stamped with time.perf_counter().  summary(t0, t1) keeps only the samples
+    taken inside [t0, t1], so the record describes the timed region itself."""
 
-    def __init__(self, device_index):
-        self.proc = None
-        self.path = None
+    NAMES = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+             ("sw_power_cap", 0x4), ("hw_power_brake", 0x80))
+
+    def __init__(self, device_index, period=0.002):
+        import threading
+        self.period = period
+        self.samples = []          # (t, sm_mhz, reasons bitmask)
+        self.max_mhz = None
+        self.source = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._handle = None
+        self._smi = None
         try:
-            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
         except Exception:
-            uuid = str(device_index)
-        self.gpu = uuid
+            self.uuid = str(device_index)
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._handle = pynvml.nvmlDeviceGetHandleByUUID(self.uuid.encode())
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM))
+            self.source = "nvml"
+        except Exception:
+            self._handle = None
+            self.source = "nvidia-smi"
+
+    def _poll_nvml(self):
+        nv, h = self._nvml, self._handle
+        getr = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                rs = int(getr(h))
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def _poll_smi(self):
+        fields = "clocks.sm,clocks.max.sm,clocks_event_reasons.active"
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", self.uuid, f"--query-gpu={fields}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip().split(",")
+                t = time.perf_counter()
+                self.max_mhz = float(out[1])
+                self.samples.append((t, float(out[0]), int(out[2].strip(), 16)))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
-        time.sleep(0.3)
+        import threading
+        target = self._poll_nvml if self._handle is not None else self._poll_smi
+        self._thread = threading.Thread(target=target, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=10)
+
+    def summary(self, t0, t1):
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside:  # a region shorter than the sampling period: the nearest sample
+            near = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:1]
+            inside = near
+        if not inside:
             return None
-        time.sleep(0.1)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 8:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return None
-        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
-        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
-        # samples under load: SM clock above idle
-        loaded = [s for s in sm if s > 0.5 * (max(sm) if sm else 1)]
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+        mhz = [s[1] for s in inside]
+        mask = 0
+        for s in inside:
+            mask |= s[2]
+        return {"sm_mhz": statistics.median(mhz), "sm_min_mhz": min(mhz), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for n, bit in self.NAMES if mask & bit], "samples": len(inside),
+                "source": self.source, "window": "timed region only"}
+
+
+def wait_event(ev):
+    """Wait for a recorded CUDA event without holding the GIL (so the clock sampler
+    thread keeps sampling), then synchronise on it."""
+    while not ev.query():
+        time.sleep(0.0002)
+    ev.synchronize()
 
 
 # ---------------------------------------------------------------------------------------
@@ -247,17 +288,37 @@ def run_ours(args):
         ssscan.ss_state_update(u["state"], u["x"], u["dt"], u["A"], u["B"], u["C"], u["D"], u["z"],
                                u["dt_bias"], y=y_dec[i & 1], stream=stream)
 
-    for i in range(args.warmup):
+    sampler = ClockSampler(local)
+    sampler.start()
+    # W declared warm-up steps, then a time-based pre-roll of the same steps until
+    # prewarm_s seconds have passed, so the timed steps run at the steady-state SM
+    # clock (a GPU that was idle starts at a low clock and ramps up under load).  The
+    # host stays at most 8 steps ahead of the GPU, and no idle gap separates the
+    # pre-roll from the timed region.
+    done = []
+    i = 0
+    t_pre = time.perf_counter()
+    while i < args.warmup or time.perf_counter() - t_pre < args.prewarm_s:
+        if len(done) >= 8:
+            done.pop(0).synchronize()
         step(i)
-    torch.cuda.synchronize(dev)
+        e = torch.cuda.Event()
+        e.record(stream)
+        done.append(e)
+        i += 1
+    prewarm_steps = i - args.warmup
+    prewarm_s = time.perf_counter() - t_pre
 
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(local)
-    sampler.start()
+    torch.cuda.synchronize(dev)
     _barrier(world)
     torch.cuda.synchronize(dev)
+    # A short GPU-side spin before the first timed event gives the host a head start,
+    # so no per-step event interval ever includes host-side launch work.
+    torch.cuda._sleep(int(1.5e-3 * 1.965e9))
+    t0 = time.perf_counter()
     start.record(stream)
     for i in range(K):
         e0, e1, e2 = ev[i]
@@ -270,13 +331,18 @@ def run_ours(args):
                                u["dt_bias"], y=y_dec[i & 1], stream=stream)
         e2.record(stream)
     end.record(stream)
+    wait_event(end)
     torch.cuda.synchronize(dev)
+    t1 = time.perf_counter()
     _barrier(world)
-    clocks = sampler.stop()
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
 
     total_ms = start.elapsed_time(end)
-    scan_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
-    dec_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    scan_list = [e[0].elapsed_time(e[1]) for e in ev]
+    dec_list = [e[1].elapsed_time(e[2]) for e in ev]
+    scan_ms = sum(scan_list) / K
+    dec_ms = sum(dec_list) / K
     total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / K
 
@@ -291,6 +357,8 @@ def run_ours(args):
         e2e = run_e2e(args, dev, stream, sets[0], ssscan)
     e2e_ms = max_over_ranks(e2e["ms_per_step"], world, dev)
 
+    plan = ssscan.ss_scan_plan(PROMPT.batch, PROMPT.channels, PROMPT.state_dim, PROMPT.seq,
+                               torch.bfloat16, has_reset=False, workspace=True, device=dev)
     hbm_gbs, sm_max_mhz, peak_kind = _peaks()
     sfu_peak = SM_COUNT_NOMINAL * MUFU_PER_CLK_PER_SM * sm_max_mhz * 1e6  # ex2/s
     scan_s = scan_ms * 1e-3
@@ -321,11 +389,16 @@ def run_ours(args):
         "peak_source": f"HBM {peak_kind} (MEASURED_PEAKS.json); SFU derived from unit counts and clock",
     }
     kernels = {
-        "scan": {"ms": round(scan_ms, 5), "elems_per_s": pw["elems"] / scan_s,
+        "scan": {"ms": round(scan_ms, 5), "ms_min": round(min(scan_list), 5),
+                 "ms_median": round(statistics.median(scan_list), 5), "ms_max": round(max(scan_list), 5),
+                 "kcycles_at_median_clock": (round(scan_ms * sm_clk, 1) if sm_clk else None),
+                 "elems_per_s": pw["elems"] / scan_s,
                  "hbm_gbs": round(scan_hbm, 1), "roofline_frac": round(t_roof_scan / scan_s, 4),
-                 "t_roof_ms": round(t_roof_scan * 1e3, 5)},
+                 "t_roof_ms": round(t_roof_scan * 1e3, 5), "launch": plan},
         "decode": {"kernel": "ss_state_update_stream_kernel (decode update)",
-                   "ms": round(dec_ms, 5), "elems_per_s": dw["elems"] / dec_s,
+                   "ms": round(dec_ms, 5), "ms_min": round(min(dec_list), 5),
+                   "ms_median": round(statistics.median(dec_list), 5), "ms_max": round(max(dec_list), 5),
+                   "elems_per_s": dw["elems"] / dec_s,
                    "hbm_gbs": round(dw["bytes"] / dec_s / 1e9, 1),
                    "hbm_frac": round(dw["bytes"] / dec_s / 1e9 / hbm_gbs, 4),
                    "roofline_frac": round(t_roof_dec / dec_s, 4),
@@ -348,13 +421,13 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32",
+        "dtype": "bf16",
         "data": "synthetic",
         "config": {
             "workload": "mamba2p8b_layer_long prompt scan (batch 1, channels 5120, state_dim 16, "
                         "seq 16384, bf16 x/dt/z/B/C/y, z gate, dt_bias, fp32 state) + decode_2p8b "
                         "update (batch 256, channels 5120, state_dim 16, bf16 I/O, fp32 state in place)",
-            "storage": "bf16",
+            "storage": "bf16 x/dt/z/B/C/y; fp32 A, D, dt_bias, state and all arithmetic",
             "elems_per_step": elems_step,
             "l2": "inputs larger than L2 (scan 673 MB + decode 179 MB per step), two rotating input sets",
             "parallelism": f"replicas x{world} (independent problems per rank, no collective)",
@@ -366,6 +439,8 @@ def run_ours(args):
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                 "steps": e2e["steps"]},
         "clocks": clocks,
+        "prewarm_s": round(prewarm_s, 3),
+        "prewarm_steps": prewarm_steps,
         "gpu_launches": 2 * K,
     }
     if rank == 0:
@@ -580,12 +655,16 @@ def run_seq_shard(args):
         sampler = ClockSampler(local)
         sampler.start()
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0 = time.perf_counter()
         start.record(stream)
         for i in range(args.warmup, args.warmup + K):
             step(i)
         end.record(stream)
+        wait_event(end)
         torch.cuda.synchronize(dev)
-        clocks = sampler.stop()
+        t1 = time.perf_counter()
+        sampler.stop()
+        clocks = sampler.summary(t0, t1)
         serial_ms = start.elapsed_time(end) / K
         per_rank = []
         for r in range(segs):
@@ -612,14 +691,17 @@ def run_seq_shard(args):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
         _barrier(world)
         torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
         for i in range(K):
             flush.zero_()                      # L2 flushed between steps, outside the timed events
             ev[i][0].record(stream)
             seqshard.seq_sharded_scan(q["x"], q["dt"], q["A"], q["B"], q["C"], q["D"], q["z"], q["dt_bias"])
             ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
+        t1 = time.perf_counter()
         _barrier(world)
-        clocks = sampler.stop()
+        sampler.stop()
+        clocks = sampler.summary(t0, t1)
         ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev) / K, world, dev)
         launches = K * (1 if world == 1 else 4)
         extra = {}
@@ -665,6 +747,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--prewarm-s", type=float, default=1.0,
+                    help="seconds of untimed steps after the warm-up steps (clock ramp-up)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")

@@ -93,8 +93,10 @@ enum { SS_DT_SOFTPLUS = 1u };
  *                  processed by persistent CTAs that pass the scan carry between
  *                  them, which balances the GPU for any shape.  Without one, each CTA
  *                  scans one group of channels over the whole sequence.  Calls that
- *                  share a workspace must be ordered (same stream, or synchronised);
- *                  after SS_ERR_TIMEOUT is reported, zero it again before reuse.
+ *                  share a workspace must be ordered (same stream, or synchronised).
+ *                  A call whose device-side waits gave up (SS_ERR_TIMEOUT, see
+ *                  ss_scan_status) also leaves the workspace ready for the next call:
+ *                  its outputs are invalid, but the workspace needs no re-zeroing.
  *
  * state_dim must be 4, 8 or 16.  Returns SS_OK or an error status.
  */
@@ -157,6 +159,24 @@ SS_API int ss_scan_fwd_conv(int64_t batch, int64_t channels, int64_t state_dim, 
                             const float *h0, uint32_t flags, void *y, float *h_last,
                             void *workspace, size_t workspace_bytes, ss_stream_t stream);
 
+/*
+ * Launch plan of ss_scan_fwd for a shape, on the current device: what the call would
+ * launch for 16-byte aligned tensors (the tile-load path) with or without resets and
+ * a workspace.  For tuning and for reporting alongside measurements; launches nothing.
+ */
+typedef struct {
+    int64_t grid;        /* CTAs launched                                        */
+    int64_t ctas_per_sm; /* resident CTAs per SM of that kernel (occupancy)      */
+    int64_t sms;         /* SMs of the current device                            */
+    int64_t groups;      /* channel groups: batch * ceil(channels / per CTA)     */
+    int64_t segments;    /* sequence segments per group (1 without a workspace)  */
+    int64_t seg_len;     /* tokens per segment                                   */
+    int64_t states_per_lane; /* state rows each scan lane owns (2 or 4)          */
+} ss_scan_plan_t;
+SS_API int ss_scan_plan(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
+                        ss_dtype_t dtype, int has_reset, int with_workspace,
+                        ss_scan_plan_t *plan);
+
 /* Workspace bytes ss_scan_fwd needs for this shape (0 for an invalid shape). */
 SS_API int64_t ss_scan_workspace_bytes(int64_t batch, int64_t channels, int64_t state_dim,
                                        int64_t seq);
@@ -169,6 +189,15 @@ SS_API int64_t ss_scan_workspace_bytes(int64_t batch, int64_t channels, int64_t 
  * SS_OK, or an error status if the query itself failed.
  */
 SS_API int ss_scan_status(const void *workspace, ss_stream_t stream, int *status);
+
+/*
+ * The device status word of calls made without a workspace (ss_scan_fwd with a NULL
+ * workspace, and every decode call) on the current device: ss_scan_status(NULL,
+ * stream, ...) as one return value.  Synchronises `stream`, reads and clears the word,
+ * and returns SS_OK, SS_ERR_TIMEOUT (a bounded device-side wait gave up; those calls'
+ * outputs are invalid) or the error status of the query itself.
+ */
+SS_API int ss_debug_status(ss_stream_t stream);
 
 /*
  * ss_scan_fwd without a caller-supplied workspace and without any allocation.
@@ -195,9 +224,10 @@ SS_API int ss_scan_status(const void *workspace, ss_stream_t stream, int *status
  * 16, i.e. batch * ceil(channels / 16) <= 992 (batch 1 at 5120 channels, or batch 8
  * at 1536, fit).
  *
- * Zero state: the scratch is zero when the library is loaded, and every scan that
- * completes leaves it ready for the next one.  After SS_ERR_TIMEOUT has been
- * reported, pass SS_SCRATCH_ZERO on the next call.
+ * Zero state: the scratch is zero when the library is loaded, and every scan leaves
+ * it ready for the next one, a scan whose waits gave up (SS_ERR_TIMEOUT) included.
+ * SS_SCRATCH_ZERO clears all SS_STATIC_SCRATCH_BYTES of it, for a caller that wants
+ * a known starting point (after a fault elsewhere in the process, say).
  *
  * Set-up: the first call on each device, with that device current, looks up the
  * scratch's address (which may load the library's device code) and configures the
@@ -264,6 +294,17 @@ SS_API int ss_state_update_conv(int64_t batch, int64_t channels, int64_t state_d
  * keep the default limit.  Synchronous; returns SS_OK or SS_ERR_CUDA.
  */
 SS_API int ss_debug_set_wait_limit(uint32_t microseconds);
+
+/*
+ * Testing aid: make later state_dim-16 scans in this process use the layout with
+ * `states_per_lane` (2 or 4) state rows per scan lane, whatever the shape; 0 restores
+ * the automatic choice (four per lane when the shape's 32-channel groups give every
+ * SM one, else two).  Results of the two layouts agree within rounding; they differ
+ * only in speed.  Other state sizes always use two.  Returns SS_OK, or
+ * SS_ERR_UNSUPPORTED for any other value.  Not thread-safe with respect to scans
+ * being issued concurrently from other host threads.
+ */
+SS_API int ss_debug_set_scan_layout(int states_per_lane);
 
 /*
  * Gated state scan (the "Mamba 2 Gated State Scan" exercise page): per batch item b,

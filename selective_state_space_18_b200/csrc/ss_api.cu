@@ -5,6 +5,7 @@
 #include "ss_scan.h"
 
 #include <atomic>
+#include <type_traits>
 #include <cstring>
 #include <cstdint>
 #include <cudaTypedefs.h> // PFN_cuTensorMapEncodeTiled
@@ -129,50 +130,61 @@ bool encode_rows(CUtensorMap *map, const void *base, int64_t inner, int64_t rows
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int N, typename T>
+template <int N, int SPL, typename T>
 bool build_maps(const ss::ScanArgs &a, ss::TmaMaps *m)
 {
-    using S = ss::ScanShape<N>;
+    using S = ss::ScanShape<N, SPL>;
     const int64_t rows = a.batch * a.channels, brows = a.batch * N;
     // B and C tiles are read by the scan warps in place: their 16-byte chunks are
-    // swizzled across the banks (64-byte rows for bf16, 128-byte rows for fp32)
-    const CUtensorMapSwizzle bc_swizzle = sizeof(T) == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    // swizzled across the banks (the swizzle the layout's lane-to-state map needs)
+    const CUtensorMapSwizzle bc_swizzle =
+        S::template swizzle<T>() == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     return encode_rows<T>(&m->x, a.x, a.seq, rows, S::kChunk, S::kChanPerCta) &&
            encode_rows<T>(&m->dt, a.dt, a.seq, rows, S::kChunk, S::kChanPerCta) &&
            encode_rows<T>(&m->B, a.B, a.seq, brows, S::kChunk, N, bc_swizzle) &&
            encode_rows<T>(&m->C, a.C, a.seq, brows, S::kChunk, N, bc_swizzle);
 }
 
-template <int N, typename T, bool R, bool V, bool E, bool C>
-int launch_scan(ss::ScanArgs a, cudaStream_t stream)
+// Launch plan of the scan kernel instance <N, SPL, T, R, V, E, C> for the shape in `a`
+// (groups, segments, segment length and grid filled in); also what ss_scan_plan
+// reports.
+template <int N, int SPL, typename T, bool R, bool V, bool E, bool C>
+int plan_scan(ss::ScanArgs &a, int64_t *grid_out, int *occ_out, int *sms_out)
 {
-    using S = ss::ScanShape<N>;
+    using S = ss::ScanShape<N, SPL>;
     constexpr size_t kSmem = S::template smem_bytes<T, V>();
-    auto kernel = ss::ss_scan_fwd_kernel<N, T, R, V, E, C>;
+    auto kernel = ss::ss_scan_fwd_kernel<N, SPL, T, R, V, E, C>;
     static std::atomic<uint64_t> smem_done{0};
     static std::atomic<int> occ_cache[64];
+    a.groups_per_batch = (a.channels + S::kChanPerCta - 1) / S::kChanPerCta;
+    if (!mul_ok(a.batch, a.groups_per_batch, &a.groups) || a.groups > 0x7fffffffLL)
+        return SS_ERR_SHAPE;
     int st = ensure_smem(kernel, kSmem, smem_done);
     if (st != SS_OK)
         return st;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || device_sm_count(&sms) != SS_OK)
+        return SS_ERR_CUDA;
+    int occ = dev < 64 ? occ_cache[dev].load(std::memory_order_acquire) : 0;
+    if (!occ) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, S::kThreads, kSmem) != cudaSuccess)
+            return SS_ERR_CUDA;
+        occ = occ > 0 ? occ : 1;
+        if (dev < 64)
+            occ_cache[dev].store(occ, std::memory_order_release);
+    }
+    *occ_out = occ;
+    *sms_out = sms;
     const int64_t nchunks = (a.seq + S::kChunk - 1) / S::kChunk;
     int64_t grid = a.groups;
     if (a.workspace) {
-        int dev = 0, sms = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || device_sm_count(&sms) != SS_OK)
-            return SS_ERR_CUDA;
-        int occ = dev < 64 ? occ_cache[dev].load(std::memory_order_acquire) : 0;
-        if (!occ) {
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, S::kThreads, kSmem) != cudaSuccess)
-                return SS_ERR_CUDA;
-            occ = occ > 0 ? occ : 1;
-            if (dev < 64)
-                occ_cache[dev].store(occ, std::memory_order_release);
-        }
         const int64_t resident = int64_t(sms) * occ;
         // about sixteen units per resident CTA (finer units balance the tail), segments
         // of at least sixteen chunks (each unit start costs a carry hand-off)
         int64_t segs = (16 * resident + a.groups - 1) / a.groups;
-        const int64_t max_segs = nchunks / 16 > 1 ? nchunks / 16 : 1;
+        // (segment indices stay below 2^24: the carry flags keep 24 bits for them)
+        int64_t max_segs = nchunks / 16 > 1 ? nchunks / 16 : 1;
+        max_segs = max_segs < (int64_t(1) << 24) - 1 ? max_segs : (int64_t(1) << 24) - 1;
         segs = segs < 1 ? 1 : (segs > max_segs ? max_segs : segs);
         const int64_t seg_chunks = (nchunks + segs - 1) / segs;
         a.seg_len = seg_chunks * S::kChunk;
@@ -182,54 +194,100 @@ int launch_scan(ss::ScanArgs a, cudaStream_t stream)
     } else {
         a.seg_len = nchunks * S::kChunk;
         a.segments = 1;
-        if (status_word_address(&a.status) != SS_OK)
-            return SS_ERR_CUDA;
     }
     if (grid > 0x7fffffffLL)
         return SS_ERR_SHAPE;
+    *grid_out = grid;
+    return SS_OK;
+}
+
+template <int N, int SPL, typename T, bool R, bool V, bool E, bool C>
+int launch_scan(ss::ScanArgs a, size_t ws_bytes, cudaStream_t stream)
+{
+    using S = ss::ScanShape<N, SPL>;
+    constexpr size_t kSmem = S::template smem_bytes<T, V>();
+    auto kernel = ss::ss_scan_fwd_kernel<N, SPL, T, R, V, E, C>;
+    int64_t grid = 0;
+    int occ = 0, sms = 0;
+    int st = plan_scan<N, SPL, T, R, V, E, C>(a, &grid, &occ, &sms);
+    if (st != SS_OK)
+        return st;
+    if (!a.workspace && status_word_address(&a.status) != SS_OK)
+        return SS_ERR_CUDA;
     ss::TmaMaps maps;
     memset(&maps, 0, sizeof(maps));
-    if (V && !build_maps<N, T>(a, &maps))
+    if (V && !build_maps<N, SPL, T>(a, &maps))
         return SS_ERR_CUDA;
     kernel<<<unsigned(grid), S::kThreads, kSmem, stream>>>(a, maps);
     return launch_status();
 }
 
-template <int N, typename T, bool E, bool C>
-int dispatch_scan_e(const ss::ScanArgs &a, bool vec, cudaStream_t s)
+template <int N, int SPL, typename T, bool E, bool C>
+int dispatch_scan_e(const ss::ScanArgs &a, bool vec, size_t ws, cudaStream_t s)
 {
     const bool r = a.reset != nullptr;
     if (r)
-        return vec ? launch_scan<N, T, true, true, E, C>(a, s) : launch_scan<N, T, true, false, E, C>(a, s);
-    return vec ? launch_scan<N, T, false, true, E, C>(a, s) : launch_scan<N, T, false, false, E, C>(a, s);
+        return vec ? launch_scan<N, SPL, T, true, true, E, C>(a, ws, s)
+                   : launch_scan<N, SPL, T, true, false, E, C>(a, ws, s);
+    return vec ? launch_scan<N, SPL, T, false, true, E, C>(a, ws, s)
+               : launch_scan<N, SPL, T, false, false, E, C>(a, ws, s);
 }
 
 // forms: plain; with per-token states (E); with the fused conv prologue (C)
-template <int N, typename T>
-int dispatch_scan_t(const ss::ScanArgs &a, bool vec, cudaStream_t s)
+template <int N, int SPL, typename T>
+int dispatch_scan_t(const ss::ScanArgs &a, bool vec, size_t ws, cudaStream_t s)
 {
     if (a.conv_w)
-        return dispatch_scan_e<N, T, false, true>(a, vec, s);
-    return a.h_all ? dispatch_scan_e<N, T, true, false>(a, vec, s) : dispatch_scan_e<N, T, false, false>(a, vec, s);
+        return dispatch_scan_e<N, SPL, T, false, true>(a, vec, ws, s);
+    return a.h_all ? dispatch_scan_e<N, SPL, T, true, false>(a, vec, ws, s)
+                   : dispatch_scan_e<N, SPL, T, false, false>(a, vec, ws, s);
 }
 
-template <int N> int64_t scan_groups(int64_t batch, int64_t channels)
+template <int N, int SPL> int64_t scan_groups(int64_t batch, int64_t channels)
 {
-    const int64_t per = ss::ScanShape<N>::kChanPerCta;
+    const int64_t per = ss::ScanShape<N, SPL>::kChanPerCta;
     return batch * ((channels + per - 1) / per);
+}
+
+// States per scan lane for a shape: at state_dim 16, four (32 channels per CTA, the
+// fewer shared-memory bytes and instructions per state) when its channel groups give
+// every SM one, else two (16 channels per CTA: twice the groups, so twice the SMs, for
+// shapes with few channels).  Smaller state sizes keep two.
+std::atomic<int> g_forced_spl{0}; // ss_debug_set_scan_layout: 0 = choose per shape
+
+int scan_spl(int64_t batch, int64_t channels, int64_t state_dim)
+{
+    if (state_dim != 16)
+        return 2;
+    const int forced = g_forced_spl.load(std::memory_order_relaxed);
+    if (forced)
+        return forced;
+    int sms = 0;
+    if (device_sm_count(&sms) != SS_OK)
+        sms = 148;
+    return scan_groups<16, 4>(batch, channels) >= int64_t(sms) ? 4 : 2;
+}
+
+template <int N, int SPL>
+int dispatch_scan_s(const ss::ScanArgs &a, ss_dtype_t dtype, bool vec, size_t ws_bytes, cudaStream_t s)
+{
+    // (a host-side check, before anything touches the device: the size the query
+    // reports, whichever layout this call picks)
+    if (a.workspace && int64_t(ws_bytes) < ss_scan_workspace_bytes(a.batch, a.channels, N, a.seq))
+        return SS_ERR_WORKSPACE;
+    if (dtype == SS_BF16)
+        return dispatch_scan_t<N, SPL, __nv_bfloat16>(a, vec, ws_bytes, s);
+    return dispatch_scan_t<N, SPL, float>(a, vec, ws_bytes, s);
 }
 
 template <int N>
 int dispatch_scan_n(ss::ScanArgs a, ss_dtype_t dtype, bool vec, size_t ws_bytes, cudaStream_t s)
 {
-    a.groups_per_batch = (a.channels + ss::ScanShape<N>::kChanPerCta - 1) / ss::ScanShape<N>::kChanPerCta;
-    if (!mul_ok(a.batch, a.groups_per_batch, &a.groups) || a.groups > 0x7fffffffLL)
-        return SS_ERR_SHAPE;
-    if (a.workspace && ws_bytes < size_t(ss::scan_workspace_bytes<N>(a.groups)))
-        return SS_ERR_WORKSPACE;
-    if (dtype == SS_BF16)
-        return dispatch_scan_t<N, __nv_bfloat16>(a, vec, s);
-    return dispatch_scan_t<N, float>(a, vec, s);
+    if constexpr (N == 16) {
+        if (scan_spl(a.batch, a.channels, N) == 4)
+            return dispatch_scan_s<16, 4>(a, dtype, vec, ws_bytes, s);
+    }
+    return dispatch_scan_s<N, 2>(a, dtype, vec, ws_bytes, s);
 }
 
 // The conv form of the decode step (w NULL: none).
@@ -376,6 +434,14 @@ const char *ss_status_string(int status)
     }
 }
 
+int ss_debug_set_scan_layout(int states_per_lane)
+{
+    if (states_per_lane != 0 && states_per_lane != 2 && states_per_lane != 4)
+        return SS_ERR_UNSUPPORTED;
+    g_forced_spl.store(states_per_lane, std::memory_order_relaxed);
+    return SS_OK;
+}
+
 int ss_debug_set_wait_limit(uint32_t microseconds)
 {
     return cudaMemcpyToSymbol(ss::g_ss_wait_limit_us, &microseconds, sizeof(microseconds)) == cudaSuccess
@@ -387,10 +453,16 @@ int64_t ss_scan_workspace_bytes(int64_t batch, int64_t channels, int64_t state_d
 {
     if (batch <= 0 || channels <= 0 || seq <= 0)
         return 0;
+    // the larger of the two layouts' needs, so the size does not depend on which one
+    // the call picks on the current device
     switch (state_dim) {
-    case 4: return ss::scan_workspace_bytes<4>(scan_groups<4>(batch, channels));
-    case 8: return ss::scan_workspace_bytes<8>(scan_groups<8>(batch, channels));
-    case 16: return ss::scan_workspace_bytes<16>(scan_groups<16>(batch, channels));
+    case 4: return ss::scan_workspace_bytes<4, 2>(scan_groups<4, 2>(batch, channels));
+    case 8: return ss::scan_workspace_bytes<8, 2>(scan_groups<8, 2>(batch, channels));
+    case 16: {
+        const int64_t a = ss::scan_workspace_bytes<16, 2>(scan_groups<16, 2>(batch, channels));
+        const int64_t b = ss::scan_workspace_bytes<16, 4>(scan_groups<16, 4>(batch, channels));
+        return a > b ? a : b;
+    }
     default: return 0;
     }
 }
@@ -417,6 +489,62 @@ int ss_scan_status(const void *workspace, ss_stream_t stream, int *status)
         return SS_ERR_CUDA;
     *status = (v & (1u << ss::kStatusTimeout)) ? SS_ERR_TIMEOUT : SS_OK;
     return SS_OK;
+}
+
+int ss_scan_plan(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, ss_dtype_t dtype,
+                 int has_reset, int with_workspace, ss_scan_plan_t *plan)
+{
+    if (!plan)
+        return SS_ERR_NULL;
+    if (batch <= 0 || channels <= 0 || seq <= 0)
+        return SS_ERR_SHAPE;
+    if (dtype != SS_F32 && dtype != SS_BF16)
+        return SS_ERR_DTYPE;
+    if (state_dim != 4 && state_dim != 8 && state_dim != 16)
+        return SS_ERR_UNSUPPORTED;
+    ss::ScanArgs a{};
+    a.batch = batch;
+    a.channels = channels;
+    a.seq = seq;
+    // any non-null value: the plan only asks whether a workspace is given
+    a.workspace = with_workspace ? reinterpret_cast<uint8_t *>(uintptr_t(256)) : nullptr;
+    int64_t grid = 0;
+    int occ = 0, sms = 0, st = SS_OK;
+    const bool r = has_reset != 0;
+    auto run = [&](auto n_tag, auto spl_tag) -> int {
+        constexpr int N = decltype(n_tag)::value, SPL = decltype(spl_tag)::value;
+        if (dtype == SS_BF16)
+            return r ? plan_scan<N, SPL, __nv_bfloat16, true, true, false, false>(a, &grid, &occ, &sms)
+                     : plan_scan<N, SPL, __nv_bfloat16, false, true, false, false>(a, &grid, &occ, &sms);
+        return r ? plan_scan<N, SPL, float, true, true, false, false>(a, &grid, &occ, &sms)
+                 : plan_scan<N, SPL, float, false, true, false, false>(a, &grid, &occ, &sms);
+    };
+    using I2 = std::integral_constant<int, 2>;
+    switch (state_dim) {
+    case 4: st = run(std::integral_constant<int, 4>(), I2()); break;
+    case 8: st = run(std::integral_constant<int, 8>(), I2()); break;
+    default:
+        st = scan_spl(batch, channels, 16) == 4 ? run(std::integral_constant<int, 16>(), std::integral_constant<int, 4>())
+                                                  : run(std::integral_constant<int, 16>(), I2());
+        break;
+    }
+    if (st != SS_OK)
+        return st;
+    plan->grid = grid;
+    plan->ctas_per_sm = occ;
+    plan->states_per_lane = state_dim == 16 ? scan_spl(batch, channels, 16) : 2;
+    plan->sms = sms;
+    plan->groups = a.groups;
+    plan->segments = a.segments;
+    plan->seg_len = a.seg_len;
+    return SS_OK;
+}
+
+int ss_debug_status(ss_stream_t stream)
+{
+    int st = SS_OK;
+    const int q = ss_scan_status(nullptr, stream, &st);
+    return q != SS_OK ? q : st;
 }
 
 } // extern "C"
@@ -847,7 +975,10 @@ int ss_scan_fwd_static_scratch(int64_t batch, int64_t channels, int64_t state_di
     if (scratch)
         *scratch = ws;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (need > 0 && (flags & SS_SCRATCH_ZERO) && cudaMemsetAsync(ws, 0, size_t(need), s) != cudaSuccess)
+    // the whole scratch: carry flags beyond this shape's part, left by an earlier call
+    // with more channel groups, must not survive the epoch going back to zero
+    if (need > 0 && (flags & SS_SCRATCH_ZERO) &&
+        cudaMemsetAsync(ws, 0, size_t(SS_STATIC_SCRATCH_BYTES), s) != cudaSuccess)
         return SS_ERR_CUDA;
     return ss_scan_fwd(batch, channels, state_dim, seq, dtype, x, dt_raw, A, B, C, D, z, dt_bias, reset, h0,
                        flags & uint32_t(SS_DT_SOFTPLUS), y, h_last, ws, SS_STATIC_SCRATCH_BYTES, stream);

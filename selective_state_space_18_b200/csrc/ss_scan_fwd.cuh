@@ -69,36 +69,61 @@ struct TmaMaps {
     CUtensorMap x, dt, B, C;
 };
 
-// Workspace layout (bytes): the caller zeroes it once; every complete call leaves
-// it ready for the next one.
+// Workspace layout (bytes): the caller zeroes it once; every call leaves it ready for
+// the next one -- also a call whose waits gave up, since every warp counts itself
+// out on every exit path and the last one resets the counters.
 struct WsHeader {
     uint32_t counter; // next work unit of this call
     uint32_t status;  // sticky error bits (1 << SS_ERR_TIMEOUT)
-    uint32_t epoch;   // advanced by the last warp of every call; tags the carry flags
     uint32_t done;    // warps finished in this call
-    uint32_t pad[12];
+    uint32_t pad0;
+    uint64_t epoch;   // advanced by the last warp of every call; tags the carry flags
+    uint32_t pad[10];
 };
 static_assert(sizeof(WsHeader) == 64, "workspace header is 64 bytes");
 
-template <int N> struct ScanShape {
+// A carry flag holds (epoch << 24) | segment: 40 bits of epoch (a flag left by an
+// earlier call never matches a later one) and 24 bits of segment index (the host
+// keeps segments below 2^24).
+constexpr int kFlagSegBits = 24;
+__device__ __forceinline__ uint64_t carry_tag(uint64_t epoch, int64_t s)
+{
+    return ((epoch & ((uint64_t(1) << 40) - 1)) << kFlagSegBits) | uint64_t(s);
+}
+
+// Geometry of the prompt-scan kernel for state_dim N with SPL states per scan lane.
+// A channel's N states are spread over kLanes = N / SPL lanes of one warp; a warp
+// covers 32 / kLanes channels, a CTA (four scan warps) kChanPerCta.  SPL = 2 (eight
+// lanes per channel at N = 16) gives the most independent warps, for shapes with few
+// channel groups.  SPL = 4 (four lanes per channel, 32 channels per CTA, one CTA per
+// SM) halves the lanes that read each token's dt and dt*x and the partial outputs
+// the epilogue stores, reads and sums, per (b, t, c): the scan is bound by the
+// exponential unit, and those shared-memory bytes and instructions are what keeps it
+// from running at that unit's rate.
+template <int N, int SPL> struct ScanShape {
     static_assert(N == 4 || N == 8 || N == 16, "state_dim must be 4, 8 or 16");
-    static constexpr int kPairs = N / 2;               // state pairs = lanes per channel
-    static constexpr int kChanPerWarp = 32 / kPairs;
-    // Roles: warps 0-3 scan, warps 4 and 6 produce, warps 5 and 7 run the epilogue,
-    // warp 8 issues the tile loads.  Warp w executes on sub-partition w % 4, so every
-    // sub-partition (and its MUFU unit) holds one scan warp and one IO warp of each CTA.
+    static_assert(SPL == 2 || (SPL == 4 && N == 16), "states per lane: 2, or 4 at state_dim 16");
+    static constexpr int kSpl = SPL;
+    static constexpr int kLanes = N / SPL;             // lanes per channel
+    static constexpr int kChanPerWarp = 32 / kLanes;
+    // Roles: warps 0-3 scan (one per SM sub-partition, so all four MUFU units work),
+    // then kIoWarps producer warps, kIoWarps epilogue warps and one issuer warp.  Warp
+    // w executes on sub-partition w % 4, so the producers and the epilogue warps are
+    // spread evenly over the sub-partitions.
     static constexpr int kScanWarps = 4;
-    static constexpr int kIssuerWarp = 8;
-    static constexpr int kWarps = 9;
+    static constexpr int kIoWarps = SPL == 4 ? 4 : 2;  // warps per IO role
+    static constexpr int kWarps = kScanWarps + 2 * kIoWarps + 1;
+    static constexpr int kIssuerWarp = kWarps - 1;
     static constexpr int kThreads = 32 * kWarps;
-    static constexpr int kIoThreads = 64;              // threads per IO role (2 warps)
+    static constexpr int kIoThreads = 32 * kIoWarps;   // threads per IO role
     static constexpr int kChanPerCta = kScanWarps * kChanPerWarp;
     static constexpr int kChunk = 32;                  // tokens per pipeline stage
     static constexpr int kBlocks = kChunk / 8;         // 8-token blocks per chunk
     static constexpr int kRow = kChunk + 4;            // padded row (floats)
     // ring depths: at N = 16 four input and three output stages (measured 5% faster
-    // than three and two) still leave room for two CTAs per SM; N = 4 and 8 put 2-4x
-    // more channels in a CTA and keep the rings short to fit
+    // than three and two) still leave room for two CTAs per SM with SPL = 2 (one CTA
+    // per SM with SPL = 4); N = 4 and 8 put 2-4x more channels in a CTA and keep the
+    // rings short to fit
     static constexpr int kStages = N == 16 ? 4 : 2, kYStages = N == 16 ? 3 : 2;
     // input stage (floats): meta | dt rows | dt*x rows | reset bias
     static constexpr int kMeta = 8;
@@ -107,7 +132,7 @@ template <int N> struct ScanShape {
     static constexpr int kRBOff = kDXOff + kChanPerCta * kRow;
     static constexpr int kInStage = kRBOff + kChunk;
     // output stage (floats): meta | partial outputs
-    static constexpr int kYChan = kPairs * kRow + 4;   // per-channel block, bank-skewed
+    static constexpr int kYChan = kLanes * kRow + 4;   // per-channel block, bank-skewed
     static constexpr int kYPOff = kMeta;
     // then x of the chunk in storage type [channels][chunk] (the fused conv form hands
     // it from the producers to the epilogue here)
@@ -124,7 +149,7 @@ template <int N> struct ScanShape {
     // slot its readers have released loading, so up to kRawStages chunks are in
     // flight.  The scan warps read B and C straight from the slot, in storage type
     // (bf16 halves their shared-memory traffic), from tiles swizzled by TMA so the
-    // N/2 state rows a warp reads at once fall into distinct banks.  On the ragged
+    // kLanes state rows a warp reads at once fall into distinct banks.  On the ragged
     // path the producers write the B and C tiles themselves in the same layout.
     static constexpr int kRawStages = N == 16 ? 8 : 4;
     // mbarriers: in_full, in_empty [kStages]; y_full, y_empty [kYStages]; raw_full,
@@ -148,6 +173,19 @@ template <int N> struct ScanShape {
     {
         return size_t(kRawStages * raw_stage_bytes<T>()) + size_t(floats<T>()) * 4 + 8 * size_t(kBars) +
                32 * size_t(kRawStages);
+    }
+    // Which states a lane owns, and how TMA swizzles the B and C tiles so that the
+    // kLanes rows a warp reads at once fall into distinct banks:
+    //  * bf16 with four states per lane: states 4g .. 4g+3 (contiguous, so the lane
+    //    moves its states, carries and per-token states as 16-byte vectors) with the
+    //    128-byte swizzle;
+    //  * otherwise states g, g + kLanes, ... (strided) with the 64-byte swizzle for
+    //    bf16 rows and the 128-byte swizzle for fp32 rows.
+    template <typename T> static constexpr bool contiguous() { return SPL == 4 && sizeof(T) == 2; }
+    template <typename T> static constexpr int swizzle() { return (sizeof(T) == 2 && SPL == 2) ? 64 : 128; }
+    template <typename T> static __device__ __forceinline__ int state(int g, int j)
+    {
+        return contiguous<T>() ? SPL * g + j : g + kLanes * j;
     }
     static_assert(kTokTasks % kIoThreads == 0, "token tasks fill whole IO lanes");
     static_assert(kInStage % 4 == 0 && kYXOff % 4 == 0, "16-byte aligned stages");
@@ -185,18 +223,14 @@ __device__ __forceinline__ ChunkMeta read_meta(const float *stage)
 }
 
 // Byte offset of 16-byte chunk `c16` of row `row` in a B or C tile of the raw ring.
-// The tile is a dense [N rows][chunk tokens] box written by TMA with the 64-byte
-// swizzle (bf16 rows of 64 bytes) or the 128-byte swizzle (fp32 rows of 128 bytes):
-// the chunk index is XORed with bits 7.. of the byte address, i.e. with row/2 mod 4
-// or row mod 8, so rows 0..7 of one chunk land in eight distinct bank groups.
-template <typename T> __device__ __forceinline__ int bc_offset(int row, int c16);
-template <> __device__ __forceinline__ int bc_offset<__nv_bfloat16>(int row, int c16)
+// The tile is a dense [N rows][chunk tokens] box (64-byte rows for bf16, 128-byte rows
+// for fp32) that TMA writes with a swizzle: the 16-byte chunk index (address bits
+// 4..6) is XORed with address bits 7.. -- two bits of them for the 64-byte swizzle,
+// three for the 128-byte one.
+template <typename T, int SWZ> __device__ __forceinline__ int bc_offset(int row, int c16)
 {
-    return row * 64 + ((c16 ^ ((row >> 1) & 3)) << 4);
-}
-template <> __device__ __forceinline__ int bc_offset<float>(int row, int c16)
-{
-    return row * 128 + ((c16 ^ (row & 7)) << 4);
+    const int lin = row * (32 * int(sizeof(T))) + (c16 << 4);
+    return SWZ == 64 ? lin ^ (((lin >> 7) & 3) << 4) : lin ^ (((lin >> 7) & 7) << 4);
 }
 
 // silu on the output gate: the exact form for fp32 outputs; for bf16 outputs the
@@ -216,9 +250,9 @@ template <> __device__ __forceinline__ float gate<__nv_bfloat16>(float v)
 // producer warp: global -> registers (one chunk ahead) -> shared-memory stage
 // ---------------------------------------------------------------------------------------
 
-template <int N, typename T, bool HAS_RESET, bool VEC, bool CONV>
+template <int N, int SPL, typename T, bool HAS_RESET, bool VEC, bool CONV>
 struct IoPrefetch {
-    using S = ScanShape<N>;
+    using S = ScanShape<N, SPL>;
     Raw8<T> bc[S::kBCPerLane];
     Raw8<T> xr[S::kTokPerLane], dr[S::kTokPerLane];
     float bias[S::kTokPerLane];
@@ -363,12 +397,12 @@ template <> __device__ __forceinline__ void smem_store8<float>(float *dst, const
 // from the task's eight inputs u (the raw x tile) and the three before them; x also
 // goes to the chunk's output stage (`ystage`, already free) for the epilogue, and the
 // last conv_k - 1 inputs of each row to conv_state_out.
-template <int N, typename T, bool HAS_RESET, bool VEC, bool CONV>
+template <int N, int SPL, typename T, bool HAS_RESET, bool VEC, bool CONV>
 __device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane,
-                                              const IoPrefetch<N, T, HAS_RESET, VEC, CONV> &f, float *stage,
+                                              const IoPrefetch<N, SPL, T, HAS_RESET, VEC, CONV> &f, float *stage,
                                               unsigned char *raw, int64_t t0, int64_t g, float *ystage)
 {
-    using S = ScanShape<N>;
+    using S = ScanShape<N, SPL>;
     const int64_t L = p.seq;
     if constexpr (!VEC) { // ragged path: B and C tiles into the raw slot, as TMA would lay them out
 #pragma unroll
@@ -381,7 +415,7 @@ __device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane,
                 constexpr int kChunksPer8 = int(sizeof(T)) / 2; // 16-byte chunks per 8 tokens
 #pragma unroll
                 for (int h = 0; h < kChunksPer8; ++h)
-                    *reinterpret_cast<uint4 *>(tile + bc_offset<T>(row, tb * kChunksPer8 + h)) =
+                    *reinterpret_cast<uint4 *>(tile + bc_offset<T, S::template swizzle<T>()>(row, tb * kChunksPer8 + h)) =
                         reinterpret_cast<const uint4 *>(&f.bc[m])[h];
             }
         }
@@ -480,12 +514,12 @@ template <> __device__ __forceinline__ float2 gate2<__nv_bfloat16>(float2 v)
 // Per-thread state of the epilogue that depends only on the channel group: the rows
 // of x, z and y of this thread's channels and their D values.  Refreshed when the
 // group changes (once per work unit), so a chunk costs no index arithmetic.
-template <int N, typename T> struct EpiCache {
-    const T *x[ScanShape<N>::kTokPerLane];
-    const T *z[ScanShape<N>::kTokPerLane];
-    T *y[ScanShape<N>::kTokPerLane];
-    T *xo[ScanShape<N>::kTokPerLane]; // fused conv form: rows of x_out (or null)
-    float d[ScanShape<N>::kTokPerLane];
+template <int N, int SPL, typename T> struct EpiCache {
+    const T *x[ScanShape<N, SPL>::kTokPerLane];
+    const T *z[ScanShape<N, SPL>::kTokPerLane];
+    T *y[ScanShape<N, SPL>::kTokPerLane];
+    T *xo[ScanShape<N, SPL>::kTokPerLane]; // fused conv form: rows of x_out (or null)
+    float d[ScanShape<N, SPL>::kTokPerLane];
     int64_t g = -1;
 };
 
@@ -493,11 +527,11 @@ template <int N, typename T> struct EpiCache {
 // L2 a few chunks earlier), issued first so their latency overlaps the partial sums.
 // In the fused conv form x is not an input: the producers left it in the output
 // stage, and it is also stored to x_out when the caller asks for it.
-template <int N, typename T, bool VEC, bool CONV>
+template <int N, int SPL, typename T, bool VEC, bool CONV>
 __device__ __forceinline__ void epilogue_chunk(const ScanArgs &p, int lane, const float *ystage, int64_t g, int64_t t0,
-                                               EpiCache<N, T> &ec)
+                                               EpiCache<N, SPL, T> &ec)
 {
-    using S = ScanShape<N>;
+    using S = ScanShape<N, SPL>;
     const int64_t L = p.seq;
     if (ec.g != g) {
         const int64_t b = g / p.groups_per_batch;
@@ -549,7 +583,7 @@ __device__ __forceinline__ void epilogue_chunk(const ScanArgs &p, int lane, cons
         for (int k = 0; k < 4; ++k)
             o[k] = make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int pr = 0; pr < S::kPairs; ++pr) {
+        for (int pr = 0; pr < S::kLanes; ++pr) {
             const float4 *src = reinterpret_cast<const float4 *>(ystage + S::kYPOff + cl * S::kYChan + pr * S::kRow + tb * 8);
             const float4 v0 = src[0], v1 = src[1];
             o[0] = __fadd2_rn(o[0], make_float2(v0.x, v0.y));
@@ -613,7 +647,7 @@ struct UnitPos {
     int32_t xrow, brow;    // first x / dt row and first B / C row of the group
 };
 
-template <int N> __device__ __forceinline__ UnitPos unit_pos(const ScanArgs &p, uint32_t u)
+template <int N, int SPL> __device__ __forceinline__ UnitPos unit_pos(const ScanArgs &p, uint32_t u)
 {
     UnitPos up;
     // units, groups and rows all fit in 32 bits (checked on the host)
@@ -624,8 +658,8 @@ template <int N> __device__ __forceinline__ UnitPos unit_pos(const ScanArgs &p, 
     up.t_begin = int64_t(s) * p.seg_len;
     const int64_t rest = p.seq - up.t_begin;
     const int64_t len = rest < p.seg_len ? rest : p.seg_len;
-    up.nck = (len + ScanShape<N>::kChunk - 1) / ScanShape<N>::kChunk;
-    up.xrow = int32_t(int64_t(b) * p.channels + int64_t(g - b * gpb) * ScanShape<N>::kChanPerCta);
+    up.nck = (len + ScanShape<N, SPL>::kChunk - 1) / ScanShape<N, SPL>::kChunk;
+    up.xrow = int32_t(int64_t(b) * p.channels + int64_t(g - b * gpb) * ScanShape<N, SPL>::kChanPerCta);
     up.brow = int32_t(b * N);
     return up;
 }
@@ -644,46 +678,51 @@ template <> __device__ __forceinline__ float2 bc_pair<float>(const uint4 &w, int
                    : make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
 }
 
-// Decays and increments of one group of four tokens for the lane's two states:
-// [token pair][state] as (token t, token t + 1).
-struct GroupTerms {
-    float2 a0[2], a1[2], v0[2], v1[2];
+// Decays and increments of one group of four tokens for the lane's SPL states:
+// [state][token pair] as (token t, token t + 1).
+template <int SPL> struct GroupTerms {
+    float2 a[SPL][2], v[SPL][2];
 };
 
-// One chunk of the recurrence for this lane's two states n0, n1 of channel `cl`:
-// dt and dt*x from the input stage, B and C from the raw slot (storage type), the
-// partial outputs C.h over the two states to `ys`.  Per pair of tokens: two packed
-// multiplies for the exponent arguments, four MUFU ex2, two packed multiplies for
-// the increments, four FMAs along the sequence, two packed ops for the readout.
+// One chunk of the recurrence for this lane's SPL states nn[] of channel `cl`: dt and
+// dt*x from the input stage, B and C from the raw slot (storage type), the partial
+// outputs C.h over the lane's states to `ys`.  Per pair of tokens and state: one
+// packed multiply for the exponent arguments, two MUFU ex2, one packed multiply for
+// the increments, two FMAs along the sequence and one packed op for the readout.
 //
 // Software pipelined over groups of four tokens: the exponentials and increments of
 // group k + 1 are issued before the sequential FMA chain of group k, so the MUFU
-// latency of one group hides behind the chain of the previous one (with only about
-// two scan warps per sub-partition there is little other work to switch to).
+// latency of one group hides behind the chain of the previous one (with one or two
+// scan warps per sub-partition there is little other work to switch to).
 //
 // EMIT: also store the state after every token to `hrow` (this channel's row of h_all
 // at the chunk's first token, N floats per token), for the first `valid` tokens.
-template <int N, typename T, bool HAS_RESET, bool EMIT>
-__device__ __forceinline__ void scan_chunk(const float *stage, const unsigned char *raw, float *ys, int cl, int n0,
-                                           int n1, float2 A0, float2 A1, float &hs0, float &hs1, float *hrow,
-                                           int64_t valid)
+template <int N, int SPL, typename T, bool HAS_RESET, bool EMIT>
+__device__ __forceinline__ void scan_chunk(const float *stage, const unsigned char *raw, float *ys, int cl,
+                                           const int (&nn)[SPL], const float2 (&A2)[SPL], float (&hs)[SPL],
+                                           float *hrow, int64_t valid)
 {
-    using S = ScanShape<N>;
+    using S = ScanShape<N, SPL>;
     constexpr int kTok = 16 / int(sizeof(T)); // tokens per 16-byte chunk of a B/C row
     constexpr int kGroups = S::kChunk / 4;
+    constexpr int SWZ = S::template swizzle<T>();
     const unsigned char *Bt = raw + S::template raw_b_off<T>();
     const unsigned char *Ct = raw + S::template raw_c_off<T>();
     const float *rbs = stage + S::kRBOff;
     const float *dts = stage + S::kDTOff + cl * S::kRow;
     const float *dxs = stage + S::kDXOff + cl * S::kRow;
-    uint4 wb0 = make_uint4(0, 0, 0, 0), wb1 = wb0, wc0 = wb0, wc1 = wb0;
-    GroupTerms gt[2];
+    uint4 wb[SPL], wc[SPL];
+#pragma unroll
+    for (int j = 0; j < SPL; ++j)
+        wb[j] = wc[j] = make_uint4(0, 0, 0, 0);
+    GroupTerms<SPL> gt[2];
     // decays and increments of group k into `f`
-    auto front = [&](int k, GroupTerms &f) {
+    auto front = [&](int k, GroupTerms<SPL> &f) {
         const int t = 4 * k;
         if (t % kTok == 0) {
-            wb0 = *reinterpret_cast<const uint4 *>(Bt + bc_offset<T>(n0, t / kTok));
-            wb1 = *reinterpret_cast<const uint4 *>(Bt + bc_offset<T>(n1, t / kTok));
+#pragma unroll
+            for (int j = 0; j < SPL; ++j)
+                wb[j] = *reinterpret_cast<const uint4 *>(Bt + bc_offset<T, SWZ>(nn[j], t / kTok));
         }
         const float4 d4 = *reinterpret_cast<const float4 *>(dts + t);
         const float4 u4 = *reinterpret_cast<const float4 *>(dxs + t);
@@ -695,19 +734,13 @@ __device__ __forceinline__ void scan_chunk(const float *stage, const unsigned ch
             const int pi = (t % kTok) / 2 + pr;
             const float2 dd = pr ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
             const float2 uu = pr ? make_float2(u4.z, u4.w) : make_float2(u4.x, u4.y);
-            float2 g0, g1;
-            if (HAS_RESET) {
-                const float2 rr = pr ? make_float2(r4.z, r4.w) : make_float2(r4.x, r4.y);
-                g0 = __ffma2_rn(dd, A0, rr);
-                g1 = __ffma2_rn(dd, A1, rr);
-            } else {
-                g0 = __fmul2_rn(dd, A0);
-                g1 = __fmul2_rn(dd, A1);
+            const float2 rr = pr ? make_float2(r4.z, r4.w) : make_float2(r4.x, r4.y);
+#pragma unroll
+            for (int j = 0; j < SPL; ++j) {
+                const float2 g = HAS_RESET ? __ffma2_rn(dd, A2[j], rr) : __fmul2_rn(dd, A2[j]);
+                f.a[j][pr] = make_float2(ex2(g.x), ex2(g.y));
+                f.v[j][pr] = __fmul2_rn(uu, bc_pair<T>(wb[j], pi));
             }
-            f.a0[pr] = make_float2(ex2(g0.x), ex2(g0.y));
-            f.a1[pr] = make_float2(ex2(g1.x), ex2(g1.y));
-            f.v0[pr] = __fmul2_rn(uu, bc_pair<T>(wb0, pi));
-            f.v1[pr] = __fmul2_rn(uu, bc_pair<T>(wb1, pi));
         }
     };
     front(0, gt[0]);
@@ -715,32 +748,49 @@ __device__ __forceinline__ void scan_chunk(const float *stage, const unsigned ch
     for (int k = 0; k < kGroups; ++k) {
         const int t = 4 * k;
         if (t % kTok == 0) {
-            wc0 = *reinterpret_cast<const uint4 *>(Ct + bc_offset<T>(n0, t / kTok));
-            wc1 = *reinterpret_cast<const uint4 *>(Ct + bc_offset<T>(n1, t / kTok));
+#pragma unroll
+            for (int j = 0; j < SPL; ++j)
+                wc[j] = *reinterpret_cast<const uint4 *>(Ct + bc_offset<T, SWZ>(nn[j], t / kTok));
         }
-        const uint4 cc0 = wc0, cc1 = wc1;
+        uint4 cc[SPL];
+#pragma unroll
+        for (int j = 0; j < SPL; ++j)
+            cc[j] = wc[j];
         if (k + 1 < kGroups)
             front(k + 1, gt[(k + 1) & 1]);
-        const GroupTerms &f = gt[k & 1];
+        const GroupTerms<SPL> &f = gt[k & 1];
         float2 yo[2];
 #pragma unroll
         for (int pr = 0; pr < 2; ++pr) {
             const int pi = (t % kTok) / 2 + pr;
-            const float h0t = fmaf(f.a0[pr].x, hs0, f.v0[pr].x);
-            hs0 = fmaf(f.a0[pr].y, h0t, f.v0[pr].y);
-            const float h1t = fmaf(f.a1[pr].x, hs1, f.v1[pr].x);
-            hs1 = fmaf(f.a1[pr].y, h1t, f.v1[pr].y);
-            const float2 yy = __fmul2_rn(bc_pair<T>(cc0, pi), make_float2(h0t, hs0));
-            yo[pr] = __ffma2_rn(bc_pair<T>(cc1, pi), make_float2(h1t, hs1), yy);
+            float hm[SPL]; // the states after token t + 2 pr (hs: after the next token)
+#pragma unroll
+            for (int j = 0; j < SPL; ++j) {
+                hm[j] = fmaf(f.a[j][pr].x, hs[j], f.v[j][pr].x);
+                hs[j] = fmaf(f.a[j][pr].y, hm[j], f.v[j][pr].y);
+            }
+            float2 yy = __fmul2_rn(bc_pair<T>(cc[0], pi), make_float2(hm[0], hs[0]));
+#pragma unroll
+            for (int j = 1; j < SPL; ++j)
+                yy = __ffma2_rn(bc_pair<T>(cc[j], pi), make_float2(hm[j], hs[j]), yy);
+            yo[pr] = yy;
             if (EMIT) {
                 const int tt = t + 2 * pr;
-                if (tt < valid) {
-                    __stcs(hrow + tt * N + n0, h0t);
-                    __stcs(hrow + tt * N + n1, h1t);
-                }
-                if (tt + 1 < valid) {
-                    __stcs(hrow + (tt + 1) * N + n0, hs0);
-                    __stcs(hrow + (tt + 1) * N + n1, hs1);
+                if constexpr (S::template contiguous<T>()) {
+                    if (tt < valid)
+                        __stcs(reinterpret_cast<float4 *>(hrow + tt * N + nn[0]),
+                               make_float4(hm[0], hm[1], hm[2], hm[3]));
+                    if (tt + 1 < valid)
+                        __stcs(reinterpret_cast<float4 *>(hrow + (tt + 1) * N + nn[0]),
+                               make_float4(hs[0], hs[1], hs[2], hs[3]));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < SPL; ++j) {
+                        if (tt < valid)
+                            __stcs(hrow + tt * N + nn[j], hm[j]);
+                        if (tt + 1 < valid)
+                            __stcs(hrow + (tt + 1) * N + nn[j], hs[j]);
+                    }
                 }
             }
         }
@@ -752,10 +802,10 @@ __device__ __forceinline__ void scan_chunk(const float *stage, const unsigned ch
 // raw-ring slot as far ahead as the ring allows and, on the TMA path (VEC), starts the
 // chunk's 2-D tile loads of x, dt, z, B and C into the slot.  Every lane returns
 // normally, so the warp reaches the kernel's end-of-call accounting as a whole.
-template <int N, typename T, bool VEC>
+template <int N, int SPL, typename T, bool VEC>
 __device__ __forceinline__ bool issuer_warp(const ScanArgs &p, const TmaMaps &maps, const CtaCtx &cx, int lane)
 {
-    using S = ScanShape<N>;
+    using S = ScanShape<N, SPL>;
     constexpr int RS = S::kRawStages;
     if (lane != 0)
         return true;
@@ -769,7 +819,7 @@ __device__ __forceinline__ bool issuer_warp(const ScanArgs &p, const TmaMaps &ma
     uint32_t u = take_unit(p, cx.ws, true);
     UnitPos up;
     if (u != kNoUnit)
-        up = unit_pos<N>(p, u);
+        up = unit_pos<N, SPL>(p, u);
     int64_t k = 0;
     for (uint32_t j = 0;; ++j) {
         const int r = int(j % RS);
@@ -806,21 +856,21 @@ __device__ __forceinline__ bool issuer_warp(const ScanArgs &p, const TmaMaps &ma
             u = take_unit(p, cx.ws, false);
             k = 0;
             if (u != kNoUnit)
-                up = unit_pos<N>(p, u);
+                up = unit_pos<N, SPL>(p, u);
         }
     }
 }
 
 // The two producer warps: each thread converts its share of every chunk (from the
 // raw slot, or straight from global memory on the ragged path) into the input stage.
-template <int N, typename T, bool HAS_RESET, bool VEC, bool CONV>
+template <int N, int SPL, typename T, bool HAS_RESET, bool VEC, bool CONV>
 __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, int pi, int lane)
 {
-    using S = ScanShape<N>;
+    using S = ScanShape<N, SPL>;
     constexpr int RS = S::kRawStages;
     constexpr int kRawBytes = S::template raw_stage_bytes<T>();
     const int tl = pi * 32 + lane; // producer thread index
-    IoPrefetch<N, T, HAS_RESET, VEC, CONV> pf;
+    IoPrefetch<N, SPL, T, HAS_RESET, VEC, CONV> pf;
     int64_t reset_g = -1;
     const uint8_t *reset_row = p.reset;
     for (uint32_t i = 0;; ++i) {
@@ -860,7 +910,7 @@ __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, in
         if (CONV && !mbar_wait(cx.y_empty + ys, ((i / S::kYStages) & 1u) ^ 1u, cx.status))
             return false;
         if (!end)
-            produce_chunk<N, T, HAS_RESET, VEC, CONV>(p, tl, pf, stage, cx.raw_base + r * kRawBytes, t0, g, ystage);
+            produce_chunk<N, SPL, T, HAS_RESET, VEC, CONV>(p, tl, pf, stage, cx.raw_base + r * kRawBytes, t0, g, ystage);
         if (tl == 0)
             write_meta(stage, t0, g, s, fl);
         if (!CONV && !mbar_wait(cx.y_empty + ys, ((i / S::kYStages) & 1u) ^ 1u, cx.status))
@@ -874,12 +924,12 @@ __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, in
 }
 
 // The two epilogue warps: partial outputs of each chunk -> y.  False on a timeout.
-template <int N, typename T, bool VEC, bool CONV>
+template <int N, int SPL, typename T, bool VEC, bool CONV>
 __device__ __forceinline__ bool epilogue_role(const ScanArgs &p, const float *y_base, uint64_t *y_full,
                                               uint64_t *y_empty, uint32_t *status, int tl)
 {
-    using S = ScanShape<N>;
-    EpiCache<N, T> ec;
+    using S = ScanShape<N, SPL>;
+    EpiCache<N, SPL, T> ec;
     for (uint32_t j = 0;; ++j) {
         const int ys = int(j % S::kYStages);
         if (!mbar_wait(y_full + ys, (j / S::kYStages) & 1u, status))
@@ -888,7 +938,7 @@ __device__ __forceinline__ bool epilogue_role(const ScanArgs &p, const float *y_
         const ChunkMeta meta = read_meta(ystage);
         if (meta.flags & kEnd)
             return true;
-        epilogue_chunk<N, T, VEC, CONV>(p, tl, ystage, meta.g, meta.t0, ec);
+        epilogue_chunk<N, SPL, T, VEC, CONV>(p, tl, ystage, meta.g, meta.t0, ec);
         mbar_arrive(y_empty + ys);
     }
 }
@@ -900,16 +950,16 @@ __device__ __forceinline__ bool epilogue_role(const ScanArgs &p, const float *y_
 // CTAs per SM to plan registers for: the states and conv forms need more registers
 // than the plain form and are bounded to two CTAs per SM wherever shared memory fits
 // two (about 113 KB each); the plain form gets there at its natural allocation.
-template <int N, typename T, bool EMIT, bool CONV> constexpr int scan_min_ctas()
+template <int N, int SPL, typename T, bool EMIT, bool CONV> constexpr int scan_min_ctas()
 {
-    return (EMIT || CONV) && ScanShape<N>::template smem_bytes<T, true>() <= 113 * 1024 ? 2 : 1;
+    return (EMIT || CONV) && ScanShape<N, SPL>::template smem_bytes<T, true>() <= 113 * 1024 ? 2 : 1;
 }
 
-template <int N, typename T, bool HAS_RESET, bool VEC, bool EMIT, bool CONV>
-__global__ void __launch_bounds__(ScanShape<N>::kThreads, (scan_min_ctas<N, T, EMIT, CONV>()))
+template <int N, int SPL, typename T, bool HAS_RESET, bool VEC, bool EMIT, bool CONV>
+__global__ void __launch_bounds__(ScanShape<N, SPL>::kThreads, (scan_min_ctas<N, SPL, T, EMIT, CONV>()))
 ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
 {
-    using S = ScanShape<N>;
+    using S = ScanShape<N, SPL>;
     constexpr int kRawRing = S::kRawStages * S::template raw_stage_bytes<T>();
     extern __shared__ __align__(1024) unsigned char smem_bytes[];
     float *const in_base = reinterpret_cast<float *>(smem_bytes + kRawRing);
@@ -922,20 +972,21 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
     WsHeader *const ws = reinterpret_cast<WsHeader *>(p.workspace);
     const bool chained = ws != nullptr;
     uint32_t *const status = chained ? &ws->status : p.status;
-    const uint32_t epoch = chained ? *reinterpret_cast<volatile uint32_t *>(&ws->epoch) : 0u;
+    const uint64_t epoch = chained ? *reinterpret_cast<volatile uint64_t *>(&ws->epoch) : 0u;
     uint64_t *const flags = chained ? reinterpret_cast<uint64_t *>(p.workspace + sizeof(WsHeader)) : nullptr;
-    float2 *const carry = chained
-        ? reinterpret_cast<float2 *>(p.workspace + sizeof(WsHeader) + 8 * p.groups * S::kScanWarps)
+    // carries: SPL floats per lane and (channel group, scan warp) slot
+    float *const carry = chained
+        ? reinterpret_cast<float *>(p.workspace + sizeof(WsHeader) + 8 * p.groups * S::kScanWarps)
         : nullptr;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S::kStages; ++s) {
-            mbar_init(in_full + s, S::kIoThreads);          // both producer warps
+            mbar_init(in_full + s, S::kIoThreads);          // the producer warps
             mbar_init(in_empty + s, 32 * S::kScanWarps);
         }
         for (int s = 0; s < S::kYStages; ++s) {
             mbar_init(y_full + s, 32 * S::kScanWarps);
-            mbar_init(y_empty + s, S::kIoThreads);          // both epilogue warps
+            mbar_init(y_empty + s, S::kIoThreads);          // the epilogue warps
         }
         for (int r = 0; r < S::kRawStages; ++r) {
             mbar_init(bars + S::kBarRawFull + r, 1);              // the issuer
@@ -960,32 +1011,44 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
         cx.raw_meta = reinterpret_cast<int64_t *>(bars + S::kBars);
         cx.ws = ws;
         cx.status = status;
+        // IO role of this warp and its index within the role: with two warps per role
+        // they alternate (sub-partitions 0 and 2 produce, 1 and 3 finish outputs), with
+        // four per role each role takes four consecutive warps (one per sub-partition)
+        const int io = warp - S::kScanWarps;
+        const bool prod = S::kIoWarps == 4 ? io < 4 : (io & 1) == 0;
+        const int ri = S::kIoWarps == 4 ? (io & 3) : (io >> 1);
         bool ok;
         if (warp == S::kIssuerWarp)
-            ok = issuer_warp<N, T, VEC>(p, maps, cx, lane);
-        else if (((warp - S::kScanWarps) & 1) == 0)
-            ok = producer<N, T, HAS_RESET, VEC, CONV>(p, cx, (warp - S::kScanWarps) >> 1, lane);
+            ok = issuer_warp<N, SPL, T, VEC>(p, maps, cx, lane);
+        else if (prod)
+            ok = producer<N, SPL, T, HAS_RESET, VEC, CONV>(p, cx, ri, lane);
         else
-            ok = epilogue_role<N, T, VEC, CONV>(p, y_base, y_full, y_empty, status,
-                                          ((warp - S::kScanWarps) >> 1) * 32 + lane);
-        if (!ok)
-            return; // gave up on a wait (SS_ERR_TIMEOUT recorded)
+            ok = epilogue_role<N, SPL, T, VEC, CONV>(p, y_base, y_full, y_empty, status, ri * 32 + lane);
+        (void)ok; // false: gave up on a wait (SS_ERR_TIMEOUT recorded); counted out below
     } else {
         // =============================== scan warps ==============================
-        const int cw = lane / S::kPairs;    // channel within the warp
-        const int sub = lane % S::kPairs;   // state pair
-        // rows n0 < N/2 and n1 >= N/2: distinct banks of the B/C tiles (and the same
-        // lane-to-state map in every form, so outputs are bit-identical across forms)
-        const int n0 = sub, n1 = sub + S::kPairs;
+        const int cw = lane / S::kLanes;    // channel within the warp
+        const int sub = lane % S::kLanes;   // state group within the channel
+        // the lane's states (the same lane-to-state map in every form of this layout, so
+        // outputs are bit-identical across the plain, states and segmented forms)
+        int nn[SPL];
+#pragma unroll
+        for (int j = 0; j < SPL; ++j)
+            nn[j] = S::template state<T>(sub, j);
         const int cl = warp * S::kChanPerWarp + cw;  // channel within the CTA
-        float hs0 = 0.0f, hs1 = 0.0f;
-        float2 A0 = make_float2(0.f, 0.f), A1 = make_float2(0.f, 0.f);
+        float hs[SPL];
+        float2 A2[SPL];
+#pragma unroll
+        for (int j = 0; j < SPL; ++j) {
+            hs[j] = 0.0f;
+            A2[j] = make_float2(0.f, 0.f);
+        }
         int64_t row = 0;
         bool cvalid = false;
         for (uint32_t j = 0;; ++j) {
             const int st = int(j % S::kStages);
             if (!mbar_wait(in_full + st, (j / S::kStages) & 1u, status))
-                return;
+                break; // timeout recorded; counted out below
             // (in_full also means: the chunk's raw slot has landed and its output
             // stage is free -- the producers waited for both before arriving)
             const float *stage = in_base + st * S::kInStage;
@@ -1001,54 +1064,63 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
                 cvalid = c_raw < p.channels;
                 const int64_t c = cvalid ? c_raw : p.channels - 1;
                 row = b * p.channels + c;
-                const float a0 = __ldg(p.A + c * N + n0) * kLog2e;
-                const float a1 = __ldg(p.A + c * N + n1) * kLog2e;
-                A0 = make_float2(a0, a0);
-                A1 = make_float2(a1, a1);
+#pragma unroll
+                for (int q = 0; q < SPL; ++q) {
+                    const float a = __ldg(p.A + c * N + nn[q]) * kLog2e;
+                    A2[q] = make_float2(a, a);
+                }
                 if (meta.s == 0) {
-                    hs0 = p.h0 ? __ldg(p.h0 + row * N + n0) : 0.0f;
-                    hs1 = p.h0 ? __ldg(p.h0 + row * N + n1) : 0.0f;
+#pragma unroll
+                    for (int q = 0; q < SPL; ++q)
+                        hs[q] = p.h0 ? __ldg(p.h0 + row * N + nn[q]) : 0.0f;
                 } else {
                     const int64_t slot = meta.g * S::kScanWarps + warp;
-                    const uint64_t want = (uint64_t(epoch) << 32) | uint64_t(meta.s);
+                    const uint64_t want = carry_tag(epoch, meta.s);
                     if (!flag_wait(flags + slot, want, status))
-                        return;
-                    const float2 h = __ldcg(carry + slot * 32 + lane);
-                    hs0 = h.x;
-                    hs1 = h.y;
+                        break; // timeout recorded; counted out below
+                    const float *cs = carry + (slot * 32 + lane) * SPL;
+#pragma unroll
+                    for (int q = 0; q < SPL; ++q)
+                        hs[q] = __ldcg(cs + q);
                 }
             }
             const int rs = int(j % S::kRawStages);
             float *hrow = nullptr;
             if (EMIT)
                 hrow = p.h_all + (row * p.seq + meta.t0) * N;
-            scan_chunk<N, T, HAS_RESET, EMIT>(stage, smem_bytes + rs * S::template raw_stage_bytes<T>(),
-                                              y_base + ysi * S::template y_stage<T>() + S::kYPOff + cl * S::kYChan + sub * S::kRow,
-                                              cl, n0, n1, A0, A1, hs0, hs1, hrow,
-                                              cvalid ? p.seq - meta.t0 : int64_t(0));
+            scan_chunk<N, SPL, T, HAS_RESET, EMIT>(stage, smem_bytes + rs * S::template raw_stage_bytes<T>(),
+                                                   y_base + ysi * S::template y_stage<T>() + S::kYPOff +
+                                                       cl * S::kYChan + sub * S::kRow,
+                                                   cl, nn, A2, hs, hrow, cvalid ? p.seq - meta.t0 : int64_t(0));
             mbar_arrive(bars + S::kBarRawEmpty + rs);
             mbar_arrive(in_empty + st);
             mbar_arrive(y_full + ysi);
             if (meta.flags & kLast) {
                 if (int64_t(meta.s) + 1 < p.segments) {
                     const int64_t slot = meta.g * S::kScanWarps + warp;
-                    __stcg(carry + slot * 32 + lane, make_float2(hs0, hs1));
+                    float *cs = carry + (slot * 32 + lane) * SPL;
+#pragma unroll
+                    for (int q = 0; q < SPL; ++q)
+                        __stcg(cs + q, hs[q]);
                     __threadfence();
                     __syncwarp();
                     if (lane == 0)
-                        st_release_gpu(flags + slot, (uint64_t(epoch) << 32) | uint64_t(meta.s + 1));
+                        st_release_gpu(flags + slot, carry_tag(epoch, meta.s + 1));
                 } else if (p.h_last && cvalid) {
-                    p.h_last[row * N + n0] = hs0;
-                    p.h_last[row * N + n1] = hs1;
+#pragma unroll
+                    for (int q = 0; q < SPL; ++q)
+                        p.h_last[row * N + nn[q]] = hs[q];
                 }
             }
         }
     }
 
     // The last warp of a chained call to finish resets the work counter and advances
-    // the epoch for the next call.  (Each warp counts itself, so no CTA-wide barrier is
-    // needed after the roles have diverged; a warp that gave up on a wait never gets
-    // here, and then the workspace stays as it is and the status word says why.)
+    // the epoch for the next call.  Each warp counts itself, so no CTA-wide barrier is
+    // needed after the roles have diverged; a warp that gave up on a wait counts itself
+    // too (every wait is bounded, so every warp gets here), so even a call that timed
+    // out leaves the workspace ready: its carry flags hold the old epoch and can never
+    // satisfy a later call's wait, and the status word says what happened.
     if (chained) {
         if (lane == 0) {
             __threadfence();
@@ -1057,16 +1129,16 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
                 ws->done = 0;
                 ws->counter = 0;
                 __threadfence();
-                atomicAdd(&ws->epoch, 1u);
+                atomicAdd(reinterpret_cast<unsigned long long *>(&ws->epoch), 1ull);
             }
         }
     }
 }
 
 // Bytes of workspace a chained call needs for `groups` channel groups.
-template <int N> constexpr int64_t scan_workspace_bytes(int64_t groups)
+template <int N, int SPL> constexpr int64_t scan_workspace_bytes(int64_t groups)
 {
-    return int64_t(sizeof(WsHeader)) + groups * ScanShape<N>::kScanWarps * (8 + 32 * 8);
+    return int64_t(sizeof(WsHeader)) + groups * ScanShape<N, SPL>::kScanWarps * (8 + 32 * SPL * 4);
 }
 
 } // namespace ss

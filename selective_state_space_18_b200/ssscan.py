@@ -9,6 +9,8 @@ error, never a fallback.
 from __future__ import annotations
 
 import ctypes
+import functools
+import itertools
 import os
 import threading
 
@@ -24,8 +26,9 @@ SS_STATIC_SCRATCH_BYTES = 1 << 20
 STATUS = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE", 4: "SS_ERR_ALIGN",
           5: "SS_ERR_UNSUPPORTED", 6: "SS_ERR_CUDA", 7: "SS_ERR_TIMEOUT", 8: "SS_ERR_ALIAS",
           9: "SS_ERR_WORKSPACE", 10: "SS_ERR_SCRATCH_LIMIT"}
-EXPORTS = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_scan_status", "ss_state_update",
-           "ss_debug_set_wait_limit", "ss_status_string", "ss_abi_version",
+EXPORTS = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_scan_plan", "ss_scan_status", "ss_debug_status",
+           "ss_state_update",
+           "ss_debug_set_wait_limit", "ss_debug_set_scan_layout", "ss_status_string", "ss_abi_version",
            "ss_scan_fwd_static_scratch", "ss_scan_fwd_states", "ss_gated_scan", "ss_scan_fwd_conv",
            "ss_state_update_conv", "ss_segment_decay", "ss_join_segments")
 ABI_MAJOR = 2
@@ -34,6 +37,13 @@ _lock = threading.Lock()
 _lib = None
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
+
+
+class ScanPlan(ctypes.Structure):
+    """ss_scan_plan_t: the launch plan of ss_scan_fwd for a shape."""
+    _fields_ = [("grid", ctypes.c_int64), ("ctas_per_sm", ctypes.c_int64), ("sms", ctypes.c_int64),
+                ("groups", ctypes.c_int64), ("segments", ctypes.c_int64), ("seg_len", ctypes.c_int64),
+                ("states_per_lane", ctypes.c_int64)]
 
 
 class SSError(RuntimeError):
@@ -76,6 +86,9 @@ def load_library(path: str = LIB_PATH):
             lib.ss_segment_decay.restype = ctypes.c_int
             lib.ss_join_segments.argtypes = [_i64, _i64, _vp, _i64, _vp, _vp, _vp]
             lib.ss_join_segments.restype = ctypes.c_int
+            lib.ss_scan_plan.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.POINTER(ScanPlan)]
+            lib.ss_scan_plan.restype = ctypes.c_int
             lib.ss_scan_workspace_bytes.argtypes = [_i64, _i64, _i64, _i64]
             lib.ss_scan_workspace_bytes.restype = _i64
             lib.ss_scan_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_int)]
@@ -87,12 +100,31 @@ def load_library(path: str = LIB_PATH):
             lib.ss_status_string.restype = ctypes.c_char_p
             lib.ss_debug_set_wait_limit.argtypes = [ctypes.c_uint32]
             lib.ss_debug_set_wait_limit.restype = ctypes.c_int
+            lib.ss_debug_set_scan_layout.argtypes = [ctypes.c_int]
+            lib.ss_debug_set_scan_layout.restype = ctypes.c_int
+            lib.ss_debug_status.argtypes = [_vp]
+            lib.ss_debug_status.restype = ctypes.c_int
             lib.ss_abi_version.argtypes = []
             lib.ss_abi_version.restype = ctypes.c_int
             if lib.ss_abi_version() >> 16 != ABI_MAJOR:
                 raise RuntimeError(f"{path}: ABI {lib.ss_abi_version() >> 16}, expected {ABI_MAJOR}")
             _lib = lib
     return _lib
+
+
+def _on_tensor_device(fn):
+    """Run a wrapper with the device of its first tensor argument current: the library
+    looks up per-device state (kernel attributes, occupancy, status words, the static
+    scratch) for the current device, which must be the one the launch goes to."""
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        dev = next((a.device for a in itertools.chain(args, kwargs.values())
+                    if isinstance(a, torch.Tensor)), None)
+        if dev is None or dev.type != "cuda":
+            return fn(*args, **kwargs)
+        with torch.cuda.device(dev):
+            return fn(*args, **kwargs)
+    return wrapper
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -150,16 +182,54 @@ def scan_workspace(batch, channels, state_dim, seq, device, stream=None):
     return ws
 
 
+def ss_scan_plan(batch, channels, state_dim, seq, dtype=torch.bfloat16, *, has_reset=False, workspace=True,
+                 device=None):
+    """Launch plan of ss_scan_fwd for this shape on `device` (16-byte aligned tensors):
+    dict(grid, ctas_per_sm, sms, groups, segments, seg_len, states_per_lane).  Launches
+    nothing."""
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    code = SS_BF16 if dtype == torch.bfloat16 else SS_F32
+    plan = ScanPlan()
+    with torch.cuda.device(device):
+        st = load_library().ss_scan_plan(batch, channels, state_dim, seq, code, int(bool(has_reset)),
+                                         int(bool(workspace)), ctypes.byref(plan))
+    if st != 0:
+        raise SSError("ss_scan_plan", st)
+    return {name: int(getattr(plan, name)) for name, _ in ScanPlan._fields_}
+
+
 def ss_scan_status(workspace=None, stream=None, device=None):
     """Read and clear the device status word of earlier scans (synchronises the
     stream): 'SS_OK' or 'SS_ERR_TIMEOUT'."""
     if device is None:
         device = workspace.device if workspace is not None else torch.device("cuda", torch.cuda.current_device())
     out = ctypes.c_int(-1)
-    st = load_library().ss_scan_status(_ptr(workspace), _stream(stream, device), ctypes.byref(out))
+    with torch.cuda.device(device):
+        st = load_library().ss_scan_status(_ptr(workspace), _stream(stream, device), ctypes.byref(out))
     if st != 0:
         raise SSError("ss_scan_status", st)
     return STATUS[out.value]
+
+
+def ss_debug_status(stream=None, device=None):
+    """Read and clear the device status word of the calls made without a workspace on
+    `device` (synchronises the stream): 'SS_OK' or 'SS_ERR_TIMEOUT'."""
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(device):
+        st = load_library().ss_debug_status(_stream(stream, device))
+    if st not in (0, 7):
+        raise SSError("ss_debug_status", st)
+    return STATUS[st]
+
+
+def ss_debug_set_scan_layout(states_per_lane: int) -> None:
+    """Force the state_dim-16 scan layout (2 or 4 states per scan lane; 0: automatic)
+    for later calls.  A testing aid: both layouts compute the same results."""
+    st = load_library().ss_debug_set_scan_layout(int(states_per_lane))
+    if st != 0:
+        raise SSError("ss_debug_set_scan_layout", st)
 
 
 def ss_debug_set_wait_limit(microseconds: int) -> None:
@@ -175,6 +245,7 @@ def _stream(stream, device):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+@_on_tensor_device
 def ss_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h0=None, *,
                 dt_softplus=True, y=None, h_last=None, return_last_state=True, stream=None,
                 workspace=True, h_all=None, return_states=False):
@@ -247,6 +318,7 @@ def ss_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h0=Non
     return y, h_last
 
 
+@_on_tensor_device
 def ss_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, *, dt_softplus=True,
                     y=None, stream=None):
     """Decode step, ``state`` [batch, channels, state_dim] fp32 updated in place.
@@ -285,6 +357,7 @@ def ss_state_update(state, x, dt, A, B, C, D=None, z=None, dt_bias=None, *, dt_s
 _scratch_addr = {}
 
 
+@_on_tensor_device
 def ss_scan_fwd_static_scratch(x, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h0=None, *,
                                dt_softplus=True, y=None, h_last=None, return_last_state=True,
                                stream=None, zero_scratch=False):
@@ -343,12 +416,14 @@ def static_scratch_status(stream=None, device=None):
     if addr is None:
         raise RuntimeError("no ss_scan_fwd_static_scratch call has run on this device")
     out = ctypes.c_int(-1)
-    st = load_library().ss_scan_status(_vp(addr), _stream(stream, device), ctypes.byref(out))
+    with torch.cuda.device(device):
+        st = load_library().ss_scan_status(_vp(addr), _stream(stream, device), ctypes.byref(out))
     if st != 0:
         raise SSError("ss_scan_status", st)
     return STATUS[out.value]
 
 
+@_on_tensor_device
 def ss_gated_scan(q, k, v, gamma, h0=None, *, stream=None):
     """Gated state scan S_t = gamma_t S_{t-1} + k_t v_t^T, y_t = q_t^T S_t.  q, k:
     [B, S, Dk]; v: [B, S, Dv] (float32 or bfloat16, same dtype); gamma: [B, S] float32;
@@ -376,6 +451,7 @@ def ss_gated_scan(q, k, v, gamma, h0=None, *, stream=None):
     return {"outputs": y, "final_state": fs}
 
 
+@_on_tensor_device
 def ss_scan_fwd_conv(u, conv_w, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h0=None, *,
                      conv_b=None, conv_state=None, dt_softplus=True, return_conv_state=True,
                      return_x=False, stream=None, workspace=True):
@@ -430,6 +506,7 @@ def ss_scan_fwd_conv(u, conv_w, dt, A, B, C, D=None, z=None, dt_bias=None, reset
     return out
 
 
+@_on_tensor_device
 def ss_state_update_conv(state, conv_state, conv_w, u, dt, A, B, C, D=None, z=None, dt_bias=None, *,
                          conv_b=None, dt_softplus=True, stream=None):
     """Decode step of the fused conv form: ``state`` [batch, channels, state_dim] fp32 and
@@ -467,6 +544,7 @@ def ss_state_update_conv(state, conv_state, conv_w, u, dt, A, B, C, D=None, z=No
     return y
 
 
+@_on_tensor_device
 def ss_segment_decay(dt, A, dt_bias=None, reset=None, *, dt_softplus=True, out=None, stream=None):
     """Decay of one segment of a sequence: [batch, channels, state_dim] fp32 =
     exp(A * sum of the segment's step sizes), 0 where the segment holds a reset.
@@ -501,6 +579,7 @@ def ss_segment_decay(dt, A, dt_bias=None, reset=None, *, dt_softplus=True, out=N
     return out
 
 
+@_on_tensor_device
 def ss_join_segments(composites, rank=None, *, carry=None, final_state=None, want_final=True, stream=None):
     """Fold gathered segment composites [segments, 2, ...] (decay, end state; fp32,
     contiguous) in segment order.  Returns (carry, final_state): the state entering

@@ -42,7 +42,9 @@ def test_shape_beyond_scratch_is_refused_before_launch():
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("dtype,resets", [("bf16", True), ("f32", False)])
-def test_static_scratch_matches_workspace_call_twice(dtype, resets):
+def test_static_scratch_matches_workspace_call_twice(orc, dtype, resets):
+    """Two calls in a row, each against ss_scan_fwd with a workspace (the entry point
+    this one stands in for) and against the float64 oracle."""
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA GPU")
     bt, ch, n, L = 2, 320, 16, 3000  # 40 groups, ragged sequence tail
@@ -50,6 +52,7 @@ def test_static_scratch_matches_workspace_call_twice(dtype, resets):
     d = dev(inp, SCAN_KEYS)
     y_ref, h_ref = ssscan.ss_scan_fwd(**d, workspace=True)
     tol = TOL[y_ref.dtype]
+    ref = orc.scan(**inp)
     y_out = torch.empty_like(y_ref)
     h_out = torch.empty_like(h_ref)
     for call in range(2):
@@ -63,17 +66,20 @@ def test_static_scratch_matches_workspace_call_twice(dtype, resets):
         assert ssscan.static_scratch_status() == "SS_OK"
         assert_close(y_out.cpu(), y_ref.cpu().double().numpy(), tol, f"y, call {call}")
         assert_close(h_out.cpu(), h_ref.cpu().double().numpy(), 1e-4, f"h_last, call {call}")
+        assert_close(y_out.cpu(), ref["y"], tol, f"y vs oracle, call {call}")
+        assert_close(h_out.cpu(), ref["h_last"], tol, f"h_last vs oracle, call {call}")
 
 
 @pytest.mark.gpu
-def test_static_scratch_zero_flag_and_chaining():
+def test_static_scratch_zero_flag_and_chaining(orc):
     """SS_SCRATCH_ZERO clears the scratch before the scan; a prompt split in two
-    calls chained through h_last equals one call."""
+    calls chained through h_last equals one call, and the oracle."""
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA GPU")
     bt, ch, n, L = 1, 512, 16, 4096
     inp = make_scan_inputs(bt, ch, n, L, "f32", seed=5)
     d = dev(inp, SCAN_KEYS)
+    ref_o = orc.scan(**inp)
     y_all, h_all = ssscan.ss_scan_fwd_static_scratch(**d, zero_scratch=True)
     half = {k: (v[..., : L // 2].contiguous() if k in ("x", "dt", "z", "B", "C") and v is not None else v)
             for k, v in d.items()}
@@ -87,3 +93,28 @@ def test_static_scratch_zero_flag_and_chaining():
     ref = y_all.cpu().double().numpy()
     assert_close(torch.cat([y1, y2], -1).cpu(), ref, 1e-4, "chained y")
     assert_close(h2.cpu(), h_all.cpu().double().numpy(), 1e-4, "chained h_last")
+    assert_close(y_all.cpu(), ref_o["y"], 1e-4, "y vs oracle")
+    assert_close(h_all.cpu(), ref_o["h_last"], 1e-4, "h_last vs oracle")
+
+
+@pytest.mark.gpu
+def test_zero_flag_clears_carry_flags_of_a_larger_shape():
+    """SS_SCRATCH_ZERO must clear the carry flags a LARGER earlier call left beyond the
+    current shape's part of the scratch: the epoch restarts at zero, and a flag left
+    by that earlier call at epoch zero would otherwise satisfy a later call's wait
+    with a stale carry.  Large call A at epoch 0, a zeroing small call, then a zeroing
+    large call B (epoch 0 again) on other inputs: B must equal ss_scan_fwd."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    big = (1, 2048, 16, 4096)   # 128 channel groups, several segments each
+    small = (1, 64, 16, 512)    # 4 groups: its part of the scratch is a small prefix
+    a = dev(make_scan_inputs(*big, "bf16", seed=11), SCAN_KEYS)
+    s = dev(make_scan_inputs(*small, "bf16", seed=12), SCAN_KEYS)
+    b = dev(make_scan_inputs(*big, "bf16", seed=13), SCAN_KEYS)
+    y_ref, h_ref = ssscan.ss_scan_fwd(**b, workspace=True)
+    ssscan.ss_scan_fwd_static_scratch(**a, zero_scratch=True)
+    ssscan.ss_scan_fwd_static_scratch(**s, zero_scratch=True)
+    y_b, h_b = ssscan.ss_scan_fwd_static_scratch(**b, zero_scratch=True)
+    torch.cuda.synchronize()
+    assert ssscan.static_scratch_status() == "SS_OK"
+    assert torch.equal(y_b, y_ref) and torch.equal(h_b, h_ref)
