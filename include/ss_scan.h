@@ -94,6 +94,15 @@ enum { SS_DT_SOFTPLUS = 1u };
  *                  them, which balances the GPU for any shape.  Without one, each CTA
  *                  scans one group of channels over the whole sequence.  Calls that
  *                  share a workspace must be ordered (same stream, or synchronised).
+ *                  For state_dim 16 with few channel groups and a long sequence (the
+ *                  single-pass schedule would leave most of the GPU idle), the size
+ *                  includes room for a two-level schedule ("s6_reset" blog draft,
+ *                  Associative Boundary Resetting): every segment of the sequence is
+ *                  scanned at once from zero for its end state, the segments'
+ *                  (decay, end state) composites are joined into each one's entering
+ *                  state, and every segment is scanned again from it.  It runs when
+ *                  the workspace has that size; it does the exponentials twice, in
+ *                  exchange for filling the GPU.
  *                  A call whose device-side waits gave up (SS_ERR_TIMEOUT, see
  *                  ss_scan_status) also leaves the workspace ready for the next call:
  *                  its outputs are invalid, but the workspace needs no re-zeroing.
@@ -172,6 +181,7 @@ typedef struct {
     int64_t segments;    /* sequence segments per group (1 without a workspace)  */
     int64_t seg_len;     /* tokens per segment                                   */
     int64_t states_per_lane; /* state rows each scan lane owns (2 or 4)          */
+    int64_t two_level;   /* 1: the two-level schedule (see ss_scan_fwd), 0: single pass */
 } ss_scan_plan_t;
 SS_API int ss_scan_plan(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
                         ss_dtype_t dtype, int has_reset, int with_workspace,
@@ -305,6 +315,16 @@ SS_API int ss_debug_set_wait_limit(uint32_t microseconds);
  * being issued concurrently from other host threads.
  */
 SS_API int ss_debug_set_scan_layout(int states_per_lane);
+
+/*
+ * Testing aid: the schedule of later state_dim-16 scans with a workspace.  mode 0
+ * (default): the two-level schedule where the shape calls for it; 1: never (always
+ * the single-pass schedule); 2: whenever the sequence has at least two segments of
+ * sixteen 32-token chunks.  ss_scan_workspace_bytes follows the same setting.  Returns
+ * SS_OK, or SS_ERR_UNSUPPORTED for any other mode.  Not thread-safe with respect to
+ * scans issued concurrently from other host threads.
+ */
+SS_API int ss_debug_set_scan_two_level(int mode);
 
 /*
  * Gated state scan (the "Mamba 2 Gated State Scan" exercise page): per batch item b,

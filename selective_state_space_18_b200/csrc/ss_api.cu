@@ -137,6 +137,8 @@ bool build_maps(const ss::ScanArgs &a, ss::TmaMaps *m)
     const int64_t rows = a.batch * a.channels, brows = a.batch * N;
     // B and C tiles are read by the scan warps in place: their 16-byte chunks are
     // swizzled across the banks (the swizzle the layout's lane-to-state map needs)
+    // (the kernel reads the tiles at a pitch of one row: the swizzle span must be that row)
+    static_assert(S::kChunk * sizeof(T) == size_t(S::template swizzle<T>()), "swizzle span = tile row");
     const CUtensorMapSwizzle bc_swizzle =
         S::template swizzle<T>() == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     return encode_rows<T>(&m->x, a.x, a.seq, rows, S::kChunk, S::kChanPerCta) &&
@@ -177,7 +179,13 @@ int plan_scan(ss::ScanArgs &a, int64_t *grid_out, int *occ_out, int *sms_out)
     *sms_out = sms;
     const int64_t nchunks = (a.seq + S::kChunk - 1) / S::kChunk;
     int64_t grid = a.groups;
-    if (a.workspace) {
+    if (a.pass != 0) {
+        // two-level passes: the segmentation comes with the call (it fixes the layout of
+        // the composites); every unit is independent, so all resident CTAs take them
+        const int64_t units = a.groups * a.segments;
+        const int64_t resident = int64_t(sms) * occ;
+        grid = units < resident ? units : resident;
+    } else if (a.workspace) {
         const int64_t resident = int64_t(sms) * occ;
         // about sixteen units per resident CTA (finer units balance the tail), segments
         // of at least sixteen chunks (each unit start costs a carry hand-off)
@@ -253,7 +261,8 @@ template <int N, int SPL> int64_t scan_groups(int64_t batch, int64_t channels)
 // fewer shared-memory bytes and instructions per state) when its channel groups give
 // every SM one, else two (16 channels per CTA: twice the groups, so twice the SMs, for
 // shapes with few channels).  Smaller state sizes keep two.
-std::atomic<int> g_forced_spl{0}; // ss_debug_set_scan_layout: 0 = choose per shape
+std::atomic<int> g_forced_spl{0};     // ss_debug_set_scan_layout: 0 = choose per shape
+std::atomic<int> g_two_level_mode{0}; // ss_debug_set_scan_two_level: 0 auto, 1 never, 2 always
 
 int scan_spl(int64_t batch, int64_t channels, int64_t state_dim)
 {
@@ -271,19 +280,185 @@ int scan_spl(int64_t batch, int64_t channels, int64_t state_dim)
 template <int N, int SPL>
 int dispatch_scan_s(const ss::ScanArgs &a, ss_dtype_t dtype, bool vec, size_t ws_bytes, cudaStream_t s)
 {
-    // (a host-side check, before anything touches the device: the size the query
-    // reports, whichever layout this call picks)
-    if (a.workspace && int64_t(ws_bytes) < ss_scan_workspace_bytes(a.batch, a.channels, N, a.seq))
-        return SS_ERR_WORKSPACE;
     if (dtype == SS_BF16)
         return dispatch_scan_t<N, SPL, __nv_bfloat16>(a, vec, ws_bytes, s);
     return dispatch_scan_t<N, SPL, float>(a, vec, ws_bytes, s);
 }
 
-template <int N>
-int dispatch_scan_n(ss::ScanArgs a, ss_dtype_t dtype, bool vec, size_t ws_bytes, cudaStream_t s)
+// ------------------------------------------------------------------------------------
+// In-GPU two-level scan over the sequence ("s6_reset" blog draft, Associative Boundary
+// Resetting: the recurrence composes associatively, so a sequence can be cut into
+// segments scanned in parallel).  For shapes with too few channel groups to fill the
+// GPU through the chained schedule (whose segments of one group run one after
+// another), every segment of every group runs at once, twice:
+//   pass 1  each segment from zero, no outputs: its end state;
+//   decay   exp(A * sum of the segment's steps), 0 where the segment holds a reset;
+//   join    each segment's entering state, h_in[s+1] = decay[s] h_in[s] + state[s],
+//           and the final state;
+//   pass 2  each segment from its entering state, with outputs.
+// This costs twice the exponentials of one pass and wins when the chained schedule
+// would leave more than half of the GPU idle.
+// ------------------------------------------------------------------------------------
+
+// Workspace of the chained (single-pass) schedule: the larger of the two layouts'
+// needs, so the size does not depend on which one the call picks on the device.
+int64_t chained_workspace_bytes(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq)
 {
+    if (batch <= 0 || channels <= 0 || seq <= 0)
+        return 0;
+    switch (state_dim) {
+    case 4: return ss::scan_workspace_bytes<4, 2>(scan_groups<4, 2>(batch, channels));
+    case 8: return ss::scan_workspace_bytes<8, 2>(scan_groups<8, 2>(batch, channels));
+    case 16: {
+        const int64_t a = ss::scan_workspace_bytes<16, 2>(scan_groups<16, 2>(batch, channels));
+        const int64_t b = ss::scan_workspace_bytes<16, 4>(scan_groups<16, 4>(batch, channels));
+        return a > b ? a : b;
+    }
+    default: return 0;
+    }
+}
+
+struct TwoLevelPlan {
+    bool use = false;
+    int spl = 4;
+    int64_t groups = 0, segs = 0, seg_len = 0, count = 0;
+    int64_t chained_bytes = 0, bytes = 0; // workspace: chained part, then 3 x segs x count floats
+};
+
+int64_t align256(int64_t b) { return (b + 255) / 256 * 256; }
+
+TwoLevelPlan two_level_plan(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq)
+{
+    TwoLevelPlan t;
+    if (state_dim != 16)
+        return t;
+    int sms = 0;
+    if (device_sm_count(&sms) != SS_OK || sms <= 0)
+        sms = 148;
+    const int64_t groups16 = scan_groups<16, 2>(batch, channels);
+    const int64_t nchunks = (seq + 31) / 32;
+    const int mode = g_two_level_mode.load(std::memory_order_relaxed);
+    // worth it when the chained schedule (two CTAs per SM of 16-channel groups) would
+    // keep fewer than half its CTA slots busy, on sequences of 64 chunks or more
+    if (mode == 1 || (mode == 0 && (groups16 >= int64_t(sms) || nchunks < 64)))
+        return t;
+    const int forced = g_forced_spl.load(std::memory_order_relaxed);
+    t.spl = forced ? forced : 4;
+    t.groups = t.spl == 4 ? scan_groups<16, 4>(batch, channels) : groups16;
+    const int64_t resident = int64_t(sms) * (t.spl == 4 ? 1 : 2);
+    int64_t segs = (8 * resident + t.groups - 1) / t.groups; // about eight units per CTA
+    const int64_t max_segs = nchunks / 16 < (int64_t(1) << 24) - 1 ? nchunks / 16 : (int64_t(1) << 24) - 1;
+    segs = segs > max_segs ? max_segs : segs;
+    if (segs < 2)
+        return t;
+    const int64_t seg_chunks = (nchunks + segs - 1) / segs;
+    t.seg_len = seg_chunks * 32;
+    t.segs = (nchunks + seg_chunks - 1) / seg_chunks;
+    if (t.segs < 2)
+        return t;
+    t.count = batch * channels * 16;
+    t.chained_bytes = t.spl == 4 ? ss::scan_workspace_bytes<16, 4>(t.groups) : ss::scan_workspace_bytes<16, 2>(t.groups);
+    t.bytes = align256(t.chained_bytes) + 3 * t.segs * t.count * 4;
+    t.use = true;
+    return t;
+}
+
+template <typename T>
+void launch_segment_decay(bool vec, bool sp, unsigned grid, const ss::SegDecayArgs &a, cudaStream_t s);
+
+template <int SPL, typename T>
+int launch_two_level(const ss::ScanArgs &a0, const TwoLevelPlan &t, bool vec, cudaStream_t s)
+{
+    uint8_t *base = a0.workspace;
+    float *state = reinterpret_cast<float *>(base + align256(t.chained_bytes));
+    float *decay = state + t.segs * t.count;
+    float *h_in = decay + t.segs * t.count;
+    ss::ScanArgs a = a0;
+    a.seg_len = t.seg_len;
+    a.segments = t.segs;
+    a.seg_stride = t.count;
+    a.seg_state = state;
+    a.seg_in = h_in;
+    const bool r = a.reset != nullptr;
+    // pass 1: the segments' end states from zero
+    a.pass = 1;
+    int st = r ? (vec ? launch_scan<16, SPL, T, true, true, false, false>(a, 0, s)
+                      : launch_scan<16, SPL, T, true, false, false, false>(a, 0, s))
+               : (vec ? launch_scan<16, SPL, T, false, true, false, false>(a, 0, s)
+                      : launch_scan<16, SPL, T, false, false, false, false>(a, 0, s));
+    if (st != SS_OK)
+        return st;
+    // the segments' decays
+    ss::SegDecayArgs d{};
+    d.dt = a.dt;
+    d.A = a.A;
+    d.dt_bias = a.dt_bias;
+    d.reset = a.reset;
+    d.decay = decay;
+    d.batch = a.batch;
+    d.channels = a.channels;
+    d.seq = a.seq;
+    d.seg_len = t.seg_len;
+    d.segments = t.segs;
+    d.out_stride = t.count;
+    d.state_dim = 16;
+    d.reset_vec = a.reset && aligned(a.reset, 16) && a.seq % 16 == 0;
+    int sms = 0;
+    if (device_sm_count(&sms) != SS_OK)
+        return SS_ERR_CUDA;
+    const int64_t items = a.batch * a.channels * t.segs;
+    const int64_t dblocks = (items + ss::kSegWarps - 1) / ss::kSegWarps;
+    const bool dvec = a.seq % 8 == 0 && aligned(a.dt, 16);
+    launch_segment_decay<T>(dvec, a.softplus != 0, unsigned(dblocks < int64_t(sms) * 8 ? dblocks : int64_t(sms) * 8),
+                            d, s);
+    if (launch_status() != SS_OK)
+        return SS_ERR_CUDA;
+    // the join: every segment's entering state, and the final state
+    ss::JoinAllArgs j{};
+    j.decay = decay;
+    j.state = state;
+    j.h0 = a.h0;
+    j.h_in = h_in;
+    j.h_last = a.h_last;
+    j.count = t.count;
+    j.segments = t.segs;
+    const int64_t jblocks = (t.count + 255) / 256;
+    ss::ss_join_all_kernel<<<unsigned(jblocks < int64_t(sms) * 8 ? jblocks : int64_t(sms) * 8), 256, 0, s>>>(j);
+    if (launch_status() != SS_OK)
+        return SS_ERR_CUDA;
+    // pass 2: every segment from its entering state, with outputs
+    a.pass = 2;
+    return r ? (vec ? launch_scan<16, SPL, T, true, true, false, false>(a, 0, s)
+                    : launch_scan<16, SPL, T, true, false, false, false>(a, 0, s))
+             : (vec ? launch_scan<16, SPL, T, false, true, false, false>(a, 0, s)
+                    : launch_scan<16, SPL, T, false, false, false, false>(a, 0, s));
+}
+
+template <int N>
+int dispatch_scan_n(ss::ScanArgs a, ss_dtype_t dtype, bool vec, size_t ws_bytes, bool allow_two_level,
+                    cudaStream_t s)
+{
+    // (a host-side check, before anything touches the device: the size the query
+    // reports -- or, where the two-level schedule is ruled out, the chained one's)
+    if (a.workspace) {
+        const int64_t need = allow_two_level ? ss_scan_workspace_bytes(a.batch, a.channels, N, a.seq)
+                                             : chained_workspace_bytes(a.batch, a.channels, N, a.seq);
+        if (int64_t(ws_bytes) < need)
+            return SS_ERR_WORKSPACE;
+    }
     if constexpr (N == 16) {
+        // the two-level schedule for the plain form, when the shape asks for it and the
+        // workspace holds its composites
+        if (allow_two_level && a.workspace && !a.h_all && !a.conv_w) {
+            const TwoLevelPlan t = two_level_plan(a.batch, a.channels, N, a.seq);
+            if (t.use && int64_t(ws_bytes) >= t.bytes) {
+                if (t.spl == 4)
+                    return dtype == SS_BF16 ? launch_two_level<4, __nv_bfloat16>(a, t, vec, s)
+                                            : launch_two_level<4, float>(a, t, vec, s);
+                return dtype == SS_BF16 ? launch_two_level<2, __nv_bfloat16>(a, t, vec, s)
+                                        : launch_two_level<2, float>(a, t, vec, s);
+            }
+        }
         if (scan_spl(a.batch, a.channels, N) == 4)
             return dispatch_scan_s<16, 4>(a, dtype, vec, ws_bytes, s);
     }
@@ -442,6 +617,14 @@ int ss_debug_set_scan_layout(int states_per_lane)
     return SS_OK;
 }
 
+int ss_debug_set_scan_two_level(int mode)
+{
+    if (mode < 0 || mode > 2)
+        return SS_ERR_UNSUPPORTED;
+    g_two_level_mode.store(mode, std::memory_order_relaxed);
+    return SS_OK;
+}
+
 int ss_debug_set_wait_limit(uint32_t microseconds)
 {
     return cudaMemcpyToSymbol(ss::g_ss_wait_limit_us, &microseconds, sizeof(microseconds)) == cudaSuccess
@@ -451,20 +634,11 @@ int ss_debug_set_wait_limit(uint32_t microseconds)
 
 int64_t ss_scan_workspace_bytes(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq)
 {
-    if (batch <= 0 || channels <= 0 || seq <= 0)
-        return 0;
-    // the larger of the two layouts' needs, so the size does not depend on which one
-    // the call picks on the current device
-    switch (state_dim) {
-    case 4: return ss::scan_workspace_bytes<4, 2>(scan_groups<4, 2>(batch, channels));
-    case 8: return ss::scan_workspace_bytes<8, 2>(scan_groups<8, 2>(batch, channels));
-    case 16: {
-        const int64_t a = ss::scan_workspace_bytes<16, 2>(scan_groups<16, 2>(batch, channels));
-        const int64_t b = ss::scan_workspace_bytes<16, 4>(scan_groups<16, 4>(batch, channels));
-        return a > b ? a : b;
-    }
-    default: return 0;
-    }
+    const int64_t chained = chained_workspace_bytes(batch, channels, state_dim, seq);
+    if (chained <= 0)
+        return chained;
+    const TwoLevelPlan t = two_level_plan(batch, channels, state_dim, seq);
+    return t.use && t.bytes > chained ? t.bytes : chained;
 }
 
 int ss_scan_status(const void *workspace, ss_stream_t stream, int *status)
@@ -533,6 +707,21 @@ int ss_scan_plan(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq
     plan->grid = grid;
     plan->ctas_per_sm = occ;
     plan->states_per_lane = state_dim == 16 ? scan_spl(batch, channels, 16) : 2;
+    plan->two_level = 0;
+    if (with_workspace) {
+        const TwoLevelPlan t = two_level_plan(batch, channels, state_dim, seq);
+        if (t.use) { // (the plain form with a workspace of ss_scan_workspace_bytes)
+            const int64_t resident = int64_t(sms) * (t.spl == 4 ? 1 : 2);
+            plan->two_level = 1;
+            plan->states_per_lane = t.spl;
+            plan->ctas_per_sm = t.spl == 4 ? 1 : 2;
+            plan->groups = t.groups;
+            plan->segments = t.segs;
+            plan->seg_len = t.seg_len;
+            plan->grid = t.groups * t.segs < resident ? t.groups * t.segs : resident;
+            plan->states_per_lane = t.spl;
+        }
+    }
     plan->sms = sms;
     plan->groups = a.groups;
     plan->segments = a.segments;
@@ -565,7 +754,8 @@ int scan_impl(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, s
               const void *x, const void *dt_raw, const float *A, const void *B, const void *C,
               const float *D, const void *z, const float *dt_bias, const uint8_t *reset,
               const float *h0, uint32_t flags, void *y, float *h_last, float *h_all, void *workspace,
-              size_t workspace_bytes, ss_stream_t stream, const ConvArgs &cv = ConvArgs())
+              size_t workspace_bytes, ss_stream_t stream, const ConvArgs &cv = ConvArgs(),
+              bool allow_two_level = true)
 {
     if (!x || !dt_raw || !A || !B || !C || !y)
         return SS_ERR_NULL;
@@ -694,9 +884,9 @@ int scan_impl(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, s
     a.workspace = static_cast<uint8_t *>(workspace);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     switch (state_dim) {
-    case 4: return dispatch_scan_n<4>(a, dtype, vec, workspace_bytes, s);
-    case 8: return dispatch_scan_n<8>(a, dtype, vec, workspace_bytes, s);
-    default: return dispatch_scan_n<16>(a, dtype, vec, workspace_bytes, s);
+    case 4: return dispatch_scan_n<4>(a, dtype, vec, workspace_bytes, allow_two_level, s);
+    case 8: return dispatch_scan_n<8>(a, dtype, vec, workspace_bytes, allow_two_level, s);
+    default: return dispatch_scan_n<16>(a, dtype, vec, workspace_bytes, allow_two_level, s);
     }
 }
 
@@ -965,7 +1155,9 @@ int ss_scan_fwd_static_scratch(int64_t batch, int64_t channels, int64_t state_di
         return SS_ERR_NULL;
     if (flags & ~uint32_t(SS_DT_SOFTPLUS | SS_SCRATCH_ZERO))
         return SS_ERR_UNSUPPORTED;
-    const int64_t need = ss_scan_workspace_bytes(batch, channels, state_dim, seq);
+    // (the chained schedule: the static scratch does not hold the two-level one's
+    // composites)
+    const int64_t need = chained_workspace_bytes(batch, channels, state_dim, seq);
     if (need > int64_t(SS_STATIC_SCRATCH_BYTES))
         return SS_ERR_SCRATCH_LIMIT;
     // (need == 0: an invalid shape, which ss_scan_fwd reports with its own status)
@@ -980,8 +1172,9 @@ int ss_scan_fwd_static_scratch(int64_t batch, int64_t channels, int64_t state_di
     if (need > 0 && (flags & SS_SCRATCH_ZERO) &&
         cudaMemsetAsync(ws, 0, size_t(SS_STATIC_SCRATCH_BYTES), s) != cudaSuccess)
         return SS_ERR_CUDA;
-    return ss_scan_fwd(batch, channels, state_dim, seq, dtype, x, dt_raw, A, B, C, D, z, dt_bias, reset, h0,
-                       flags & uint32_t(SS_DT_SOFTPLUS), y, h_last, ws, SS_STATIC_SCRATCH_BYTES, stream);
+    return scan_impl(batch, channels, state_dim, seq, dtype, x, dt_raw, A, B, C, D, z, dt_bias, reset, h0,
+                     flags & uint32_t(SS_DT_SOFTPLUS), y, h_last, nullptr, ws, SS_STATIC_SCRATCH_BYTES, stream,
+                     ConvArgs(), false);
 }
 
 
@@ -1021,6 +1214,9 @@ int ss_segment_decay(int64_t batch, int64_t channels, int64_t state_dim, int64_t
     a.channels = channels;
     a.seq = seq;
     a.state_dim = int(state_dim);
+    a.seg_len = seq;
+    a.segments = 1;
+    a.out_stride = 0;
     a.reset_vec = reset && aligned(reset, 16) && seq % 16 == 0;
     int sms = 0;
     if (device_sm_count(&sms) != SS_OK)

@@ -61,6 +61,16 @@ struct ScanArgs {
     int64_t segments;         // ceil(seq / seg_len); 1 without a workspace
     uint8_t *workspace;       // nullptr: one CTA per channel group, one segment
     uint32_t *status;         // status word when there is no workspace
+    // In-GPU two-level scan over the sequence (no carries between segments):
+    //  pass 1: every segment starts from zero, no outputs; its end state goes to
+    //          seg_state[s * seg_stride + (b * channels + c) * N + n];
+    //  pass 2: every segment starts from seg_in[s * seg_stride + ...] (the joined
+    //          entering state) and writes y; h_last comes from the join.
+    // pass 0 is the single-pass scan (chained segments, or one CTA per group).
+    int pass;
+    float *seg_state;
+    const float *seg_in;
+    int64_t seg_stride;
 };
 
 // Tensor maps of the TMA path: x, dt as [batch * channels rows][seq] and B, C as
@@ -174,19 +184,16 @@ template <int N, int SPL> struct ScanShape {
         return size_t(kRawStages * raw_stage_bytes<T>()) + size_t(floats<T>()) * 4 + 8 * size_t(kBars) +
                32 * size_t(kRawStages);
     }
-    // Which states a lane owns, and how TMA swizzles the B and C tiles so that the
-    // kLanes rows a warp reads at once fall into distinct banks:
-    //  * bf16 with four states per lane: states 4g .. 4g+3 (contiguous, so the lane
-    //    moves its states, carries and per-token states as 16-byte vectors) with the
-    //    128-byte swizzle;
-    //  * otherwise states g, g + kLanes, ... (strided) with the 64-byte swizzle for
-    //    bf16 rows and the 128-byte swizzle for fp32 rows.
-    template <typename T> static constexpr bool contiguous() { return SPL == 4 && sizeof(T) == 2; }
-    template <typename T> static constexpr int swizzle() { return (sizeof(T) == 2 && SPL == 2) ? 64 : 128; }
-    template <typename T> static __device__ __forceinline__ int state(int g, int j)
-    {
-        return contiguous<T>() ? SPL * g + j : g + kLanes * j;
-    }
+    // The lane with state group g owns states g, g + kLanes, g + 2 kLanes, ...; the B and
+    // C tiles are swizzled by TMA with the swizzle whose span is exactly one tile row
+    // (64 bytes for bf16 rows of 32 tokens, 128 bytes for fp32 rows), so the rows a
+    // warp reads at once fall into distinct banks: with 64-byte rows, rows g and g + 1
+    // lie in different halves of the banks and rows g and g + 2 differ in the chunk the
+    // swizzle selects; with 128-byte rows, the swizzle alone separates eight rows.  (A
+    // swizzle span wider than the row is not used: TMA lays such a box out at the span's
+    // pitch, not the row's.)
+    template <typename T> static constexpr int swizzle() { return sizeof(T) == 2 ? 64 : 128; }
+    template <typename T> static __device__ __forceinline__ int state(int g, int j) { return g + kLanes * j; }
     static_assert(kTokTasks % kIoThreads == 0, "token tasks fill whole IO lanes");
     static_assert(kInStage % 4 == 0 && kYXOff % 4 == 0, "16-byte aligned stages");
 };
@@ -776,21 +783,12 @@ __device__ __forceinline__ void scan_chunk(const float *stage, const unsigned ch
             yo[pr] = yy;
             if (EMIT) {
                 const int tt = t + 2 * pr;
-                if constexpr (S::template contiguous<T>()) {
-                    if (tt < valid)
-                        __stcs(reinterpret_cast<float4 *>(hrow + tt * N + nn[0]),
-                               make_float4(hm[0], hm[1], hm[2], hm[3]));
-                    if (tt + 1 < valid)
-                        __stcs(reinterpret_cast<float4 *>(hrow + (tt + 1) * N + nn[0]),
-                               make_float4(hs[0], hs[1], hs[2], hs[3]));
-                } else {
 #pragma unroll
-                    for (int j = 0; j < SPL; ++j) {
-                        if (tt < valid)
-                            __stcs(hrow + tt * N + nn[j], hm[j]);
-                        if (tt + 1 < valid)
-                            __stcs(hrow + (tt + 1) * N + nn[j], hs[j]);
-                    }
+                for (int j = 0; j < SPL; ++j) {
+                    if (tt < valid)
+                        __stcs(hrow + tt * N + nn[j], hm[j]);
+                    if (tt + 1 < valid)
+                        __stcs(hrow + (tt + 1) * N + nn[j], hs[j]);
                 }
             }
         }
@@ -938,7 +936,8 @@ __device__ __forceinline__ bool epilogue_role(const ScanArgs &p, const float *y_
         const ChunkMeta meta = read_meta(ystage);
         if (meta.flags & kEnd)
             return true;
-        epilogue_chunk<N, SPL, T, VEC, CONV>(p, tl, ystage, meta.g, meta.t0, ec);
+        if (p.pass != 1) // (the first pass of the two-level scan has no outputs)
+            epilogue_chunk<N, SPL, T, VEC, CONV>(p, tl, ystage, meta.g, meta.t0, ec);
         mbar_arrive(y_empty + ys);
     }
 }
@@ -1069,7 +1068,16 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
                     const float a = __ldg(p.A + c * N + nn[q]) * kLog2e;
                     A2[q] = make_float2(a, a);
                 }
-                if (meta.s == 0) {
+                if (p.pass == 1) {
+#pragma unroll
+                    for (int q = 0; q < SPL; ++q)
+                        hs[q] = 0.0f;
+                } else if (p.pass == 2) {
+                    const float *src = p.seg_in + meta.s * p.seg_stride + row * N;
+#pragma unroll
+                    for (int q = 0; q < SPL; ++q)
+                        hs[q] = __ldcg(src + nn[q]);
+                } else if (meta.s == 0) {
 #pragma unroll
                     for (int q = 0; q < SPL; ++q)
                         hs[q] = p.h0 ? __ldg(p.h0 + row * N + nn[q]) : 0.0f;
@@ -1096,7 +1104,16 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
             mbar_arrive(in_empty + st);
             mbar_arrive(y_full + ysi);
             if (meta.flags & kLast) {
-                if (int64_t(meta.s) + 1 < p.segments) {
+                if (p.pass == 1) {
+                    if (cvalid) {
+                        float *dst = p.seg_state + meta.s * p.seg_stride + row * N;
+#pragma unroll
+                        for (int q = 0; q < SPL; ++q)
+                            __stcg(dst + nn[q], hs[q]);
+                    }
+                } else if (p.pass == 2) {
+                    // the final state was produced by the join
+                } else if (int64_t(meta.s) + 1 < p.segments) {
                     const int64_t slot = meta.g * S::kScanWarps + warp;
                     float *cs = carry + (slot * 32 + lane) * SPL;
 #pragma unroll

@@ -61,7 +61,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
 }
 
 // 2-D tile load global -> this CTA's shared memory through a tensor map, completing
-// on `bar` (plain tile mode: no multicast, no swizzle).  c0 is the innermost
+// on `bar` (tile mode, no multicast; the tensor map decides the swizzle: none for the
+// x and dt tiles, a span of one tile row for the B and C tiles).  c0 is the innermost
 // (contiguous) coordinate.
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int32_t c0, int32_t c1,
                                             uint64_t *bar)

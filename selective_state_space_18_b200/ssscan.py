@@ -28,7 +28,8 @@ STATUS = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE", 4:
           9: "SS_ERR_WORKSPACE", 10: "SS_ERR_SCRATCH_LIMIT"}
 EXPORTS = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_scan_plan", "ss_scan_status", "ss_debug_status",
            "ss_state_update",
-           "ss_debug_set_wait_limit", "ss_debug_set_scan_layout", "ss_status_string", "ss_abi_version",
+           "ss_debug_set_wait_limit", "ss_debug_set_scan_layout", "ss_debug_set_scan_two_level",
+           "ss_status_string", "ss_abi_version",
            "ss_scan_fwd_static_scratch", "ss_scan_fwd_states", "ss_gated_scan", "ss_scan_fwd_conv",
            "ss_state_update_conv", "ss_segment_decay", "ss_join_segments")
 ABI_MAJOR = 2
@@ -43,7 +44,7 @@ class ScanPlan(ctypes.Structure):
     """ss_scan_plan_t: the launch plan of ss_scan_fwd for a shape."""
     _fields_ = [("grid", ctypes.c_int64), ("ctas_per_sm", ctypes.c_int64), ("sms", ctypes.c_int64),
                 ("groups", ctypes.c_int64), ("segments", ctypes.c_int64), ("seg_len", ctypes.c_int64),
-                ("states_per_lane", ctypes.c_int64)]
+                ("states_per_lane", ctypes.c_int64), ("two_level", ctypes.c_int64)]
 
 
 class SSError(RuntimeError):
@@ -102,6 +103,8 @@ def load_library(path: str = LIB_PATH):
             lib.ss_debug_set_wait_limit.restype = ctypes.c_int
             lib.ss_debug_set_scan_layout.argtypes = [ctypes.c_int]
             lib.ss_debug_set_scan_layout.restype = ctypes.c_int
+            lib.ss_debug_set_scan_two_level.argtypes = [ctypes.c_int]
+            lib.ss_debug_set_scan_two_level.restype = ctypes.c_int
             lib.ss_debug_status.argtypes = [_vp]
             lib.ss_debug_status.restype = ctypes.c_int
             lib.ss_abi_version.argtypes = []
@@ -185,8 +188,8 @@ def scan_workspace(batch, channels, state_dim, seq, device, stream=None):
 def ss_scan_plan(batch, channels, state_dim, seq, dtype=torch.bfloat16, *, has_reset=False, workspace=True,
                  device=None):
     """Launch plan of ss_scan_fwd for this shape on `device` (16-byte aligned tensors):
-    dict(grid, ctas_per_sm, sms, groups, segments, seg_len, states_per_lane).  Launches
-    nothing."""
+    dict(grid, ctas_per_sm, sms, groups, segments, seg_len, states_per_lane, two_level).
+    Launches nothing."""
     if device is None:
         device = torch.device("cuda", torch.cuda.current_device())
     code = SS_BF16 if dtype == torch.bfloat16 else SS_F32
@@ -230,6 +233,14 @@ def ss_debug_set_scan_layout(states_per_lane: int) -> None:
     st = load_library().ss_debug_set_scan_layout(int(states_per_lane))
     if st != 0:
         raise SSError("ss_debug_set_scan_layout", st)
+
+
+def ss_debug_set_scan_two_level(mode: int) -> None:
+    """Schedule of later state_dim-16 scans with a workspace: 0 automatic, 1 never the
+    two-level schedule, 2 whenever the sequence allows it.  A testing aid."""
+    st = load_library().ss_debug_set_scan_two_level(int(mode))
+    if st != 0:
+        raise SSError("ss_debug_set_scan_two_level", st)
 
 
 def ss_debug_set_wait_limit(microseconds: int) -> None:

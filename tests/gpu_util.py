@@ -1,5 +1,7 @@
 """Helpers shared by the GPU test files: move seeded inputs to the device, call the
 C ABI through the binding, and compare with the oracle elementwise."""
+import contextlib
+
 import numpy as np
 import torch
 
@@ -41,3 +43,19 @@ def assert_close(out, ref, tol, what=""):
     e = rel_err(out, ref)
     assert e <= tol, f"{what}: max |d|/(1+|ref|) = {e:.3e} > {tol:.0e}"
     return e
+
+
+@contextlib.contextmanager
+def schedule(two_level=None, layout=None):
+    """Pin the scan's schedule for the block: two_level 0 (automatic), 1 (never: the
+    single-pass schedule, chained segments or one CTA per group) or 2 (whenever the
+    sequence allows); layout 2 or 4 state rows per scan lane (0: automatic)."""
+    if two_level is not None:
+        ssscan.ss_debug_set_scan_two_level(two_level)
+    if layout is not None:
+        ssscan.ss_debug_set_scan_layout(layout)
+    try:
+        yield
+    finally:
+        ssscan.ss_debug_set_scan_two_level(0)
+        ssscan.ss_debug_set_scan_layout(0)

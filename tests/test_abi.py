@@ -119,7 +119,12 @@ def test_workspace_size_query(lib):
     small = lib.ss_scan_workspace_bytes(2, 16, 16, 64)
     big = lib.ss_scan_workspace_bytes(2, 1600, 16, 64)
     assert 64 < small < big
-    assert lib.ss_scan_workspace_bytes(2, 16, 16, 1 << 20) == small  # independent of seq
+    # with enough channel groups to fill the GPU (the chained schedule), independent of seq
+    assert lib.ss_scan_workspace_bytes(2, 2400, 16, 1 << 20) == lib.ss_scan_workspace_bytes(2, 2400, 16, 64)
+    # few groups and a long sequence: the two-level schedule's composites are included
+    # (three floats per state element and segment)
+    long_few = lib.ss_scan_workspace_bytes(1, 512, 16, 65536)
+    assert long_few > lib.ss_scan_workspace_bytes(1, 512, 16, 64) + 3 * 4 * 512 * 16
     assert lib.ss_scan_workspace_bytes(2, 16, 5, 64) == 0
     assert lib.ss_scan_workspace_bytes(0, 16, 16, 64) == 0
     for n in (4, 8, 16):

@@ -8,7 +8,7 @@ ever publish.  The wait limit is shortened to 2 ms for the duration of the test 
 import pytest
 import torch
 
-from gpu_util import SCAN_KEYS, assert_close, dev
+from gpu_util import SCAN_KEYS, assert_close, dev, schedule
 from selective_state_space_18_b200 import ssscan
 from selective_state_space_18_b200.inputs import make_scan_inputs
 
@@ -19,6 +19,14 @@ pytestmark = pytest.mark.gpu
 def _cuda():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA GPU")
+
+
+@pytest.fixture(autouse=True)
+def _single_pass():
+    """The carry waits these tests block belong to the single-pass (chained) schedule;
+    the two-level schedule has none."""
+    with schedule(two_level=1):
+        yield
 
 
 def _block_first_segment(ws, groups):

@@ -8,7 +8,7 @@ import contextlib
 import pytest
 import torch
 
-from gpu_util import SCAN_KEYS, TOL, assert_close, dev, gpu_scan
+from gpu_util import SCAN_KEYS, TOL, assert_close, dev, gpu_scan, schedule
 from selective_state_space_18_b200 import ssscan
 from selective_state_space_18_b200.inputs import make_scan_inputs, make_workload
 
@@ -54,7 +54,7 @@ def test_layout_matches_oracle(orc, spl, case):
                            reset_mean_doc=60 if resets else 0, a_perturb=True)
     ref = orc.scan(**inp)
     tol = TOL[inp["x"].dtype]
-    with layout(spl):
+    with layout(spl), schedule(two_level=1):
         y_seg, h_seg = gpu_scan(inp, workspace=True)
         y_one, h_one = gpu_scan(inp, workspace=False)
     assert_close(y_seg, ref["y"], tol, "y")

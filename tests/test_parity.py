@@ -4,7 +4,7 @@ inputs, elementwise: max |out - ref| <= 1e-4 (1 + |ref|) for fp32 tensors and
 import pytest
 import torch
 
-from gpu_util import TOL, assert_close, gpu_scan, gpu_update
+from gpu_util import TOL, assert_close, gpu_scan, gpu_update, schedule
 from selective_state_space_18_b200.inputs import make_scan_inputs, make_update_inputs, make_workload
 
 pytestmark = pytest.mark.gpu
@@ -233,12 +233,13 @@ def test_segmented_schedule_is_bit_identical(shape):
     bt, ch, n, L, dt_, doc = shape
     inp = make_scan_inputs(bt, ch, n, L, dt_, seed=L + ch, h0=True, reset_mean_doc=doc)
     d = {k: (None if v is None else v.cuda()) for k, v in inp.items()}
-    y_static, h_static = ssscan.ss_scan_fwd(**d, workspace=False)
-    y_seg, h_seg = ssscan.ss_scan_fwd(**d)
-    ws = torch.zeros(int(ssscan.load_library().ss_scan_workspace_bytes(bt, ch, n, L)),
-                     dtype=torch.uint8, device="cuda")
-    outs = [ssscan.ss_scan_fwd(**d, workspace=ws) for _ in range(4)]
-    torch.cuda.synchronize()
+    with schedule(two_level=1):  # the single-pass schedule (chained segments)
+        y_static, h_static = ssscan.ss_scan_fwd(**d, workspace=False)
+        y_seg, h_seg = ssscan.ss_scan_fwd(**d)
+        ws = torch.zeros(int(ssscan.load_library().ss_scan_workspace_bytes(bt, ch, n, L)),
+                         dtype=torch.uint8, device="cuda")
+        outs = [ssscan.ss_scan_fwd(**d, workspace=ws) for _ in range(4)]
+        torch.cuda.synchronize()
     assert torch.equal(y_static, y_seg) and torch.equal(h_static, h_seg)
     for y, h in outs:
         assert torch.equal(y, y_seg) and torch.equal(h, h_seg)
