@@ -360,7 +360,12 @@ def run_ours(args):
     plan = ssscan.ss_scan_plan(PROMPT.batch, PROMPT.channels, PROMPT.state_dim, PROMPT.seq,
                                torch.bfloat16, has_reset=False, workspace=True, device=dev)
     hbm_gbs, sm_max_mhz, peak_kind = _peaks()
-    sfu_peak = SM_COUNT_NOMINAL * MUFU_PER_CLK_PER_SM * sm_max_mhz * 1e6  # ex2/s
+    # the special-function unit's rate, measured on this GPU after the timed region
+    # (results per SM clock; the peak takes it at the maximum SM clock)
+    ex2_rate, ex2_rates = ssscan.mufu_rate("ex2", device=dev)
+    tanh_rate, _ = ssscan.mufu_rate("tanh", device=dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    sfu_peak = sms * ex2_rate * sm_max_mhz * 1e6  # ex2/s
     scan_s = scan_ms * 1e-3
     dec_s = dec_ms * 1e-3
     scan_exps_rate = pw["exps"] / scan_s
@@ -376,8 +381,12 @@ def run_ours(args):
         "peak": round(sfu_peak / 1e9, 2),
         "unit": "Gexp/s",
         "frac": round(scan_exps_rate / sfu_peak, 4),
-        "peak_basis": f"{SM_COUNT_NOMINAL} SMs x {MUFU_PER_CLK_PER_SM} ex2/clk x {sm_max_mhz:.0f} MHz (max SM clock)",
-        "frac_at_measured_clock": (round(scan_exps_rate / (SM_COUNT_NOMINAL * MUFU_PER_CLK_PER_SM * sm_clk * 1e6), 4)
+        "peak_basis": (f"{sms} SMs x {ex2_rate:.2f} ex2/clk/SM (measured: ss_debug_mufu_probe, median over SMs) "
+                       f"x {sm_max_mhz:.0f} MHz (max SM clock)"),
+        "sfu_probe": {"ex2_per_clk_per_sm": round(ex2_rate, 3), "ex2_min": round(ex2_rates[0], 3),
+                      "ex2_max": round(ex2_rates[-1], 3), "tanh_per_clk_per_sm": round(tanh_rate, 3),
+                      "nominal": MUFU_PER_CLK_PER_SM},
+        "frac_at_measured_clock": (round(scan_exps_rate / (sms * ex2_rate * sm_clk * 1e6), 4)
                                    if sm_clk else None),
         "exps_per_launch": pw["exps"],
         "algorithmic_bytes_per_launch": pw["bytes"],
@@ -386,7 +395,7 @@ def run_ours(args):
         "hbm_frac": round(scan_hbm / hbm_gbs, 4),
         "roofline_frac": round(t_roof_scan / scan_s, 4),
         "traffic": _measured_traffic("ss_scan_fwd_kernel"),
-        "peak_source": f"HBM {peak_kind} (MEASURED_PEAKS.json); SFU derived from unit counts and clock",
+        "peak_source": f"HBM {peak_kind} (MEASURED_PEAKS.json); SFU measured per clock, at the max clock",
     }
     kernels = {
         "scan": {"ms": round(scan_ms, 5), "ms_min": round(min(scan_list), 5),

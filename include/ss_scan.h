@@ -402,6 +402,29 @@ SS_API int ss_segment_decay(int64_t batch, int64_t channels, int64_t state_dim, 
 SS_API int ss_join_segments(int64_t segments, int64_t count, const float *composites, int64_t rank,
                             float *carry, float *final_state, ss_stream_t stream);
 
+/*
+ * Measurement aid: the throughput of the special-function unit that bounds the prompt
+ * scan (its exponentials).  Launches `blocks` CTAs of 512 threads (one per SM when
+ * blocks is the SM count) that each run 8 independent chains of `iters` operations:
+ * op 0 = ex2.approx.ftz.f32 (the decays), op 1 = tanh.approx.f32 (the bf16 output
+ * gate).  cycles (device, [blocks] int64) receives each CTA's SM clock cycles for its
+ * loop; sink (device, [512] float) is written only to keep the work live; the host
+ * gets *ops_per_block, so ops / cycles is the unit's results per clock per SM.
+ * Asynchronous on `stream`; returns SS_OK or an error status.
+ */
+SS_API int ss_debug_mufu_probe(int op, int64_t iters, int64_t blocks, long long *cycles, float *sink,
+                               int64_t *ops_per_block, ss_stream_t stream);
+
+/*
+ * Debug build with index checks (libssscan_bounds.so, compiled with SS_BOUNDS_CHECK):
+ * every runtime-computed global and shared-memory index of the scan and decode kernels
+ * is checked before its access; a failed check skips the access and records the
+ * number of its site (the first one wins) in a device word, without a trap.  This call
+ * synchronises `stream`, stores that site in *site (0: no failed check) and clears it.
+ * In the normal build it stores -1 and returns SS_ERR_UNSUPPORTED.
+ */
+SS_API int ss_debug_bounds_status(ss_stream_t stream, int *site);
+
 /* Human-readable name of a status code (static string, never NULL). */
 SS_API const char *ss_status_string(int status);
 

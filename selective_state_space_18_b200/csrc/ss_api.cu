@@ -617,6 +617,27 @@ int ss_debug_set_scan_layout(int states_per_lane)
     return SS_OK;
 }
 
+int ss_debug_bounds_status(ss_stream_t stream, int *site)
+{
+    if (!site)
+        return SS_ERR_NULL;
+#ifdef SS_BOUNDS_CHECK
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t v = 0;
+    const uint32_t zero = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess ||
+        cudaMemcpyFromSymbol(&v, ss::g_ss_bounds_site, sizeof(v)) != cudaSuccess ||
+        cudaMemcpyToSymbol(ss::g_ss_bounds_site, &zero, sizeof(zero)) != cudaSuccess)
+        return SS_ERR_CUDA;
+    *site = int(v);
+    return SS_OK;
+#else
+    (void)stream;
+    *site = -1;
+    return SS_ERR_UNSUPPORTED;
+#endif
+}
+
 int ss_debug_set_scan_two_level(int mode)
 {
     if (mode < 0 || mode > 2)

@@ -16,6 +16,25 @@ namespace ss {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// ---- debug build with index checks (compile with -DSS_BOUNDS_CHECK) ----------------
+//
+// SS_IN_BOUNDS(cond, site) is `cond` in the checked build and `true` otherwise.  In
+// the checked build a false condition records the site's number in g_ss_bounds_site
+// (the first one wins) and the caller skips the access it guards: no trap, so the
+// kernel finishes and the host reads the site with ss_debug_bounds_status.
+#ifdef SS_BOUNDS_CHECK
+__device__ uint32_t g_ss_bounds_site;
+__device__ __forceinline__ bool ss_bounds_ok(bool ok, uint32_t site)
+{
+    if (!ok)
+        atomicCAS(&g_ss_bounds_site, 0u, site);
+    return ok;
+}
+#define SS_IN_BOUNDS(cond, site) ::ss::ss_bounds_ok((cond), (site))
+#else
+#define SS_IN_BOUNDS(cond, site) true
+#endif
+
 // 2^x on the MUFU unit (flush-to-zero: results below 2^-126 become +0, and
 // 2^-inf = +0, which the reset fold relies on).
 __device__ __forceinline__ float ex2(float x)

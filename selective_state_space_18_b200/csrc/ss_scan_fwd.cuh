@@ -307,6 +307,8 @@ struct IoPrefetch {
             if (q < S::kBCTasks) {
                 const int r = q % (2 * N), tb = q / (2 * N);
                 const T *src = r < N ? Bb + r * L : Cb + (r - N) * L;
+                if (!SS_IN_BOUNDS(b < p.batch, 120))
+                    continue;
                 if (VEC)
                     bc[m].load_vec(src, t0 + tb * 8, L);
                 else
@@ -321,6 +323,8 @@ struct IoPrefetch {
             c = c < p.channels ? c : p.channels - 1;
             const int64_t row = b * p.channels + c;
             const int64_t t = t0 + tb * 8;
+            if (!SS_IN_BOUNDS(row < p.batch * p.channels && t0 < L, 121))
+                continue;
             const T *xrow = static_cast<const T *>(p.x) + row * L;
             const T *drow = static_cast<const T *>(p.dt) + row * L;
             if (VEC) {
@@ -421,9 +425,11 @@ __device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane,
                 const int row = r < N ? r : r - N;
                 constexpr int kChunksPer8 = int(sizeof(T)) / 2; // 16-byte chunks per 8 tokens
 #pragma unroll
-                for (int h = 0; h < kChunksPer8; ++h)
-                    *reinterpret_cast<uint4 *>(tile + bc_offset<T, S::template swizzle<T>()>(row, tb * kChunksPer8 + h)) =
-                        reinterpret_cast<const uint4 *>(&f.bc[m])[h];
+                for (int h = 0; h < kChunksPer8; ++h) {
+                    const int o = bc_offset<T, S::template swizzle<T>()>(row, tb * kChunksPer8 + h);
+                    if (SS_IN_BOUNDS(o >= 0 && o + 16 <= N * S::kChunk * int(sizeof(T)), 123))
+                        *reinterpret_cast<uint4 *>(tile + o) = reinterpret_cast<const uint4 *>(&f.bc[m])[h];
+                }
             }
         }
     }
@@ -464,7 +470,7 @@ __device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane,
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int64_t pos = tl + j;
-                        if (pos >= L - H && pos < L)
+                        if (pos >= L - H && pos < L && SS_IN_BOUNDS(row < p.batch * p.channels, 125))
                             p.conv_state_out[row * H + (pos - (L - H))] = U[3 + j];
                     }
                     if (tl == 0)
@@ -550,6 +556,7 @@ __device__ __forceinline__ void epilogue_chunk(const ScanArgs &p, int lane, cons
             const bool valid = c_raw < p.channels;
             const int64_t c = valid ? c_raw : p.channels - 1;
             const int64_t off = (b * p.channels + c) * L;
+            (void)SS_IN_BOUNDS(b < p.batch && c < p.channels && t0 < L, 130);
             ec.x[m] = static_cast<const T *>(p.x) + off;
             ec.z[m] = p.z ? static_cast<const T *>(p.z) + off : nullptr;
             ec.y[m] = valid ? static_cast<T *>(p.y) + off : nullptr;
@@ -728,8 +735,11 @@ __device__ __forceinline__ void scan_chunk(const float *stage, const unsigned ch
         const int t = 4 * k;
         if (t % kTok == 0) {
 #pragma unroll
-            for (int j = 0; j < SPL; ++j)
-                wb[j] = *reinterpret_cast<const uint4 *>(Bt + bc_offset<T, SWZ>(nn[j], t / kTok));
+            for (int j = 0; j < SPL; ++j) {
+                const int o = bc_offset<T, SWZ>(nn[j], t / kTok);
+                if (SS_IN_BOUNDS(o >= 0 && o + 16 <= N * S::kChunk * int(sizeof(T)), 112))
+                    wb[j] = *reinterpret_cast<const uint4 *>(Bt + o);
+            }
         }
         const float4 d4 = *reinterpret_cast<const float4 *>(dts + t);
         const float4 u4 = *reinterpret_cast<const float4 *>(dxs + t);
@@ -756,8 +766,11 @@ __device__ __forceinline__ void scan_chunk(const float *stage, const unsigned ch
         const int t = 4 * k;
         if (t % kTok == 0) {
 #pragma unroll
-            for (int j = 0; j < SPL; ++j)
-                wc[j] = *reinterpret_cast<const uint4 *>(Ct + bc_offset<T, SWZ>(nn[j], t / kTok));
+            for (int j = 0; j < SPL; ++j) {
+                const int o = bc_offset<T, SWZ>(nn[j], t / kTok);
+                if (SS_IN_BOUNDS(o >= 0 && o + 16 <= N * S::kChunk * int(sizeof(T)), 113))
+                    wc[j] = *reinterpret_cast<const uint4 *>(Ct + o);
+            }
         }
         uint4 cc[SPL];
 #pragma unroll
@@ -843,6 +856,9 @@ __device__ __forceinline__ bool issuer_warp(const ScanArgs &p, const TmaMaps &ma
             uint64_t *bar = cx.raw_full + r;
             mbar_arrive_expect_tx(bar, tx_bytes);
             const int32_t tt = int32_t(t0), xrow = up.xrow, brow = up.brow;
+            (void)SS_IN_BOUNDS(t0 < p.seq && int64_t(xrow) < p.batch * p.channels &&
+                                   int64_t(brow) + N <= p.batch * N && r < S::kRawStages,
+                               140);
             tma_load_2d(dst + S::template raw_x_off<T>(), &maps.x, tt, xrow, bar);
             tma_load_2d(dst + S::template raw_dt_off<T>(), &maps.dt, tt, xrow, bar);
             tma_load_2d(dst + S::template raw_b_off<T>(), &maps.B, tt, brow, bar);
@@ -889,7 +905,10 @@ __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, in
                     reset_g = g;
                     reset_row = p.reset + int64_t(uint32_t(g) / uint32_t(p.groups_per_batch)) * p.seq;
                 }
-                pf.rbyte = (tl < S::kChunk && t0 + tl < p.seq) ? uint32_t(__ldg(reset_row + t0 + tl)) : 0u;
+                pf.rbyte = (tl < S::kChunk && t0 + tl < p.seq &&
+                            SS_IN_BOUNDS(uint32_t(g) / uint32_t(p.groups_per_batch) < uint64_t(p.batch), 122))
+                               ? uint32_t(__ldg(reset_row + t0 + tl))
+                               : 0u;
             }
         }
         mbar_arrive(cx.raw_empty + r); // this thread's reads of slot r are done
@@ -1058,11 +1077,16 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
                 break;
             }
             if (meta.flags & kFirst) {
+                if (!SS_IN_BOUNDS(meta.g < p.groups && meta.s < p.segments && meta.t0 < p.seq, 101))
+                    break;
                 const int64_t b = meta.g / p.groups_per_batch;
                 const int64_t c_raw = (meta.g % p.groups_per_batch) * S::kChanPerCta + cl;
                 cvalid = c_raw < p.channels;
                 const int64_t c = cvalid ? c_raw : p.channels - 1;
                 row = b * p.channels + c;
+#pragma unroll
+                if (!SS_IN_BOUNDS(c < p.channels && row < p.batch * p.channels && nn[SPL - 1] < N, 109))
+                    break;
 #pragma unroll
                 for (int q = 0; q < SPL; ++q) {
                     const float a = __ldg(p.A + c * N + nn[q]) * kLog2e;
@@ -1073,6 +1097,8 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
                     for (int q = 0; q < SPL; ++q)
                         hs[q] = 0.0f;
                 } else if (p.pass == 2) {
+                    if (!SS_IN_BOUNDS(p.seg_stride >= p.batch * p.channels * N, 107))
+                        break;
                     const float *src = p.seg_in + meta.s * p.seg_stride + row * N;
 #pragma unroll
                     for (int q = 0; q < SPL; ++q)
@@ -1083,6 +1109,8 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
                         hs[q] = p.h0 ? __ldg(p.h0 + row * N + nn[q]) : 0.0f;
                 } else {
                     const int64_t slot = meta.g * S::kScanWarps + warp;
+                    if (!SS_IN_BOUNDS(slot < p.groups * S::kScanWarps, 103))
+                        break;
                     const uint64_t want = carry_tag(epoch, meta.s);
                     if (!flag_wait(flags + slot, want, status))
                         break; // timeout recorded; counted out below
@@ -1094,8 +1122,11 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
             }
             const int rs = int(j % S::kRawStages);
             float *hrow = nullptr;
-            if (EMIT)
+            if (EMIT) {
+                if (!SS_IN_BOUNDS(row < p.batch * p.channels && meta.t0 < p.seq, 110))
+                    break;
                 hrow = p.h_all + (row * p.seq + meta.t0) * N;
+            }
             scan_chunk<N, SPL, T, HAS_RESET, EMIT>(stage, smem_bytes + rs * S::template raw_stage_bytes<T>(),
                                                    y_base + ysi * S::template y_stage<T>() + S::kYPOff +
                                                        cl * S::kYChan + sub * S::kRow,
@@ -1105,7 +1136,7 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
             mbar_arrive(y_full + ysi);
             if (meta.flags & kLast) {
                 if (p.pass == 1) {
-                    if (cvalid) {
+                    if (cvalid && SS_IN_BOUNDS(p.seg_stride >= p.batch * p.channels * N, 106)) {
                         float *dst = p.seg_state + meta.s * p.seg_stride + row * N;
 #pragma unroll
                         for (int q = 0; q < SPL; ++q)
@@ -1115,6 +1146,8 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
                     // the final state was produced by the join
                 } else if (int64_t(meta.s) + 1 < p.segments) {
                     const int64_t slot = meta.g * S::kScanWarps + warp;
+                    if (!SS_IN_BOUNDS(slot < p.groups * S::kScanWarps, 104))
+                        continue;
                     float *cs = carry + (slot * 32 + lane) * SPL;
 #pragma unroll
                     for (int q = 0; q < SPL; ++q)
@@ -1123,7 +1156,7 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
                     __syncwarp();
                     if (lane == 0)
                         st_release_gpu(flags + slot, carry_tag(epoch, meta.s + 1));
-                } else if (p.h_last && cvalid) {
+                } else if (p.h_last && cvalid && SS_IN_BOUNDS(row < p.batch * p.channels, 105)) {
 #pragma unroll
                     for (int q = 0; q < SPL; ++q)
                         p.h_last[row * N + nn[q]] = hs[q];

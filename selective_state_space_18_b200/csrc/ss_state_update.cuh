@@ -88,7 +88,9 @@ ss_state_update_kernel(const UpdateArgs p)
 #pragma unroll
     for (int it = 0; it < kUpdateItems; ++it) {
         const float *sp = p.state + (b * p.channels + chan(it)) * N + 4 * lane_q;
-        s[it] = VEC ? __ldcs(reinterpret_cast<const float4 *>(sp)) : make_float4(sp[0], sp[1], sp[2], sp[3]);
+        s[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (SS_IN_BOUNDS(b < p.batch && chan(it) < p.channels, 210))
+            s[it] = VEC ? __ldcs(reinterpret_cast<const float4 *>(sp)) : make_float4(sp[0], sp[1], sp[2], sp[3]);
     }
     float xs[kUpdateItems], ds[kUpdateItems];
 #pragma unroll
@@ -120,7 +122,7 @@ ss_state_update_kernel(const UpdateArgs p)
 #pragma unroll
         for (int off = Q / 2; off >= 1; off >>= 1)
             yp += __shfl_xor_sync(0xffffffffu, yp, off);
-        if (valid) {
+        if (valid && SS_IN_BOUNDS(row < p.batch * p.channels, 211)) {
             float *sp = p.state + row * N + 4 * lane_q;
             if (VEC)
                 __stcs(reinterpret_cast<float4 *>(sp), st);
@@ -247,6 +249,10 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
         // (bulk_cs: channels % 4 == 0, so row0 * H * 4 and nch * H * 4 are multiples of 16)
         const uint32_t csbytes = (CONV && da.bulk_cs) ? uint32_t(nch * (da.conv_k - 1) * 4) : 0u;
         unsigned char *dst = dsm + size_t(stage) * kStage;
+        if (!SS_IN_BOUNDS(b < p.batch && nch > 0 && row0 + nch <= p.batch * p.channels && stage < kDecStages &&
+                              nch * N * 4 <= kDecTileBytes,
+                          202))
+            return false;
         mbar_arrive_expect_tx(full + stage, sbytes + nvec * vbytes + bcbytes + csbytes);
         bulk_load(dst, p.state + row0 * N, sbytes, full + stage);
         if (nvec) {
@@ -310,6 +316,10 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
             break;
         const int64_t c0 = cb * D::kChanPerTile;
         const int nq = int(nchan(cb) * Q); // valid quarters in this tile
+        if (!SS_IN_BOUNDS(cb < da.ncb && nq > 0 && nq <= kDecQuarters, 201)) {
+            ok = false;
+            break;
+        }
         if (cb != cached_cb) {
             cached_cb = cb;
 #pragma unroll
@@ -475,7 +485,7 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
                 yp += __shfl_xor_sync(0xffffffffu, yp, off);
             if constexpr (CONV) {
                 __syncwarp(); // every lane of the row has read the conv state
-                if (valid && lane_q == 0 && H > 0) {
+                if (valid && lane_q == 0 && H > 0 && SS_IN_BOUNDS(c0 + q / Q < p.channels, 207)) {
                     const int64_t row = b * p.channels + c0 + q / Q;
                     float *csr = da.conv_state + row * H;
                     // shift: drop the oldest input (entry 0, whose register now holds u),
@@ -487,7 +497,7 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
                     csr[H - 1] = cs[it][0];
                 }
             }
-            if (valid) {
+            if (valid && SS_IN_BOUNDS(c0 + q / Q < p.channels && b < p.batch, 204)) {
                 const int64_t row = b * p.channels + c0 + q / Q;
                 __stcs(reinterpret_cast<float4 *>(p.state + row * N) + lane_q, st);
                 if (lane_q == 0) {

@@ -18,6 +18,8 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libssscan.so")
+# the same sources compiled with SS_BOUNDS_CHECK (a debug build, for the index-check tests)
+BOUNDS_LIB_PATH = os.path.join(_PKG, "libssscan_bounds.so")
 
 SS_F32, SS_BF16 = 0, 1
 SS_DT_SOFTPLUS = 1
@@ -29,7 +31,7 @@ STATUS = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE", 4:
 EXPORTS = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_scan_plan", "ss_scan_status", "ss_debug_status",
            "ss_state_update",
            "ss_debug_set_wait_limit", "ss_debug_set_scan_layout", "ss_debug_set_scan_two_level",
-           "ss_status_string", "ss_abi_version",
+           "ss_status_string", "ss_abi_version", "ss_debug_mufu_probe", "ss_debug_bounds_status",
            "ss_scan_fwd_static_scratch", "ss_scan_fwd_states", "ss_gated_scan", "ss_scan_fwd_conv",
            "ss_state_update_conv", "ss_segment_decay", "ss_join_segments")
 ABI_MAJOR = 2
@@ -105,6 +107,10 @@ def load_library(path: str = LIB_PATH):
             lib.ss_debug_set_scan_layout.restype = ctypes.c_int
             lib.ss_debug_set_scan_two_level.argtypes = [ctypes.c_int]
             lib.ss_debug_set_scan_two_level.restype = ctypes.c_int
+            lib.ss_debug_mufu_probe.argtypes = [ctypes.c_int, _i64, _i64, _vp, _vp, ctypes.POINTER(_i64), _vp]
+            lib.ss_debug_mufu_probe.restype = ctypes.c_int
+            lib.ss_debug_bounds_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int)]
+            lib.ss_debug_bounds_status.restype = ctypes.c_int
             lib.ss_debug_status.argtypes = [_vp]
             lib.ss_debug_status.restype = ctypes.c_int
             lib.ss_abi_version.argtypes = []
@@ -241,6 +247,28 @@ def ss_debug_set_scan_two_level(mode: int) -> None:
     st = load_library().ss_debug_set_scan_two_level(int(mode))
     if st != 0:
         raise SSError("ss_debug_set_scan_two_level", st)
+
+
+def mufu_rate(op="ex2", iters=1 << 16, device=None):
+    """Measured results per clock per SM of the special-function unit (op "ex2" or
+    "tanh"): one 512-thread CTA per SM, the SM cycle counter around the loop.  Returns
+    (median rate, [per-SM rates])."""
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    code = {"ex2": 0, "tanh": 1}[op]
+    with torch.cuda.device(device):
+        sms = torch.cuda.get_device_properties(device).multi_processor_count
+        cycles = torch.zeros(sms, dtype=torch.int64, device=device)
+        sink = torch.zeros(512, dtype=torch.float32, device=device)
+        ops = _i64(0)
+        st = load_library().ss_debug_mufu_probe(code, int(iters), sms, _ptr(cycles), _ptr(sink),
+                                                ctypes.byref(ops), _stream(None, device))
+        if st != 0:
+            raise SSError("ss_debug_mufu_probe", st)
+        torch.cuda.synchronize(device)
+    rates = [ops.value / float(c) for c in cycles.cpu().tolist() if c > 0]
+    rates.sort()
+    return rates[len(rates) // 2], rates
 
 
 def ss_debug_set_wait_limit(microseconds: int) -> None:

@@ -295,3 +295,12 @@ def test_join_segments_checks(lib):
     assert call(carry=ctypes.c_void_p(P[0].value + 1024)) == "SS_ERR_ALIAS"  # inside the composites
     assert call(final=ctypes.c_void_p(P[1].value + 512)) == "SS_ERR_ALIAS"   # overlaps carry
     assert call(count=1 << 62) == "SS_ERR_SHAPE"
+
+
+def test_mufu_probe_checks(lib):
+    ops = ctypes.c_int64(0)
+    P = [ctypes.c_void_p(0x7f0000000000 + i * 0x100000000) for i in range(2)]
+    assert lib.ss_debug_mufu_probe(0, 16, 4, None, P[1], ctypes.byref(ops), None) == 1
+    assert lib.ss_debug_mufu_probe(2, 16, 4, P[0], P[1], ctypes.byref(ops), None) == 5
+    assert lib.ss_debug_mufu_probe(0, 0, 4, P[0], P[1], ctypes.byref(ops), None) == 2
+    assert lib.ss_debug_mufu_probe(1, 16, 0, P[0], P[1], ctypes.byref(ops), None) == 2
