@@ -17,10 +17,16 @@ the maximum over ranks of the device-timed region.  Rank 0 prints one JSON line.
 
 times the prompt scan alone with its one sequence cut into a segment per rank
 (strong scaling; one NCCL all-gather of segment composites per step).
+
+    python bench.py --form {scan-130m,scan-packed,states,conv,conv-decode,gated,
+                            segment-decay,two-level,single-pass-small} [--steps K]
+
+times one kernel form on its own workload (one GPU) and prints its own JSON line.
 """
 from __future__ import annotations
 
 import argparse
+import gc
 import hashlib
 import json
 import math
@@ -315,9 +321,14 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     _barrier(world)
     torch.cuda.synchronize(dev)
-    # A short GPU-side spin before the first timed event gives the host a head start,
-    # so no per-step event interval ever includes host-side launch work.
-    torch.cuda._sleep(int(1.5e-3 * 1.965e9))
+    # The host must never let the GPU's queue run dry inside a timed interval (a host
+    # stall between a step's first event and its launch would be timed as GPU work):
+    # no garbage collection during the timed loop, and a 10 ms GPU-side spin before the
+    # first timed event, so the host is ahead of the GPU by that much from the start
+    # (it enqueues a step in well under the GPU's step time).
+    gc.collect()
+    gc.disable()
+    torch.cuda._sleep(int(10e-3 * 1.965e9))
     t0 = time.perf_counter()
     start.record(stream)
     for i in range(K):
@@ -331,9 +342,11 @@ def run_ours(args):
                                u["dt_bias"], y=y_dec[i & 1], stream=stream)
         e2.record(stream)
     end.record(stream)
+    t_enq = time.perf_counter()
     wait_event(end)
     torch.cuda.synchronize(dev)
     t1 = time.perf_counter()
+    gc.enable()
     _barrier(world)
     sampler.stop()
     clocks = sampler.summary(t0, t1)
@@ -400,6 +413,7 @@ def run_ours(args):
     kernels = {
         "scan": {"ms": round(scan_ms, 5), "ms_min": round(min(scan_list), 5),
                  "ms_median": round(statistics.median(scan_list), 5), "ms_max": round(max(scan_list), 5),
+                 "max_step": scan_list.index(max(scan_list)),
                  "kcycles_at_median_clock": (round(scan_ms * sm_clk, 1) if sm_clk else None),
                  "elems_per_s": pw["elems"] / scan_s,
                  "hbm_gbs": round(scan_hbm, 1), "roofline_frac": round(t_roof_scan / scan_s, 4),
@@ -449,6 +463,7 @@ def run_ours(args):
                 "steps": e2e["steps"]},
         "clocks": clocks,
         "prewarm_s": round(prewarm_s, 3),
+        "host_enqueue_ms": round((t_enq - t0) * 1e3, 2),
         "prewarm_steps": prewarm_steps,
         "gpu_launches": 2 * K,
     }
@@ -749,6 +764,178 @@ def run_seq_shard(args):
         dist.destroy_process_group()
 
 
+# ---------------------------------------------------------------------------------------
+# the next rows' kernels, one at a time (--form)
+# ---------------------------------------------------------------------------------------
+
+FORMS = ("scan-130m", "scan-packed", "states", "conv", "conv-decode", "gated", "segment-decay",
+         "two-level", "single-pass-small")
+
+
+def run_form(args):
+    """Time one kernel form on its workload with the protocol of the headline step
+    (pre-roll, GPU-side head start, CUDA events per call, clocks sampled inside the
+    timed region) and print one JSON line with its own roofline."""
+    from selective_state_space_18_b200 import ssscan
+    from selective_state_space_18_b200.inputs import make_gated_inputs, make_scan_inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    ssscan.load_library()
+    form = args.form
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    hbm_gbs, sm_max_mhz, peak_kind = _peaks()
+    bf16 = torch.bfloat16
+    nsets = 2
+    g = torch.Generator().manual_seed(4242)
+
+    def to_dev(d):
+        return {k: (None if v is None else v.to(dev)) for k, v in d.items()}
+
+    if form in ("scan-130m", "scan-packed", "states", "conv", "two-level", "single-pass-small"):
+        wname = {"scan-130m": "mamba130m_layer", "scan-packed": "packed_resets"}.get(form, "mamba2p8b_layer_long")
+        w = WORKLOADS[wname]
+        if form in ("two-level", "single-pass-small"):
+            shape = (1, 1024, 16, 65536)
+            mk = lambda sd: make_scan_inputs(*shape, "bf16", seed=sd, a_perturb=True)
+            desc = "batch 1, channels 1024, state_dim 16, seq 65536, bf16, z gate, dt_bias"
+        else:
+            shape = (w.batch, w.channels, w.state_dim, w.seq)
+            mk = lambda sd: make_workload(w, seed=sd)
+            desc = f"{wname}: batch {w.batch}, channels {w.channels}, state_dim {w.state_dim}, seq {w.seq}, bf16"
+        if form == "states":
+            nsets = 1  # 5.4 GB of states per call: one set already far exceeds L2
+        sets = [to_dev(mk(w.seed + 1000 * i)) for i in range(nsets)]
+        bt, ch, n, L = shape
+        rows, elems = bt * ch, bt * ch * n * L
+        keys = ("x", "dt", "A", "B", "C", "D", "z", "dt_bias", "reset", "h0")
+        y = torch.empty(bt, ch, L, device=dev, dtype=bf16)
+        hl = torch.empty(bt, ch, n, device=dev)
+        if form == "states":
+            hall = torch.empty(bt, ch, L, n, device=dev)
+        if form == "conv":
+            cw = (torch.randn(ch, 4, generator=g) * 0.5).to(dev)
+            cb = (torch.randn(ch, generator=g) * 0.1).to(dev)
+        if form == "single-pass-small":
+            ssscan.ss_debug_set_scan_two_level(1)
+
+        def call(i):
+            d = sets[i % nsets]
+            a = [d[k] for k in keys]
+            if form == "states":
+                ssscan.ss_scan_fwd(*a, y=y, h_last=hl, h_all=hall)
+            elif form == "conv":
+                ssscan.ss_scan_fwd_conv(d["x"], cw, d["dt"], d["A"], d["B"], d["C"], d["D"], d["z"], d["dt_bias"],
+                                        conv_b=cb, return_conv_state=False)
+            else:
+                ssscan.ss_scan_fwd(*a, y=y, h_last=hl)
+        exps = rows * L * (n + 2)
+        byts = 4 * rows * L * 2 + 2 * bt * n * L * 2 + rows * n * 4
+        if form == "states":
+            byts += rows * L * n * 4
+        kernel = {"states": "ss_scan_fwd_kernel (states form)", "conv": "ss_scan_fwd_kernel (fused conv form)",
+                  "two-level": "ss_scan_fwd_kernel x2 + ss_segment_decay_kernel + ss_join_all_kernel (two-level)",
+                  "single-pass-small": "ss_scan_fwd_kernel (single pass, chained segments)"}.get(form, "ss_scan_fwd_kernel")
+        bound = "hbm" if form == "states" else "alu"
+        metric_elems = elems
+    elif form == "conv-decode":
+        w = DECODE
+        sets = [to_dev(make_workload(w, seed=w.seed + 1000 * i)) for i in range(nsets)]
+        cw = (torch.randn(w.channels, 4, generator=g) * 0.5).to(dev)
+        cs = [torch.randn(w.batch, w.channels, 3, generator=g).to(dev) for _ in range(nsets)]
+        y = torch.empty(w.batch, w.channels, device=dev, dtype=bf16)
+
+        def call(i):
+            u = sets[i % nsets]
+            ssscan.ss_state_update_conv(u["state"], cs[i % nsets], cw, u["x"], u["dt"], u["A"], u["B"], u["C"],
+                                        u["D"], u["z"], u["dt_bias"])
+        rows = w.batch * w.channels
+        byts = decode_work()["bytes"] + 2 * rows * 3 * 4 + w.channels * 4 * 4
+        exps, bound, kernel = rows * (w.state_dim + 3), "hbm", "ss_state_update_stream_kernel (fused conv form)"
+        metric_elems = rows * w.state_dim
+        desc = "decode_2p8b with the conv form (conv_k 4, fp32 conv state in place)"
+    elif form == "gated":
+        B_, S_, dk, dv = 512, 2048, 128, 64
+        sets = [to_dev(make_gated_inputs(B_, S_, dk, dv, "bf16", seed=77 + i)) for i in range(nsets)]
+
+        def call(i):
+            d = sets[i % nsets]
+            ssscan.ss_gated_scan(d["q"], d["k"], d["v"], d["gamma"])
+        metric_elems = B_ * S_ * dk * dv
+        lane_ops = 3 * metric_elems
+        byts = B_ * S_ * (2 * dk + 2 * dv) * 2 + B_ * S_ * 4 + B_ * dk * dv * 2
+        exps, bound, kernel = 0, "fp32-pipe", "ss_gated_scan_kernel"
+        desc = f"gated state scan: batch {B_}, seq {S_}, dk {dk}, dv {dv}, bf16"
+    elif form == "segment-decay":
+        w = PROMPT
+        Ls = 1816  # one segment of the 2.8B-layer prompt cut into 8
+        full = make_workload(w, seed=w.seed)
+        sets = [{"dt": full["dt"][..., i * Ls:(i + 1) * Ls].contiguous().to(dev), "A": full["A"].to(dev),
+                 "dt_bias": full["dt_bias"].to(dev)} for i in range(nsets)]
+        out = torch.empty(w.batch, w.channels, w.state_dim, device=dev)
+
+        def call(i):
+            d = sets[i % nsets]
+            ssscan.ss_segment_decay(d["dt"], d["A"], d["dt_bias"], out=out)
+        rows = w.batch * w.channels
+        byts = rows * Ls * 2 + rows * w.state_dim * 4 * 2 + w.channels * 4
+        exps, bound, kernel = rows * Ls, "hbm", "ss_segment_decay_kernel"
+        metric_elems = rows * Ls
+        desc = "segment decay: batch 1, channels 5120, one 1816-token segment of the 2.8B-layer prompt, bf16"
+    else:
+        raise SystemExit(f"unknown form {form}")
+
+    stream = torch.cuda.current_stream(dev)
+    sampler = ClockSampler(0)
+    sampler.start()
+    t_pre, i = time.perf_counter(), 0
+    while i < args.warmup or time.perf_counter() - t_pre < args.prewarm_s:
+        call(i)
+        i += 1
+        if i % 8 == 0:
+            torch.cuda.synchronize(dev)
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    gc.collect()
+    gc.disable()
+    torch.cuda._sleep(int(10e-3 * 1.965e9))
+    t0 = time.perf_counter()
+    for k in range(K):
+        ev[k][0].record(stream)
+        call(k)
+        ev[k][1].record(stream)
+    wait_event(ev[-1][1])
+    torch.cuda.synchronize(dev)
+    t1 = time.perf_counter()
+    gc.enable()
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
+    ssscan.ss_debug_set_scan_two_level(0)
+    ts = [a.elapsed_time(b) for a, b in ev]
+    ms = sum(ts) / K
+    sec = ms * 1e-3
+    ex2_rate, _ = ssscan.mufu_rate("ex2", device=dev)
+    sfu_peak = sms * ex2_rate * sm_max_mhz * 1e6
+    roof = {"bound": bound, "algorithmic_bytes_per_launch": byts, "hbm_achieved_gbs": round(byts / sec / 1e9, 1),
+            "hbm_frac": round(byts / sec / 1e9 / hbm_gbs, 4), "hbm_peak_gbs": hbm_gbs}
+    if bound == "alu":
+        roof.update({"unit_peak": "MUFU ex2", "exps_per_launch": exps, "achieved_gexp_s": round(exps / sec / 1e9, 2),
+                     "peak_gexp_s": round(sfu_peak / 1e9, 2), "frac": round(exps / sec / sfu_peak, 4)})
+    elif bound == "hbm":
+        roof["frac"] = roof["hbm_frac"]
+    else:
+        peak_ops = sms * 128 * sm_max_mhz * 1e6
+        roof.update({"lane_ops_per_launch": lane_ops, "peak_lane_ops_s": peak_ops,
+                     "frac": round(lane_ops / sec / peak_ops, 4)})
+    line = {"form": form, "kernel": kernel, "workload": desc, "ms": round(ms, 5),
+            "ms_median": round(statistics.median(ts), 5), "ms_min": round(min(ts), 5),
+            "ms_max": round(max(ts), 5),
+            "elems_per_s": metric_elems / sec, "steps": K, "warmup": args.warmup, "sets": nsets,
+            "roofline": roof, "clocks": clocks, "peaks": f"HBM {peak_kind}; SFU {ex2_rate:.2f} ex2/clk/SM measured"}
+    print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -767,10 +954,14 @@ def main(argv=None):
                     help="time the prompt scan with its sequence cut into one segment per rank (strong scaling)")
     ap.add_argument("--emulate-ranks", type=int, default=1,
                     help="with --seq-shard on one process: run this many segments on the one GPU")
+    ap.add_argument("--form", choices=FORMS, default=None,
+                    help="time one kernel form of the next rows on its own workload instead of the step")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.form:
+        run_form(args)
+    elif args.impl == "reference":
         run_reference(args)
     elif args.seq_shard:
         run_seq_shard(args)

@@ -308,9 +308,9 @@ SS_API int ss_debug_set_wait_limit(uint32_t microseconds);
 /*
  * Testing aid: make later state_dim-16 scans in this process use the layout with
  * `states_per_lane` (2 or 4) state rows per scan lane, whatever the shape; 0 restores
- * the automatic choice (four per lane when the shape's 32-channel groups give every
- * SM one, else two).  Results of the two layouts agree within rounding; they differ
- * only in speed.  Other state sizes always use two.  Returns SS_OK, or
+ * the default (two per lane, the faster layout as measured).  Results of the two
+ * layouts agree within rounding; they differ only in speed.  Other state sizes always
+ * use two.  Returns SS_OK, or
  * SS_ERR_UNSUPPORTED for any other value.  Not thread-safe with respect to scans
  * being issued concurrently from other host threads.
  */

@@ -257,10 +257,12 @@ template <int N, int SPL> int64_t scan_groups(int64_t batch, int64_t channels)
     return batch * ((channels + per - 1) / per);
 }
 
-// States per scan lane for a shape: at state_dim 16, four (32 channels per CTA, the
-// fewer shared-memory bytes and instructions per state) when its channel groups give
-// every SM one, else two (16 channels per CTA: twice the groups, so twice the SMs, for
-// shapes with few channels).  Smaller state sizes keep two.
+// States per scan lane: two.  Four per lane (32 channels per CTA, one CTA per SM)
+// moves fewer shared-memory bytes and issues fewer instructions per state, but leaves
+// one scan warp per SM sub-partition for the 2.8B-layer shape, and measured slower
+// (0.738 against 0.637 ms): a lone warp cannot hide the exponential unit's throttling
+// and the FMA chains' latency as two warps do.  It stays selectable
+// (ss_debug_set_scan_layout) and tested.
 std::atomic<int> g_forced_spl{0};     // ss_debug_set_scan_layout: 0 = choose per shape
 std::atomic<int> g_two_level_mode{0}; // ss_debug_set_scan_two_level: 0 auto, 1 never, 2 always
 
@@ -271,10 +273,9 @@ int scan_spl(int64_t batch, int64_t channels, int64_t state_dim)
     const int forced = g_forced_spl.load(std::memory_order_relaxed);
     if (forced)
         return forced;
-    int sms = 0;
-    if (device_sm_count(&sms) != SS_OK)
-        sms = 148;
-    return scan_groups<16, 4>(batch, channels) >= int64_t(sms) ? 4 : 2;
+    (void)batch;
+    (void)channels;
+    return 2;
 }
 
 template <int N, int SPL>
@@ -343,7 +344,7 @@ TwoLevelPlan two_level_plan(int64_t batch, int64_t channels, int64_t state_dim, 
     if (mode == 1 || (mode == 0 && (groups16 >= int64_t(sms) || nchunks < 64)))
         return t;
     const int forced = g_forced_spl.load(std::memory_order_relaxed);
-    t.spl = forced ? forced : 4;
+    t.spl = forced ? forced : 2;
     t.groups = t.spl == 4 ? scan_groups<16, 4>(batch, channels) : groups16;
     const int64_t resident = int64_t(sms) * (t.spl == 4 ? 1 : 2);
     int64_t segs = (8 * resident + t.groups - 1) / t.groups; // about eight units per CTA
