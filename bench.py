@@ -303,6 +303,8 @@ def run_ours(args):
     # pre-roll from the timed region.
     done = []
     i = 0
+    gc.collect()
+    gc.disable()  # no collector pauses from here to the end of the timed region
     t_pre = time.perf_counter()
     while i < args.warmup or time.perf_counter() - t_pre < args.prewarm_s:
         if len(done) >= 8:
@@ -312,8 +314,10 @@ def run_ours(args):
         e.record(stream)
         done.append(e)
         i += 1
+    torch.cuda.synchronize(dev)
     prewarm_steps = i - args.warmup
     prewarm_s = time.perf_counter() - t_pre
+    step_s = prewarm_s / max(1, i)  # (an upper bound on the GPU's time per step)
 
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
@@ -322,13 +326,13 @@ def run_ours(args):
     _barrier(world)
     torch.cuda.synchronize(dev)
     # The host must never let the GPU's queue run dry inside a timed interval (a host
-    # stall between a step's first event and its launch would be timed as GPU work):
-    # no garbage collection during the timed loop, and a 10 ms GPU-side spin before the
-    # first timed event, so the host is ahead of the GPU by that much from the start
-    # (it enqueues a step in well under the GPU's step time).
-    gc.collect()
-    gc.disable()
-    torch.cuda._sleep(int(10e-3 * 1.965e9))
+    # stall between a step's first event and its launch would be timed as GPU work), and
+    # the GPU must not idle or run light right before it: untimed steps worth about
+    # 10 ms of GPU work go first, so the GPU is busy with the step's own work while the
+    # host enqueues the timed steps (garbage collection stays off throughout).
+    head = max(3, min(64, int(10e-3 / max(step_s, 1e-5)) + 1))
+    for h in range(head):
+        step(i + h)
     t0 = time.perf_counter()
     start.record(stream)
     for i in range(K):
@@ -463,6 +467,7 @@ def run_ours(args):
                 "steps": e2e["steps"]},
         "clocks": clocks,
         "prewarm_s": round(prewarm_s, 3),
+        "head_start_steps": head,
         "host_enqueue_ms": round((t_enq - t0) * 1e3, 2),
         "prewarm_steps": prewarm_steps,
         "gpu_launches": 2 * K,
@@ -888,6 +893,10 @@ def run_form(args):
     stream = torch.cuda.current_stream(dev)
     sampler = ClockSampler(0)
     sampler.start()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    gc.collect()
+    gc.disable()
     t_pre, i = time.perf_counter(), 0
     while i < args.warmup or time.perf_counter() - t_pre < args.prewarm_s:
         call(i)
@@ -895,11 +904,9 @@ def run_form(args):
         if i % 8 == 0:
             torch.cuda.synchronize(dev)
     torch.cuda.synchronize(dev)
-    K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    gc.collect()
-    gc.disable()
-    torch.cuda._sleep(int(10e-3 * 1.965e9))
+    call_s = (time.perf_counter() - t_pre) / max(1, i)
+    for h in range(max(3, min(64, int(10e-3 / max(call_s, 1e-5)) + 1))):  # head start, untimed
+        call(i + h)
     t0 = time.perf_counter()
     for k in range(K):
         ev[k][0].record(stream)

@@ -143,6 +143,7 @@ bool build_maps(const ss::ScanArgs &a, ss::TmaMaps *m)
         S::template swizzle<T>() == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     return encode_rows<T>(&m->x, a.x, a.seq, rows, S::kChunk, S::kChanPerCta) &&
            encode_rows<T>(&m->dt, a.dt, a.seq, rows, S::kChunk, S::kChanPerCta) &&
+           (!a.z || encode_rows<T>(&m->z, a.z, a.seq, rows, S::kChunk, S::kChanPerCta)) &&
            encode_rows<T>(&m->B, a.B, a.seq, brows, S::kChunk, N, bc_swizzle) &&
            encode_rows<T>(&m->C, a.C, a.seq, brows, S::kChunk, N, bc_swizzle);
 }

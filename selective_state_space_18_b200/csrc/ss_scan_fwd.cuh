@@ -73,10 +73,12 @@ struct ScanArgs {
     int64_t seg_stride;
 };
 
-// Tensor maps of the TMA path: x, dt as [batch * channels rows][seq] and B, C as
-// [batch * state_dim rows][seq], boxes of one chunk of tokens.
+// Tensor maps of the TMA path: x, dt (and z) as [batch * channels rows][seq] and B, C
+// as [batch * state_dim rows][seq], boxes of one chunk of tokens.  z is not loaded into
+// shared memory: the issuer only prefetches each chunk's z tile into L2, several chunks
+// before the epilogue reads it with plain loads.
 struct TmaMaps {
-    CUtensorMap x, dt, B, C;
+    CUtensorMap x, dt, B, C, z;
 };
 
 // Workspace layout (bytes): the caller zeroes it once; every call leaves it ready for
@@ -825,6 +827,8 @@ __device__ __forceinline__ bool issuer_warp(const ScanArgs &p, const TmaMaps &ma
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.dt)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.B)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.C)) : "memory");
+        if (p.z)
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.z)) : "memory");
     }
     constexpr uint32_t tx_bytes = uint32_t((2 * S::kChanPerCta + 2 * N) * S::kChunk * sizeof(T));
     uint32_t u = take_unit(p, cx.ws, true);
@@ -863,6 +867,8 @@ __device__ __forceinline__ bool issuer_warp(const ScanArgs &p, const TmaMaps &ma
             tma_load_2d(dst + S::template raw_dt_off<T>(), &maps.dt, tt, xrow, bar);
             tma_load_2d(dst + S::template raw_b_off<T>(), &maps.B, tt, brow, bar);
             tma_load_2d(dst + S::template raw_c_off<T>(), &maps.C, tt, brow, bar);
+            if (p.z && p.pass != 1) // the epilogue's z, from HBM into L2 ahead of time
+                tma_prefetch_l2_2d(&maps.z, tt, xrow);
         } else {
             mbar_arrive(cx.raw_full + r);
         }

@@ -73,6 +73,16 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
                  : "memory");
 }
 
+// Prefetch a 2-D tile into L2 through a tensor map (nothing is written to shared
+// memory and nothing is waited for): a later plain load of the tile then hits L2.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int32_t c0, int32_t c1)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1)
+                 : "memory");
+}
+
 // Orders this thread's earlier generic-proxy shared-memory accesses before later
 // asynchronous-proxy (TMA) writes to the same memory.
 __device__ __forceinline__ void fence_proxy_async_smem()
