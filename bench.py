@@ -107,6 +107,16 @@ def _measured_traffic(kernel):
     return entry.get("dram_bytes_per_launch")
 
 
+def _tensor_peak_tflops():
+    """Dense bf16 tensor throughput (TFLOP/s): the measured burst figure when present,
+    else the pool's earlier measurement."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except (OSError, ValueError, KeyError):
+        return 1590.0
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -773,8 +783,8 @@ def run_seq_shard(args):
 # the next rows' kernels, one at a time (--form)
 # ---------------------------------------------------------------------------------------
 
-FORMS = ("scan-130m", "scan-packed", "states", "conv", "conv-decode", "gated", "segment-decay",
-         "two-level", "single-pass-small")
+FORMS = ("scan-130m", "scan-packed", "states", "conv", "conv-decode", "gated", "gated-recurrent",
+         "segment-decay", "two-level", "single-pass-small")
 
 
 def run_form(args):
@@ -859,9 +869,11 @@ def run_form(args):
         exps, bound, kernel = rows * (w.state_dim + 3), "hbm", "ss_state_update_stream_kernel (fused conv form)"
         metric_elems = rows * w.state_dim
         desc = "decode_2p8b with the conv form (conv_k 4, fp32 conv state in place)"
-    elif form == "gated":
+    elif form in ("gated", "gated-recurrent"):
         B_, S_, dk, dv = 512, 2048, 128, 64
         sets = [to_dev(make_gated_inputs(B_, S_, dk, dv, "bf16", seed=77 + i)) for i in range(nsets)]
+        if form == "gated-recurrent":
+            ssscan.ss_debug_set_gated_path(1)
 
         def call(i):
             d = sets[i % nsets]
@@ -869,7 +881,14 @@ def run_form(args):
         metric_elems = B_ * S_ * dk * dv
         lane_ops = 3 * metric_elems
         byts = B_ * S_ * (2 * dk + 2 * dv) * 2 + B_ * S_ * 4 + B_ * dk * dv * 2
-        exps, bound, kernel = 0, "fp32-pipe", "ss_gated_scan_kernel"
+        if form == "gated":
+            # the chunked form's matrix products per 128-token chunk: Q K^T, (L o S) V, Q H
+            # and K^T (w o V)
+            C_ = 128
+            flops = 2 * B_ * (S_ // C_) * (C_ * C_ * dk + C_ * C_ * dv + C_ * dk * dv + dk * C_ * dv)
+            exps, bound, kernel = 0, "tensor", "ss_gated_tc_kernel (chunked, tcgen05)"
+        else:
+            exps, bound, kernel = 0, "fp32-pipe", "ss_gated_scan_kernel (token by token)"
         desc = f"gated state scan: batch {B_}, seq {S_}, dk {dk}, dv {dv}, bf16"
     elif form == "segment-decay":
         w = PROMPT
@@ -919,6 +938,7 @@ def run_form(args):
     sampler.stop()
     clocks = sampler.summary(t0, t1)
     ssscan.ss_debug_set_scan_two_level(0)
+    ssscan.ss_debug_set_gated_path(0)
     ts = [a.elapsed_time(b) for a, b in ev]
     ms = sum(ts) / K
     sec = ms * 1e-3
@@ -931,6 +951,11 @@ def run_form(args):
                      "peak_gexp_s": round(sfu_peak / 1e9, 2), "frac": round(exps / sec / sfu_peak, 4)})
     elif bound == "hbm":
         roof["frac"] = roof["hbm_frac"]
+    elif bound == "tensor":
+        peak_tf = _tensor_peak_tflops()
+        roof.update({"flops_per_launch": flops, "achieved_tflops": round(flops / sec / 1e12, 2),
+                     "peak_tflops": peak_tf, "frac": round(flops / sec / 1e12 / peak_tf, 4),
+                     "fp32_pipe_equivalent": round(lane_ops / sec / (sms * 128 * sm_max_mhz * 1e6), 4)})
     else:
         peak_ops = sms * 128 * sm_max_mhz * 1e6
         roof.update({"lane_ops_per_launch": lane_ops, "peak_lane_ops_s": peak_ops,

@@ -327,6 +327,14 @@ SS_API int ss_debug_set_scan_layout(int states_per_lane);
 SS_API int ss_debug_set_scan_two_level(int mode);
 
 /*
+ * Testing aid: the kernel of later ss_gated_scan calls.  mode 0 (default): the
+ * chunked tensor-core form where it applies (see ss_gated_scan), 1: always the
+ * token-by-token recurrence, 2: as 0.  Returns SS_OK, or SS_ERR_UNSUPPORTED for any
+ * other mode.
+ */
+SS_API int ss_debug_set_gated_path(int mode);
+
+/*
  * Gated state scan (the "Mamba 2 Gated State Scan" exercise page): per batch item b,
  *
  *   S_t = gamma[b,t] * S_{t-1} + k[b,t,:] v[b,t,:]^T      (Dk x Dv state, fp32)
@@ -341,10 +349,16 @@ SS_API int ss_debug_set_scan_two_level(int mode);
  *   outputs     : [batch, seq, dv]  dtype (output)
  *   final_state : [batch, dk, dv]   dtype (output)
  *
- * All arithmetic is fp32; results are rounded to the dtype of q, as the page asks.
- * dk must be at most 128 (SS_ERR_UNSUPPORTED otherwise); dv is unrestricted.  Inputs
- * are not modified; outputs must not overlap inputs or each other (SS_ERR_ALIAS).
- * Asynchronous on `stream`; returns SS_OK or an error status.
+ * Results are rounded to the dtype of q, as the page asks.  dk must be at most 128
+ * (SS_ERR_UNSUPPORTED otherwise); dv is unrestricted.  Two kernels:
+ *  - bf16 with dk = 128, dv a multiple of 64 and 16-byte aligned tensors: the chunked
+ *    form on the tensor cores -- per 128-token chunk, Q K^T, the decay-masked scores
+ *    times V, Q times the entering state, and K^T times the decay-weighted V as
+ *    tcgen05 matrix products (bf16 operands, fp32 accumulation), the state itself in
+ *    fp32;
+ *  - every other case: the recurrence token by token, all arithmetic in fp32.
+ * Inputs are not modified; outputs must not overlap inputs or each other
+ * (SS_ERR_ALIAS).  Asynchronous on `stream`; returns SS_OK or an error status.
  */
 SS_API int ss_gated_scan(int64_t batch, int64_t seq, int64_t dk, int64_t dv, ss_dtype_t dtype,
                          const void *q, const void *k, const void *v, const float *gamma,

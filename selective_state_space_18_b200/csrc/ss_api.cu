@@ -13,6 +13,7 @@
 #include "ss_scan_fwd.cuh"
 #include "ss_state_update.cuh"
 #include "ss_gated_scan.cuh"
+#include "ss_gated_tc.cuh"
 #include "ss_segment.cuh"
 
 namespace {
@@ -265,6 +266,7 @@ template <int N, int SPL> int64_t scan_groups(int64_t batch, int64_t channels)
 // and the FMA chains' latency as two warps do.  It stays selectable
 // (ss_debug_set_scan_layout) and tested.
 std::atomic<int> g_forced_spl{0};     // ss_debug_set_scan_layout: 0 = choose per shape
+std::atomic<int> g_gated_path{0};     // ss_debug_set_gated_path: 0 auto, 1 recurrent, 2 tensor cores
 std::atomic<int> g_two_level_mode{0}; // ss_debug_set_scan_two_level: 0 auto, 1 never, 2 always
 
 int scan_spl(int64_t batch, int64_t channels, int64_t state_dim)
@@ -640,6 +642,14 @@ int ss_debug_bounds_status(ss_stream_t stream, int *site)
 #endif
 }
 
+int ss_debug_set_gated_path(int mode)
+{
+    if (mode < 0 || mode > 2)
+        return SS_ERR_UNSUPPORTED;
+    g_gated_path.store(mode, std::memory_order_relaxed);
+    return SS_OK;
+}
+
 int ss_debug_set_scan_two_level(int mode)
 {
     if (mode < 0 || mode > 2)
@@ -937,8 +947,68 @@ template <int RG, typename T> int dispatch_gated_v(const ss::GatedArgs &a, cudaS
     return vec ? launch_gated<RG, T, true>(a, s) : launch_gated<RG, T, false>(a, s);
 }
 
+// 3-D map over [batch][seq][inner] bf16 with boxes of 64 x 128 x 1 and the 128-byte
+// swizzle (rows past seq read as zeros, per batch item).
+bool encode_bsi(CUtensorMap *map, const void *base, int64_t batch, int64_t seq, int64_t inner)
+{
+    PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
+    if (!enc)
+        return false;
+    const cuuint64_t dims[3] = {cuuint64_t(inner), cuuint64_t(seq), cuuint64_t(batch)};
+    const cuuint64_t strides[2] = {cuuint64_t(inner) * 2, cuuint64_t(seq) * cuuint64_t(inner) * 2};
+    const cuuint32_t box[3] = {64, uint32_t(ss::kGtChunk), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The chunked tensor-core form: bf16, dk = 128, dv a multiple of 64, 16-byte aligned
+// rows (the tile loads and the vector stores).
+bool gated_tc_eligible(const ss::GatedArgs &a, bool bf16)
+{
+    const int mode = g_gated_path.load(std::memory_order_relaxed);
+    if (mode == 1 || !bf16)
+        return false;
+    return a.dk == ss::kGtDk && a.dv % ss::kGtNv == 0 && a.seq < (int64_t(1) << 31) &&
+           a.batch < (int64_t(1) << 31) && aligned(a.q, 16) && aligned(a.k, 16) && aligned(a.v, 16) &&
+           aligned(a.y, 16) && aligned(a.final_state, 16);
+}
+
+int launch_gated_tc(const ss::GatedArgs &g, cudaStream_t stream)
+{
+    static std::atomic<uint64_t> smem_done{0};
+    const int st = ensure_smem(ss::ss_gated_tc_kernel, size_t(ss::GtSmem::kBytes), smem_done);
+    if (st != SS_OK)
+        return st;
+    ss::GatedTcArgs a{};
+    a.batch = g.batch;
+    a.seq = g.seq;
+    a.dv = g.dv;
+    a.gamma = g.gamma;
+    a.h0 = g.h0;
+    a.y = static_cast<__nv_bfloat16 *>(g.y);
+    a.final_state = static_cast<__nv_bfloat16 *>(g.final_state);
+    a.col_tiles = int(g.dv / ss::kGtNv);
+    int64_t grid = 0;
+    if (!mul_ok(g.batch, a.col_tiles, &grid) || grid > 0x7fffffffLL)
+        return SS_ERR_SHAPE;
+    ss::GatedTcMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (!encode_bsi(&maps.q, g.q, g.batch, g.seq, g.dk) || !encode_bsi(&maps.k, g.k, g.batch, g.seq, g.dk) ||
+        !encode_bsi(&maps.v, g.v, g.batch, g.seq, g.dv))
+        return SS_ERR_CUDA;
+    uint32_t *status = nullptr;
+    if (status_word_address(&status) != SS_OK)
+        return SS_ERR_CUDA;
+    ss::ss_gated_tc_kernel<<<unsigned(grid), ss::kGtThreads, ss::GtSmem::kBytes, stream>>>(a, maps, status);
+    return launch_status();
+}
+
 template <typename T> int dispatch_gated(const ss::GatedArgs &a, cudaStream_t s)
 {
+    if (gated_tc_eligible(a, sizeof(T) == 2))
+        return launch_gated_tc(a, s);
     if (a.dk <= 32)
         return dispatch_gated_v<4, T>(a, s);
     if (a.dk <= 64)

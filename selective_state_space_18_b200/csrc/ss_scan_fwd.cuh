@@ -1090,7 +1090,6 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
                 cvalid = c_raw < p.channels;
                 const int64_t c = cvalid ? c_raw : p.channels - 1;
                 row = b * p.channels + c;
-#pragma unroll
                 if (!SS_IN_BOUNDS(c < p.channels && row < p.batch * p.channels && nn[SPL - 1] < N, 109))
                     break;
 #pragma unroll

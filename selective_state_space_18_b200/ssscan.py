@@ -31,6 +31,7 @@ STATUS = {0: "SS_OK", 1: "SS_ERR_NULL", 2: "SS_ERR_SHAPE", 3: "SS_ERR_DTYPE", 4:
 EXPORTS = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_scan_plan", "ss_scan_status", "ss_debug_status",
            "ss_state_update",
            "ss_debug_set_wait_limit", "ss_debug_set_scan_layout", "ss_debug_set_scan_two_level",
+           "ss_debug_set_gated_path",
            "ss_status_string", "ss_abi_version", "ss_debug_mufu_probe", "ss_debug_bounds_status",
            "ss_scan_fwd_static_scratch", "ss_scan_fwd_states", "ss_gated_scan", "ss_scan_fwd_conv",
            "ss_state_update_conv", "ss_segment_decay", "ss_join_segments")
@@ -105,6 +106,8 @@ def load_library(path: str = LIB_PATH):
             lib.ss_debug_set_wait_limit.restype = ctypes.c_int
             lib.ss_debug_set_scan_layout.argtypes = [ctypes.c_int]
             lib.ss_debug_set_scan_layout.restype = ctypes.c_int
+            lib.ss_debug_set_gated_path.argtypes = [ctypes.c_int]
+            lib.ss_debug_set_gated_path.restype = ctypes.c_int
             lib.ss_debug_set_scan_two_level.argtypes = [ctypes.c_int]
             lib.ss_debug_set_scan_two_level.restype = ctypes.c_int
             lib.ss_debug_mufu_probe.argtypes = [ctypes.c_int, _i64, _i64, _vp, _vp, ctypes.POINTER(_i64), _vp]
@@ -269,6 +272,14 @@ def mufu_rate(op="ex2", iters=1 << 16, device=None):
     rates = [ops.value / float(c) for c in cycles.cpu().tolist() if c > 0]
     rates.sort()
     return rates[len(rates) // 2], rates
+
+
+def ss_debug_set_gated_path(mode: int) -> None:
+    """Kernel of later ss_gated_scan calls: 0 automatic (the tensor-core chunked form
+    where it applies), 1 always the token-by-token recurrence.  A testing aid."""
+    st = load_library().ss_debug_set_gated_path(int(mode))
+    if st != 0:
+        raise SSError("ss_debug_set_gated_path", st)
 
 
 def ss_debug_set_wait_limit(microseconds: int) -> None:

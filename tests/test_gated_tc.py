@@ -1,0 +1,93 @@
+"""The chunked tensor-core form of the gated state scan ("Mamba 2 Gated State Scan"
+exercise page: S_t = gamma_t S_{t-1} + k_t v_t^T, y_t = q_t^T S_t), which ss_gated_scan
+runs for bf16 inputs with dk = 128 and dv a multiple of 64: every output and the final
+state against the float64 oracle, and against the token-by-token kernel on the same
+inputs, both within the bf16 tolerance -- across ragged chunk tails, several value
+tiles, an initial state, and gates of exactly 0 and 1 (on chunk boundaries too)."""
+import contextlib
+
+import pytest
+import torch
+
+from gpu_util import TOL, assert_close
+from selective_state_space_18_b200 import ssscan
+from selective_state_space_18_b200.inputs import make_gated_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+
+
+@contextlib.contextmanager
+def recurrent():
+    ssscan.ss_debug_set_gated_path(1)
+    try:
+        yield
+    finally:
+        ssscan.ss_debug_set_gated_path(0)
+
+
+def _gpu(inp):
+    d = {k: (None if v is None else v.cuda()) for k, v in inp.items()}
+    out = ssscan.ss_gated_scan(**d)
+    torch.cuda.synchronize()
+    return out["outputs"].cpu(), out["final_state"].cpu()
+
+
+def _check(orc, inp, what):
+    y, fs = _gpu(inp)
+    with recurrent():
+        y1, fs1 = _gpu(inp)
+    ref = orc.gated_scan(**inp)
+    tol = TOL[torch.bfloat16]
+    assert_close(y, ref["outputs"], tol, f"{what}: outputs")
+    assert_close(fs, ref["final_state"], tol, f"{what}: final_state")
+    assert_close(y, y1.double().numpy(), tol, f"{what}: outputs against the recurrent kernel")
+    assert_close(fs, fs1.double().numpy(), tol, f"{what}: final_state against the recurrent kernel")
+
+
+@pytest.mark.parametrize("shape", [(2, 128, 64), (3, 300, 64), (2, 1000, 128), (1, 2048, 192), (5, 1, 64),
+                                   (2, 127, 64), (1, 4100, 64)])
+@pytest.mark.parametrize("h0", [False, True])
+def test_chunked_form_matches_oracle(orc, shape, h0):
+    B, S, dv = shape
+    inp = make_gated_inputs(B, S, 128, dv, "bf16", seed=1900 + B * S + dv, h0=h0)
+    _check(orc, inp, f"{shape}")
+
+
+@pytest.mark.parametrize("pattern", ["zeros_on_boundaries", "all_ones", "all_zeros", "zero_first"])
+def test_exact_gates(orc, pattern):
+    B, S, dv = 2, 520, 64
+    inp = make_gated_inputs(B, S, 128, dv, "bf16", seed=1950, h0=True)
+    g = inp["gamma"].clone()
+    if pattern == "zeros_on_boundaries":
+        g[:, ::128] = 0.0          # the state is discarded exactly where a chunk starts
+        g[1, 255] = 0.0            # and on a chunk's last token
+    elif pattern == "all_ones":
+        g[:] = 1.0                 # no decay: the state is a running sum
+    elif pattern == "all_zeros":
+        g[:] = 0.0                 # every token stands alone: S_t = k_t v_t^T
+    else:
+        g[:, 0] = 0.0              # the initial state is discarded at once
+    inp["gamma"] = g.contiguous()
+    _check(orc, inp, pattern)
+
+
+def test_chunked_form_chains_through_its_final_state(orc):
+    """Two calls chained through the final state (given back as h0, fp32) equal one
+    call over the whole sequence within the bf16 tolerance (the final state between
+    the calls is rounded to bf16, as the page's output dtype asks)."""
+    inp = make_gated_inputs(2, 700, 128, 64, "bf16", seed=1960)
+    y, fs = _gpu(inp)
+    a = {k: v[:, :384].contiguous() for k, v in inp.items() if v is not None}
+    b = {k: v[:, 384:].contiguous() for k, v in inp.items() if v is not None}
+    ya, fa = _gpu(a)
+    b["h0"] = fa.float()
+    yb, fb = _gpu(b)
+    tol = TOL[torch.bfloat16]
+    assert_close(torch.cat([ya, yb], 1), y.double().numpy(), tol, "outputs")
+    assert_close(fb, fs.double().numpy(), tol, "final_state")
