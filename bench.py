@@ -84,25 +84,37 @@ def decode_work(w=DECODE):
     return {"elems": w.batch * w.channels * w.state_dim, "bytes": bytes_, "exps": exps}
 
 
-def _kernel_source_hash():
+# the sources each kernel's device code is compiled from
+KERNEL_SOURCES = {
+    "ss_scan_fwd_kernel": ("ss_scan_fwd.cuh", "ss_device.cuh", "ss_sync.cuh"),
+    "ss_state_update_stream_kernel": ("ss_state_update.cuh", "ss_device.cuh", "ss_sync.cuh"),
+    "ss_gated_tc_kernel": ("ss_gated_tc.cuh", "ss_device.cuh", "ss_sync.cuh"),
+}
+
+
+def _kernel_source_hash(kernel):
+    """Hash of the sources of `kernel`'s device code (its own header and the shared
+    device headers)."""
     h = hashlib.sha256()
-    for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(CSRC, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in sorted(KERNEL_SOURCES[kernel]):
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
-def _measured_traffic(kernel):
+def _measured_traffic(kernel, launch=None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    current kernel sources (else None)."""
+    current device code of that kernel and, where the entry records one, with the same
+    launch plan (else None)."""
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
     except (OSError, ValueError):
         return None
     entry = rec.get(kernel)
-    if not entry or entry.get("source_hash") != _kernel_source_hash():
+    if not entry or entry.get("source_hash") != _kernel_source_hash(kernel):
+        return None
+    if "launch" in entry and launch is not None and entry["launch"] != launch:
         return None
     return entry.get("dram_bytes_per_launch")
 
@@ -421,7 +433,7 @@ def run_ours(args):
         "hbm_peak_gbs": hbm_gbs,
         "hbm_frac": round(scan_hbm / hbm_gbs, 4),
         "roofline_frac": round(t_roof_scan / scan_s, 4),
-        "traffic": _measured_traffic("ss_scan_fwd_kernel"),
+        "traffic": _measured_traffic("ss_scan_fwd_kernel", {k: plan[k] for k in ("grid", "segments", "seg_len")}),
         "peak_source": f"HBM {peak_kind} (MEASURED_PEAKS.json); SFU measured per clock, at the max clock",
     }
     kernels = {
@@ -493,40 +505,64 @@ def run_e2e(args, dev, stream, inputs, ssscan):
     """Same step through the public API with the per-step inputs in pinned host memory:
     H2D copies of x, dt_raw, z, B, C (both calls), the two kernels, and D2H of y,
     h_last and the decode output, all inside the timed region.  A, D, dt_bias and the
-    decode state (the cache) stay resident on the device."""
+    decode state (the cache) stay resident on the device.
+
+    The steps are pipelined the way a serving loop would run them: step i's inputs go up
+    on a copy stream while step i-1's kernels run on `stream` and step i-2's results come
+    down on a third stream (PCIe is full duplex, and the copy engines are not the SMs).
+    Device input and output buffers are double-buffered; events order each buffer's
+    reuse, so no copy overwrites data a kernel still reads and no kernel overwrites a
+    result before it has reached the host.  The timed region runs from the first H2D
+    copy of the first timed step to the last D2H copy of the last one."""
     p, u = inputs
     per_step = {"p": ("x", "dt", "z", "B", "C"), "u": ("x", "dt", "z", "B", "C")}
     host = {("p", k): p[k].cpu().pin_memory() for k in per_step["p"]}
     host.update({("u", k): u[k].cpu().pin_memory() for k in per_step["u"]})
-    devb = {key: torch.empty_like(t, device=dev) for key, t in host.items()}
-    y = torch.empty_like(p["x"])
-    hl = torch.empty(PROMPT.batch, PROMPT.channels, PROMPT.state_dim, device=dev)
-    yd = torch.empty(DECODE.batch, DECODE.channels, device=dev, dtype=u["x"].dtype)
-    out_host = [torch.empty_like(y, device="cpu").pin_memory(), torch.empty_like(hl, device="cpu").pin_memory(),
-                torch.empty_like(yd, device="cpu").pin_memory()]
+    devb = [{key: torch.empty_like(t, device=dev) for key, t in host.items()} for _ in range(2)]
+    y = [torch.empty_like(p["x"]) for _ in range(2)]
+    hl = [torch.empty(PROMPT.batch, PROMPT.channels, PROMPT.state_dim, device=dev) for _ in range(2)]
+    yd = [torch.empty(DECODE.batch, DECODE.channels, device=dev, dtype=u["x"].dtype) for _ in range(2)]
+    out_host = [[torch.empty_like(t, device="cpu").pin_memory() for t in (y[b], hl[b], yd[b])] for b in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in out_host)
+    d2h = sum(t.numel() * t.element_size() for t in out_host[0])
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
+    uploaded, computed, downloaded = ev(), ev(), ev()
+    used = [False, False]
 
-    def one():
-        for key, t in host.items():
-            devb[key].copy_(t, non_blocking=True)
-        ssscan.ss_scan_fwd(devb[("p", "x")], devb[("p", "dt")], p["A"], devb[("p", "B")], devb[("p", "C")],
-                           p["D"], devb[("p", "z")], p["dt_bias"], None, None, y=y, h_last=hl, stream=stream)
-        ssscan.ss_state_update(u["state"], devb[("u", "x")], devb[("u", "dt")], u["A"], devb[("u", "B")],
-                               devb[("u", "C")], u["D"], devb[("u", "z")], u["dt_bias"], y=yd, stream=stream)
-        out_host[0].copy_(y, non_blocking=True)
-        out_host[1].copy_(hl, non_blocking=True)
-        out_host[2].copy_(yd, non_blocking=True)
+    def one(i):
+        b = i & 1
+        with torch.cuda.stream(up):
+            if used[b]:
+                up.wait_event(computed[b])          # step i-2's kernels are done with devb[b]
+            for key, t in host.items():
+                devb[b][key].copy_(t, non_blocking=True)
+            uploaded[b].record(up)
+        stream.wait_event(uploaded[b])
+        if used[b]:
+            stream.wait_event(downloaded[b])        # step i-2's results have left y[b] ...
+        d = devb[b]
+        ssscan.ss_scan_fwd(d[("p", "x")], d[("p", "dt")], p["A"], d[("p", "B")], d[("p", "C")],
+                           p["D"], d[("p", "z")], p["dt_bias"], None, None, y=y[b], h_last=hl[b], stream=stream)
+        ssscan.ss_state_update(u["state"], d[("u", "x")], d[("u", "dt")], u["A"], d[("u", "B")],
+                               d[("u", "C")], u["D"], d[("u", "z")], u["dt_bias"], y=yd[b], stream=stream)
+        computed[b].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(computed[b])
+            for h, t in zip(out_host[b], (y[b], hl[b], yd[b])):
+                h.copy_(t, non_blocking=True)
+            downloaded[b].record(down)
+        used[b] = True
 
-    for _ in range(2):
-        one()
+    for i in range(2):
+        one(i)
     torch.cuda.synchronize(dev)
     steps = max(3, min(args.steps, args.e2e_steps))
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(stream)
-    for _ in range(steps):
-        one()
-    e.record(stream)
+    s.record(up)
+    for i in range(steps):
+        one(i)
+    e.record(down)
     torch.cuda.synchronize(dev)
     return {"ms_per_step": s.elapsed_time(e) / steps, "h2d": h2d, "d2h": d2h, "steps": steps}
 

@@ -964,7 +964,7 @@ bool encode_bsi(CUtensorMap *map, const void *base, int64_t batch, int64_t seq, 
 }
 
 // The chunked tensor-core form: bf16, dk = 128, dv a multiple of 64, 16-byte aligned
-// rows (the tile loads and the vector stores).
+// rows (the tile loads, the vector loads of h0 and the vector stores).
 bool gated_tc_eligible(const ss::GatedArgs &a, bool bf16)
 {
     const int mode = g_gated_path.load(std::memory_order_relaxed);
@@ -972,7 +972,7 @@ bool gated_tc_eligible(const ss::GatedArgs &a, bool bf16)
         return false;
     return a.dk == ss::kGtDk && a.dv % ss::kGtNv == 0 && a.seq < (int64_t(1) << 31) &&
            a.batch < (int64_t(1) << 31) && aligned(a.q, 16) && aligned(a.k, 16) && aligned(a.v, 16) &&
-           aligned(a.y, 16) && aligned(a.final_state, 16);
+           aligned(a.y, 16) && aligned(a.final_state, 16) && (!a.h0 || aligned(a.h0, 16));
 }
 
 int launch_gated_tc(const ss::GatedArgs &g, cudaStream_t stream)

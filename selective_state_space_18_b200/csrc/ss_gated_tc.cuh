@@ -12,20 +12,37 @@
 //   H'   = P_127 H  +  sum_j w_j k_j v_j^T
 // i.e. four matrix products per chunk:
 //   S  = Q K^T          [128 x 128, K = dk]      scores
-//   Yi = (L o S) V      [128 x 64,  K = 128]     within the chunk
 //   Yh = Q H            [128 x 64,  K = dk]      from the entering state
+//   Yi = (L o S) V      [128 x 64,  K = 128]     within the chunk
 //   dH = K^T (w o V)    [dk x 64,   K = 128]     the state's increment
-// run as tcgen05.mma (bf16 operands staged in shared memory by TMA or by the CUDA
-// cores, fp32 accumulators in tensor memory), and the element-wise parts on the CUDA
-// cores: the decay mask from a block scan of log2(gamma), y = Yi + P o Yh, and the
-// fp32 state H' = P_127 H + dH, which each thread keeps in registers for one row.
-// The decays are exact products in log space: L[i,j] = exp2(sum_{j<s<=i} log2 gamma_s),
-// and exactly 0 where a gate of 0 lies in (j, i] (tracked as the last zero's index).
+// run as tcgen05.mma (bf16 x bf16 -> fp32 accumulators in tensor memory), and the
+// element-wise parts on the CUDA cores: the decay mask from a block scan of the gates,
+// y = Yi + P o Yh, and the fp32 state H' = P_127 H + dH, kept in registers.
 //
-// Precision: the operands of the products are bf16 -- q, k, v exactly (they are bf16
-// inputs); L o S, w o V and H rounded to bf16 -- with fp32 accumulation; the state
-// itself stays fp32.  The result is within the bf16 output tolerance of the fp32
-// recurrence (tested against the float64 oracle); fp32 inputs use the recurrent kernel.
+// Decays.  The gates are scanned in log space with the zero gates and the signs kept
+// apart, so every real gate is taken as the recurrence takes it: lam_i = sum of
+// log2|gamma_s| over s <= i (zero gates add 0), z_i = index of the last zero gate <= i,
+// par_i = parity of the negative gates <= i.  Then L[i,j] = 0 if z_i > j, else
+// (-1)^(par_i ^ par_j) exp2(lam_i - lam_j).  (A gate below the smallest normal float
+// counts as zero: the terms it scales are below 1e-38 of the others.)  For a 32-column
+// block below the diagonal block (every j before every i of the row block) the decay
+// factors through the block's last column j1: L[i,j] = L[i,j1] L[j1,j], one
+// exponential per row and one per column instead of one per element -- used when every
+// gate of the chunk has |gamma| <= 1, so that neither factor can overflow (otherwise
+// every element takes the direct form).
+//
+// Precision.  q, k, v are bf16 inputs and enter the products exactly.  The fp32
+// intermediates that are operands (L o S, w o V and the state H) are each split into a
+// bf16 high part and a bf16 residual (x = hi + lo to about 2^-17 relative), and each of
+// their products runs as two MMAs into the same fp32 accumulator: the result follows
+// fp32 intermediate arithmetic far below the bf16 rounding of the outputs.
+//
+// One CTA: 256 threads, 8 warps; warp w works on tensor-memory lanes 32 (w % 4) .. +31
+// (rows of the scores, outputs and state) and on column half w / 4.  Thread 0 issues the
+// tile loads (TMA) and the MMAs.  The k and v tiles are double-buffered (the next
+// chunk's are in flight during this one); the q tile is reloaded as soon as the
+// products that read it are done.  L o S goes to tensor memory (tcgen05.st) and enters
+// Yi as the A operand from there.
 #pragma once
 
 #include <cuda.h>
@@ -37,27 +54,33 @@ namespace ss {
 constexpr int kGtChunk = 128;   // tokens per chunk (the MMA's M)
 constexpr int kGtDk = 128;      // key size of this kernel
 constexpr int kGtNv = 64;       // value columns per CTA
-constexpr int kGtThreads = 128; // thread i owns score/output row i and state row i
+constexpr int kGtThreads = 256; // 8 warps: lane quarter w % 4, column half w / 4
 constexpr uint32_t kGtTmemCols = 512;
-// tensor-memory columns of the accumulators
-constexpr uint32_t kGtColS = 0, kGtColYi = 128, kGtColYh = 192, kGtColDH = 256;
+// tensor-memory columns: fp32 accumulators S, Yi, Yh, dH; L o S as packed bf16 pairs
+// (high and low parts, 64 columns = 128 elements each)
+constexpr uint32_t kGtColS = 0, kGtColMhi = 128, kGtColMlo = 192, kGtColYi = 256, kGtColYh = 320,
+                   kGtColDH = 384;
 
-// shared memory (bytes from a 1024-byte aligned base): every tile is 128 rows of 128
-// bytes per 64-element block, written with the 128-byte swizzle
+// shared memory (bytes from a 1024-byte aligned base): every tile is rows of 128 bytes
+// per 64-element block, written with the 128-byte swizzle
 struct GtSmem {
-    static constexpr int kQ = 0;              // q chunk: 2 blocks [128 tokens x 64 keys]
-    static constexpr int kK = kQ + 32768;     // k chunk: 2 blocks
-    static constexpr int kV = kK + 32768;     // v chunk: [128 tokens x 64 values]
-    static constexpr int kM = kV + 16384;     // L o S: 2 blocks [128 rows i x 64 cols j]
-    static constexpr int kH = kM + 32768;     // H in bf16: [128 keys x 64 values]
-    static constexpr int kW = kH + 16384;     // w o V: [128 tokens x 64 values]
-    static constexpr int kLam = kW + 16384;   // log2 prefix of the chunk's gates [128] fp32
-    static constexpr int kZ = kLam + 512;     // index of the last zero gate <= i [128] int
-    static constexpr int kRed = kZ + 512;     // block-scan partials [4 warps x 2]
-    static constexpr int kBar = kRed + 64;    // mbarriers: load, mma1, mma2
-    static constexpr int kTmem = kBar + 32;   // tensor-memory base address
+    static constexpr int kQ = 0;                // q chunk: 2 blocks [128 tokens x 64 keys]
+    static constexpr int kK = kQ + 32768;       // k chunk: 2 stages of 2 blocks
+    static constexpr int kV = kK + 2 * 32768;   // v chunk: 2 stages of [128 tokens x 64 values]
+    static constexpr int kHhi = kV + 2 * 16384; // H, high and low bf16 parts: [128 keys x 64 values]
+    static constexpr int kHlo = kHhi + 16384;
+    static constexpr int kWhi = kHlo + 16384;   // w o V, high and low parts: [128 tokens x 64 values]
+    static constexpr int kWlo = kWhi + 16384;
+    static constexpr int kLam = kWlo + 16384;   // lam_j [128] fp32
+    static constexpr int kG = kLam + 512;       // L[j1(j), j] [128] fp32 (column factors)
+    static constexpr int kZ = kG + 512;         // z_j [128] int
+    static constexpr int kSg = kZ + 512;        // (-1)^par_j [128] fp32
+    static constexpr int kRed = kSg + 512;      // per lane quarter: log sum, last zero, parity, |gamma| > 1
+    static constexpr int kBar = kRed + 64;      // mbarriers: q, kv[2], s, yh, mma2
+    static constexpr int kTmem = kBar + 64;     // tensor-memory base address
     static constexpr int kBytes = kTmem + 16 + 1024; // + alignment slack
 };
+static_assert(GtSmem::kBytes <= 227 * 1024, "shared memory of the gated tensor-core kernel");
 
 struct GatedTcArgs {
     int64_t batch, seq, dv;
@@ -65,7 +88,7 @@ struct GatedTcArgs {
     const float *h0;          // [batch, dk, dv] or null
     __nv_bfloat16 *y;         // [batch, seq, dv]
     __nv_bfloat16 *final_state; // [batch, dk, dv]
-    int col_tiles;            // ceil(dv / 64)
+    int col_tiles;            // dv / 64
 };
 
 struct GatedTcMaps {
@@ -100,6 +123,16 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
                  "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
                  : "memory");
 }
+// D[tmem] (+)= A[tmem] B[smem]: A is M x 16 with row m in lane m and its 16 bf16
+// elements packed in pairs (lower index in the low half) into 8 columns from a_tmem.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
 // Arrive on `bar` once every MMA this thread issued before has completed.
 __device__ __forceinline__ void umma_commit(uint64_t *bar)
 {
@@ -126,6 +159,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
     for (int i = 0; i < 32; ++i)
         v[i] = __uint_as_float(r[i]);
 }
+
+// 16 consecutive 32-bit columns of this warp's 32 lanes from registers (thread t writes
+// lane (warp's first lane + t)); complete once tmem_st_wait returns.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+                 "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+                 "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor (the tcgen05 "smem descriptor"): start address, leading
 // and stride byte offsets (all in 16-byte units), version 1, the 128-byte swizzle
@@ -163,255 +208,386 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
                  : "memory");
 }
 
-// One CTA per (batch item, 64-column value tile); 128 threads; thread 0 issues the
-// tile loads and the MMAs.  `status` records a timeout of a bounded wait.
+// x = hi + lo with hi = bf16(x) and lo = bf16(x - hi), for a pair of values, as packed
+// pairs (element 0 in the low half).  x - hi is exact in fp32.
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t &hi, uint32_t &lo)
+{
+    hi = pack_bf16x2(x0, x1);
+    lo = pack_bf16x2(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xffff0000u));
+}
+
+// The 8 bf16 values of a 16-byte chunk, scaled by w, split into high and low parts.
+__device__ __forceinline__ void scale_split8(uint4 v, float w, uint4 &hi, uint4 &lo)
+{
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        split_bf16x2(__uint_as_float(in[e] << 16) * w, __uint_as_float(in[e] & 0xffff0000u) * w, h[e], l[e]);
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// One CTA per (batch item, 64-column value tile).  `status` records a timeout of a
+// bounded wait.
 __global__ void __launch_bounds__(kGtThreads, 1)
 ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps, uint32_t *status)
 {
     extern __shared__ unsigned char gt_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(gt_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + GtSmem::kBar);
-    uint64_t *bar_load = bars, *bar_mma1 = bars + 1, *bar_mma2 = bars + 2;
+    uint64_t *bar_q = bars, *bar_kv = bars + 1 /* [2] */, *bar_s = bars + 3, *bar_yh = bars + 4, *bar_2 = bars + 5;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + GtSmem::kTmem);
     float *s_lam = reinterpret_cast<float *>(sm + GtSmem::kLam);
+    float *s_g = reinterpret_cast<float *>(sm + GtSmem::kG);
     int *s_z = reinterpret_cast<int *>(sm + GtSmem::kZ);
-    float *s_red = reinterpret_cast<float *>(sm + GtSmem::kRed);
+    float *s_sg = reinterpret_cast<float *>(sm + GtSmem::kSg);
+    uint32_t *s_red = reinterpret_cast<uint32_t *>(sm + GtSmem::kRed);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q4 = warp & 3, half = warp >> 2;
+    const int r = 32 * q4 + lane; // this thread's row: a token of the chunk, a key of the state
     const int64_t b = blockIdx.x / a.col_tiles;
     const int n0 = int(blockIdx.x % a.col_tiles) * kGtNv;
     const int64_t nchunks = (a.seq + kGtChunk - 1) / kGtChunk;
     const uint32_t s_base = smem_u32(sm);
 
     if (tid == 0) {
-        mbar_init(bar_load, 1);
-        mbar_init(bar_mma1, 1);
-        mbar_init(bar_mma2, 1);
+        mbar_init(bar_q, 1);
+        mbar_init(bar_kv, 1);
+        mbar_init(bar_kv + 1, 1);
+        mbar_init(bar_s, 1);
+        mbar_init(bar_yh, 1);
+        mbar_init(bar_2, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, kGtTmemCols);
         tmem_relinquish();
     }
-    // the entering state: this thread's row d = tid, fp32, in registers
-    float H[kGtNv];
+    // the entering state: key row r, value columns 32 half .. +31 of the tile, fp32
+    float H[32];
+    {
+        const float *src = a.h0 ? a.h0 + (b * kGtDk + r) * a.dv + n0 + 32 * half : nullptr;
 #pragma unroll
-    for (int n = 0; n < kGtNv; ++n) {
-        const int col = n0 + n;
-        H[n] = (a.h0 && col < a.dv) ? __ldg(a.h0 + (b * kGtDk + tid) * a.dv + col) : 0.0f;
+        for (int e = 0; e < 32; e += 4) {
+            const float4 v = src ? __ldg(reinterpret_cast<const float4 *>(src + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            H[e] = v.x;
+            H[e + 1] = v.y;
+            H[e + 2] = v.z;
+            H[e + 3] = v.w;
+        }
     }
-    // and its bf16 copy, the B operand of Q H
+    // and its high and low bf16 parts, the B operands of Q H
     auto store_h = [&]() {
 #pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) {
-            const float *h = H + 8 * c16;
-            *reinterpret_cast<uint4 *>(sm + GtSmem::kH + sw128_off(tid, c16)) =
-                make_uint4(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]),
-                           pack_bf16x2(h[6], h[7]));
+        for (int cc = 0; cc < 4; ++cc) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                split_bf16x2(H[8 * cc + 2 * e], H[8 * cc + 2 * e + 1], hi[e], lo[e]);
+            const uint32_t off = sw128_off(r, 4 * half + cc);
+            *reinterpret_cast<uint4 *>(sm + GtSmem::kHhi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4 *>(sm + GtSmem::kHlo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
     };
     store_h();
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); // generic writes -> MMA reads
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
-    const uint32_t lane_base = uint32_t(32 * warp) << 16; // this warp's tensor-memory lanes
+    const uint32_t lane_base = uint32_t(32 * q4) << 16; // this warp's tensor-memory lanes
+    // L o S is 0 above the diagonal in every chunk: those blocks of its tensor-memory
+    // copy are written once, here, and never again
+#pragma unroll
+    for (int bb = 0; bb < 2; ++bb) {
+        const int jb = 2 * half + bb;
+        if (jb > q4) {
+            const uint32_t zero[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+            tmem_st16(tmem + lane_base + kGtColMhi + 16 * jb, zero);
+            tmem_st16(tmem + lane_base + kGtColMlo + 16 * jb, zero);
+        }
+    }
+    tmem_st_wait();
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); // H writes -> MMA reads
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
 
-    constexpr uint32_t kLoadBytes = 2 * 16384 + 2 * 16384 + 16384;
-    auto issue_loads = [&](int64_t c) {
-        mbar_arrive_expect_tx(bar_load, kLoadBytes);
-        const int32_t t0 = int32_t(c * kGtChunk), bb = int32_t(b);
-        tma_load_3d(sm + GtSmem::kQ, &maps.q, 0, t0, bb, bar_load);
-        tma_load_3d(sm + GtSmem::kQ + 16384, &maps.q, 64, t0, bb, bar_load);
-        tma_load_3d(sm + GtSmem::kK, &maps.k, 0, t0, bb, bar_load);
-        tma_load_3d(sm + GtSmem::kK + 16384, &maps.k, 64, t0, bb, bar_load);
-        tma_load_3d(sm + GtSmem::kV, &maps.v, n0, t0, bb, bar_load);
+    const int32_t b32 = int32_t(b);
+    auto issue_q = [&](int64_t c) {
+        mbar_arrive_expect_tx(bar_q, 32768);
+        const int32_t t0 = int32_t(c * kGtChunk);
+        tma_load_3d(sm + GtSmem::kQ, &maps.q, 0, t0, b32, bar_q);
+        tma_load_3d(sm + GtSmem::kQ + 16384, &maps.q, 64, t0, b32, bar_q);
     };
+    auto issue_kv = [&](int64_t c) {
+        const int st = int(c & 1);
+        mbar_arrive_expect_tx(bar_kv + st, 32768 + 16384);
+        const int32_t t0 = int32_t(c * kGtChunk);
+        tma_load_3d(sm + GtSmem::kK + st * 32768, &maps.k, 0, t0, b32, bar_kv + st);
+        tma_load_3d(sm + GtSmem::kK + st * 32768 + 16384, &maps.k, 64, t0, b32, bar_kv + st);
+        tma_load_3d(sm + GtSmem::kV + st * 16384, &maps.v, n0, t0, b32, bar_kv + st);
+    };
+    // thread 0's record of the asynchronous work (phases issued and phases waited for,
+    // per barrier), for draining after a timeout
+    int64_t nq_issued = 0, nq_waited = 0, nkv0_issued = 0, nkv1_issued = 0, nkv0_waited = 0, nkv1_waited = 0;
+    int64_t ns_committed = 0, ns_waited = 0, nyh_committed = 0, nyh_waited = 0, n2_committed = 0, n2_waited = 0;
     if (tid == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.q)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.k)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.v)) : "memory");
-        issue_loads(0);
+        issue_q(0);
+        nq_issued = 1;
+        issue_kv(0);
+        nkv0_issued = 1;
+        if (nchunks > 1) {
+            issue_kv(1);
+            nkv1_issued = 1;
+        }
     }
 
-    // (thread 0's record of the asynchronous work in flight, for draining after a timeout)
-    int64_t loads_issued = tid == 0 ? 1 : 0, loads_done = 0, mma_issued = 0, mma_done = 0;
-    constexpr uint32_t kIdS = idesc_bf16(128, 128, 0, 0);  // Q (K-major) x K (K-major)
-    constexpr uint32_t kIdY = idesc_bf16(128, kGtNv, 0, 1); // (L o S) or Q (K-major) x V or H (MN-major)
+    constexpr uint32_t kIdS = idesc_bf16(128, 128, 0, 0);   // Q (K-major) x K (K-major)
+    constexpr uint32_t kIdY = idesc_bf16(128, kGtNv, 0, 1); // Q or L o S (K-major) x H or V (MN-major)
     constexpr uint32_t kIdH = idesc_bf16(128, kGtNv, 1, 1); // K^T (MN-major) x (w o V) (MN-major)
+    constexpr float kTiny = 1.17549435e-38f;                // smallest normal float
+    const float *gam = a.gamma + b * a.seq;
+    float gm_next = r < a.seq ? __ldg(gam + r) : 1.0f; // past the end: no decay
     bool ok = true;
     for (int64_t c = 0; c < nchunks && ok; ++c) {
-        const uint32_t ph = uint32_t(c & 1);
+        const int st = int(c & 1);
+        const uint32_t ph = uint32_t(c & 1), ph_kv = uint32_t((c >> 1) & 1);
         const int64_t t0 = c * kGtChunk;
-        // ---- gates: block scan of log2(gamma) and of the last zero gate --------------
-        const int64_t t = t0 + tid;
-        const float gm = t < a.seq ? __ldg(a.gamma + b * a.seq + t) : 1.0f; // past the end: no decay
-        float lg = gm > 0.0f ? __log2f(gm) : 0.0f;
-        int zl = gm == 0.0f ? tid : -1;
+        // ---- gates: scans of log2|gamma|, of the last zero gate and of the sign parity
+        // over this lane quarter's 32 tokens (both column halves compute the same) -------
+        const float gm = gm_next;
+        gm_next = t0 + kGtChunk + r < a.seq ? __ldg(gam + t0 + kGtChunk + r) : 1.0f; // the next chunk's
+        const bool zero_gate = fabsf(gm) < kTiny;
+        float lg = zero_gate ? 0.0f : __log2f(fabsf(gm));
+        int zl = zero_gate ? r : -1;
+        uint32_t par = (!zero_gate && gm < 0.0f) ? 1u : 0u;
+        const uint32_t big = __any_sync(0xffffffffu, !(fabsf(gm) <= 1.0f)) ? 1u : 0u; // |gamma| > 1, or NaN
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float up = __shfl_up_sync(0xffffffffu, lg, o);
             const int uz = __shfl_up_sync(0xffffffffu, zl, o);
+            const uint32_t upar = __shfl_up_sync(0xffffffffu, par, o);
             if (lane >= o) {
                 lg += up;
                 zl = max(zl, uz);
+                par ^= upar;
             }
         }
-        if (lane == 31) {
-            s_red[2 * warp] = lg;
-            s_red[2 * warp + 1] = __int_as_float(zl);
+        if (half == 0 && lane == 31) {
+            s_red[4 * q4] = __float_as_uint(lg);
+            s_red[4 * q4 + 1] = uint32_t(zl);
+            s_red[4 * q4 + 2] = par;
+            s_red[4 * q4 + 3] = big;
         }
-        // ---- the chunk's tiles (every thread observes the load), then S = Q K^T and
-        // Yh = Q H ------------------------------------------------------------------------
-        if (!mbar_wait(bar_load, ph, status))
+        // ---- the chunk's tiles, then (thread 0) S = Q K^T and Yh = Q H ----------------
+        if (!mbar_wait(bar_q, ph, status) || !mbar_wait(bar_kv + st, ph_kv, status))
             ok = false;
-        else if (tid == 0)
-            loads_done = c + 1;
         if (tid == 0 && ok) {
-            {
-                tc_fence_after();
+            nq_waited = c + 1;
+            (st ? nkv1_waited : nkv0_waited) = (c >> 1) + 1;
+            tc_fence_after();
+            const uint32_t qb = s_base + GtSmem::kQ, kb = s_base + GtSmem::kK + st * 32768;
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) { // K = 128 keys in slices of 16
-                    const uint32_t qa = s_base + GtSmem::kQ + (ks >> 2) * 16384 + (ks & 3) * 32;
-                    const uint32_t ka = s_base + GtSmem::kK + (ks >> 2) * 16384 + (ks & 3) * 32;
-                    umma_bf16(tmem + kGtColS, sw128_desc(qa, 16, 1024), sw128_desc(ka, 16, 1024), kIdS, ks > 0);
-                    const uint32_t ha = s_base + GtSmem::kH + ks * 2048; // 16 key rows of H
-                    umma_bf16(tmem + kGtColYh, sw128_desc(qa, 16, 1024), sw128_desc(ha, 16384, 1024), kIdY, ks > 0);
-                }
-                umma_commit(bar_mma1);
-                mma_issued = c + 1;
+            for (int ks = 0; ks < 8; ++ks) { // K = 128 keys in slices of 16
+                const uint32_t o = (ks >> 2) * 16384 + (ks & 3) * 32;
+                umma_bf16(tmem + kGtColS, sw128_desc(qb + o, 16, 1024), sw128_desc(kb + o, 16, 1024), kIdS, ks > 0);
             }
-        }
-        __syncthreads();
-        {
-            float off = 0.0f;
-            int zoff = -1;
-            for (int w = 0; w < warp; ++w) {
-                off += s_red[2 * w];
-                zoff = max(zoff, __float_as_int(s_red[2 * w + 1]));
+            umma_commit(bar_s);
+            ns_committed = c + 1;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t qd = sw128_desc(qb + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                const uint32_t ho = ks * 2048; // 16 key rows of H
+                umma_bf16(tmem + kGtColYh, qd, sw128_desc(s_base + GtSmem::kHhi + ho, 16384, 1024), kIdY, ks > 0);
+                umma_bf16(tmem + kGtColYh, qd, sw128_desc(s_base + GtSmem::kHlo + ho, 16384, 1024), kIdY, 1);
             }
-            lg += off;
-            zl = max(zl, zoff);
-            s_lam[tid] = lg;
-            s_z[tid] = zl;
+            umma_commit(bar_yh);
+            nyh_committed = c + 1;
         }
-        if (!__syncthreads_and(ok ? 1 : 0)) { // thread 0 could not get the tiles
+        if (!__syncthreads_and(ok ? 1 : 0)) {
             ok = false;
             break;
         }
-        const float lam_i = lg;
-        const int z_i = zl;
-        const float p_i = z_i >= 0 ? 0.0f : ex2(lam_i);                 // P_i
-        const float lam_end = s_lam[kGtChunk - 1];
-        const int z_end = s_z[kGtChunk - 1];
-        const float p_end = z_end >= 0 ? 0.0f : ex2(lam_end);           // P_127
-        // ---- w o V: thread j scales row j of v by w_j ---------------------------------
+        // ---- prefixes over the chunk for this row, and the chunk's totals --------------
+        float off = 0.0f;
+        int zoff = -1, z_end = -1;
+        uint32_t poff = 0, par_end = 0, any_big = 0;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const int wz = int(s_red[4 * w + 1]);
+            const uint32_t wp = s_red[4 * w + 2];
+            if (w < q4) {
+                off += __uint_as_float(s_red[4 * w]);
+                zoff = max(zoff, wz);
+                poff ^= wp;
+            }
+            z_end = max(z_end, wz);
+            par_end ^= wp;
+            any_big |= s_red[4 * w + 3];
+        }
+        const float lam_r = lg + off;
+        const int z_r = max(zl, zoff);
+        const uint32_t par_r = par ^ poff;
+        const float sg_r = par_r ? -1.0f : 1.0f;
+        // lam of token 127, summed in the order its own row prefix was
+        const float lam_end = __uint_as_float(s_red[12]) +
+                              ((__uint_as_float(s_red[0]) + __uint_as_float(s_red[4])) + __uint_as_float(s_red[8]));
+        if (half == 0) {
+            // the column factor L[j1, r], j1 the last token of this lane quarter
+            const float lam_j1 = __uint_as_float(s_red[4 * q4]) + off;
+            const int z_j1 = max(int(s_red[4 * q4 + 1]), zoff);
+            const uint32_t par_j1 = s_red[4 * q4 + 2] ^ poff;
+            s_lam[r] = lam_r;
+            s_z[r] = z_r;
+            s_sg[r] = sg_r;
+            s_g[r] = z_j1 > r ? 0.0f : ((par_j1 ^ par_r) ? -1.0f : 1.0f) * ex2(lam_j1 - lam_r);
+        }
+        const float p_r = z_r >= 0 ? 0.0f : sg_r * ex2(lam_r);                             // P_r
+        const float p_end = z_end >= 0 ? 0.0f : (par_end ? -1.0f : 1.0f) * ex2(lam_end);  // P_127
+        __syncthreads();
+        // ---- w o V: token row r, this half's 32 value columns, as high / low parts ----
         {
-            const float w_j = z_end > tid ? 0.0f : ex2(lam_end - lam_i);
+            const float w_r = z_end > r ? 0.0f : ((par_end ^ par_r) ? -1.0f : 1.0f) * ex2(lam_end - lam_r);
 #pragma unroll
-            for (int c16 = 0; c16 < 8; ++c16) {
-                const uint4 vv = *reinterpret_cast<const uint4 *>(sm + GtSmem::kV + sw128_off(tid, c16));
-                const uint32_t in[4] = {vv.x, vv.y, vv.z, vv.w};
-                uint32_t out[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    out[e] = pack_bf16x2(__uint_as_float(in[e] << 16) * w_j, __uint_as_float(in[e] & 0xffff0000u) * w_j);
-                *reinterpret_cast<uint4 *>(sm + GtSmem::kW + sw128_off(tid, c16)) =
-                    make_uint4(out[0], out[1], out[2], out[3]);
+            for (int cc = 0; cc < 4; ++cc) {
+                const uint32_t o = sw128_off(r, 4 * half + cc);
+                uint4 hi, lo;
+                scale_split8(*reinterpret_cast<const uint4 *>(sm + GtSmem::kV + st * 16384 + o), w_r, hi, lo);
+                *reinterpret_cast<uint4 *>(sm + GtSmem::kWhi + o) = hi;
+                *reinterpret_cast<uint4 *>(sm + GtSmem::kWlo + o) = lo;
             }
         }
-        // ---- L o S: thread i masks and decays row i of the scores -------------------
-        if (!mbar_wait(bar_mma1, ph, status)) {
+        // ---- L o S: row r, this half's 64 columns, into tensor memory -----------------
+        if (!mbar_wait(bar_s, ph, status))
             ok = false;
-        }
+        else if (tid == 0)
+            ns_waited = c + 1;
+        ok = __all_sync(0xffffffffu, ok); // the tensor-memory accesses below are warp-collective
         tc_fence_after();
         if (ok) {
 #pragma unroll 1
-            for (int jb = 0; jb < 4; ++jb) { // 32 columns at a time
+            for (int bb = 0; bb < 2; ++bb) {
+                const int jb = 2 * half + bb;
+                if (jb > q4)
+                    continue; // above the diagonal: the zeros written once
                 float s[32];
                 tmem_ld32(tmem + lane_base + kGtColS + 32 * jb, s);
+                uint32_t hi[16], lo[16];
+                if (jb < q4 && !any_big) {
+                    // below the diagonal block: L[r, j] = L[r, j1] L[j1, j]
+                    const int j1 = 32 * jb + 31;
+                    const float f = z_r > j1 ? 0.0f : sg_r * s_sg[j1] * ex2(lam_r - s_lam[j1]);
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    float m[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int j = 32 * jb + 8 * q8 + e;
-                        const bool valid = j <= tid && z_i <= j;
-                        m[e] = valid ? s[8 * q8 + e] * ex2(lam_i - s_lam[j]) : 0.0f;
+                    for (int e = 0; e < 32; e += 4) {
+                        const float4 g = *reinterpret_cast<const float4 *>(s_g + 32 * jb + e);
+                        split_bf16x2(s[e] * g.x * f, s[e + 1] * g.y * f, hi[e / 2], lo[e / 2]);
+                        split_bf16x2(s[e + 2] * g.z * f, s[e + 3] * g.w * f, hi[e / 2 + 1], lo[e / 2 + 1]);
                     }
-                    const int j0 = 32 * jb + 8 * q8;
-                    *reinterpret_cast<uint4 *>(sm + GtSmem::kM + (j0 >> 6) * 16384 + sw128_off(tid, (j0 & 63) >> 3)) =
-                        make_uint4(pack_bf16x2(m[0], m[1]), pack_bf16x2(m[2], m[3]), pack_bf16x2(m[4], m[5]),
-                                   pack_bf16x2(m[6], m[7]));
+                } else {
+                    // the diagonal block (or a chunk with gates above 1 in magnitude):
+                    // element by element
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                        const int j = 32 * jb + e;
+                        const float4 lj = *reinterpret_cast<const float4 *>(s_lam + j);
+                        const float4 sj = *reinterpret_cast<const float4 *>(s_sg + j);
+                        const float ljv[4] = {lj.x, lj.y, lj.z, lj.w}, sjv[4] = {sj.x, sj.y, sj.z, sj.w};
+                        float m[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const bool valid = j + u <= r && z_r <= j + u;
+                            m[u] = valid ? s[e + u] * (sg_r * sjv[u]) * ex2(lam_r - ljv[u]) : 0.0f;
+                        }
+                        split_bf16x2(m[0], m[1], hi[e / 2], lo[e / 2]);
+                        split_bf16x2(m[2], m[3], hi[e / 2 + 1], lo[e / 2 + 1]);
+                    }
+                }
+                tmem_st16(tmem + lane_base + kGtColMhi + 16 * jb, hi);
+                tmem_st16(tmem + lane_base + kGtColMlo + 16 * jb, lo);
+            }
+            tmem_st_wait();
+        }
+        // the q tile is free once Q H is done (long done by now): the next chunk's q
+        if (tid == 0 && ok) {
+            if (!mbar_wait(bar_yh, ph, status)) {
+                ok = false;
+            } else {
+                nyh_waited = c + 1;
+                if (c + 1 < nchunks) {
+                    issue_q(c + 1);
+                    nq_issued = c + 2;
                 }
             }
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); // w o V writes -> MMA reads
         tc_fence_before();
         if (!__syncthreads_and(ok ? 1 : 0)) {
             ok = false;
             break;
         }
-        // ---- Yi = (L o S) V and dH = K^T (w o V) ---------------------------------------
+        // ---- Yi = (L o S) V and dH = K^T (w o V), each over high + low parts -----------
         if (tid == 0) {
             tc_fence_after();
+            const uint32_t vb = s_base + GtSmem::kV + st * 16384, kb = s_base + GtSmem::kK + st * 32768;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) { // K = 128 tokens in slices of 16
-                const uint32_t ma = s_base + GtSmem::kM + (ks >> 2) * 16384 + (ks & 3) * 32;
-                const uint32_t va = s_base + GtSmem::kV + ks * 2048;
-                umma_bf16(tmem + kGtColYi, sw128_desc(ma, 16, 1024), sw128_desc(va, 16384, 1024), kIdY, ks > 0);
-                const uint32_t kt = s_base + GtSmem::kK + ks * 2048; // keys x 16 tokens (MN-major)
-                const uint32_t wa = s_base + GtSmem::kW + ks * 2048;
-                umma_bf16(tmem + kGtColDH, sw128_desc(kt, 16384, 1024), sw128_desc(wa, 16384, 1024), kIdH, ks > 0);
+                const uint64_t vd = sw128_desc(vb + ks * 2048, 16384, 1024);
+                umma_bf16_ts(tmem + kGtColYi, tmem + kGtColMhi + 8 * ks, vd, kIdY, ks > 0);
+                umma_bf16_ts(tmem + kGtColYi, tmem + kGtColMlo + 8 * ks, vd, kIdY, 1);
+                const uint64_t kd = sw128_desc(kb + ks * 2048, 16384, 1024); // keys x 16 tokens (MN-major)
+                umma_bf16(tmem + kGtColDH, kd, sw128_desc(s_base + GtSmem::kWhi + ks * 2048, 16384, 1024), kIdH,
+                          ks > 0);
+                umma_bf16(tmem + kGtColDH, kd, sw128_desc(s_base + GtSmem::kWlo + ks * 2048, 16384, 1024), kIdH, 1);
             }
-            umma_commit(bar_mma2);
+            umma_commit(bar_2);
+            n2_committed = c + 1;
         }
-        if (!mbar_wait(bar_mma2, ph, status))
+        if (!mbar_wait(bar_2, ph, status))
             ok = false;
         else if (tid == 0)
-            mma_done = c + 1;
+            n2_waited = c + 1;
+        ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
-        // the chunk's tiles are free: start the next chunk's loads now
-        if (tid == 0 && ok && c + 1 < nchunks) {
-            issue_loads(c + 1);
-            loads_issued = c + 2;
+        // this chunk's k / v stage is free: the chunk after next goes there
+        if (tid == 0 && ok && c + 2 < nchunks) {
+            issue_kv(c + 2);
+            (st ? nkv1_issued : nkv0_issued) = (c >> 1) + 2;
         }
         if (ok) {
-            // ---- y = Yi + P o Yh for this thread's row i ----------------------------------
-            const bool row_ok = t0 + tid < a.seq;
-#pragma unroll 1
-            for (int nb = 0; nb < 2; ++nb) {
+            // ---- y = Yi + P o Yh: row r, this half's 32 columns ---------------------------
+            {
                 float yi[32], yh[32];
-                tmem_ld32(tmem + lane_base + kGtColYi + 32 * nb, yi);
-                tmem_ld32(tmem + lane_base + kGtColYh + 32 * nb, yh);
-                if (row_ok) {
-                    __nv_bfloat16 *dst = a.y + (b * a.seq + t0 + tid) * a.dv + n0 + 32 * nb;
+                tmem_ld32(tmem + lane_base + kGtColYi + 32 * half, yi);
+                tmem_ld32(tmem + lane_base + kGtColYh + 32 * half, yh);
+                if (t0 + r < a.seq) {
+                    __nv_bfloat16 *dst = a.y + (b * a.seq + t0 + r) * a.dv + n0 + 32 * half;
 #pragma unroll
                     for (int q8 = 0; q8 < 4; ++q8) {
                         float o[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
-                            o[e] = fmaf(p_i, yh[8 * q8 + e], yi[8 * q8 + e]);
-                        const int col = n0 + 32 * nb + 8 * q8;
-                        if (col + 8 <= a.dv)
-                            *reinterpret_cast<uint4 *>(dst + 8 * q8) =
-                                make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
-                                           pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+                            o[e] = fmaf(p_r, yh[8 * q8 + e], yi[8 * q8 + e]);
+                        *reinterpret_cast<uint4 *>(dst + 8 * q8) =
+                            make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                                       pack_bf16x2(o[6], o[7]));
                     }
                 }
             }
-            // ---- H' = P_127 H + dH for this thread's key row ------------------------------
-#pragma unroll
-            for (int nb = 0; nb < 2; ++nb) {
+            // ---- H' = P_127 H + dH: key row r, this half's 32 columns ---------------------
+            {
                 float dh[32];
-                tmem_ld32(tmem + lane_base + kGtColDH + 32 * nb, dh);
+                tmem_ld32(tmem + lane_base + kGtColDH + 32 * half, dh);
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
-                    H[32 * nb + e] = fmaf(p_end, H[32 * nb + e], dh[e]);
+                    H[e] = fmaf(p_end, H[e], dh[e]);
             }
             store_h();
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); // H writes -> MMA reads
         tc_fence_before();
         if (!__syncthreads_and(ok ? 1 : 0)) {
             ok = false;
@@ -419,23 +595,28 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
         }
     }
     if (ok) {
+        __nv_bfloat16 *dst = a.final_state + (b * kGtDk + r) * a.dv + n0 + 32 * half;
 #pragma unroll
-        for (int n = 0; n < kGtNv; n += 2) {
-            const int col = n0 + n;
-            if (col < a.dv) {
-                __nv_bfloat16 *dst = a.final_state + (b * kGtDk + tid) * a.dv + col;
-                *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(H[n], H[n + 1]);
-            }
+        for (int q8 = 0; q8 < 4; ++q8) {
+            const float *h = H + 8 * q8;
+            *reinterpret_cast<uint4 *>(dst + 8 * q8) = make_uint4(
+                pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
         }
     } else if (tid == 0) {
         // a wait gave up: let the loads and MMAs still in flight finish (the drain waits
         // keep the default limit) before the tensor memory is freed
-        if (loads_issued > loads_done)
-            mbar_wait(bar_load, uint32_t((loads_issued - 1) & 1), nullptr);
-        if (mma_issued > mma_done) {
-            mbar_wait(bar_mma1, uint32_t((mma_issued - 1) & 1), nullptr);
-            mbar_wait(bar_mma2, uint32_t((mma_issued - 1) & 1), nullptr);
-        }
+        if (nq_issued > nq_waited)
+            mbar_wait(bar_q, uint32_t((nq_issued - 1) & 1), nullptr);
+        if (nkv0_issued > nkv0_waited)
+            mbar_wait(bar_kv, uint32_t((nkv0_issued - 1) & 1), nullptr);
+        if (nkv1_issued > nkv1_waited)
+            mbar_wait(bar_kv + 1, uint32_t((nkv1_issued - 1) & 1), nullptr);
+        if (ns_committed > ns_waited)
+            mbar_wait(bar_s, uint32_t((ns_committed - 1) & 1), nullptr);
+        if (nyh_committed > nyh_waited)
+            mbar_wait(bar_yh, uint32_t((nyh_committed - 1) & 1), nullptr);
+        if (n2_committed > n2_waited)
+            mbar_wait(bar_2, uint32_t((n2_committed - 1) & 1), nullptr);
     }
     tc_fence_before();
     __syncthreads();

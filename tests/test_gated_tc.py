@@ -59,11 +59,16 @@ def test_chunked_form_matches_oracle(orc, shape, h0):
     _check(orc, inp, f"{shape}")
 
 
-@pytest.mark.parametrize("pattern", ["zeros_on_boundaries", "all_ones", "all_zeros", "zero_first"])
+@pytest.mark.parametrize("pattern", ["zeros_on_boundaries", "all_ones", "all_zeros", "zero_first", "negative",
+                                     "above_one", "tiny"])
 def test_exact_gates(orc, pattern):
+    """Gates the decay mask must take exactly as the recurrence does: zeros (the state
+    is discarded), ones, negative gates (signs of the products), magnitudes above 1 (the
+    element-by-element form of the mask) and gates below the smallest normal float."""
     B, S, dv = 2, 520, 64
     inp = make_gated_inputs(B, S, 128, dv, "bf16", seed=1950, h0=True)
     g = inp["gamma"].clone()
+    gen = torch.Generator().manual_seed(1951)
     if pattern == "zeros_on_boundaries":
         g[:, ::128] = 0.0          # the state is discarded exactly where a chunk starts
         g[1, 255] = 0.0            # and on a chunk's last token
@@ -71,9 +76,18 @@ def test_exact_gates(orc, pattern):
         g[:] = 1.0                 # no decay: the state is a running sum
     elif pattern == "all_zeros":
         g[:] = 0.0                 # every token stands alone: S_t = k_t v_t^T
-    else:
+    elif pattern == "zero_first":
         g[:, 0] = 0.0              # the initial state is discarded at once
-    inp["gamma"] = g.contiguous()
+    elif pattern == "negative":
+        flip = torch.rand(g.shape, generator=gen) < 0.3
+        g = torch.where(flip, -g, g)  # about a third of the gates negative
+        g[0, 130] = -1.0
+    elif pattern == "above_one":
+        g = 0.9 + 0.2 * torch.rand(g.shape, generator=gen)  # |gamma| in [0.9, 1.1]
+        g[1, 300:310] = 1.5
+    else:
+        g[:, 5::37] = 1e-39        # subnormal gates: the terms they scale vanish
+    inp["gamma"] = g.float().contiguous()
     _check(orc, inp, pattern)
 
 
