@@ -222,25 +222,36 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
     uint64_t *empty = full + kDecStages;
     const int tid = threadIdx.x, lane_q = tid & (Q - 1);
 
-    // the k-th tile of this CTA: batch row b, channel block cb (false past the end)
-    auto tile_of = [&](int64_t k, int64_t &b, int64_t &cb) -> bool {
-        if (da.fixed_cb) {
-            cb = blockIdx.x % da.ncb;
-            b = blockIdx.x / da.ncb + k * (gridDim.x / da.ncb);
-        } else {
-            const int64_t t = blockIdx.x + k * gridDim.x;
-            b = t / da.ncb;
-            cb = t - b * da.ncb;
+    // Tile k of this CTA is tile blockIdx.x + k * gridDim.x of the (batch row, channel
+    // block) order; walked incrementally, without a division per tile.  (With fixed_cb
+    // the grid is a multiple of the channel blocks, so the CTA keeps its channel block.)
+    struct TileWalk {
+        int64_t b, cb, db, dcb, ncb;
+        __device__ __forceinline__ void start(int64_t n)
+        {
+            ncb = n;
+            b = int64_t(blockIdx.x) / n;
+            cb = int64_t(blockIdx.x) - b * n;
+            db = int64_t(gridDim.x) / n;
+            dcb = int64_t(gridDim.x) - db * n;
         }
-        return b < p.batch;
+        __device__ __forceinline__ void next()
+        {
+            b += db;
+            cb += dcb;
+            if (cb >= ncb) {
+                cb -= ncb;
+                ++b;
+            }
+        }
     };
     auto nchan = [&](int64_t cb) -> int64_t {
         const int64_t rest = p.channels - cb * D::kChanPerTile;
         return rest < D::kChanPerTile ? rest : D::kChanPerTile;
     };
-    auto issue = [&](int64_t k, int stage) -> bool {
-        int64_t b, cb;
-        if (!tile_of(k, b, cb))
+    auto issue = [&](const TileWalk &w, int stage) -> bool {
+        const int64_t b = w.b, cb = w.cb;
+        if (b >= p.batch)
             return false;
         const int64_t nch = nchan(cb), row0 = b * p.channels + cb * D::kChanPerTile;
         const uint32_t sbytes = uint32_t(nch * N * 4), vbytes = uint32_t(nch * int64_t(sizeof(T)));
@@ -283,7 +294,9 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
         // the copy-issuing warp: tile k goes into stage k % kDecStages once the
         // consumers have released tile k - kDecStages
         if (tid == kDecThreads) {
-            for (int64_t k = 0;; ++k) {
+            TileWalk w;
+            w.start(da.ncb);
+            for (int64_t k = 0;; ++k, w.next()) {
                 const int s = int(k % kDecStages);
                 if (k >= kDecStages &&
                     !mbar_wait(empty + s, (uint32_t(k / kDecStages) & 1u) ^ 1u, status)) {
@@ -293,7 +306,7 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
                         mbar_wait(full + int(j % kDecStages), uint32_t(j / kDecStages) & 1u, nullptr);
                     break;
                 }
-                if (!issue(k, s))
+                if (!issue(w, s))
                     break;
             }
         }
@@ -310,9 +323,11 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
     const int H = CONV ? da.conv_k - 1 : 0;
     int64_t cached_cb = -1;
     bool ok = true;
-    for (int64_t k = 0;; ++k) {
-        int64_t b, cb;
-        if (!tile_of(k, b, cb))
+    TileWalk w;
+    w.start(da.ncb);
+    for (int64_t k = 0;; ++k, w.next()) {
+        const int64_t b = w.b, cb = w.cb;
+        if (b >= p.batch)
             break;
         const int64_t c0 = cb * D::kChanPerTile;
         const int nq = int(nchan(cb) * Q); // valid quarters in this tile
@@ -464,6 +479,11 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
             for (int it = 0; it < kDecItems; ++it)
                 dsp[it] = ds[it] + bias[it];
         }
+        // the tile's rows start at row0: item it of this thread is quarter
+        // q = tid + it * kDecThreads, i.e. float4 q of the tile's state and row q / Q
+        const int64_t row0 = b * p.channels + c0;
+        float4 *const st_tile = reinterpret_cast<float4 *>(p.state) + row0 * Q;
+        float ysum[kDecItems];
 #pragma unroll
         for (int it = 0; it < kDecItems; ++it) {
             const int q = tid + it * kDecThreads;
@@ -483,6 +503,7 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
 #pragma unroll
             for (int off = Q / 2; off >= 1; off >>= 1)
                 yp += __shfl_xor_sync(0xffffffffu, yp, off);
+            ysum[it] = yp; // (every lane of the row holds the row's sum)
             if constexpr (CONV) {
                 __syncwarp(); // every lane of the row has read the conv state
                 if (valid && lane_q == 0 && H > 0 && SS_IN_BOUNDS(c0 + q / Q < p.channels, 207)) {
@@ -497,15 +518,28 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
                     csr[H - 1] = cs[it][0];
                 }
             }
-            if (valid && SS_IN_BOUNDS(c0 + q / Q < p.channels && b < p.batch, 204)) {
-                const int64_t row = b * p.channels + c0 + q / Q;
-                __stcs(reinterpret_cast<float4 *>(p.state + row * N) + lane_q, st);
-                if (lane_q == 0) {
-                    float v = fmaf(dco[it], xs[it], yp);
-                    if (p.z)
-                        v *= silu(zs[it]);
-                    Elem<T>::store(static_cast<T *>(p.y) + row, v);
+            if (valid && SS_IN_BOUNDS(c0 + q / Q < p.channels && b < p.batch, 204))
+                __stcs(st_tile + q, st);
+        }
+        // y of the items' rows: the Q lanes of a row finish one item each in turn (lane
+        // j the items it with it % Q == j), instead of one lane finishing them all
+#pragma unroll
+        for (int m = 0; m < kDecItems / Q; ++m) {
+            float yv = ysum[m * Q], xv = xs[m * Q], zv = zs[m * Q], dv = dco[m * Q];
+#pragma unroll
+            for (int j = 1; j < Q; ++j)
+                if (lane_q == j) {
+                    yv = ysum[m * Q + j];
+                    xv = xs[m * Q + j];
+                    zv = zs[m * Q + j];
+                    dv = dco[m * Q + j];
                 }
+            const int q = tid + (m * Q + lane_q) * kDecThreads;
+            if (q < nq && SS_IN_BOUNDS(c0 + q / Q < p.channels && b < p.batch, 208)) {
+                float v = fmaf(dv, xv, yv);
+                if (p.z)
+                    v *= silu(zv);
+                Elem<T>::store(static_cast<T *>(p.y) + row0 + q / Q, v);
             }
         }
         // this warp is done reading the stage
