@@ -37,9 +37,14 @@
 // their products runs as two MMAs into the same fp32 accumulator: the result follows
 // fp32 intermediate arithmetic far below the bf16 rounding of the outputs.
 //
-// One CTA: 256 threads, 8 warps; warp w works on tensor-memory lanes 32 (w % 4) .. +31
-// (rows of the scores, outputs and state) and on column half w / 4.  Thread 0 issues the
-// tile loads (TMA) and the MMAs.  The k and v tiles are double-buffered (the next
+// One CTA: 8 compute warps and one issuer warp.  Compute warp w works on tensor-memory
+// lanes 32 (w % 4) .. +31 (rows of the scores, outputs and state) and on column half
+// w / 4.  The issuer warp's lane 0 issues every tile load (TMA) and every MMA, each as
+// soon as its inputs are ready; the compute warps tell it through two mbarriers (L o S
+// and w o V written; the epilogue done) and wait only for products to complete, so the
+// scores of a chunk are computed while the previous chunk's epilogue runs and Q H while
+// the mask is built.  (Issuing an MMA blocks the issuing thread for about as long as
+// the tensor core takes to run it.)  The k and v tiles are double-buffered (the next
 // chunk's are in flight during this one); the q tile is reloaded as soon as the
 // products that read it are done.  L o S goes to tensor memory (tcgen05.st) and enters
 // Yi as the A operand from there.
@@ -54,7 +59,9 @@ namespace ss {
 constexpr int kGtChunk = 128;   // tokens per chunk (the MMA's M)
 constexpr int kGtDk = 128;      // key size of this kernel
 constexpr int kGtNv = 64;       // value columns per CTA
-constexpr int kGtThreads = 256; // 8 warps: lane quarter w % 4, column half w / 4
+constexpr int kGtComputeWarps = 8; // warp w: tensor-memory lane quarter w % 4, column half w / 4
+constexpr int kGtComputeThreads = 32 * kGtComputeWarps;
+constexpr int kGtThreads = kGtComputeThreads + 32; // + the issuer warp
 constexpr uint32_t kGtTmemCols = 512;
 // tensor-memory columns: fp32 accumulators S, Yi, Yh, dH; L o S as packed bf16 pairs
 // (high and low parts, 64 columns = 128 elements each)
@@ -76,7 +83,7 @@ struct GtSmem {
     static constexpr int kZ = kG + 512;         // z_j [128] int
     static constexpr int kSg = kZ + 512;        // (-1)^par_j [128] fp32
     static constexpr int kRed = kSg + 512;      // per lane quarter: log sum, last zero, parity, |gamma| > 1
-    static constexpr int kBar = kRed + 64;      // mbarriers: q, kv[2], s, yh, mma2
+    static constexpr int kBar = kRed + 64;      // mbarriers: q, kv[2], s, yh, mma2, mw, epi
     static constexpr int kTmem = kBar + 64;     // tensor-memory base address
     static constexpr int kBytes = kTmem + 16 + 1024; // + alignment slack
 };
@@ -140,11 +147,12 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar)
                  : "memory");
 }
 
-// 32 consecutive fp32 columns of this warp's 32 tensor-memory lanes: thread t gets lane
-// (warp's first lane + t).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+// 32 consecutive fp32 columns of this warp's 32 tensor-memory lanes (thread t gets lane
+// (warp's first lane + t)), as raw 32-bit words, without waiting: several loads go out
+// together and one tmem_ld_wait(), followed by tmem_ld_fence() on each destination,
+// completes them.
+__device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t (&r)[32])
 {
-    uint32_t r[32];
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
                  "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
                  "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
@@ -154,10 +162,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
                    "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
                    "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
                  : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-        v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Ties every later use of `r` to a point after the wait (the registers a tcgen05.ld
+// writes are only valid once the wait has returned).
+__device__ __forceinline__ void tmem_ld_fence(uint32_t (&r)[32])
+{
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
 }
 
 // 16 consecutive 32-bit columns of this warp's 32 lanes from registers (thread t writes
@@ -228,15 +244,37 @@ __device__ __forceinline__ void scale_split8(uint4 v, float w, uint4 &hi, uint4 
     lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
+// Named barrier 1 over the compute warps (the issuer warp takes no part): plain, and
+// with an AND over every thread's predicate, so the compute warps leave the chunk loop
+// together (a warp that left alone would strand the others at the barrier).
+__device__ __forceinline__ void gt_compute_sync()
+{
+    asm volatile("bar.sync 1, %0;" ::"n"(kGtComputeThreads) : "memory");
+}
+__device__ __forceinline__ bool gt_compute_sync_and(bool v)
+{
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                 "bar.red.and.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r)
+                 : "r"(uint32_t(v)), "n"(kGtComputeThreads)
+                 : "memory");
+    return r != 0;
+}
+
 // One CTA per (batch item, 64-column value tile).  `status` records a timeout of a
 // bounded wait.
 __global__ void __launch_bounds__(kGtThreads, 1)
 ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps, uint32_t *status)
 {
     extern __shared__ unsigned char gt_raw[];
-    unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(gt_raw) + 1023) & ~uintptr_t(1023));
+    // the 1024-byte aligned base, as an offset into the shared array (a pointer that went
+    // through an integer would lose its address space: every access through it would
+    // compile to a generic load or store)
+    unsigned char *sm = gt_raw + ((1024u - (smem_u32(gt_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + GtSmem::kBar);
     uint64_t *bar_q = bars, *bar_kv = bars + 1 /* [2] */, *bar_s = bars + 3, *bar_yh = bars + 4, *bar_2 = bars + 5;
+    uint64_t *bar_mw = bars + 6, *bar_epi = bars + 7;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + GtSmem::kTmem);
     float *s_lam = reinterpret_cast<float *>(sm + GtSmem::kLam);
     float *s_g = reinterpret_cast<float *>(sm + GtSmem::kG);
@@ -244,7 +282,8 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
     float *s_sg = reinterpret_cast<float *>(sm + GtSmem::kSg);
     uint32_t *s_red = reinterpret_cast<uint32_t *>(sm + GtSmem::kRed);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int q4 = warp & 3, half = warp >> 2;
+    const bool issuer = warp == kGtComputeWarps;
+    const int q4 = warp & 3, half = (warp >> 2) & 1;
     const int r = 32 * q4 + lane; // this thread's row: a token of the chunk, a key of the state
     const int64_t b = blockIdx.x / a.col_tiles;
     const int n0 = int(blockIdx.x % a.col_tiles) * kGtNv;
@@ -258,6 +297,8 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
         mbar_init(bar_s, 1);
         mbar_init(bar_yh, 1);
         mbar_init(bar_2, 1);
+        mbar_init(bar_mw, kGtComputeWarps);  // one arrival per compute warp
+        mbar_init(bar_epi, kGtComputeWarps);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -266,11 +307,14 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
     }
     // the entering state: key row r, value columns 32 half .. +31 of the tile, fp32
     float H[32];
-    {
-        const float *src = a.h0 ? a.h0 + (b * kGtDk + r) * a.dv + n0 + 32 * half : nullptr;
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+        H[e] = 0.0f;
+    if (!issuer && a.h0) {
+        const float *src = a.h0 + (b * kGtDk + r) * a.dv + n0 + 32 * half;
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-            const float4 v = src ? __ldg(reinterpret_cast<const float4 *>(src + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(src + e));
             H[e] = v.x;
             H[e + 1] = v.y;
             H[e + 2] = v.z;
@@ -290,333 +334,394 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
             *reinterpret_cast<uint4 *>(sm + GtSmem::kHlo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
     };
-    store_h();
+    if (!issuer)
+        store_h();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
     const uint32_t lane_base = uint32_t(32 * q4) << 16; // this warp's tensor-memory lanes
-    // L o S is 0 above the diagonal in every chunk: those blocks of its tensor-memory
-    // copy are written once, here, and never again
+    if (!issuer) {
+        // L o S is 0 above the diagonal in every chunk: those blocks of its tensor-memory
+        // copy are written once, here, and never again
 #pragma unroll
-    for (int bb = 0; bb < 2; ++bb) {
-        const int jb = 2 * half + bb;
-        if (jb > q4) {
-            const uint32_t zero[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-            tmem_st16(tmem + lane_base + kGtColMhi + 16 * jb, zero);
-            tmem_st16(tmem + lane_base + kGtColMlo + 16 * jb, zero);
+        for (int bb = 0; bb < 2; ++bb) {
+            const int jb = 2 * half + bb;
+            if (jb > q4) {
+                const uint32_t zero[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                tmem_st16(tmem + lane_base + kGtColMhi + 16 * jb, zero);
+                tmem_st16(tmem + lane_base + kGtColMlo + 16 * jb, zero);
+            }
         }
+        tmem_st_wait();
     }
-    tmem_st_wait();
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); // H writes -> MMA reads
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
-    const int32_t b32 = int32_t(b);
-    auto issue_q = [&](int64_t c) {
-        mbar_arrive_expect_tx(bar_q, 32768);
-        const int32_t t0 = int32_t(c * kGtChunk);
-        tma_load_3d(sm + GtSmem::kQ, &maps.q, 0, t0, b32, bar_q);
-        tma_load_3d(sm + GtSmem::kQ + 16384, &maps.q, 64, t0, b32, bar_q);
-    };
-    auto issue_kv = [&](int64_t c) {
-        const int st = int(c & 1);
-        mbar_arrive_expect_tx(bar_kv + st, 32768 + 16384);
-        const int32_t t0 = int32_t(c * kGtChunk);
-        tma_load_3d(sm + GtSmem::kK + st * 32768, &maps.k, 0, t0, b32, bar_kv + st);
-        tma_load_3d(sm + GtSmem::kK + st * 32768 + 16384, &maps.k, 64, t0, b32, bar_kv + st);
-        tma_load_3d(sm + GtSmem::kV + st * 16384, &maps.v, n0, t0, b32, bar_kv + st);
-    };
-    // thread 0's record of the asynchronous work (phases issued and phases waited for,
-    // per barrier), for draining after a timeout
-    int64_t nq_issued = 0, nq_waited = 0, nkv0_issued = 0, nkv1_issued = 0, nkv0_waited = 0, nkv1_waited = 0;
-    int64_t ns_committed = 0, ns_waited = 0, nyh_committed = 0, nyh_waited = 0, n2_committed = 0, n2_waited = 0;
-    if (tid == 0) {
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.q)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.k)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.v)) : "memory");
-        issue_q(0);
-        nq_issued = 1;
-        issue_kv(0);
-        nkv0_issued = 1;
-        if (nchunks > 1) {
-            issue_kv(1);
-            nkv1_issued = 1;
-        }
-    }
-
     constexpr uint32_t kIdS = idesc_bf16(128, 128, 0, 0);   // Q (K-major) x K (K-major)
     constexpr uint32_t kIdY = idesc_bf16(128, kGtNv, 0, 1); // Q or L o S (K-major) x H or V (MN-major)
     constexpr uint32_t kIdH = idesc_bf16(128, kGtNv, 1, 1); // K^T (MN-major) x (w o V) (MN-major)
-    constexpr float kTiny = 1.17549435e-38f;                // smallest normal float
-    const float *gam = a.gamma + b * a.seq;
-    float gm_next = r < a.seq ? __ldg(gam + r) : 1.0f; // past the end: no decay
     bool ok = true;
-    for (int64_t c = 0; c < nchunks && ok; ++c) {
-        const int st = int(c & 1);
-        const uint32_t ph = uint32_t(c & 1), ph_kv = uint32_t((c >> 1) & 1);
-        const int64_t t0 = c * kGtChunk;
-        // ---- gates: scans of log2|gamma|, of the last zero gate and of the sign parity
-        // over this lane quarter's 32 tokens (both column halves compute the same) -------
-        const float gm = gm_next;
-        gm_next = t0 + kGtChunk + r < a.seq ? __ldg(gam + t0 + kGtChunk + r) : 1.0f; // the next chunk's
-        const bool zero_gate = fabsf(gm) < kTiny;
-        float lg = zero_gate ? 0.0f : __log2f(fabsf(gm));
-        int zl = zero_gate ? r : -1;
-        uint32_t par = (!zero_gate && gm < 0.0f) ? 1u : 0u;
-        const uint32_t big = __any_sync(0xffffffffu, !(fabsf(gm) <= 1.0f)) ? 1u : 0u; // |gamma| > 1, or NaN
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float up = __shfl_up_sync(0xffffffffu, lg, o);
-            const int uz = __shfl_up_sync(0xffffffffu, zl, o);
-            const uint32_t upar = __shfl_up_sync(0xffffffffu, par, o);
-            if (lane >= o) {
-                lg += up;
-                zl = max(zl, uz);
-                par ^= upar;
+    if (issuer) {
+        // ======================= the issuer warp (lane 0 works) =======================
+        // Per chunk c, in order: S(c) once the chunk's tiles have landed and the mask of
+        // chunk c-1 is done with the score columns; Yh(c) once the epilogue of c-1 has
+        // stored H(c) and read its accumulators; the k / v tiles of c+1 into the stage
+        // chunk c-1 used, once that chunk's products are done; the q tile of c+1 once
+        // Yh(c) (the last reader of q) is done; dH(c) and Yi(c) once the compute warps
+        // have written L o S and w o V.  The compute warps never wait for an issue, only
+        // for products to complete.
+        if (lane == 0) {
+            const int32_t b32 = int32_t(b);
+            auto issue_q = [&](int64_t c) {
+                mbar_arrive_expect_tx(bar_q, 32768);
+                const int32_t t0 = int32_t(c * kGtChunk);
+                tma_load_3d(sm + GtSmem::kQ, &maps.q, 0, t0, b32, bar_q);
+                tma_load_3d(sm + GtSmem::kQ + 16384, &maps.q, 64, t0, b32, bar_q);
+            };
+            auto issue_kv = [&](int64_t c) {
+                const int st = int(c & 1);
+                mbar_arrive_expect_tx(bar_kv + st, 32768 + 16384);
+                const int32_t t0 = int32_t(c * kGtChunk);
+                tma_load_3d(sm + GtSmem::kK + st * 32768, &maps.k, 0, t0, b32, bar_kv + st);
+                tma_load_3d(sm + GtSmem::kK + st * 32768 + 16384, &maps.k, 64, t0, b32, bar_kv + st);
+                tma_load_3d(sm + GtSmem::kV + st * 16384, &maps.v, n0, t0, b32, bar_kv + st);
+            };
+            // phases issued (or committed) per barrier, for draining after a timeout
+            int64_t nq = 0, nkv0 = 0, nkv1 = 0, ns = 0, nyh = 0, n2 = 0;
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.q)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.k)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.v)) : "memory");
+            issue_q(0);
+            nq = 1;
+            issue_kv(0);
+            nkv0 = 1;
+            if (nchunks > 1) {
+                issue_kv(1);
+                nkv1 = 1;
             }
-        }
-        if (half == 0 && lane == 31) {
-            s_red[4 * q4] = __float_as_uint(lg);
-            s_red[4 * q4 + 1] = uint32_t(zl);
-            s_red[4 * q4 + 2] = par;
-            s_red[4 * q4 + 3] = big;
-        }
-        // ---- the chunk's tiles, then (thread 0) S = Q K^T and Yh = Q H ----------------
-        if (!mbar_wait(bar_q, ph, status) || !mbar_wait(bar_kv + st, ph_kv, status))
-            ok = false;
-        if (tid == 0 && ok) {
-            nq_waited = c + 1;
-            (st ? nkv1_waited : nkv0_waited) = (c >> 1) + 1;
-            tc_fence_after();
-            const uint32_t qb = s_base + GtSmem::kQ, kb = s_base + GtSmem::kK + st * 32768;
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) { // K = 128 keys in slices of 16
-                const uint32_t o = (ks >> 2) * 16384 + (ks & 3) * 32;
-                umma_bf16(tmem + kGtColS, sw128_desc(qb + o, 16, 1024), sw128_desc(kb + o, 16, 1024), kIdS, ks > 0);
-            }
-            umma_commit(bar_s);
-            ns_committed = c + 1;
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t qd = sw128_desc(qb + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                const uint32_t ho = ks * 2048; // 16 key rows of H
-                umma_bf16(tmem + kGtColYh, qd, sw128_desc(s_base + GtSmem::kHhi + ho, 16384, 1024), kIdY, ks > 0);
-                umma_bf16(tmem + kGtColYh, qd, sw128_desc(s_base + GtSmem::kHlo + ho, 16384, 1024), kIdY, 1);
-            }
-            umma_commit(bar_yh);
-            nyh_committed = c + 1;
-        }
-        if (!__syncthreads_and(ok ? 1 : 0)) {
-            ok = false;
-            break;
-        }
-        // ---- prefixes over the chunk for this row, and the chunk's totals --------------
-        float off = 0.0f;
-        int zoff = -1, z_end = -1;
-        uint32_t poff = 0, par_end = 0, any_big = 0;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            const int wz = int(s_red[4 * w + 1]);
-            const uint32_t wp = s_red[4 * w + 2];
-            if (w < q4) {
-                off += __uint_as_float(s_red[4 * w]);
-                zoff = max(zoff, wz);
-                poff ^= wp;
-            }
-            z_end = max(z_end, wz);
-            par_end ^= wp;
-            any_big |= s_red[4 * w + 3];
-        }
-        const float lam_r = lg + off;
-        const int z_r = max(zl, zoff);
-        const uint32_t par_r = par ^ poff;
-        const float sg_r = par_r ? -1.0f : 1.0f;
-        // lam of token 127, summed in the order its own row prefix was
-        const float lam_end = __uint_as_float(s_red[12]) +
-                              ((__uint_as_float(s_red[0]) + __uint_as_float(s_red[4])) + __uint_as_float(s_red[8]));
-        if (half == 0) {
-            // the column factor L[j1, r], j1 the last token of this lane quarter
-            const float lam_j1 = __uint_as_float(s_red[4 * q4]) + off;
-            const int z_j1 = max(int(s_red[4 * q4 + 1]), zoff);
-            const uint32_t par_j1 = s_red[4 * q4 + 2] ^ poff;
-            s_lam[r] = lam_r;
-            s_z[r] = z_r;
-            s_sg[r] = sg_r;
-            s_g[r] = z_j1 > r ? 0.0f : ((par_j1 ^ par_r) ? -1.0f : 1.0f) * ex2(lam_j1 - lam_r);
-        }
-        const float p_r = z_r >= 0 ? 0.0f : sg_r * ex2(lam_r);                             // P_r
-        const float p_end = z_end >= 0 ? 0.0f : (par_end ? -1.0f : 1.0f) * ex2(lam_end);  // P_127
-        __syncthreads();
-        // ---- w o V: token row r, this half's 32 value columns, as high / low parts ----
-        {
-            const float w_r = z_end > r ? 0.0f : ((par_end ^ par_r) ? -1.0f : 1.0f) * ex2(lam_end - lam_r);
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                const uint32_t o = sw128_off(r, 4 * half + cc);
-                uint4 hi, lo;
-                scale_split8(*reinterpret_cast<const uint4 *>(sm + GtSmem::kV + st * 16384 + o), w_r, hi, lo);
-                *reinterpret_cast<uint4 *>(sm + GtSmem::kWhi + o) = hi;
-                *reinterpret_cast<uint4 *>(sm + GtSmem::kWlo + o) = lo;
-            }
-        }
-        // ---- L o S: row r, this half's 64 columns, into tensor memory -----------------
-        if (!mbar_wait(bar_s, ph, status))
-            ok = false;
-        else if (tid == 0)
-            ns_waited = c + 1;
-        ok = __all_sync(0xffffffffu, ok); // the tensor-memory accesses below are warp-collective
-        tc_fence_after();
-        if (ok) {
-#pragma unroll 1
-            for (int bb = 0; bb < 2; ++bb) {
-                const int jb = 2 * half + bb;
-                if (jb > q4)
-                    continue; // above the diagonal: the zeros written once
-                float s[32];
-                tmem_ld32(tmem + lane_base + kGtColS + 32 * jb, s);
-                uint32_t hi[16], lo[16];
-                if (jb < q4 && !any_big) {
-                    // below the diagonal block: L[r, j] = L[r, j1] L[j1, j]
-                    const int j1 = 32 * jb + 31;
-                    const float f = z_r > j1 ? 0.0f : sg_r * s_sg[j1] * ex2(lam_r - s_lam[j1]);
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        const float4 g = *reinterpret_cast<const float4 *>(s_g + 32 * jb + e);
-                        split_bf16x2(s[e] * g.x * f, s[e + 1] * g.y * f, hi[e / 2], lo[e / 2]);
-                        split_bf16x2(s[e + 2] * g.z * f, s[e + 3] * g.w * f, hi[e / 2 + 1], lo[e / 2 + 1]);
-                    }
-                } else {
-                    // the diagonal block (or a chunk with gates above 1 in magnitude):
-                    // element by element
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        const int j = 32 * jb + e;
-                        const float4 lj = *reinterpret_cast<const float4 *>(s_lam + j);
-                        const float4 sj = *reinterpret_cast<const float4 *>(s_sg + j);
-                        const float ljv[4] = {lj.x, lj.y, lj.z, lj.w}, sjv[4] = {sj.x, sj.y, sj.z, sj.w};
-                        float m[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const bool valid = j + u <= r && z_r <= j + u;
-                            m[u] = valid ? s[e + u] * (sg_r * sjv[u]) * ex2(lam_r - ljv[u]) : 0.0f;
-                        }
-                        split_bf16x2(m[0], m[1], hi[e / 2], lo[e / 2]);
-                        split_bf16x2(m[2], m[3], hi[e / 2 + 1], lo[e / 2 + 1]);
-                    }
+            for (int64_t c = 0; c < nchunks; ++c) {
+                const int st = int(c & 1);
+                const uint32_t ph = uint32_t(c & 1), pp = uint32_t((c - 1) & 1);
+                if (!mbar_wait(bar_q, ph, status) || !mbar_wait(bar_kv + st, uint32_t((c >> 1) & 1), status) ||
+                    (c > 0 && !mbar_wait(bar_mw, pp, status))) {
+                    ok = false;
+                    break;
                 }
-                tmem_st16(tmem + lane_base + kGtColMhi + 16 * jb, hi);
-                tmem_st16(tmem + lane_base + kGtColMlo + 16 * jb, lo);
-            }
-            tmem_st_wait();
-        }
-        // the q tile is free once Q H is done (long done by now): the next chunk's q
-        if (tid == 0 && ok) {
-            if (!mbar_wait(bar_yh, ph, status)) {
-                ok = false;
-            } else {
-                nyh_waited = c + 1;
+                tc_fence_after();
+                const uint32_t qb = s_base + GtSmem::kQ, kb = s_base + GtSmem::kK + st * 32768;
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) { // K = 128 keys in slices of 16
+                    const uint32_t o = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    umma_bf16(tmem + kGtColS, sw128_desc(qb + o, 16, 1024), sw128_desc(kb + o, 16, 1024), kIdS,
+                              ks > 0);
+                }
+                umma_commit(bar_s);
+                ns = c + 1;
+                if (c > 0 && !mbar_wait(bar_epi, pp, status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t qd = sw128_desc(qb + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                    const uint32_t ho = ks * 2048; // 16 key rows of H
+                    umma_bf16(tmem + kGtColYh, qd, sw128_desc(s_base + GtSmem::kHhi + ho, 16384, 1024), kIdY,
+                              ks > 0);
+                    umma_bf16(tmem + kGtColYh, qd, sw128_desc(s_base + GtSmem::kHlo + ho, 16384, 1024), kIdY, 1);
+                }
+                umma_commit(bar_yh);
+                nyh = c + 1;
+                if (c > 0 && c + 1 < nchunks) {
+                    if (!mbar_wait(bar_2, pp, status)) { // chunk c-1's products: its stage is free
+                        ok = false;
+                        break;
+                    }
+                    issue_kv(c + 1);
+                    ((c + 1) & 1 ? nkv1 : nkv0) = ((c + 1) >> 1) + 1;
+                }
+                if (!mbar_wait(bar_yh, ph, status)) {
+                    ok = false;
+                    break;
+                }
                 if (c + 1 < nchunks) {
                     issue_q(c + 1);
-                    nq_issued = c + 2;
+                    nq = c + 2;
+                }
+                if (!mbar_wait(bar_mw, ph, status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t vb = s_base + GtSmem::kV + st * 16384;
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) { // K = 128 tokens in slices of 16
+                    const uint64_t kd = sw128_desc(kb + ks * 2048, 16384, 1024); // keys x 16 tokens (MN-major)
+                    umma_bf16(tmem + kGtColDH, kd, sw128_desc(s_base + GtSmem::kWhi + ks * 2048, 16384, 1024),
+                              kIdH, ks > 0);
+                    umma_bf16(tmem + kGtColDH, kd, sw128_desc(s_base + GtSmem::kWlo + ks * 2048, 16384, 1024),
+                              kIdH, 1);
+                }
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t vd = sw128_desc(vb + ks * 2048, 16384, 1024);
+                    umma_bf16_ts(tmem + kGtColYi, tmem + kGtColMhi + 8 * ks, vd, kIdY, ks > 0);
+                    umma_bf16_ts(tmem + kGtColYi, tmem + kGtColMlo + 8 * ks, vd, kIdY, 1);
+                }
+                umma_commit(bar_2);
+                n2 = c + 1;
+            }
+            // Let every load and product still in flight finish before the tensor memory
+            // is freed: the latest phase of each barrier (already complete on the normal
+            // path; the drain waits keep the default limit)
+            if (nq)
+                mbar_wait(bar_q, uint32_t((nq - 1) & 1), nullptr);
+            if (nkv0)
+                mbar_wait(bar_kv, uint32_t((nkv0 - 1) & 1), nullptr);
+            if (nkv1)
+                mbar_wait(bar_kv + 1, uint32_t((nkv1 - 1) & 1), nullptr);
+            if (ns)
+                mbar_wait(bar_s, uint32_t((ns - 1) & 1), nullptr);
+            if (nyh)
+                mbar_wait(bar_yh, uint32_t((nyh - 1) & 1), nullptr);
+            if (n2)
+                mbar_wait(bar_2, uint32_t((n2 - 1) & 1), nullptr);
+        }
+    } else {
+        // ======================= the compute warps =======================================
+        // Per chunk c: w o V(c) and L o S(c) (then the issuer runs dH(c) and Yi(c)); while
+        // those products run, the gate scan of chunk c+1; then the epilogue of chunk c.
+        constexpr float kTiny = 1.17549435e-38f; // smallest normal float
+        const float *gam = a.gamma + b * a.seq;
+        float gm_next = r < a.seq ? __ldg(gam + r) : 1.0f; // past the end: no decay
+        // chunk values of this row from the gate scan
+        float lam_r = 0.0f, sg_r = 1.0f, p_r = 0.0f, p_end = 0.0f, lam_end = 0.0f;
+        int z_r = -1, z_end = -1;
+        uint32_t par_r = 0, par_end = 0, any_big = 0;
+        // The gate scan of chunk c: scans of log2|gamma|, of the last zero gate and of the
+        // sign parity over each lane quarter's 32 tokens (both column halves compute the
+        // same), then the prefixes of row r, the chunk's totals and the arrays the mask
+        // reads.  Between two barriers of the compute warps: the first comes after every
+        // compute warp has finished the previous chunk's mask (the last reader of those
+        // arrays), and ends the loop for all of them at once when any has seen a failed
+        // wait (false).
+        auto scan_gates = [&](int64_t c) -> bool {
+            const int64_t t0 = c * kGtChunk;
+            const float gm = gm_next;
+            gm_next = t0 + kGtChunk + r < a.seq ? __ldg(gam + t0 + kGtChunk + r) : 1.0f; // the next chunk's
+            const bool zero_gate = fabsf(gm) < kTiny;
+            float lg = zero_gate ? 0.0f : __log2f(fabsf(gm));
+            int zl = zero_gate ? r : -1;
+            uint32_t par = (!zero_gate && gm < 0.0f) ? 1u : 0u;
+            const uint32_t big = __any_sync(0xffffffffu, !(fabsf(gm) <= 1.0f)) ? 1u : 0u; // |gamma| > 1, or NaN
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float up = __shfl_up_sync(0xffffffffu, lg, o);
+                const int uz = __shfl_up_sync(0xffffffffu, zl, o);
+                const uint32_t upar = __shfl_up_sync(0xffffffffu, par, o);
+                if (lane >= o) {
+                    lg += up;
+                    zl = max(zl, uz);
+                    par ^= upar;
                 }
             }
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); // w o V writes -> MMA reads
-        tc_fence_before();
-        if (!__syncthreads_and(ok ? 1 : 0)) {
-            ok = false;
-            break;
-        }
-        // ---- Yi = (L o S) V and dH = K^T (w o V), each over high + low parts -----------
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t vb = s_base + GtSmem::kV + st * 16384, kb = s_base + GtSmem::kK + st * 32768;
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) { // K = 128 tokens in slices of 16
-                const uint64_t vd = sw128_desc(vb + ks * 2048, 16384, 1024);
-                umma_bf16_ts(tmem + kGtColYi, tmem + kGtColMhi + 8 * ks, vd, kIdY, ks > 0);
-                umma_bf16_ts(tmem + kGtColYi, tmem + kGtColMlo + 8 * ks, vd, kIdY, 1);
-                const uint64_t kd = sw128_desc(kb + ks * 2048, 16384, 1024); // keys x 16 tokens (MN-major)
-                umma_bf16(tmem + kGtColDH, kd, sw128_desc(s_base + GtSmem::kWhi + ks * 2048, 16384, 1024), kIdH,
-                          ks > 0);
-                umma_bf16(tmem + kGtColDH, kd, sw128_desc(s_base + GtSmem::kWlo + ks * 2048, 16384, 1024), kIdH, 1);
+            if (half == 0 && lane == 31) {
+                s_red[4 * q4] = __float_as_uint(lg);
+                s_red[4 * q4 + 1] = uint32_t(zl);
+                s_red[4 * q4 + 2] = par;
+                s_red[4 * q4 + 3] = big;
             }
-            umma_commit(bar_2);
-            n2_committed = c + 1;
-        }
-        if (!mbar_wait(bar_2, ph, status))
-            ok = false;
-        else if (tid == 0)
-            n2_waited = c + 1;
-        ok = __all_sync(0xffffffffu, ok);
-        tc_fence_after();
-        // this chunk's k / v stage is free: the chunk after next goes there
-        if (tid == 0 && ok && c + 2 < nchunks) {
-            issue_kv(c + 2);
-            (st ? nkv1_issued : nkv0_issued) = (c >> 1) + 2;
-        }
-        if (ok) {
-            // ---- y = Yi + P o Yh: row r, this half's 32 columns ---------------------------
-            {
-                float yi[32], yh[32];
-                tmem_ld32(tmem + lane_base + kGtColYi + 32 * half, yi);
-                tmem_ld32(tmem + lane_base + kGtColYh + 32 * half, yh);
-                if (t0 + r < a.seq) {
-                    __nv_bfloat16 *dst = a.y + (b * a.seq + t0 + r) * a.dv + n0 + 32 * half;
+            if (!gt_compute_sync_and(ok))
+                return false;
+            float off = 0.0f;
+            int zoff = -1;
+            uint32_t poff = 0;
+            z_end = -1;
+            par_end = 0;
+            any_big = 0;
 #pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8) {
-                        float o[8];
+            for (int w = 0; w < 4; ++w) {
+                const int wz = int(s_red[4 * w + 1]);
+                const uint32_t wp = s_red[4 * w + 2];
+                if (w < q4) {
+                    off += __uint_as_float(s_red[4 * w]);
+                    zoff = max(zoff, wz);
+                    poff ^= wp;
+                }
+                z_end = max(z_end, wz);
+                par_end ^= wp;
+                any_big |= s_red[4 * w + 3];
+            }
+            lam_r = lg + off;
+            z_r = max(zl, zoff);
+            par_r = par ^ poff;
+            sg_r = par_r ? -1.0f : 1.0f;
+            // lam of token 127, summed in the order its own row prefix was
+            lam_end = __uint_as_float(s_red[12]) +
+                      ((__uint_as_float(s_red[0]) + __uint_as_float(s_red[4])) + __uint_as_float(s_red[8]));
+            if (half == 0) {
+                // the column factor L[j1, r], j1 the last token of this lane quarter
+                const float lam_j1 = __uint_as_float(s_red[4 * q4]) + off;
+                const int z_j1 = max(int(s_red[4 * q4 + 1]), zoff);
+                const uint32_t par_j1 = s_red[4 * q4 + 2] ^ poff;
+                s_lam[r] = lam_r;
+                s_z[r] = z_r;
+                s_sg[r] = sg_r;
+                s_g[r] = z_j1 > r ? 0.0f : ((par_j1 ^ par_r) ? -1.0f : 1.0f) * ex2(lam_j1 - lam_r);
+            }
+            p_r = z_r >= 0 ? 0.0f : sg_r * ex2(lam_r);                            // P_r
+            p_end = z_end >= 0 ? 0.0f : (par_end ? -1.0f : 1.0f) * ex2(lam_end); // P_127
+            gt_compute_sync();
+            return true;
+        };
+        bool run = scan_gates(0);
+        for (int64_t c = 0; run && c < nchunks; ++c) {
+            const int st = int(c & 1);
+            const uint32_t ph = uint32_t(c & 1), ph_kv = uint32_t((c >> 1) & 1);
+            const int64_t t0 = c * kGtChunk;
+            // ---- w o V: token row r, this half's 32 value columns, as high / low parts
+            // (the v tile has landed; dH of the previous chunk, the last reader of w o V,
+            // completed before that chunk's epilogue) --------------------------------------
+            if (!mbar_wait(bar_kv + st, ph_kv, status))
+                ok = false;
+            if (ok) {
+                const float w_r = z_end > r ? 0.0f : ((par_end ^ par_r) ? -1.0f : 1.0f) * ex2(lam_end - lam_r);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            o[e] = fmaf(p_r, yh[8 * q8 + e], yi[8 * q8 + e]);
-                        *reinterpret_cast<uint4 *>(dst + 8 * q8) =
-                            make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
-                                       pack_bf16x2(o[6], o[7]));
+                for (int cc = 0; cc < 4; ++cc) {
+                    const uint32_t o = sw128_off(r, 4 * half + cc);
+                    uint4 hi, lo;
+                    scale_split8(*reinterpret_cast<const uint4 *>(sm + GtSmem::kV + st * 16384 + o), w_r, hi, lo);
+                    *reinterpret_cast<uint4 *>(sm + GtSmem::kWhi + o) = hi;
+                    *reinterpret_cast<uint4 *>(sm + GtSmem::kWlo + o) = lo;
+                }
+            }
+            // ---- L o S: row r, this half's 64 columns, into tensor memory -------------
+            if (!mbar_wait(bar_s, ph, status))
+                ok = false;
+            ok = __all_sync(0xffffffffu, ok); // the tensor-memory accesses below are warp-collective
+            tc_fence_after();
+            if (ok) {
+#pragma unroll 1
+                for (int bb = 0; bb < 2; ++bb) {
+                    const int jb = 2 * half + bb;
+                    if (jb > q4)
+                        continue; // above the diagonal: the zeros written once
+                    uint32_t sr[32];
+                    tmem_ld32_issue(tmem + lane_base + kGtColS + 32 * jb, sr);
+                    tmem_ld_wait();
+                    tmem_ld_fence(sr);
+                    float s[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        s[e] = __uint_as_float(sr[e]);
+                    uint32_t hi[16], lo[16];
+                    if (jb < q4 && !any_big) {
+                        // below the diagonal block: L[r, j] = L[r, j1] L[j1, j]
+                        const int j1 = 32 * jb + 31;
+                        const float f = z_r > j1 ? 0.0f : sg_r * s_sg[j1] * ex2(lam_r - s_lam[j1]);
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            const float4 gv = *reinterpret_cast<const float4 *>(s_g + 32 * jb + e);
+                            split_bf16x2(s[e] * gv.x * f, s[e + 1] * gv.y * f, hi[e / 2], lo[e / 2]);
+                            split_bf16x2(s[e + 2] * gv.z * f, s[e + 3] * gv.w * f, hi[e / 2 + 1], lo[e / 2 + 1]);
+                        }
+                    } else {
+                        // the diagonal block (or a chunk with gates above 1 in magnitude):
+                        // element by element
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            const int j = 32 * jb + e;
+                            const float4 lj = *reinterpret_cast<const float4 *>(s_lam + j);
+                            const float4 sj = *reinterpret_cast<const float4 *>(s_sg + j);
+                            const float ljv[4] = {lj.x, lj.y, lj.z, lj.w}, sjv[4] = {sj.x, sj.y, sj.z, sj.w};
+                            float m[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const bool valid = j + u <= r && z_r <= j + u;
+                                m[u] = valid ? s[e + u] * (sg_r * sjv[u]) * ex2(lam_r - ljv[u]) : 0.0f;
+                            }
+                            split_bf16x2(m[0], m[1], hi[e / 2], lo[e / 2]);
+                            split_bf16x2(m[2], m[3], hi[e / 2 + 1], lo[e / 2 + 1]);
+                        }
+                    }
+                    tmem_st16(tmem + lane_base + kGtColMhi + 16 * jb, hi);
+                    tmem_st16(tmem + lane_base + kGtColMlo + 16 * jb, lo);
+                }
+                tmem_st_wait();
+            }
+            // L o S and w o V of this warp are written: tell the issuer (after a failed
+            // wait too, so that it does not wait in vain; the loop ends at the next barrier)
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); // w o V writes -> MMA reads
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_mw);
+            // ---- while dH(c) and Yi(c) run: the gate scan of the next chunk -----------
+            const float p_rc = p_r, p_endc = p_end; // this chunk's, for its epilogue
+            run = c + 1 < nchunks ? scan_gates(c + 1) : gt_compute_sync_and(ok);
+            if (!run) {
+                ok = false;
+                break;
+            }
+            // ---- the chunk's products: y = Yi + P o Yh and H' = P_127 H + dH ------------
+            if (!mbar_wait(bar_2, ph, status))
+                ok = false;
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+            if (ok) {
+                {
+                    uint32_t yir[32], yhr[32];
+                    tmem_ld32_issue(tmem + lane_base + kGtColYi + 32 * half, yir);
+                    tmem_ld32_issue(tmem + lane_base + kGtColYh + 32 * half, yhr);
+                    tmem_ld_wait();
+                    tmem_ld_fence(yir);
+                    tmem_ld_fence(yhr);
+                    if (t0 + r < a.seq) {
+                        __nv_bfloat16 *dst = a.y + (b * a.seq + t0 + r) * a.dv + n0 + 32 * half;
+#pragma unroll
+                        for (int q8 = 0; q8 < 4; ++q8) {
+                            float o[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                o[e] = fmaf(p_rc, __uint_as_float(yhr[8 * q8 + e]), __uint_as_float(yir[8 * q8 + e]));
+                            *reinterpret_cast<uint4 *>(dst + 8 * q8) =
+                                make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                                           pack_bf16x2(o[6], o[7]));
+                        }
                     }
                 }
-            }
-            // ---- H' = P_127 H + dH: key row r, this half's 32 columns ---------------------
-            {
-                float dh[32];
-                tmem_ld32(tmem + lane_base + kGtColDH + 32 * half, dh);
+                {
+                    uint32_t dhr[32];
+                    tmem_ld32_issue(tmem + lane_base + kGtColDH + 32 * half, dhr);
+                    tmem_ld_wait();
+                    tmem_ld_fence(dhr);
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    H[e] = fmaf(p_end, H[e], dh[e]);
+                    for (int e = 0; e < 32; ++e)
+                        H[e] = fmaf(p_endc, H[e], __uint_as_float(dhr[e]));
+                }
+                store_h();
             }
-            store_h();
+            // this warp has read its accumulators and stored its part of H(c+1)
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); // H writes -> MMA reads
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_epi);
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); // H writes -> MMA reads
-        tc_fence_before();
-        if (!__syncthreads_and(ok ? 1 : 0)) {
+        if (!run)
             ok = false;
-            break;
-        }
-    }
-    if (ok) {
-        __nv_bfloat16 *dst = a.final_state + (b * kGtDk + r) * a.dv + n0 + 32 * half;
+        if (ok) {
+            __nv_bfloat16 *dst = a.final_state + (b * kGtDk + r) * a.dv + n0 + 32 * half;
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-            const float *h = H + 8 * q8;
-            *reinterpret_cast<uint4 *>(dst + 8 * q8) = make_uint4(
-                pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
+            for (int q8 = 0; q8 < 4; ++q8) {
+                const float *h = H + 8 * q8;
+                *reinterpret_cast<uint4 *>(dst + 8 * q8) = make_uint4(
+                    pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
+            }
         }
-    } else if (tid == 0) {
-        // a wait gave up: let the loads and MMAs still in flight finish (the drain waits
-        // keep the default limit) before the tensor memory is freed
-        if (nq_issued > nq_waited)
-            mbar_wait(bar_q, uint32_t((nq_issued - 1) & 1), nullptr);
-        if (nkv0_issued > nkv0_waited)
-            mbar_wait(bar_kv, uint32_t((nkv0_issued - 1) & 1), nullptr);
-        if (nkv1_issued > nkv1_waited)
-            mbar_wait(bar_kv + 1, uint32_t((nkv1_issued - 1) & 1), nullptr);
-        if (ns_committed > ns_waited)
-            mbar_wait(bar_s, uint32_t((ns_committed - 1) & 1), nullptr);
-        if (nyh_committed > nyh_waited)
-            mbar_wait(bar_yh, uint32_t((nyh_committed - 1) & 1), nullptr);
-        if (n2_committed > n2_waited)
-            mbar_wait(bar_2, uint32_t((n2_committed - 1) & 1), nullptr);
     }
     tc_fence_before();
     __syncthreads();
