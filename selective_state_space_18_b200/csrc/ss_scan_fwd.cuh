@@ -271,6 +271,11 @@ struct IoPrefetch {
     // three conv inputs before each task's first token
     float cw[CONV ? S::kTokPerLane : 1][4], cb[CONV ? S::kTokPerLane : 1];
     float halo[CONV ? S::kTokPerLane : 1][3];
+    // (TMA path) the last three inputs of each task's block in the previous chunk, and
+    // which chunk that was: the next chunk of the same rows takes its first block's halo
+    // from them
+    float tail[CONV ? S::kTokPerLane : 1][3] = {};
+    int64_t tail_g = -1, tail_t0 = -1;
 
     __device__ __forceinline__ void load_bias(const ScanArgs &p, int lane, int64_t g)
     {
@@ -388,8 +393,40 @@ struct IoPrefetch {
             dr[m].load_smem(rd + cl * S::kChunk + tb * 8);
         }
         load_bias(p, lane, g);
-        if constexpr (CONV)
-            load_halo(p, lane, g, t0);
+        if constexpr (CONV) {
+            // The halo of a task's block: the block before it in the same row of the tile,
+            // or, for the first block, the previous chunk's last block -- held by lane
+            // (lane | kBlocks - 1) of this warp one chunk ago when that chunk was this
+            // row group's previous one (chunks of a unit reach the producers in order);
+            // only the first chunk of a unit reads global memory (or the conv state).
+            static_assert(S::kBlocks == 4 && S::kIoThreads % S::kBlocks == 0, "task (channel, block) layout");
+            const bool follows = g == tail_g && t0 == tail_t0 + S::kChunk;
+            if (!follows)
+                load_halo(p, lane, g, t0);
+#pragma unroll
+            for (int m = 0; m < S::kTokPerLane; ++m) {
+                const int q = lane + S::kIoThreads * m;
+                const int cl = q / S::kBlocks, tb = q % S::kBlocks;
+                float prev[3];
+#pragma unroll
+                for (int k = 0; k < 3; ++k)
+                    prev[k] = __shfl_sync(0xffffffffu, tail[m][k], (lane & 31) | (S::kBlocks - 1));
+                if (tb > 0) {
+#pragma unroll
+                    for (int k = 0; k < 3; ++k)
+                        halo[m][k] = Elem<T>::load_smem(rx + cl * S::kChunk + tb * 8 - 3 + k);
+                } else if (follows) {
+#pragma unroll
+                    for (int k = 0; k < 3; ++k)
+                        halo[m][k] = prev[k];
+                }
+#pragma unroll
+                for (int k = 0; k < 3; ++k)
+                    tail[m][k] = xr[m].get(5 + k);
+            }
+            tail_g = g;
+            tail_t0 = t0;
+        }
     }
 };
 

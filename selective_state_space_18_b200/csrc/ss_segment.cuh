@@ -36,7 +36,7 @@ struct SegDecayArgs {
 };
 
 constexpr int kSegWarps = 8;
-constexpr int kSegBatch = 4; // 16-byte loads in flight per lane
+constexpr int kSegBatch = 8; // 16-byte loads in flight per lane (a 2048-token bf16 row in one round trip)
 
 // One warp per (b, c) row and segment, grid-strided: the lanes sum the segment's
 // step sizes (8 elements per 16-byte vector when VEC), OR the batch row's reset flags
