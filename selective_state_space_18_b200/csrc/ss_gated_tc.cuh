@@ -37,9 +37,9 @@
 // their products runs as two MMAs into the same fp32 accumulator: the result follows
 // fp32 intermediate arithmetic far below the bf16 rounding of the outputs.
 //
-// One CTA: 8 compute warps and one issuer warp.  Compute warp w works on tensor-memory
-// lanes 32 (w % 4) .. +31 (rows of the scores, outputs and state) and on column half
-// w / 4.  The issuer warp's lane 0 issues every tile load (TMA) and every MMA, each as
+// One CTA: 16 compute warps and one issuer warp.  Compute warp w works on tensor-memory
+// lanes 32 (w % 4) .. +31 (rows of the scores, outputs and state) and on column group
+// w / 4 (a quarter of the value columns and one 32-column block of the scores).  The issuer warp's lane 0 issues every tile load (TMA) and every MMA, each as
 // soon as its inputs are ready; the compute warps tell it through two mbarriers (L o S
 // and w o V written; the epilogue done) and wait only for products to complete, so the
 // scores of a chunk are computed while the previous chunk's epilogue runs and Q H while
@@ -59,8 +59,12 @@ namespace ss {
 constexpr int kGtChunk = 128;   // tokens per chunk (the MMA's M)
 constexpr int kGtDk = 128;      // key size of this kernel
 constexpr int kGtNv = 64;       // value columns per CTA
-constexpr int kGtComputeWarps = 8; // warp w: tensor-memory lane quarter w % 4, column half w / 4
+constexpr int kGtComputeWarps = 16; // warp w: tensor-memory lane quarter w % 4, column group w / 4
 constexpr int kGtComputeThreads = 32 * kGtComputeWarps;
+constexpr int kGtColGroups = kGtComputeWarps / 4;     // column groups per lane quarter
+constexpr int kGtVCols = 64 / kGtColGroups;           // value columns per compute thread
+constexpr int kGtSBlocks = 4 / kGtColGroups;          // 32-column score blocks per compute thread
+static_assert(kGtColGroups == 2 || kGtColGroups == 4, "compute warps: 8 or 16");
 constexpr int kGtThreads = kGtComputeThreads + 32; // + the issuer warp
 constexpr uint32_t kGtTmemCols = 512;
 // tensor-memory columns: fp32 accumulators S, Yi, Yh, dH; L o S as packed bf16 pairs
@@ -164,6 +168,31 @@ __device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t (&r)[32
                  : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// 16 consecutive 32-bit columns, as tmem_ld32_issue.
+__device__ __forceinline__ void tmem_ld16_issue(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                   "=r"(r[15])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_fence(uint32_t (&r)[16])
+{
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]));
+}
+// NC (16 or 32) consecutive columns of this warp's lanes (issue only).
+template <int NC> __device__ __forceinline__ void tmem_ld_n_issue(uint32_t taddr, uint32_t (&r)[NC])
+{
+    if constexpr (NC == 16)
+        tmem_ld16_issue(taddr, r);
+    else
+        tmem_ld32_issue(taddr, r);
+}
 // Ties every later use of `r` to a point after the wait (the registers a tcgen05.ld
 // writes are only valid once the wait has returned).
 __device__ __forceinline__ void tmem_ld_fence(uint32_t (&r)[32])
@@ -283,7 +312,7 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
     uint32_t *s_red = reinterpret_cast<uint32_t *>(sm + GtSmem::kRed);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool issuer = warp == kGtComputeWarps;
-    const int q4 = warp & 3, half = (warp >> 2) & 1;
+    const int q4 = warp & 3, cg = (warp >> 2) % kGtColGroups; // lane quarter, column group
     const int r = 32 * q4 + lane; // this thread's row: a token of the chunk, a key of the state
     const int64_t b = blockIdx.x / a.col_tiles;
     const int n0 = int(blockIdx.x % a.col_tiles) * kGtNv;
@@ -305,15 +334,16 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
         tmem_alloc(tmem_slot, kGtTmemCols);
         tmem_relinquish();
     }
-    // the entering state: key row r, value columns 32 half .. +31 of the tile, fp32
-    float H[32];
+    // the entering state: key row r, value columns kGtVCols cg .. + kGtVCols - 1 of the
+    // tile, fp32
+    float H[kGtVCols];
 #pragma unroll
-    for (int e = 0; e < 32; ++e)
+    for (int e = 0; e < kGtVCols; ++e)
         H[e] = 0.0f;
     if (!issuer && a.h0) {
-        const float *src = a.h0 + (b * kGtDk + r) * a.dv + n0 + 32 * half;
+        const float *src = a.h0 + (b * kGtDk + r) * a.dv + n0 + kGtVCols * cg;
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
+        for (int e = 0; e < kGtVCols; e += 4) {
             const float4 v = __ldg(reinterpret_cast<const float4 *>(src + e));
             H[e] = v.x;
             H[e + 1] = v.y;
@@ -324,12 +354,12 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
     // and its high and low bf16 parts, the B operands of Q H
     auto store_h = [&]() {
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < kGtVCols / 8; ++cc) {
             uint32_t hi[4], lo[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 split_bf16x2(H[8 * cc + 2 * e], H[8 * cc + 2 * e + 1], hi[e], lo[e]);
-            const uint32_t off = sw128_off(r, 4 * half + cc);
+            const uint32_t off = sw128_off(r, (kGtVCols / 8) * cg + cc);
             *reinterpret_cast<uint4 *>(sm + GtSmem::kHhi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
             *reinterpret_cast<uint4 *>(sm + GtSmem::kHlo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
@@ -345,8 +375,8 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
         // L o S is 0 above the diagonal in every chunk: those blocks of its tensor-memory
         // copy are written once, here, and never again
 #pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-            const int jb = 2 * half + bb;
+        for (int bb = 0; bb < kGtSBlocks; ++bb) {
+            const int jb = kGtSBlocks * cg + bb;
             if (jb > q4) {
                 const uint32_t zero[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
                 tmem_st16(tmem + lane_base + kGtColMhi + 16 * jb, zero);
@@ -528,7 +558,7 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
                     par ^= upar;
                 }
             }
-            if (half == 0 && lane == 31) {
+            if (cg == 0 && lane == 31) {
                 s_red[4 * q4] = __float_as_uint(lg);
                 s_red[4 * q4 + 1] = uint32_t(zl);
                 s_red[4 * q4 + 2] = par;
@@ -562,7 +592,7 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
             // lam of token 127, summed in the order its own row prefix was
             lam_end = __uint_as_float(s_red[12]) +
                       ((__uint_as_float(s_red[0]) + __uint_as_float(s_red[4])) + __uint_as_float(s_red[8]));
-            if (half == 0) {
+            if (cg == 0) {
                 // the column factor L[j1, r], j1 the last token of this lane quarter
                 const float lam_j1 = __uint_as_float(s_red[4 * q4]) + off;
                 const int z_j1 = max(int(s_red[4 * q4 + 1]), zoff);
@@ -582,7 +612,7 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
             const int st = int(c & 1);
             const uint32_t ph = uint32_t(c & 1), ph_kv = uint32_t((c >> 1) & 1);
             const int64_t t0 = c * kGtChunk;
-            // ---- w o V: token row r, this half's 32 value columns, as high / low parts
+            // ---- w o V: token row r, this thread's kGtVCols value columns, high / low parts
             // (the v tile has landed; dH of the previous chunk, the last reader of w o V,
             // completed before that chunk's epilogue) --------------------------------------
             if (!mbar_wait(bar_kv + st, ph_kv, status))
@@ -590,23 +620,23 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
             if (ok) {
                 const float w_r = z_end > r ? 0.0f : ((par_end ^ par_r) ? -1.0f : 1.0f) * ex2(lam_end - lam_r);
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const uint32_t o = sw128_off(r, 4 * half + cc);
+                for (int cc = 0; cc < kGtVCols / 8; ++cc) {
+                    const uint32_t o = sw128_off(r, (kGtVCols / 8) * cg + cc);
                     uint4 hi, lo;
                     scale_split8(*reinterpret_cast<const uint4 *>(sm + GtSmem::kV + st * 16384 + o), w_r, hi, lo);
                     *reinterpret_cast<uint4 *>(sm + GtSmem::kWhi + o) = hi;
                     *reinterpret_cast<uint4 *>(sm + GtSmem::kWlo + o) = lo;
                 }
             }
-            // ---- L o S: row r, this half's 64 columns, into tensor memory -------------
+            // ---- L o S: row r, this thread's 32 kGtSBlocks columns, into tensor memory
             if (!mbar_wait(bar_s, ph, status))
                 ok = false;
             ok = __all_sync(0xffffffffu, ok); // the tensor-memory accesses below are warp-collective
             tc_fence_after();
             if (ok) {
 #pragma unroll 1
-                for (int bb = 0; bb < 2; ++bb) {
-                    const int jb = 2 * half + bb;
+                for (int bb = 0; bb < kGtSBlocks; ++bb) {
+                    const int jb = kGtSBlocks * cg + bb;
                     if (jb > q4)
                         continue; // above the diagonal: the zeros written once
                     uint32_t sr[32];
@@ -673,16 +703,16 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
             tc_fence_after();
             if (ok) {
                 {
-                    uint32_t yir[32], yhr[32];
-                    tmem_ld32_issue(tmem + lane_base + kGtColYi + 32 * half, yir);
-                    tmem_ld32_issue(tmem + lane_base + kGtColYh + 32 * half, yhr);
+                    uint32_t yir[kGtVCols], yhr[kGtVCols];
+                    tmem_ld_n_issue<kGtVCols>(tmem + lane_base + kGtColYi + kGtVCols * cg, yir);
+                    tmem_ld_n_issue<kGtVCols>(tmem + lane_base + kGtColYh + kGtVCols * cg, yhr);
                     tmem_ld_wait();
                     tmem_ld_fence(yir);
                     tmem_ld_fence(yhr);
                     if (t0 + r < a.seq) {
-                        __nv_bfloat16 *dst = a.y + (b * a.seq + t0 + r) * a.dv + n0 + 32 * half;
+                        __nv_bfloat16 *dst = a.y + (b * a.seq + t0 + r) * a.dv + n0 + kGtVCols * cg;
 #pragma unroll
-                        for (int q8 = 0; q8 < 4; ++q8) {
+                        for (int q8 = 0; q8 < kGtVCols / 8; ++q8) {
                             float o[8];
 #pragma unroll
                             for (int e = 0; e < 8; ++e)
@@ -694,12 +724,12 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
                     }
                 }
                 {
-                    uint32_t dhr[32];
-                    tmem_ld32_issue(tmem + lane_base + kGtColDH + 32 * half, dhr);
+                    uint32_t dhr[kGtVCols];
+                    tmem_ld_n_issue<kGtVCols>(tmem + lane_base + kGtColDH + kGtVCols * cg, dhr);
                     tmem_ld_wait();
                     tmem_ld_fence(dhr);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
+                    for (int e = 0; e < kGtVCols; ++e)
                         H[e] = fmaf(p_endc, H[e], __uint_as_float(dhr[e]));
                 }
                 store_h();
@@ -714,9 +744,9 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
         if (!run)
             ok = false;
         if (ok) {
-            __nv_bfloat16 *dst = a.final_state + (b * kGtDk + r) * a.dv + n0 + 32 * half;
+            __nv_bfloat16 *dst = a.final_state + (b * kGtDk + r) * a.dv + n0 + kGtVCols * cg;
 #pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
+            for (int q8 = 0; q8 < kGtVCols / 8; ++q8) {
                 const float *h = H + 8 * q8;
                 *reinterpret_cast<uint4 *>(dst + 8 * q8) = make_uint4(
                     pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]), pack_bf16x2(h[4], h[5]), pack_bf16x2(h[6], h[7]));
