@@ -67,8 +67,9 @@ constexpr int kGtSBlocks = 4 / kGtColGroups;          // 32-column score blocks 
 static_assert(kGtColGroups == 2 || kGtColGroups == 4, "compute warps: 8 or 16");
 constexpr int kGtThreads = kGtComputeThreads + 32; // + the issuer warp
 constexpr uint32_t kGtTmemCols = 512;
-// tensor-memory columns: fp32 accumulators S, Yi, Yh, dH; L o S as packed bf16 pairs
-// (high and low parts, 64 columns = 128 elements each)
+// tensor-memory columns: fp32 accumulators S, Yi, Yh, and dH as two 64-column halves
+// (the products with the high and the low part of w o V, summed in the epilogue); L o S
+// as packed bf16 pairs (high and low parts, 64 columns = 128 elements each)
 constexpr uint32_t kGtColS = 0, kGtColMhi = 128, kGtColMlo = 192, kGtColYi = 256, kGtColYh = 320,
                    kGtColDH = 384;
 
@@ -392,7 +393,10 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
 
     constexpr uint32_t kIdS = idesc_bf16(128, 128, 0, 0);   // Q (K-major) x K (K-major)
     constexpr uint32_t kIdY = idesc_bf16(128, kGtNv, 0, 1); // Q or L o S (K-major) x H or V (MN-major)
-    constexpr uint32_t kIdH = idesc_bf16(128, kGtNv, 1, 1); // K^T (MN-major) x (w o V) (MN-major)
+    // K^T (MN-major) x [w o V high | w o V low] (MN-major, N = 128: the low part's tile lies
+    // one 64-column block after the high part's, the stride between N blocks)
+    constexpr uint32_t kIdH = idesc_bf16(128, 2 * kGtNv, 1, 1);
+    static_assert(GtSmem::kWlo == GtSmem::kWhi + 16384, "w o V high and low parts one block apart");
     bool ok = true;
     if (issuer) {
         // ======================= the issuer warp (lane 0 works) =======================
@@ -492,8 +496,6 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
                     const uint64_t kd = sw128_desc(kb + ks * 2048, 16384, 1024); // keys x 16 tokens (MN-major)
                     umma_bf16(tmem + kGtColDH, kd, sw128_desc(s_base + GtSmem::kWhi + ks * 2048, 16384, 1024),
                               kIdH, ks > 0);
-                    umma_bf16(tmem + kGtColDH, kd, sw128_desc(s_base + GtSmem::kWlo + ks * 2048, 16384, 1024),
-                              kIdH, 1);
                 }
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
@@ -724,13 +726,15 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
                     }
                 }
                 {
-                    uint32_t dhr[kGtVCols];
+                    uint32_t dhr[kGtVCols], dlr[kGtVCols];
                     tmem_ld_n_issue<kGtVCols>(tmem + lane_base + kGtColDH + kGtVCols * cg, dhr);
+                    tmem_ld_n_issue<kGtVCols>(tmem + lane_base + kGtColDH + kGtNv + kGtVCols * cg, dlr);
                     tmem_ld_wait();
                     tmem_ld_fence(dhr);
+                    tmem_ld_fence(dlr);
 #pragma unroll
                     for (int e = 0; e < kGtVCols; ++e)
-                        H[e] = fmaf(p_endc, H[e], __uint_as_float(dhr[e]));
+                        H[e] = fmaf(p_endc, H[e], __uint_as_float(dhr[e]) + __uint_as_float(dlr[e]));
                 }
                 store_h();
             }
