@@ -329,8 +329,12 @@ SS_API int ss_debug_set_scan_two_level(int mode);
 /*
  * Testing aid: the kernel of later ss_gated_scan calls.  mode 0 (default): the
  * chunked tensor-core form where it applies (see ss_gated_scan), 1: always the
- * token-by-token recurrence, 2: as 0.  Returns SS_OK, or SS_ERR_UNSUPPORTED for any
- * other mode.
+ * token-by-token recurrence, 2: as 0, 3: as 0, and in the tensor-core form the compute
+ * warps withhold their first "L o S written" arrival, so the issuing warp's wait for it
+ * can never be satisfied: the call ends on the wait time limit (shorten it with
+ * ss_debug_set_wait_limit) with SS_ERR_TIMEOUT in the status word and no output
+ * written (a failure-path test aid: nothing faults, every wait is bounded).  Returns
+ * SS_OK, or SS_ERR_UNSUPPORTED for any other mode.
  */
 SS_API int ss_debug_set_gated_path(int mode);
 
@@ -344,7 +348,7 @@ SS_API int ss_debug_set_gated_path(int mode);
  *
  *   q, k        : [batch, seq, dk]  dtype (SS_F32 or SS_BF16)
  *   v           : [batch, seq, dv]  dtype
- *   gamma       : [batch, seq]      float32, in [0, 1]
+ *   gamma       : [batch, seq]      float32, any real value (the page's gates are in [0, 1])
  *   h0          : [batch, dk, dv]   float32, nullable
  *   outputs     : [batch, seq, dv]  dtype (output)
  *   final_state : [batch, dk, dv]   dtype (output)

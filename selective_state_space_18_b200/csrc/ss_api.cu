@@ -266,7 +266,7 @@ template <int N, int SPL> int64_t scan_groups(int64_t batch, int64_t channels)
 // and the FMA chains' latency as two warps do.  It stays selectable
 // (ss_debug_set_scan_layout) and tested.
 std::atomic<int> g_forced_spl{0};     // ss_debug_set_scan_layout: 0 = choose per shape
-std::atomic<int> g_gated_path{0};     // ss_debug_set_gated_path: 0 auto, 1 recurrent, 2 tensor cores
+std::atomic<int> g_gated_path{0};     // ss_debug_set_gated_path: 0 auto, 1 recurrent, 2 auto, 3 auto + held arrival
 std::atomic<int> g_two_level_mode{0}; // ss_debug_set_scan_two_level: 0 auto, 1 never, 2 always
 
 int scan_spl(int64_t batch, int64_t channels, int64_t state_dim)
@@ -644,7 +644,7 @@ int ss_debug_bounds_status(ss_stream_t stream, int *site)
 
 int ss_debug_set_gated_path(int mode)
 {
-    if (mode < 0 || mode > 2)
+    if (mode < 0 || mode > 3)
         return SS_ERR_UNSUPPORTED;
     g_gated_path.store(mode, std::memory_order_relaxed);
     return SS_OK;
@@ -990,6 +990,7 @@ int launch_gated_tc(const ss::GatedArgs &g, cudaStream_t stream)
     a.y = static_cast<__nv_bfloat16 *>(g.y);
     a.final_state = static_cast<__nv_bfloat16 *>(g.final_state);
     a.col_tiles = int(g.dv / ss::kGtNv);
+    a.hold_first_mw = g_gated_path.load(std::memory_order_relaxed) == 3 ? 1 : 0;
     int64_t grid = 0;
     if (!mul_ok(g.batch, a.col_tiles, &grid) || grid > 0x7fffffffLL)
         return SS_ERR_SHAPE;

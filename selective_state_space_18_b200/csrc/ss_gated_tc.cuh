@@ -101,6 +101,7 @@ struct GatedTcArgs {
     __nv_bfloat16 *y;         // [batch, seq, dv]
     __nv_bfloat16 *final_state; // [batch, dk, dv]
     int col_tiles;            // dv / 64
+    int hold_first_mw;        // failure-path test aid: withhold the first "L o S written" arrival
 };
 
 struct GatedTcMaps {
@@ -689,7 +690,7 @@ ss_gated_tc_kernel(const GatedTcArgs a, const __grid_constant__ GatedTcMaps maps
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); // w o V writes -> MMA reads
             tc_fence_before();
             __syncwarp();
-            if (lane == 0)
+            if (lane == 0 && !(a.hold_first_mw && c == 0))
                 mbar_arrive(bar_mw);
             // ---- while dH(c) and Yi(c) run: the gate scan of the next chunk -----------
             const float p_rc = p_r, p_endc = p_end; // this chunk's, for its epilogue

@@ -276,7 +276,9 @@ def mufu_rate(op="ex2", iters=1 << 16, device=None):
 
 def ss_debug_set_gated_path(mode: int) -> None:
     """Kernel of later ss_gated_scan calls: 0 automatic (the tensor-core chunked form
-    where it applies), 1 always the token-by-token recurrence.  A testing aid."""
+    where it applies), 1 always the token-by-token recurrence, 3 automatic with the
+    tensor-core form's first "L o S written" arrival withheld (its wait runs out on the
+    wait limit: a failure-path test aid).  A testing aid."""
     st = load_library().ss_debug_set_gated_path(int(mode))
     if st != 0:
         raise SSError("ss_debug_set_gated_path", st)

@@ -105,3 +105,30 @@ def test_chunked_form_chains_through_its_final_state(orc):
     tol = TOL[torch.bfloat16]
     assert_close(torch.cat([ya, yb], 1), y.double().numpy(), tol, "outputs")
     assert_close(fb, fs.double().numpy(), tol, "final_state")
+
+
+def test_timed_out_waits_report_and_recover(orc):
+    """Failure detection in the tensor-core form without a GPU fault: with the compute
+    warps' first "L o S written" arrival withheld (a flag nothing sets) and the wait
+    limit cut to 2 ms, the issuer's wait for it gives up, the status word reports
+    SS_ERR_TIMEOUT, and the kernel still drains its loads and products before freeing
+    its tensor memory -- the next call, normal again, gives the normal answer."""
+    inp = make_gated_inputs(2, 2048, 128, 64, "bf16", seed=1970, h0=True)
+    d = {k: (None if v is None else v.cuda()) for k, v in inp.items()}
+    assert ssscan.ss_debug_status() == "SS_OK"
+    ssscan.ss_debug_set_wait_limit(2000)
+    ssscan.ss_debug_set_gated_path(3)
+    try:
+        ssscan.ss_gated_scan(**d)
+        torch.cuda.synchronize()
+        assert ssscan.ss_debug_status() == "SS_ERR_TIMEOUT"
+    finally:
+        ssscan.ss_debug_set_gated_path(0)
+        ssscan.ss_debug_set_wait_limit(0)
+    out = ssscan.ss_gated_scan(**d)
+    torch.cuda.synchronize()
+    assert ssscan.ss_debug_status() == "SS_OK"
+    ref = orc.gated_scan(**inp)
+    tol = TOL[torch.bfloat16]
+    assert_close(out["outputs"].cpu(), ref["outputs"], tol, "outputs after the timeout")
+    assert_close(out["final_state"].cpu(), ref["final_state"], tol, "final_state after the timeout")
