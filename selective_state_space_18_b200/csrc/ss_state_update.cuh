@@ -362,15 +362,21 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
         }
         // the conv state of each item's row (read by the row's lanes before its first
         // lane writes the shifted state back, below)
-        float cs[CONV ? kDecItems : 1][3];
-        if (CONV && !da.bulk_cs) {
+        // conv form: each lane evaluates, and shifts the conv state of, its own items
+        // (item v * Q + lane_q of its row group for v < kMine): their state rows only
+        float csm[kMine][3];
+        int own_cl[kMine];
+        if constexpr (CONV) {
 #pragma unroll
-            for (int it = 0; it < kDecItems; ++it) {
-                const int q = tid + it * kDecThreads;
-                const int64_t row = b * p.channels + c0 + (q < nq ? q : nq - 1) / Q;
+            for (int v = 0; v < kMine; ++v) {
+                const int q = tid + (v * Q + lane_q) * kDecThreads;
+                own_cl[v] = (q < nq ? q : nq - 1) / Q;
+                if (!da.bulk_cs) {
+                    const int64_t row = b * p.channels + c0 + own_cl[v];
 #pragma unroll
-                for (int j = 0; j < 3; ++j)
-                    cs[it][j] = j < H ? __ldg(da.conv_state + row * H + j) : 0.0f;
+                    for (int j = 0; j < 3; ++j)
+                        csm[v][j] = j < H ? __ldg(da.conv_state + row * H + j) : 0.0f;
+                }
             }
         }
         // the small operands first: their latency overlaps the wait for the state
@@ -414,15 +420,14 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
                 zs[it] = p.z ? Elem<T>::load_smem(sz + cl) : 0.0f;
             }
         }
-        if (CONV && da.bulk_cs) { // the conv state arrived with the tile
-            const float *scs = reinterpret_cast<const float *>(sb + D::kCSOff);
+        if constexpr (CONV) {
+            if (da.bulk_cs) { // the conv state arrived with the tile
+                const float *scs = reinterpret_cast<const float *>(sb + D::kCSOff);
 #pragma unroll
-            for (int it = 0; it < kDecItems; ++it) {
-                const int q = tid + it * kDecThreads;
-                const int cl = (q < nq ? q : nq - 1) / Q;
+                for (int v = 0; v < kMine; ++v)
 #pragma unroll
-                for (int j = 0; j < 3; ++j)
-                    cs[it][j] = j < H ? scs[cl * H + j] : 0.0f;
+                    for (int j = 0; j < 3; ++j)
+                        csm[v][j] = j < H ? scs[own_cl[v] * H + j] : 0.0f;
             }
         }
         if constexpr (CONV) {
@@ -432,30 +437,33 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
             float xm[kMine];
 #pragma unroll
             for (int v = 0; v < kMine; ++v) {
-                // this lane's item v * Q + lane_q: its input and conv state, selected
-                // with compile-time indices
-                float uu = xs[v * Q], s0 = cs[v * Q][0], s1 = cs[v * Q][1], s2 = cs[v * Q][2];
+                // this lane's item v * Q + lane_q: its input, selected with compile-time
+                // indices
+                float uu = xs[v * Q];
 #pragma unroll
                 for (int j = 1; j < Q; ++j)
-                    if (lane_q == j) {
+                    if (lane_q == j)
                         uu = xs[v * Q + j];
-                        s0 = cs[v * Q + j][0];
-                        s1 = cs[v * Q + j][1];
-                        s2 = cs[v * Q + j][2];
-                    }
                 float a = fmaf(cu_w[v], uu, cbi[v]); // entries e >= H hold 0, and so do their taps
-                a = fmaf(cs_w[v][0], s0, a);
-                a = fmaf(cs_w[v][1], s1, a);
-                a = fmaf(cs_w[v][2], s2, a);
+                a = fmaf(cs_w[v][0], csm[v][0], a);
+                a = fmaf(cs_w[v][1], csm[v][1], a);
+                a = fmaf(cs_w[v][2], csm[v][2], a);
                 xm[v] = silu(a);
+                // the row's conv state shifts by one input: drop the oldest, append u
+                // (only this lane reads or writes this row's conv state)
+                const int q = tid + (v * Q + lane_q) * kDecThreads;
+                if (q < nq && H > 0 && SS_IN_BOUNDS(c0 + own_cl[v] < p.channels, 207)) {
+                    float *csr = da.conv_state + (b * p.channels + c0 + own_cl[v]) * H;
+#pragma unroll
+                    for (int j = 0; j < 3; ++j)
+                        if (j < H)
+                            csr[j] = j + 1 < H ? csm[v][j + 1 < 3 ? j + 1 : 0] : uu;
+                }
             }
             const int xbase = (tid & 31) & ~(Q - 1);
 #pragma unroll
-            for (int it = 0; it < kDecItems; ++it) {
-                const float u = xs[it];
+            for (int it = 0; it < kDecItems; ++it)
                 xs[it] = Q == 1 ? xm[it] : __shfl_sync(0xffffffffu, xm[it / Q], xbase | (it % Q));
-                cs[it][0] = u; // keep u for the state shift below
-            }
         }
         // dt of the four items: the Q lanes of a row share them, so lane j computes
         // the softplus of the items it with it % Q == j and the row's lanes exchange
@@ -504,20 +512,6 @@ ss_state_update_stream_kernel(const DecArgs da, uint32_t *status)
             for (int off = Q / 2; off >= 1; off >>= 1)
                 yp += __shfl_xor_sync(0xffffffffu, yp, off);
             ysum[it] = yp; // (every lane of the row holds the row's sum)
-            if constexpr (CONV) {
-                __syncwarp(); // every lane of the row has read the conv state
-                if (valid && lane_q == 0 && H > 0 && SS_IN_BOUNDS(c0 + q / Q < p.channels, 207)) {
-                    const int64_t row = b * p.channels + c0 + q / Q;
-                    float *csr = da.conv_state + row * H;
-                    // shift: drop the oldest input (entry 0, whose register now holds u),
-                    // keep entries 1 .. H-1 from registers, append u
-#pragma unroll
-                    for (int j = 0; j < 2; ++j)
-                        if (j + 1 < H)
-                            csr[j] = cs[it][j + 1];
-                    csr[H - 1] = cs[it][0];
-                }
-            }
             if (valid && SS_IN_BOUNDS(c0 + q / Q < p.channels && b < p.batch, 204))
                 __stcs(st_tile + q, st);
         }
