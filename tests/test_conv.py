@@ -133,3 +133,31 @@ def test_decode_conv_continues_the_fused_prompt(dtype):
     assert_close(y.cpu(), full["y"][:, :, -1].double().numpy(), tol, "y")
     assert_close(st.cpu(), full["h_last"].double().numpy(), max(tol, 1e-5), "state")
     assert torch.equal(cs.cpu(), full["conv_state"])
+
+
+def test_layer_workload_full_size_sampled(orc):
+    """The fused conv form at the 2.8B layer shape it is timed on (1 x 5120 x 16 x 16384,
+    bf16, conv_k 4 with a bias, no conv state, in the benchmark's launch configuration):
+    every output and final-state entry of sampled channels -- the first and last channel
+    group and both sides of a group boundary -- against the oracle composition run on
+    those channels."""
+    from selective_state_space_18_b200.inputs import make_workload
+    inp = make_workload("mamba2p8b_layer_long")
+    ch = inp["x"].shape[1]
+    g = torch.Generator().manual_seed(4242)
+    cw = torch.randn(ch, 4, generator=g) * 0.5
+    cb = torch.randn(ch, generator=g) * 0.1
+    d = {k: (None if v is None else v.cuda()) for k, v in inp.items()}
+    out = ssscan.ss_scan_fwd_conv(d["x"], cw.cuda(), d["dt"], d["A"], d["B"], d["C"], d["D"], d["z"], d["dt_bias"],
+                                  conv_b=cb.cuda(), return_conv_state=False)
+    torch.cuda.synchronize()
+    chans = [0, 1, 15, 16, 2559, 2560, 5118, 5119]
+    y, h = out["y"][:, chans].cpu(), out["h_last"][:, chans].cpu()
+    sub = {"u": inp["x"][:, chans], "conv_w": cw[chans], "conv_b": cb[chans], "conv_state": None,
+           "dt": inp["dt"][:, chans], "A": inp["A"][chans], "B": inp["B"], "C": inp["C"],
+           "D": None if inp["D"] is None else inp["D"][chans], "z": None if inp["z"] is None else inp["z"][:, chans],
+           "dt_bias": None if inp["dt_bias"] is None else inp["dt_bias"][chans], "reset": inp.get("reset"),
+           "h0": None if inp.get("h0") is None else inp["h0"][:, chans]}
+    cv, sc = _oracle(orc, sub)
+    assert_close(y, sc["y"], TOL[torch.bfloat16], "y")
+    assert_close(h, sc["h_last"], 1e-2, "h_last")

@@ -132,3 +132,24 @@ def test_timed_out_waits_report_and_recover(orc):
     tol = TOL[torch.bfloat16]
     assert_close(out["outputs"].cpu(), ref["outputs"], tol, "outputs after the timeout")
     assert_close(out["final_state"].cpu(), ref["final_state"], tol, "final_state after the timeout")
+
+
+def test_bench_workload_full_size_sampled(orc):
+    """The workload the gated benchmark times, at full size and in its launch
+    configuration (512 items x 2048 tokens, dk 128, dv 64, bf16, the same seed): every
+    output and final-state entry of sampled items -- the first, second, middle and last
+    item, so the first and last CTAs of the grid -- against the oracle run on those items."""
+    inp = make_gated_inputs(512, 2048, 128, 64, "bf16", seed=77)
+    d = {k: (None if v is None else v.cuda()) for k, v in inp.items()}
+    out = ssscan.ss_gated_scan(d["q"], d["k"], d["v"], d["gamma"])
+    torch.cuda.synchronize()
+    assert ssscan.ss_debug_status() == "SS_OK"
+    items = [0, 1, 255, 256, 510, 511]
+    y = out["outputs"][items].cpu()
+    fs = out["final_state"][items].cpu()
+    tol = TOL[torch.bfloat16]
+    for i, b in enumerate(items):
+        sub = {k: (v[b:b + 1] if v is not None else None) for k, v in inp.items()}
+        ref = orc.gated_scan(**sub)
+        assert_close(y[i:i + 1], ref["outputs"], tol, f"outputs item {b}")
+        assert_close(fs[i:i + 1], ref["final_state"], tol, f"final_state item {b}")
