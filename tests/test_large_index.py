@@ -112,3 +112,31 @@ def test_decode_beyond_int32_state_elements(orc, batch, channels):
                      C=before["C"], D=small["D"], z=before["z"], dt_bias=small["dt_bias"])
     assert_close(ys, ref["y"], TOL[torch.bfloat16], "y")
     assert_close(st, ref["state"], 1e-4, "state")
+
+
+def test_gated_tensor_core_beyond_int32_elements(orc):
+    """The gated state scan's tensor-core form with q and k of more than 2^31 elements
+    (8200 x 2048 x 128 bf16, 4.3 GB each; dv 64): every output and final-state entry of
+    sampled batch items (the first, the last and two around the middle) against the oracle.
+    Inputs drawn on the device as the input module draws them: q, k standard normal over
+    sqrt(dk), v standard normal, gamma mostly in [0.5, 1) with about 1% exact zeros and 1%
+    exact ones."""
+    batch, seq, dk, dv = 8200, 2048, 128, 64
+    assert batch * seq * dk > 2**31
+    gd = torch.Generator(device="cuda").manual_seed(2600)
+    sc = dk ** -0.5
+    d = {"q": (torch.randn(batch, seq, dk, generator=gd, device="cuda") * sc).to(torch.bfloat16),
+         "k": (torch.randn(batch, seq, dk, generator=gd, device="cuda") * sc).to(torch.bfloat16),
+         "v": torch.randn(batch, seq, dv, generator=gd, device="cuda", dtype=torch.bfloat16)}
+    g = 0.5 + 0.5 * torch.rand(batch, seq, generator=gd, device="cuda")
+    u = torch.rand(batch, seq, generator=gd, device="cuda")
+    d["gamma"] = torch.where(u < 0.01, torch.zeros_like(g), torch.where(u > 0.99, torch.ones_like(g), g)).contiguous()
+    out = ssscan.ss_gated_scan(d["q"], d["k"], d["v"], d["gamma"])
+    assert ssscan.ss_debug_status() == "SS_OK"
+    items = [0, batch // 2 - 1, batch // 2, batch - 1]
+    y, fs = out["outputs"][items].cpu(), out["final_state"][items].cpu()
+    del out
+    for i, b in enumerate(items):
+        ref = orc.gated_scan(**{k: v[b:b + 1].cpu() for k, v in d.items()})
+        assert_close(y[i:i + 1], ref["outputs"], TOL[torch.bfloat16], f"outputs item {b}")
+        assert_close(fs[i:i + 1], ref["final_state"], TOL[torch.bfloat16], f"final_state item {b}")
