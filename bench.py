@@ -119,24 +119,35 @@ def _measured_traffic(kernel, launch=None):
     return entry.get("dram_bytes_per_launch")
 
 
+def _measured_peak(key):
+    """A figure of MEASURED_PEAKS.json as a positive float: the value itself, or the
+    "value" of an object.  None when the file, the key or a usable number is missing."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            v = json.load(f)[key]
+        if isinstance(v, dict):
+            v = v["value"]
+        v = float(v)
+        return v if v > 0 and math.isfinite(v) else None
+    except (OSError, ValueError, KeyError, TypeError):
+        return None
+
+
 def _tensor_peak_tflops():
     """Dense bf16 tensor throughput (TFLOP/s): the measured burst figure when present,
     else the pool's earlier measurement."""
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            return float(json.load(f)["bf16_tflops"])
-    except (OSError, ValueError, KeyError):
-        return 1590.0
+    v = _measured_peak("bf16_tflops")
+    return 1590.0 if v is None else v
 
 
 def _peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    try:
-        with open(path) as f:
-            p = json.load(f)
-        return float(p["hbm_gbs"]), float(p.get("sm_max_mhz", 1965.0)), "measured"
-    except (OSError, ValueError, KeyError):
+    """(HBM GB/s, SM max MHz, basis): the measured copy bandwidth when present, else the
+    pool's earlier measurement."""
+    hbm = _measured_peak("hbm_gbs")
+    if hbm is None:
         return FALLBACK_HBM_GBS, 1965.0, "fallback"
+    mhz = _measured_peak("sm_max_mhz")
+    return hbm, 1965.0 if mhz is None else mhz, "measured"
 
 
 # ---------------------------------------------------------------------------------------
@@ -435,7 +446,8 @@ def run_ours(args):
         "hbm_frac": round(scan_hbm / hbm_gbs, 4),
         "roofline_frac": round(t_roof_scan / scan_s, 4),
         "traffic": _measured_traffic("ss_scan_fwd_kernel", {k: plan[k] for k in ("grid", "segments", "seg_len")}),
-        "peak_source": f"HBM {peak_kind} (MEASURED_PEAKS.json); SFU measured per clock, at the max clock",
+        "peak_source": (f"HBM {'measured (MEASURED_PEAKS.json)' if peak_kind == 'measured' else 'fallback'} "
+                        f"{hbm_gbs:.0f} GB/s; SFU measured per clock, at the max clock"),
     }
     kernels = {
         "scan": {"ms": round(scan_ms, 5), "ms_min": round(min(scan_list), 5),

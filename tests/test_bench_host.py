@@ -29,3 +29,24 @@ def test_summary_of_a_region_shorter_than_the_period_takes_the_nearest_sample():
 
 def test_summary_without_samples_is_none():
     assert _sampler([]).summary(0.0, 1.0) is None
+
+
+def test_measured_peaks_are_read_whatever_the_file_holds(tmp_path, monkeypatch):
+    """The roofline denominators come from MEASURED_PEAKS.json when it holds usable
+    numbers (plain or as an object's "value"), and fall back to the pool's earlier
+    measurement for a missing file, a missing key or a value that is not a number."""
+    import json
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench._peaks() == (bench.FALLBACK_HBM_GBS, 1965.0, "fallback")
+    assert bench._tensor_peak_tflops() == 1590.0
+    f = tmp_path / "MEASURED_PEAKS.json"
+    f.write_text(json.dumps({"hbm_gbs": 6547.2, "bf16_tflops": 1585.0}))
+    assert bench._peaks() == (6547.2, 1965.0, "measured")
+    assert bench._tensor_peak_tflops() == 1585.0
+    f.write_text(json.dumps({"hbm_gbs": {"value": 6500.0}, "bf16_tflops": {"burst": 1}, "sm_max_mhz": 1965}))
+    assert bench._peaks() == (6500.0, 1965.0, "measured")
+    assert bench._tensor_peak_tflops() == 1590.0
+    f.write_text(json.dumps({"hbm_gbs": [1, 2]}))
+    assert bench._peaks()[2] == "fallback"
+    f.write_text("not json")
+    assert bench._peaks()[2] == "fallback"
