@@ -922,7 +922,8 @@ def run_form(args):
                                         conv_b=cb, return_conv_state=False)
             else:
                 ssscan.ss_scan_fwd(*a, y=y, h_last=hl)
-        exps = rows * L * (n + 2)
+        # N decays, the softplus and the gate per (b, t, c); the fused conv form adds its SiLU
+        exps = rows * L * (n + 3 if form == "conv" else n + 2)
         byts = 4 * rows * L * 2 + 2 * bt * n * L * 2 + rows * n * 4
         if form == "states":
             byts += rows * L * n * 4
