@@ -47,7 +47,7 @@ def _load():
         if _lib is None:
             lib = ctypes.CDLL(build())
             lib.ss_oracle_scan.argtypes = [_i64, _i64, _i64, _i64] + [_dp] * 8 + [
-                _u8p, _dp, ctypes.c_int, _dp, _dp, _dp, ctypes.c_int]
+                _u8p, _dp, ctypes.c_int, _dp, _dp, _dp, _dp, ctypes.c_int]
             lib.ss_oracle_scan.restype = ctypes.c_int
             lib.ss_oracle_tree_scan.argtypes = [_i64, _i64, _i64, _i64] + [_dp] * 8 + [
                 _u8p, _dp, ctypes.c_int, _dp, _dp, ctypes.c_int]
@@ -123,20 +123,22 @@ def _scan_args(x, dt, A, B, C, D, z, dt_bias, reset, h0):
 
 
 def scan(x, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h0=None, *,
-         dt_softplus=True, return_states=False, nthreads=None):
-    """Token-loop oracle.  Returns dict(y [b,c,L], h_last [b,c,n], h_all [b,c,L,n] or None)."""
+         dt_softplus=True, return_states=False, return_betas=False, nthreads=None):
+    """Token-loop oracle.  Returns dict(y [b,c,L], h_last [b,c,n], h_all [b,c,L,n] or None,
+    betas [b,c,L] (the step size of every token) or None)."""
     (bt, ch, n, L), (x, dt, A, B, C, D, z, dt_bias, reset, h0) = _scan_args(
         x, dt, A, B, C, D, z, dt_bias, reset, h0)
     y = np.empty((bt, ch, L))
     h_last = np.empty((bt, ch, n))
     h_all = np.empty((bt, ch, L, n)) if return_states else None
+    betas = np.empty((bt, ch, L)) if return_betas else None
     lib = _load()
     st = lib.ss_oracle_scan(bt, ch, n, L, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
                             _ptr(D), _ptr(z), _ptr(dt_bias), _ptr(reset, _u8p), _ptr(h0),
-                            int(bool(dt_softplus)), _ptr(y), _ptr(h_last), _ptr(h_all),
+                            int(bool(dt_softplus)), _ptr(y), _ptr(h_last), _ptr(h_all), _ptr(betas),
                             int(nthreads or num_threads()))
     _check(st, "ss_oracle_scan")
-    return {"y": y, "h_last": h_last, "h_all": h_all}
+    return {"y": y, "h_last": h_last, "h_all": h_all, "betas": betas}
 
 
 def tree_scan(x, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h0=None, *,

@@ -27,6 +27,10 @@
  * h0, h_last, decode state [batch, channels, state_dim].  Every array is
  * contiguous float64 except reset (uint8).
  *
+ * The token loop can also return the state after every token (h_all) and the step
+ * size of every token (betas [batch, channels, seq]: dt_t itself, which the nnterp
+ * page exposes per token and channel; its log decay dt_t * A[c,n] is that times A).
+ *
  * Two independent orderings of the same recurrence are provided:
  *   ss_oracle_scan      -- the token loop, in sequence order;
  *   ss_oracle_tree_scan -- an inclusive associative scan (recursive doubling) of
@@ -91,7 +95,7 @@ int ss_oracle_scan(int64_t batch, int64_t channels, int64_t state_dim, int64_t s
                    const double *x, const double *dt, const double *A, const double *B,
                    const double *C, const double *D, const double *z, const double *dt_bias,
                    const uint8_t *reset, const double *h0, int dt_softplus,
-                   double *y, double *h_last, double *h_all, int nthreads)
+                   double *y, double *h_last, double *h_all, double *betas, int nthreads)
 {
     if (!x || !dt || !A || !B || !C || !y)
         return ORC_ERR_NULL;
@@ -118,6 +122,8 @@ int ss_oracle_scan(int64_t batch, int64_t channels, int64_t state_dim, int64_t s
         for (int64_t t = 0; t < seq; ++t) {
             const int64_t idx = row * seq + t;
             const double d = orc_step(dt, dt_bias, dt_softplus, idx, c);
+            if (betas) /* the step size of this token (nnterp selective_scan, "betas") */
+                betas[idx] = d;
             const double xv = x[idx];
             if (reset && reset[b * seq + t]) {
                 /* state zeroed before this token's update */

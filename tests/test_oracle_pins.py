@@ -414,3 +414,49 @@ def test_decode_update_batch_independent_and_copy(orc):
         out = orc.update(**one)
         np.testing.assert_array_equal(out["y"][0], full["y"][b])
         np.testing.assert_array_equal(out["state"][0], full["state"][b])
+
+
+# --------------------------------------------------------------------------------------
+# 7. Per-token step sizes ("betas" of the nnterp selective_scan page) and log decays
+# --------------------------------------------------------------------------------------
+
+def test_betas_closed_forms(orc):
+    """The step size per token and channel: softplus(0) = ln 2 (dt_raw = -bias),
+    softplus(r) - softplus(-r) = r, the raw sum when the softplus is off, and the bias
+    added per channel before the softplus."""
+    arr = lambda v: np.array(v, dtype=np.float64)
+    r = arr([0.0, 0.3, -0.3, 2.0, -2.0, 40.0, -40.0])
+    L = r.size
+    kw = dict(x=np.ones((1, 2, L)), dt=np.stack([r, r])[None] - arr([0.5, -1.25])[None, :, None],
+              A=-np.ones((2, 1)), B=np.ones((1, 1, L)), C=np.ones((1, 1, L)), dt_bias=arr([0.5, -1.25]))
+    b = orc.scan(**kw, return_betas=True)["betas"]
+    for c in range(2):
+        assert b[0, c, 0] == pytest.approx(math.log(2), rel=1e-15)
+        for i in (1, 3, 5):
+            assert b[0, c, i] - b[0, c, i + 1] == pytest.approx(r[i], rel=1e-15)
+    raw = orc.scan(**kw, dt_softplus=False, return_betas=True)["betas"]
+    np.testing.assert_allclose(raw[0], np.stack([r, r]), rtol=0, atol=1e-15)
+
+
+def test_betas_are_the_recurrence_steps(orc):
+    """With B = 0 the state only decays: h_t = h0 exp(A sum_{s<=t} beta_s), so the
+    states after every token follow from the betas and A alone (the log decays beta_t A
+    summed); and with A = 0, C = x = 1, D = 0, the output increments by exactly
+    beta_t B_t at each token."""
+    inp = _small(71, b=2, c=3, n=4, L=20, h0=True)
+    inp["B"] = inp["B"] * 0
+    out = orc.scan(**inp, return_states=True, return_betas=True)
+    betas = out["betas"]
+    A = _np(inp["A"])
+    want = _np(inp["h0"])[:, :, None, :] * np.exp(A[None, :, None, :] * np.cumsum(betas, axis=2)[..., None])
+    assert _rel(out["h_all"], want) < 1e-13
+    inp = _small(72, b=1, c=2, n=1, L=16, z=False, D=False)
+    inp["A"] = inp["A"] * 0
+    inp["C"] = inp["C"] * 0 + 1
+    inp["x"] = inp["x"] * 0 + 1
+    out = orc.scan(**inp, return_betas=True)
+    inc = np.diff(np.concatenate([np.zeros((1, 2, 1)), out["y"]], axis=2), axis=2)
+    assert _rel(inc, out["betas"] * _np(inp["B"])[:, 0:1, :]) < 1e-13
+    # and they are the softplus of the biased raw steps, token by token, in place
+    want = _softplus(_np(inp["dt"]) + _np(inp["dt_bias"])[None, :, None])
+    assert _rel(out["betas"], want) < 1e-15
