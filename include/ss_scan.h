@@ -117,23 +117,30 @@ SS_API int ss_scan_fwd(int64_t batch, int64_t channels, int64_t state_dim, int64
                        size_t workspace_bytes, ss_stream_t stream);
 
 /*
- * ss_scan_fwd that also returns the state after every token (nnterp selective_scan:
- * the interpretability readers ask for the state after each token; TransformerLens
- * ssm_mixer: the unrolled state S_t at every position):
+ * ss_scan_fwd that also returns, per token, what the interpretability readers ask for
+ * (nnterp selective_scan: the state after each token, the step size per token and
+ * channel, and the log decay dt * A; TransformerLens ssm_mixer: the unrolled state S_t
+ * at every position):
  *
- *   h_all : [batch, channels, seq, state_dim] float32 output, required;
+ *   h_all : [batch, channels, seq, state_dim] float32 output (nullable);
  *           h_all[b,c,t,:] = h_t of row (b, c), resets and h0 included.
+ *   betas : [batch, channels, seq] float32 output (nullable): the step size of every
+ *           token, dt[b,c,t] = softplus(dt_raw[b,c,t] + dt_bias[c]) (without the
+ *           softplus when SS_DT_SOFTPLUS is clear), the value the scan itself uses.
+ *           The per-token log decay of state n is betas[b,c,t] * A[c,n].
+ * At least one of the two must be given (SS_ERR_NULL otherwise).
  *
  * Everything else is as for ss_scan_fwd (same outputs, bit-identical y and h_last).
- * h_all must not overlap any other buffer (SS_ERR_ALIAS).  The extra traffic is
- * 4 * state_dim bytes per (b, t, c) written once, so this form is bound by HBM
- * bandwidth rather than by the exponentials.
+ * h_all and betas must not overlap any other buffer or each other (SS_ERR_ALIAS).  The
+ * extra traffic is 4 * state_dim bytes per (b, t, c) for h_all and 4 for betas, each
+ * written once, so with h_all this form is bound by HBM bandwidth rather than by the
+ * exponentials.
  */
 SS_API int ss_scan_fwd_states(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
                               ss_dtype_t dtype, const void *x, const void *dt_raw, const float *A,
                               const void *B, const void *C, const float *D, const void *z,
                               const float *dt_bias, const uint8_t *reset, const float *h0,
-                              uint32_t flags, void *y, float *h_last, float *h_all,
+                              uint32_t flags, void *y, float *h_last, float *h_all, float *betas,
                               void *workspace, size_t workspace_bytes, ss_stream_t stream);
 
 /*

@@ -18,7 +18,7 @@
 
 namespace {
 
-constexpr int kAbiMajor = 2, kAbiMinor = 2;
+constexpr int kAbiMajor = 3, kAbiMinor = 0;
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -249,8 +249,8 @@ int dispatch_scan_t(const ss::ScanArgs &a, bool vec, size_t ws, cudaStream_t s)
 {
     if (a.conv_w)
         return dispatch_scan_e<N, SPL, T, false, true>(a, vec, ws, s);
-    return a.h_all ? dispatch_scan_e<N, SPL, T, true, false>(a, vec, ws, s)
-                   : dispatch_scan_e<N, SPL, T, false, false>(a, vec, ws, s);
+    return (a.h_all || a.betas) ? dispatch_scan_e<N, SPL, T, true, false>(a, vec, ws, s)
+                                : dispatch_scan_e<N, SPL, T, false, false>(a, vec, ws, s);
 }
 
 template <int N, int SPL> int64_t scan_groups(int64_t batch, int64_t channels)
@@ -453,7 +453,7 @@ int dispatch_scan_n(ss::ScanArgs a, ss_dtype_t dtype, bool vec, size_t ws_bytes,
     if constexpr (N == 16) {
         // the two-level schedule for the plain form, when the shape asks for it and the
         // workspace holds its composites
-        if (allow_two_level && a.workspace && !a.h_all && !a.conv_w) {
+        if (allow_two_level && a.workspace && !a.h_all && !a.betas && !a.conv_w) {
             const TwoLevelPlan t = two_level_plan(a.batch, a.channels, N, a.seq);
             if (t.use && int64_t(ws_bytes) >= t.bytes) {
                 if (t.spl == 4)
@@ -774,7 +774,7 @@ int ss_debug_status(ss_stream_t stream)
 namespace {
 
 // ss_scan_fwd and ss_scan_fwd_states: validation, then the launch.  h_all (nullable)
-// receives the state after every token.
+// receives the state after every token, betas (nullable) every token's step size.
 // Fused conv prologue of ss_scan_fwd_conv (w NULL: none); x is then the conv input.
 struct ConvArgs {
     const float *w = nullptr, *b = nullptr, *state = nullptr;
@@ -786,8 +786,8 @@ struct ConvArgs {
 int scan_impl(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, ss_dtype_t dtype,
               const void *x, const void *dt_raw, const float *A, const void *B, const void *C,
               const float *D, const void *z, const float *dt_bias, const uint8_t *reset,
-              const float *h0, uint32_t flags, void *y, float *h_last, float *h_all, void *workspace,
-              size_t workspace_bytes, ss_stream_t stream, const ConvArgs &cv = ConvArgs(),
+              const float *h0, uint32_t flags, void *y, float *h_last, float *h_all, float *betas,
+              void *workspace, size_t workspace_bytes, ss_stream_t stream, const ConvArgs &cv = ConvArgs(),
               bool allow_two_level = true)
 {
     if (!x || !dt_raw || !A || !B || !C || !y)
@@ -844,9 +844,20 @@ int scan_impl(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, s
         if (overlaps(h_all, abytes, y, ybytes) || (h_last && overlaps(h_all, abytes, h_last, hbytes)))
             return SS_ERR_ALIAS;
     }
+    const size_t bbytes = betas ? size_t(elems) * 4 : 0; // betas
+    if (betas) {
+        if (!aligned(betas, 4))
+            return SS_ERR_ALIGN;
+        for (int i = 0; i < 10; ++i)
+            if (overlaps(betas, bbytes, in_p[i], in_n[i]))
+                return SS_ERR_ALIAS;
+        if (overlaps(betas, bbytes, y, ybytes) || (h_last && overlaps(betas, bbytes, h_last, hbytes)) ||
+            (h_all && overlaps(betas, bbytes, h_all, abytes)))
+            return SS_ERR_ALIAS;
+    }
     size_t cbytes = 0; // conv state
     if (cv.w) {
-        if (cv.k < 1 || cv.k > 4 || h_all)
+        if (cv.k < 1 || cv.k > 4 || h_all || betas)
             return SS_ERR_UNSUPPORTED;
         const float *f32c[] = {cv.w, cv.b, cv.state, cv.state_out};
         for (const float *q : f32c)
@@ -882,6 +893,7 @@ int scan_impl(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, s
         if (overlaps(workspace, workspace_bytes, y, ybytes) ||
             (h_last && overlaps(workspace, workspace_bytes, h_last, hbytes)) ||
             (h_all && overlaps(workspace, workspace_bytes, h_all, abytes)) ||
+            (betas && overlaps(workspace, workspace_bytes, betas, bbytes)) ||
             (cv.x_out && overlaps(workspace, workspace_bytes, cv.x_out, ybytes)) ||
             (cv.state_out && overlaps(workspace, workspace_bytes, cv.state_out, cbytes)))
             return SS_ERR_ALIAS;
@@ -907,6 +919,7 @@ int scan_impl(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, s
     a.y = y;
     a.h_last = h_last;
     a.h_all = h_all;
+    a.betas = betas;
     a.conv_w = cv.w;
     a.conv_b = cv.b;
     a.conv_state = cv.state;
@@ -1088,7 +1101,7 @@ int ss_scan_fwd(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq,
                 size_t workspace_bytes, ss_stream_t stream)
 {
     return scan_impl(batch, channels, state_dim, seq, dtype, x, dt_raw, A, B, C, D, z, dt_bias, reset, h0, flags, y,
-                     h_last, nullptr, workspace, workspace_bytes, stream);
+                     h_last, nullptr, nullptr, workspace, workspace_bytes, stream);
 }
 
 int ss_scan_fwd_conv(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, ss_dtype_t dtype,
@@ -1110,19 +1123,19 @@ int ss_scan_fwd_conv(int64_t batch, int64_t channels, int64_t state_dim, int64_t
     cv.x_out = x_out;
     cv.k = int(conv_k);
     return scan_impl(batch, channels, state_dim, seq, dtype, u, dt_raw, A, B, C, D, z, dt_bias, reset, h0, flags, y,
-                     h_last, nullptr, workspace, workspace_bytes, stream, cv);
+                     h_last, nullptr, nullptr, workspace, workspace_bytes, stream, cv);
 }
 
 int ss_scan_fwd_states(int64_t batch, int64_t channels, int64_t state_dim, int64_t seq, ss_dtype_t dtype,
                        const void *x, const void *dt_raw, const float *A, const void *B, const void *C,
                        const float *D, const void *z, const float *dt_bias, const uint8_t *reset,
-                       const float *h0, uint32_t flags, void *y, float *h_last, float *h_all, void *workspace,
-                       size_t workspace_bytes, ss_stream_t stream)
+                       const float *h0, uint32_t flags, void *y, float *h_last, float *h_all, float *betas,
+                       void *workspace, size_t workspace_bytes, ss_stream_t stream)
 {
-    if (!h_all)
+    if (!h_all && !betas)
         return SS_ERR_NULL;
     return scan_impl(batch, channels, state_dim, seq, dtype, x, dt_raw, A, B, C, D, z, dt_bias, reset, h0, flags, y,
-                     h_last, h_all, workspace, workspace_bytes, stream);
+                     h_last, h_all, betas, workspace, workspace_bytes, stream);
 }
 
 } // extern "C"
@@ -1267,7 +1280,7 @@ int ss_scan_fwd_static_scratch(int64_t batch, int64_t channels, int64_t state_di
         cudaMemsetAsync(ws, 0, size_t(SS_STATIC_SCRATCH_BYTES), s) != cudaSuccess)
         return SS_ERR_CUDA;
     return scan_impl(batch, channels, state_dim, seq, dtype, x, dt_raw, A, B, C, D, z, dt_bias, reset, h0,
-                     flags & uint32_t(SS_DT_SOFTPLUS), y, h_last, nullptr, ws, SS_STATIC_SCRATCH_BYTES, stream,
+                     flags & uint32_t(SS_DT_SOFTPLUS), y, h_last, nullptr, nullptr, ws, SS_STATIC_SCRATCH_BYTES, stream,
                      ConvArgs(), false);
 }
 

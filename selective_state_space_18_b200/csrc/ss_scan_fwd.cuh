@@ -47,6 +47,7 @@ struct ScanArgs {
     void *y;
     float *h_last;
     float *h_all;             // nullable: the state after every token [b, c, L, N] fp32
+    float *betas;             // nullable: the step size dt of every token [b, c, L] fp32
     // fused causal conv + SiLU prologue (x above is then the conv's input u):
     const float *conv_w;      // [channels, conv_k] taps
     const float *conv_b;      // [channels] bias (nullable)
@@ -447,7 +448,7 @@ template <> __device__ __forceinline__ void smem_store8<float>(float *dst, const
 // from the task's eight inputs u (the raw x tile) and the three before them; x also
 // goes to the chunk's output stage (`ystage`, already free) for the epilogue, and the
 // last conv_k - 1 inputs of each row to conv_state_out.
-template <int N, int SPL, typename T, bool HAS_RESET, bool VEC, bool CONV>
+template <int N, int SPL, typename T, bool HAS_RESET, bool VEC, bool CONV, bool EMIT>
 __device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane,
                                               const IoPrefetch<N, SPL, T, HAS_RESET, VEC, CONV> &f, float *stage,
                                               unsigned char *raw, int64_t t0, int64_t g, float *ystage)
@@ -542,6 +543,25 @@ __device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane,
         pd[1] = make_float4(dtv[2].x, dtv[2].y, dtv[3].x, dtv[3].y);
         px[0] = make_float4(dxv[0].x, dxv[0].y, dxv[1].x, dxv[1].y);
         px[1] = make_float4(dxv[2].x, dxv[2].y, dxv[3].x, dxv[3].y);
+        if constexpr (EMIT) {
+            // the step sizes of this block's tokens, as the scan uses them
+            const uint32_t gpb = uint32_t(p.groups_per_batch), b32 = uint32_t(g) / gpb;
+            const int64_t c = int64_t(uint32_t(g) - b32 * gpb) * S::kChanPerCta + cl;
+            if (p.betas && c < p.channels && tl < L &&
+                SS_IN_BOUNDS(int64_t(b32) < p.batch && (int64_t(b32) * p.channels + c) * L + tl < p.batch * p.channels * L, 126)) {
+                float *dst = p.betas + (int64_t(b32) * p.channels + c) * L + tl;
+                if (tl + 8 <= L && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+                    __stcs(reinterpret_cast<float4 *>(dst), make_float4(dtv[0].x, dtv[0].y, dtv[1].x, dtv[1].y));
+                    __stcs(reinterpret_cast<float4 *>(dst) + 1, make_float4(dtv[2].x, dtv[2].y, dtv[3].x, dtv[3].y));
+                } else {
+                    const float v[8] = {dtv[0].x, dtv[0].y, dtv[1].x, dtv[1].y, dtv[2].x, dtv[2].y, dtv[3].x, dtv[3].y};
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (tl + j < L)
+                            __stcs(dst + j, v[j]);
+                }
+            }
+        }
     }
 }
 
@@ -920,7 +940,7 @@ __device__ __forceinline__ bool issuer_warp(const ScanArgs &p, const TmaMaps &ma
 
 // The two producer warps: each thread converts its share of every chunk (from the
 // raw slot, or straight from global memory on the ragged path) into the input stage.
-template <int N, int SPL, typename T, bool HAS_RESET, bool VEC, bool CONV>
+template <int N, int SPL, typename T, bool HAS_RESET, bool VEC, bool CONV, bool EMIT>
 __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, int pi, int lane)
 {
     using S = ScanShape<N, SPL>;
@@ -970,7 +990,8 @@ __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, in
         if (CONV && !mbar_wait(cx.y_empty + ys, ((i / S::kYStages) & 1u) ^ 1u, cx.status))
             return false;
         if (!end)
-            produce_chunk<N, SPL, T, HAS_RESET, VEC, CONV>(p, tl, pf, stage, cx.raw_base + r * kRawBytes, t0, g, ystage);
+            produce_chunk<N, SPL, T, HAS_RESET, VEC, CONV, EMIT>(p, tl, pf, stage, cx.raw_base + r * kRawBytes, t0, g,
+                                                                 ystage);
         if (tl == 0)
             write_meta(stage, t0, g, s, fl);
         if (!CONV && !mbar_wait(cx.y_empty + ys, ((i / S::kYStages) & 1u) ^ 1u, cx.status))
@@ -1082,7 +1103,7 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
         if (warp == S::kIssuerWarp)
             ok = issuer_warp<N, SPL, T, VEC>(p, maps, cx, lane);
         else if (prod)
-            ok = producer<N, SPL, T, HAS_RESET, VEC, CONV>(p, cx, ri, lane);
+            ok = producer<N, SPL, T, HAS_RESET, VEC, CONV, EMIT>(p, cx, ri, lane);
         else
             ok = epilogue_role<N, SPL, T, VEC, CONV>(p, y_base, y_full, y_empty, status, ri * 32 + lane);
         (void)ok; // false: gave up on a wait (SS_ERR_TIMEOUT recorded); counted out below
@@ -1164,7 +1185,7 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
             }
             const int rs = int(j % S::kRawStages);
             float *hrow = nullptr;
-            if (EMIT) {
+            if (EMIT && p.h_all) { // (the emitting form may be asked for the step sizes alone)
                 if (!SS_IN_BOUNDS(row < p.batch * p.channels && meta.t0 < p.seq, 110))
                     break;
                 hrow = p.h_all + (row * p.seq + meta.t0) * N;
@@ -1172,7 +1193,8 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
             scan_chunk<N, SPL, T, HAS_RESET, EMIT>(stage, smem_bytes + rs * S::template raw_stage_bytes<T>(),
                                                    y_base + ysi * S::template y_stage<T>() + S::kYPOff +
                                                        cl * S::kYChan + sub * S::kRow,
-                                                   cl, nn, A2, hs, hrow, cvalid ? p.seq - meta.t0 : int64_t(0));
+                                                   cl, nn, A2, hs, hrow,
+                                                   (cvalid && hrow) ? p.seq - meta.t0 : int64_t(0));
             mbar_arrive(bars + S::kBarRawEmpty + rs);
             mbar_arrive(in_empty + st);
             mbar_arrive(y_full + ysi);

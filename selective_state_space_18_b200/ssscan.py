@@ -35,7 +35,7 @@ EXPORTS = ("ss_scan_fwd", "ss_scan_workspace_bytes", "ss_scan_plan", "ss_scan_st
            "ss_status_string", "ss_abi_version", "ss_debug_mufu_probe", "ss_debug_bounds_status",
            "ss_scan_fwd_static_scratch", "ss_scan_fwd_states", "ss_gated_scan", "ss_scan_fwd_conv",
            "ss_state_update_conv", "ss_segment_decay", "ss_join_segments")
-ABI_MAJOR = 2
+ABI_MAJOR = 3
 
 _lock = threading.Lock()
 _lib = None
@@ -72,7 +72,7 @@ def load_library(path: str = LIB_PATH):
                 ctypes.c_uint32, _vp, _vp, _vp, ctypes.c_size_t, _vp]
             lib.ss_scan_fwd.restype = ctypes.c_int
             lib.ss_scan_fwd_states.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 10 + [
-                ctypes.c_uint32, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+                ctypes.c_uint32, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
             lib.ss_scan_fwd_states.restype = ctypes.c_int
             lib.ss_scan_fwd_static_scratch.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_int] + [_vp] * 10 + [
                 ctypes.c_uint32, _vp, _vp, ctypes.POINTER(_vp), _vp]
@@ -300,12 +300,15 @@ def _stream(stream, device):
 @_on_tensor_device
 def ss_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h0=None, *,
                 dt_softplus=True, y=None, h_last=None, return_last_state=True, stream=None,
-                workspace=True, h_all=None, return_states=False):
+                workspace=True, h_all=None, return_states=False, betas=None, return_betas=False):
     """Prompt scan.  x, dt, z: [batch, channels, seq]; B, C: [batch, state_dim, seq];
     A: [channels, state_dim] fp32; D, dt_bias: [channels] fp32; reset: [batch, seq]
     bool/uint8; h0: [batch, channels, state_dim] fp32.  Returns (y, h_last), or
     (y, h_last, h_all) with the state after every token [batch, channels, seq,
-    state_dim] fp32 when return_states is set or h_all is given (ss_scan_fwd_states).
+    state_dim] fp32 when return_states is set or h_all is given (ss_scan_fwd_states),
+    or (y, h_last, h_all or None, betas) with every token's step size [batch, channels,
+    seq] fp32 as well when return_betas is set or betas is given (the log decays are
+    betas[..., None] * A[:, None, :] per batch row).
 
     workspace: True (a cached per-stream workspace: segmented, balanced schedule),
     False (none: one CTA per channel group) or a zero-initialised uint8 tensor."""
@@ -347,6 +350,11 @@ def ss_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h0=Non
         h_all = torch.empty(bt, ch, L, n, device=dev, dtype=torch.float32)
     elif h_all is not None:
         h_all = _out(h_all, "h_all", dev, torch.float32, (bt, ch, L, n))
+    steps = return_betas or betas is not None
+    if betas is None and steps:
+        betas = torch.empty(bt, ch, L, device=dev, dtype=torch.float32)
+    elif betas is not None:
+        betas = _out(betas, "betas", dev, torch.float32, (bt, ch, L))
     if workspace is True:
         workspace = scan_workspace(bt, ch, n, L, dev, stream)
     elif workspace is False or workspace is None:
@@ -354,14 +362,14 @@ def ss_scan_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, reset=None, h0=Non
     elif workspace.device != dev or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous uint8 tensor on the inputs' device")
     ws_bytes = 0 if workspace is None else workspace.numel()
-    if states:
+    if states or steps:
         st = lib.ss_scan_fwd_states(bt, ch, n, L, code, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
                                     _ptr(D), _ptr(z), _ptr(dt_bias), _ptr(reset), _ptr(h0), flags,
-                                    _ptr(y), _ptr(h_last), _ptr(h_all), _ptr(workspace), ws_bytes,
+                                    _ptr(y), _ptr(h_last), _ptr(h_all), _ptr(betas), _ptr(workspace), ws_bytes,
                                     _stream(stream, dev))
         if st != 0:
             raise SSError("ss_scan_fwd_states", st)
-        return y, h_last, h_all
+        return (y, h_last, h_all, betas) if steps else (y, h_last, h_all)
     st = lib.ss_scan_fwd(bt, ch, n, L, code, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
                          _ptr(D), _ptr(z), _ptr(dt_bias), _ptr(reset), _ptr(h0), flags,
                          _ptr(y), _ptr(h_last), _ptr(workspace), ws_bytes, _stream(stream, dev))

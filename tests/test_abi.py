@@ -181,18 +181,24 @@ def test_missing_library_is_an_error(tmp_path):
 def _scan_states(lib, h_all, **kw):
     a = dict(batch=2, channels=16, state_dim=16, seq=64, dtype=ssscan.SS_BF16, x=P[0], dt=P[1],
              A=P[2], B=P[3], C=P[4], D=None, z=None, dt_bias=None, reset=None, h0=None,
-             flags=1, y=P[5], h_last=None, ws=None, ws_bytes=0, stream=None)
+             flags=1, y=P[5], h_last=None, betas=None, ws=None, ws_bytes=0, stream=None)
     a.update(kw)
     return lib.ss_scan_fwd_states(a["batch"], a["channels"], a["state_dim"], a["seq"], a["dtype"],
                                   a["x"], a["dt"], a["A"], a["B"], a["C"], a["D"], a["z"], a["dt_bias"],
-                                  a["reset"], a["h0"], a["flags"], a["y"], a["h_last"], h_all, a["ws"],
-                                  a["ws_bytes"], a["stream"])
+                                  a["reset"], a["h0"], a["flags"], a["y"], a["h_last"], h_all, a["betas"],
+                                  a["ws"], a["ws_bytes"], a["stream"])
 
 
 def test_scan_states_checks(lib):
-    """ss_scan_fwd_states: the per-token state output is required, 4-byte aligned and
-    overlaps nothing; the other arguments are checked as for ss_scan_fwd."""
+    """ss_scan_fwd_states: at least one per-token output (states or step sizes), each
+    4-byte aligned and overlapping nothing, the other arguments checked as for
+    ss_scan_fwd."""
     assert ssscan.STATUS[_scan_states(lib, None)] == "SS_ERR_NULL"
+    assert ssscan.STATUS[_scan_states(lib, None, betas=ctypes.c_void_p(P[10].value + 2))] == "SS_ERR_ALIGN"
+    assert ssscan.STATUS[_scan_states(lib, None, betas=ctypes.c_void_p(P[1].value + 64))] == "SS_ERR_ALIAS"
+    assert ssscan.STATUS[_scan_states(lib, P[9], betas=ctypes.c_void_p(P[9].value + 4096))] == "SS_ERR_ALIAS"
+    assert ssscan.STATUS[_scan_states(lib, None, betas=ctypes.c_void_p(P[5].value + 8))] == "SS_ERR_ALIAS"
+    assert ssscan.STATUS[_scan_states(lib, None, betas=P[10], state_dim=5)] == "SS_ERR_UNSUPPORTED"
     assert ssscan.STATUS[_scan_states(lib, ctypes.c_void_p(P[9].value + 2))] == "SS_ERR_ALIGN"
     assert ssscan.STATUS[_scan_states(lib, ctypes.c_void_p(P[0].value + 64))] == "SS_ERR_ALIAS"
     assert ssscan.STATUS[_scan_states(lib, ctypes.c_void_p(P[5].value))] == "SS_ERR_ALIAS"

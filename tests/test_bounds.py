@@ -92,6 +92,8 @@ def test_scan_forms_pass_every_check(checked, shape, layout):
                 _run_both(checked, lambda: ssscan.ss_scan_fwd(**d))
                 _run_both(checked, lambda: ssscan.ss_scan_fwd(**d, workspace=False))
         _run_both(checked, lambda: ssscan.ss_scan_fwd(**d, return_states=True))
+        _run_both(checked, lambda: ssscan.ss_scan_fwd(**d, return_states=True, return_betas=True))
+        _run_both(checked, lambda: ssscan.ss_scan_fwd(**d, return_betas=True))  # (y, h_last, None, betas)
         _run_both(checked, lambda: tuple(ssscan.ss_scan_fwd_conv(
             d["x"], w, d["dt"], d["A"], d["B"], d["C"], d["D"], d["z"], d["dt_bias"], d["reset"], d["h0"],
             conv_state=cs, return_x=True).values()))

@@ -110,3 +110,62 @@ def test_states_layer_workload_full_size_sampled(orc):
         assert_close(hs[i], ref["h_all"][0, 0], 1e-4, f"h_all channel {c}")
         assert_close(hls[i], ref["h_last"][0, 0], 1e-4, f"h_last channel {c}")
         assert_close(ys[i], ref["y"][0, 0], TOL[torch.bfloat16], f"y channel {c}")
+
+
+# ---- the step size of every token ("betas" of the nnterp selective_scan page) ------------
+
+@pytest.mark.parametrize("n", [4, 8, 16])
+@pytest.mark.parametrize("dtype,L", [("f32", 100), ("bf16", 264), ("bf16", 77), ("f32", 31)])
+@pytest.mark.parametrize("softplus", [True, False])
+def test_betas_match_oracle(orc, n, dtype, L, softplus):
+    """Every token's step size against the oracle's, with the states, across tile-load
+    and ragged lengths; and the log decays betas * A against the oracle's dt * A."""
+    inp = make_scan_inputs(2, 40, n, L, dtype, seed=430 + n + L, h0=True, reset_mean_doc=30)
+    if not softplus:  # positive steps without the softplus (the bias is negative): the raw steps alone
+        inp["dt"] = (inp["dt"].float().abs() * 0.1).to(inp["dt"].dtype)
+        inp["dt_bias"] = None
+    d = dev(inp, SCAN_KEYS)
+    y, h, hall, betas = ssscan.ss_scan_fwd(**d, dt_softplus=softplus, return_states=True, return_betas=True)
+    torch.cuda.synchronize()
+    ref = orc.scan(**inp, dt_softplus=softplus, return_states=True, return_betas=True)
+    assert_close(betas.cpu(), ref["betas"], 1e-4, "betas")
+    assert_close(hall.cpu(), ref["h_all"], 1e-4, "h_all")
+    assert_close(y.cpu(), ref["y"], TOL[inp["x"].dtype], "y")
+    A = inp["A"].double().numpy()
+    assert_close(betas.cpu()[..., None] * inp["A"][None, :, None, :], ref["betas"][..., None] * A[None, :, None, :],
+                 1e-4, "log decays")
+
+
+def test_betas_alone_change_nothing_else():
+    """The step sizes asked for without the states: y and h_last bit-identical to the
+    plain scan's, the step sizes bit-identical to those emitted beside the states, in
+    either schedule."""
+    inp = make_scan_inputs(3, 96, 16, 1500, "bf16", seed=440, h0=True, reset_mean_doc=200)
+    d = dev(inp, SCAN_KEYS)
+    for ws in (True, False):
+        y0, h0 = ssscan.ss_scan_fwd(**d, workspace=ws)
+        y1, h1, none, b1 = ssscan.ss_scan_fwd(**d, workspace=ws, return_betas=True)
+        _, _, _, b2 = ssscan.ss_scan_fwd(**d, workspace=ws, return_states=True, return_betas=True)
+        torch.cuda.synchronize()
+        assert none is None
+        assert torch.equal(y0, y1) and torch.equal(h0, h1)
+        assert torch.equal(b1, b2)
+
+
+def test_betas_sampled_rows_medium(orc):
+    """Many channel groups and a ragged tail: every token's step size of sampled rows."""
+    inp = make_scan_inputs(2, 512, 16, 3001, "bf16", seed=441)
+    _, _, _, betas = ssscan.ss_scan_fwd(**dev(inp, SCAN_KEYS), return_betas=True)
+    torch.cuda.synchronize()
+    rows = [(0, 0), (0, 17), (1, 255), (1, 511), (0, 300)]
+    for b, c in rows:
+        one = dict(inp)
+        for k in ("x", "dt", "z"):
+            one[k] = inp[k][b:b + 1, c:c + 1]
+        one["B"], one["C"] = inp["B"][b:b + 1], inp["C"][b:b + 1]
+        one["A"] = inp["A"][c:c + 1]
+        for k in ("D", "dt_bias"):
+            one[k] = inp[k][c:c + 1] if inp[k] is not None else None
+        one["h0"], one["reset"] = None, None
+        ref = orc.scan(**one, return_betas=True)
+        assert_close(betas[b, c].cpu(), ref["betas"][0, 0], 1e-4, f"betas row {(b, c)}")
