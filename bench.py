@@ -859,7 +859,7 @@ def run_seq_shard(args):
 # the next rows' kernels, one at a time (--form)
 # ---------------------------------------------------------------------------------------
 
-FORMS = ("scan-130m", "scan-packed", "states", "conv", "conv-decode", "gated", "gated-recurrent",
+FORMS = ("scan-130m", "scan-packed", "states", "betas", "conv", "conv-decode", "gated", "gated-recurrent",
          "segment-decay", "two-level", "single-pass-small")
 
 
@@ -885,7 +885,7 @@ def run_form(args):
     def to_dev(d):
         return {k: (None if v is None else v.to(dev)) for k, v in d.items()}
 
-    if form in ("scan-130m", "scan-packed", "states", "conv", "two-level", "single-pass-small"):
+    if form in ("scan-130m", "scan-packed", "states", "betas", "conv", "two-level", "single-pass-small"):
         wname = {"scan-130m": "mamba130m_layer", "scan-packed": "packed_resets"}.get(form, "mamba2p8b_layer_long")
         w = WORKLOADS[wname]
         if form in ("two-level", "single-pass-small"):
@@ -906,6 +906,8 @@ def run_form(args):
         hl = torch.empty(bt, ch, n, device=dev)
         if form == "states":
             hall = torch.empty(bt, ch, L, n, device=dev)
+        if form == "betas":
+            betas = torch.empty(bt, ch, L, device=dev)
         if form == "conv":
             cw = (torch.randn(ch, 4, generator=g) * 0.5).to(dev)
             cb = (torch.randn(ch, generator=g) * 0.1).to(dev)
@@ -917,6 +919,8 @@ def run_form(args):
             a = [d[k] for k in keys]
             if form == "states":
                 ssscan.ss_scan_fwd(*a, y=y, h_last=hl, h_all=hall)
+            elif form == "betas":
+                ssscan.ss_scan_fwd(*a, y=y, h_last=hl, betas=betas)
             elif form == "conv":
                 ssscan.ss_scan_fwd_conv(d["x"], cw, d["dt"], d["A"], d["B"], d["C"], d["D"], d["z"], d["dt_bias"],
                                         conv_b=cb, return_conv_state=False)
@@ -927,7 +931,10 @@ def run_form(args):
         byts = 4 * rows * L * 2 + 2 * bt * n * L * 2 + rows * n * 4
         if form == "states":
             byts += rows * L * n * 4
+        if form == "betas":
+            byts += rows * L * 4
         kernel = {"states": "ss_scan_fwd_kernel (states form)", "conv": "ss_scan_fwd_kernel (fused conv form)",
+                  "betas": "ss_scan_fwd_kernel (emitting form, step sizes only)",
                   "two-level": "ss_scan_fwd_kernel x2 + ss_segment_decay_kernel + ss_join_all_kernel (two-level)",
                   "single-pass-small": "ss_scan_fwd_kernel (single pass, chained segments)"}.get(form, "ss_scan_fwd_kernel")
         bound = "hbm" if form == "states" else "alu"

@@ -152,7 +152,7 @@ bool build_maps(const ss::ScanArgs &a, ss::TmaMaps *m)
 // Launch plan of the scan kernel instance <N, SPL, T, R, V, E, C> for the shape in `a`
 // (groups, segments, segment length and grid filled in); also what ss_scan_plan
 // reports.
-template <int N, int SPL, typename T, bool R, bool V, bool E, bool C>
+template <int N, int SPL, typename T, bool R, bool V, int E, bool C>
 int plan_scan(ss::ScanArgs &a, int64_t *grid_out, int *occ_out, int *sms_out)
 {
     using S = ss::ScanShape<N, SPL>;
@@ -211,7 +211,7 @@ int plan_scan(ss::ScanArgs &a, int64_t *grid_out, int *occ_out, int *sms_out)
     return SS_OK;
 }
 
-template <int N, int SPL, typename T, bool R, bool V, bool E, bool C>
+template <int N, int SPL, typename T, bool R, bool V, int E, bool C>
 int launch_scan(ss::ScanArgs a, size_t ws_bytes, cudaStream_t stream)
 {
     using S = ss::ScanShape<N, SPL>;
@@ -232,7 +232,7 @@ int launch_scan(ss::ScanArgs a, size_t ws_bytes, cudaStream_t stream)
     return launch_status();
 }
 
-template <int N, int SPL, typename T, bool E, bool C>
+template <int N, int SPL, typename T, int E, bool C>
 int dispatch_scan_e(const ss::ScanArgs &a, bool vec, size_t ws, cudaStream_t s)
 {
     const bool r = a.reset != nullptr;
@@ -243,14 +243,17 @@ int dispatch_scan_e(const ss::ScanArgs &a, bool vec, size_t ws, cudaStream_t s)
                : launch_scan<N, SPL, T, false, false, E, C>(a, ws, s);
 }
 
-// forms: plain; with per-token states (E); with the fused conv prologue (C)
+// forms: plain (E 0); with per-token states and optionally step sizes (E 1); with the
+// step sizes alone (E 2); with the fused conv prologue (C)
 template <int N, int SPL, typename T>
 int dispatch_scan_t(const ss::ScanArgs &a, bool vec, size_t ws, cudaStream_t s)
 {
     if (a.conv_w)
-        return dispatch_scan_e<N, SPL, T, false, true>(a, vec, ws, s);
-    return (a.h_all || a.betas) ? dispatch_scan_e<N, SPL, T, true, false>(a, vec, ws, s)
-                                : dispatch_scan_e<N, SPL, T, false, false>(a, vec, ws, s);
+        return dispatch_scan_e<N, SPL, T, 0, true>(a, vec, ws, s);
+    if (a.h_all) // the states (and the step sizes when asked for)
+        return dispatch_scan_e<N, SPL, T, 1, false>(a, vec, ws, s);
+    return a.betas ? dispatch_scan_e<N, SPL, T, 2, false>(a, vec, ws, s) // the step sizes alone
+                   : dispatch_scan_e<N, SPL, T, 0, false>(a, vec, ws, s);
 }
 
 template <int N, int SPL> int64_t scan_groups(int64_t batch, int64_t channels)

@@ -448,7 +448,7 @@ template <> __device__ __forceinline__ void smem_store8<float>(float *dst, const
 // from the task's eight inputs u (the raw x tile) and the three before them; x also
 // goes to the chunk's output stage (`ystage`, already free) for the epilogue, and the
 // last conv_k - 1 inputs of each row to conv_state_out.
-template <int N, int SPL, typename T, bool HAS_RESET, bool VEC, bool CONV, bool EMIT>
+template <int N, int SPL, typename T, bool HAS_RESET, bool VEC, bool CONV, int EMIT>
 __device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane,
                                               const IoPrefetch<N, SPL, T, HAS_RESET, VEC, CONV> &f, float *stage,
                                               unsigned char *raw, int64_t t0, int64_t g, float *ystage)
@@ -543,7 +543,7 @@ __device__ __forceinline__ void produce_chunk(const ScanArgs &p, int lane,
         pd[1] = make_float4(dtv[2].x, dtv[2].y, dtv[3].x, dtv[3].y);
         px[0] = make_float4(dxv[0].x, dxv[0].y, dxv[1].x, dxv[1].y);
         px[1] = make_float4(dxv[2].x, dxv[2].y, dxv[3].x, dxv[3].y);
-        if constexpr (EMIT) {
+        if constexpr (EMIT != 0) {
             // the step sizes of this block's tokens, as the scan uses them
             const uint32_t gpb = uint32_t(p.groups_per_batch), b32 = uint32_t(g) / gpb;
             const int64_t c = int64_t(uint32_t(g) - b32 * gpb) * S::kChanPerCta + cl;
@@ -768,9 +768,9 @@ template <int SPL> struct GroupTerms {
 // latency of one group hides behind the chain of the previous one (with one or two
 // scan warps per sub-partition there is little other work to switch to).
 //
-// EMIT: also store the state after every token to `hrow` (this channel's row of h_all
-// at the chunk's first token, N floats per token), for the first `valid` tokens.
-template <int N, int SPL, typename T, bool HAS_RESET, bool EMIT>
+// EMIT == 1: also store the state after every token to `hrow` (this channel's row of
+// h_all at the chunk's first token, N floats per token), for the first `valid` tokens.
+template <int N, int SPL, typename T, bool HAS_RESET, int EMIT>
 __device__ __forceinline__ void scan_chunk(const float *stage, const unsigned char *raw, float *ys, int cl,
                                            const int (&nn)[SPL], const float2 (&A2)[SPL], float (&hs)[SPL],
                                            float *hrow, int64_t valid)
@@ -853,7 +853,7 @@ __device__ __forceinline__ void scan_chunk(const float *stage, const unsigned ch
             for (int j = 1; j < SPL; ++j)
                 yy = __ffma2_rn(bc_pair<T>(cc[j], pi), make_float2(hm[j], hs[j]), yy);
             yo[pr] = yy;
-            if (EMIT) {
+            if (EMIT == 1) {
                 const int tt = t + 2 * pr;
 #pragma unroll
                 for (int j = 0; j < SPL; ++j) {
@@ -940,7 +940,7 @@ __device__ __forceinline__ bool issuer_warp(const ScanArgs &p, const TmaMaps &ma
 
 // The two producer warps: each thread converts its share of every chunk (from the
 // raw slot, or straight from global memory on the ragged path) into the input stage.
-template <int N, int SPL, typename T, bool HAS_RESET, bool VEC, bool CONV, bool EMIT>
+template <int N, int SPL, typename T, bool HAS_RESET, bool VEC, bool CONV, int EMIT>
 __device__ __forceinline__ bool producer(const ScanArgs &p, const CtaCtx &cx, int pi, int lane)
 {
     using S = ScanShape<N, SPL>;
@@ -1032,12 +1032,12 @@ __device__ __forceinline__ bool epilogue_role(const ScanArgs &p, const float *y_
 // CTAs per SM to plan registers for: the states and conv forms need more registers
 // than the plain form and are bounded to two CTAs per SM wherever shared memory fits
 // two (about 113 KB each); the plain form gets there at its natural allocation.
-template <int N, int SPL, typename T, bool EMIT, bool CONV> constexpr int scan_min_ctas()
+template <int N, int SPL, typename T, int EMIT, bool CONV> constexpr int scan_min_ctas()
 {
-    return (EMIT || CONV) && ScanShape<N, SPL>::template smem_bytes<T, true>() <= 113 * 1024 ? 2 : 1;
+    return (EMIT != 0 || CONV) && ScanShape<N, SPL>::template smem_bytes<T, true>() <= 113 * 1024 ? 2 : 1;
 }
 
-template <int N, int SPL, typename T, bool HAS_RESET, bool VEC, bool EMIT, bool CONV>
+template <int N, int SPL, typename T, bool HAS_RESET, bool VEC, int EMIT, bool CONV>
 __global__ void __launch_bounds__(ScanShape<N, SPL>::kThreads, (scan_min_ctas<N, SPL, T, EMIT, CONV>()))
 ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
 {
@@ -1185,7 +1185,7 @@ ss_scan_fwd_kernel(const ScanArgs p, const __grid_constant__ TmaMaps maps)
             }
             const int rs = int(j % S::kRawStages);
             float *hrow = nullptr;
-            if (EMIT && p.h_all) { // (the emitting form may be asked for the step sizes alone)
+            if (EMIT == 1 && p.h_all) {
                 if (!SS_IN_BOUNDS(row < p.batch * p.channels && meta.t0 < p.seq, 110))
                     break;
                 hrow = p.h_all + (row * p.seq + meta.t0) * N;
