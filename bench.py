@@ -442,6 +442,10 @@ def run_ours(args):
         "frac_at_measured_clock": (round(scan_exps_rate / (sms * ex2_rate * sm_clk * 1e6), 4)
                                    if sm_clk else None),
         "exps_per_launch": pw["exps"],
+        # every MUFU op the kernel issues, per (b, t, c) of this bf16 workload: the N decays,
+        # the softplus's exponential (its log1p is a polynomial on the FMA pipe) and the
+        # gate's tanh (sigmoid(z) = (1 + tanh(z/2)) / 2): no MUFU log or reciprocal
+        "mufu_ops_per_launch": pw["exps"] if PROMPT.dtype == "bf16" else None,
         "algorithmic_bytes_per_launch": pw["bytes"],
         "hbm_achieved_gbs": round(scan_hbm, 1),
         "hbm_peak_gbs": hbm_gbs,
